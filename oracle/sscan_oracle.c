@@ -1,0 +1,218 @@
+/*
+ * sscan_oracle.c -- fp64 CPU oracle for the selective-scan (S6) forward.
+ *
+ * TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only the test suite, the smoke
+ * check and the CPU-baseline leg of the benchmark load this library.  It
+ * shares no code, header, table or helper with the CUDA path, and the CUDA
+ * path never calls it.
+ *
+ * What it computes is the plain definition of the forward pass, one
+ * sequential loop over time per (batch b, channel d) row, in double
+ * precision:
+ *
+ *   Abar[t,n] = exp(delta[b,t,d] * A[d,n])                      (ZOH of A)
+ *   Euler:  bu[t,n] = delta[b,t,d] * B[b,t,n] * u[b,t,d]
+ *   ZOH:    bu[t,n] = (exp(delta*A[d,n]) - 1) / A[d,n] * B[b,t,n] * u[b,t,d]
+ *   h[n]    = Abar[t,n] * h[n] + bu[t,n]          h before t=0 is h0 (or 0)
+ *   y[b,t,d] = sum_n C[b,t,n] * h[n]              (state AFTER token t)
+ *   h_final[b,d,n] = h[n] after the last token
+ *
+ * Sources (page title, section):
+ *  - "tm_ssm_selective" (Transformer Math page on selective SSMs), section
+ *    "Discretization becomes a per-token operation": per-token ZOH
+ *    Abar = exp(Delta_t A) elementwise for diagonal A, the exact ZOH input
+ *    term (Delta A)^-1 (exp(Delta A) - I) Delta B, its Euler limit Delta B
+ *    ("what implementations actually use"), the diagonal recurrence and the
+ *    readout y_t = sum_n C_t[n] x_t[:, n]; shapes from section
+ *    "The mechanism: parameters as functions of the input".
+ *  - "12. Selective State Space", the selective_scan reference loop: the
+ *    tensors u, delta:(batch, seq, d_inner), A:(d_inner, d_state),
+ *    B, C:(batch, seq, d_state), the state update followed by the readout
+ *    of the updated state at the same step.
+ *  - "Mamba & Mamba-2 Architecture", section 1 (shapes B,C:[B,L,N],
+ *    Delta:[B,L,D], A:[D,N]) and the numpy listing in section "Code"
+ *    (update, then y_t = c_t . h).
+ *
+ * Readings where the pages leave a step open:
+ *  - y at step t reads the state after token t's update (all listings agree).
+ *  - h0 is an optional input (the pages start from zero); NULL means zero.
+ *  - ZOH with A[d,n] == 0 takes the limit (exp(Delta*A)-1)/A -> Delta.
+ *  - Delta arrives already positive: softplus belongs to the projection
+ *    layer that produces it, not to the scan.
+ *
+ * Rows are independent (each (b,d) row has its own state), so rows are
+ * spread over POSIX threads; the per-row arithmetic is the same sequential
+ * loop whatever the thread count, so results do not depend on it.
+ *
+ * Build: gcc -O2 -ffp-contract=off -fPIC -shared -pthread ... -lm
+ * (-ffp-contract=off keeps every multiply and add separately rounded).
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+/* One (b,d) row: the sequential recurrence over L tokens.
+ *   u[t*su], dl[t*sd]   input and step size of this channel at token t
+ *   a[n]                the channel's diagonal A row
+ *   Bm[t*N+n], Cm[t*N+n] the batch's input / output projections
+ *   h0[n]               initial state, or NULL for zero
+ *   y[t*sy]             output of this channel at token t
+ *   hfin[n]             final state, or NULL
+ *   h                   scratch of N doubles */
+static void scan_row(int64_t L, int64_t N,
+                     const double *u, int64_t su,
+                     const double *dl, int64_t sd,
+                     const double *a,
+                     const double *Bm, const double *Cm,
+                     const double *h0, int zoh,
+                     double *y, int64_t sy, double *hfin, double *h)
+{
+    for (int64_t n = 0; n < N; ++n)
+        h[n] = h0 ? h0[n] : 0.0;
+    for (int64_t t = 0; t < L; ++t) {
+        const double delta = dl[t * sd];
+        const double x = u[t * su];
+        const double *Bt = Bm + t * N;
+        const double *Ct = Cm + t * N;
+        double acc = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+            const double abar = exp(delta * a[n]);
+            double bbar;
+            if (zoh)
+                bbar = (a[n] != 0.0) ? expm1(delta * a[n]) / a[n] * Bt[n] : delta * Bt[n];
+            else
+                bbar = delta * Bt[n];
+            h[n] = abar * h[n] + bbar * x;
+            acc += Ct[n] * h[n];
+        }
+        y[t * sy] = acc;
+    }
+    if (hfin)
+        for (int64_t n = 0; n < N; ++n)
+            hfin[n] = h[n];
+}
+
+/* How a row index maps onto the caller's arrays. */
+typedef struct {
+    int64_t B, L, D, N;
+    int rows_mode;            /* 0: all B*D rows of full tensors; 1: an explicit row list */
+    const double *u, *dl, *A, *Bm, *Cm, *h0;
+    double *y, *hfin;
+    const int64_t *row_b;     /* rows_mode 1: batch index of each row */
+    int64_t nrows;
+    int zoh;
+} job_t;
+
+typedef struct {
+    const job_t *job;
+    int64_t r0, r1;
+    int status;
+} slice_t;
+
+static void run_row(const job_t *j, int64_t r, double *h)
+{
+    const int64_t L = j->L, N = j->N, D = j->D;
+    if (j->rows_mode == 0) {
+        /* full tensors: u,delta,y [B][L][D]; A [D][N]; B,C [B][L][N]; h0,h_final [B][D][N] */
+        const int64_t b = r / D, d = r % D;
+        scan_row(L, N,
+                 j->u + b * L * D + d, D,
+                 j->dl + b * L * D + d, D,
+                 j->A + d * N,
+                 j->Bm + b * L * N, j->Cm + b * L * N,
+                 j->h0 ? j->h0 + (b * D + d) * N : NULL, j->zoh,
+                 j->y + b * L * D + d, D,
+                 j->hfin ? j->hfin + (b * D + d) * N : NULL, h);
+    } else {
+        /* row list: u,delta,y [R][L]; A,h0,h_final [R][N]; B,C [B][L][N] indexed by row_b[r] */
+        const int64_t b = j->row_b[r];
+        scan_row(L, N,
+                 j->u + r * L, 1,
+                 j->dl + r * L, 1,
+                 j->A + r * N,
+                 j->Bm + b * L * N, j->Cm + b * L * N,
+                 j->h0 ? j->h0 + r * N : NULL, j->zoh,
+                 j->y + r * L, 1,
+                 j->hfin ? j->hfin + r * N : NULL, h);
+    }
+}
+
+static void *run_slice(void *arg)
+{
+    slice_t *s = (slice_t *)arg;
+    double *h = (double *)malloc(sizeof(double) * (size_t)(s->job->N > 0 ? s->job->N : 1));
+    if (!h) { s->status = 2; return NULL; }
+    for (int64_t r = s->r0; r < s->r1; ++r)
+        run_row(s->job, r, h);
+    free(h);
+    s->status = 0;
+    return NULL;
+}
+
+static int run_job(const job_t *j, int64_t nrows, int nthreads)
+{
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 1024) nthreads = 1024;
+    if ((int64_t)nthreads > nrows) nthreads = (int)(nrows > 0 ? nrows : 1);
+    slice_t *sl = (slice_t *)calloc((size_t)nthreads, sizeof(slice_t));
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!sl || !th) { free(sl); free(th); return 2; }
+    int rc = 0, started = 0;
+    for (int i = 0; i < nthreads; ++i) {
+        sl[i].job = j;
+        sl[i].r0 = nrows * i / nthreads;
+        sl[i].r1 = nrows * (i + 1) / nthreads;
+        sl[i].status = 1;
+        if (i == nthreads - 1) break;          /* the calling thread takes the last slice */
+        if (pthread_create(&th[i], NULL, run_slice, &sl[i]) != 0) { rc = 3; break; }
+        ++started;
+    }
+    if (rc == 0) run_slice(&sl[nthreads - 1]);
+    for (int i = 0; i < started; ++i) pthread_join(th[i], NULL);
+    for (int i = 0; rc == 0 && i < nthreads; ++i)
+        if (sl[i].status != 0) rc = sl[i].status;
+    free(sl);
+    free(th);
+    return rc;
+}
+
+/* Full forward over contiguous row-major tensors.
+ *   u, delta, y : [B][L][D]     A : [D][N]     Bm, Cm : [B][L][N]
+ *   h0, h_final : [B][D][N]     (either may be NULL)
+ * Returns 0 on success, 1 for bad sizes or pointers, 2/3 on allocation or
+ * thread-creation failure. */
+int sscan_oracle_forward(int64_t B, int64_t L, int64_t D, int64_t N,
+                         const double *u, const double *delta, const double *A,
+                         const double *Bm, const double *Cm, const double *h0,
+                         int zoh, double *y, double *h_final, int nthreads)
+{
+    if (B < 0 || L < 0 || D < 0 || N < 0) return 1;
+    if (B == 0 || D == 0) return 0;
+    if (N > 0 && (!A || ((L > 0) && (!Bm || !Cm)))) return 1;
+    if (L > 0 && (!u || !delta || !y)) return 1;
+    job_t j = {B, L, D, N, 0, u, delta, A, Bm, Cm, h0, y, h_final, NULL, B * D, zoh};
+    return run_job(&j, B * D, nthreads);
+}
+
+/* The same recurrence on an explicit list of R rows (for sampling large
+ * problems row by row; rows are independent, so a sampled row is exact).
+ *   row_b      : [R]     batch index of each row (indexes Bm/Cm)
+ *   u_rows, delta_rows, y_rows : [R][L]   the row's channel, gathered
+ *   A_rows, h0_rows, hfin_rows : [R][N]   (h0_rows / hfin_rows may be NULL)
+ *   Bm, Cm     : [Bn][L][N] */
+int sscan_oracle_rows(int64_t R, int64_t L, int64_t N, int64_t Bn,
+                      const int64_t *row_b,
+                      const double *u_rows, const double *delta_rows, const double *A_rows,
+                      const double *Bm, const double *Cm, const double *h0_rows,
+                      int zoh, double *y_rows, double *hfin_rows, int nthreads)
+{
+    if (R < 0 || L < 0 || N < 0 || Bn < 0) return 1;
+    if (R == 0) return 0;
+    if (!row_b) return 1;
+    for (int64_t r = 0; r < R; ++r)
+        if (row_b[r] < 0 || row_b[r] >= Bn) return 1;
+    job_t j = {Bn, L, 0, N, 1, u_rows, delta_rows, A_rows, Bm, Cm, h0_rows,
+               y_rows, hfin_rows, row_b, R, zoh};
+    return run_job(&j, R, nthreads);
+}
