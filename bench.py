@@ -1,0 +1,368 @@
+#!/usr/bin/env python
+"""Benchmark of the selective-scan forward on B200 (one process per GPU).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+For N > 1 launch one rank per GPU with torch.distributed.run; each rank runs the
+same shape on its own shard of the job (batch rows are independent, so there is
+no data-path collective: weak scaling), the timed region is bracketed by a
+barrier and a device synchronise, and the slowest rank's time is reported.
+
+A step is one full forward over the workload (discretise, recurrence, readout,
+final state) with inputs already resident in HBM.  Rank 0 prints one JSON line.
+``--impl reference`` times the fp64 CPU oracle instead (host cores, rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from selective_state_space_32_b200 import workloads as W  # noqa: E402
+
+METRIC = "selective-scan elements (B*L*D)/s"
+UNIT = "elements/s"
+L2_BYTES = 126 * 1024 * 1024
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+SM_COUNT = 148
+SM_MAX_MHZ = 1965.0
+# ALU roofline of one state update on B200 (per SM per clock): 16 MUFU ex2 and
+# 128 FP32 FMA-pipe lanes.  An update needs one 2^x and four FMA-pipe ops
+# (delta*A, B*(delta*u), Abar*h + Bbar u, y += C*h); a 2^x can instead be
+# computed on the FMA pipe with eight ops (range reduction + degree-5
+# polynomial).  Balancing the two pipes: f = 4/15 of the exps in software gives
+# 16 / (1 - 4/15) = 21.8 updates per SM per clock.
+ALU_UPDATES_PER_SM_CLK = 16.0 / (1.0 - 4.0 / 15.0)
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p.get("sm_max_mhz", SM_MAX_MHZ)), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, SM_MAX_MHZ, "fallback"
+
+
+# ---------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for k, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------- CPU oracle --
+
+def cpu_oracle_rate(g, w, min_seconds=10.0, max_seconds=30.0):
+    """Time the fp64 oracle as it stands on this host's cores: full passes over the
+    workload until at least ``min_seconds`` elapsed.  Returns (elements/s, cores, sample)."""
+    from oracle import oracle as O
+    v = {k: (None if g[k] is None else W.as_f32(g[k], g["dtype"]).astype(np.float64))
+         for k in ("u", "delta", "B", "C")}
+    A = g["A"].astype(np.float64)
+    h0 = None if g["h0"] is None else g["h0"].astype(np.float64)
+    cores = O.host_threads()
+    n, t0 = 0, time.perf_counter()
+    while True:
+        O.forward(v["u"], v["delta"], A, v["B"], v["C"], h0, w.zoh, nthreads=cores)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or el + el / n > max_seconds:
+            break
+    return n * w.elements / el, cores, f"{n} full pass(es) over the workload ({w.elements} elements each) in {el:.2f} s"
+
+
+# -------------------------------------------------------------- our arm --
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from selective_state_space_32_b200 import sscan as S
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = W.WORKLOADS[args.workload]
+    # shard: rank r owns batch rows [r*B, (r+1)*B) of an N*B-row job (own seed)
+    g = W.generate(w.B, w.L, w.D, w.N, w.dtype, w.h0_std, w.reset_frac,
+                   seed=W.SEED_BASE + w.index + 1000 * rank)
+    tdt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+
+    def host(x, dt):
+        if x is None:
+            return None
+        if dt == "bf16":
+            t = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16)
+        else:
+            t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+        return t.pin_memory()
+
+    hin = {"u": host(g["u"], w.dtype), "delta": host(g["delta"], w.dtype),
+           "A": host(g["A"], "f32"), "B": host(g["B"], w.dtype), "C": host(g["C"], w.dtype),
+           "h0": host(g["h0"], "f32")}
+    din = {k: (None if v is None else v.to(dev)) for k, v in hin.items()}
+    plan = S.Plan(w.B, w.L, w.D, w.N, tdt, w.zoh)
+    ws = plan.new_workspace(dev)
+    y = torch.empty((w.B, w.L, w.D), dtype=tdt, device=dev)
+    hf = torch.empty((w.B, w.D, w.N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        plan.forward(din["u"], din["delta"], din["A"], din["B"], din["C"], din["h0"],
+                     y=y, h_final=hf, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if plan.status(stream) != S.OK:
+        raise RuntimeError("device status word reported an error during warm-up")
+
+    # ---- timed region: K steps, events around every launch (kernel time) ----
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    kern_ms = [a.elapsed_time(b) for a, b in ev]
+    if plan.status(stream) != S.OK:
+        raise RuntimeError("device status word reported an error in the timed region")
+
+    # ---- end to end: host buffers through the public API, copies inside ----
+    out_h = (torch.empty(y.shape, dtype=y.dtype).pin_memory(),
+             torch.empty(hf.shape, dtype=hf.dtype).pin_memory())
+    e2e_steps = max(1, min(args.steps, 20))
+
+    def e2e_step():
+        S.forward_host(hin["u"], hin["delta"], hin["A"], hin["B"], hin["C"], hin["h0"],
+                       zoh=w.zoh, device=dev, out=out_h)
+
+    for _ in range(min(args.warmup, 3)):
+        e2e_step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    h2d = sum(v.numel() * v.element_size() for v in hin.values() if v is not None)
+    d2h = sum(v.numel() * v.element_size() for v in out_h)
+
+    # ---- max over ranks ----
+    t = torch.tensor([elapsed_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_ms, e2e_ms = float(t[0]), float(t[1])
+
+    if rank != 0:
+        return None
+    hbm_peak, sm_max, peak_src = load_peaks()
+    kmean = sum(kern_ms) / len(kern_ms)
+    value = w.elements * args.steps * world / (elapsed_ms / 1e3)
+    alg_bytes = w.algorithmic_bytes()
+    hbm_achieved = alg_bytes / (kmean / 1e3) / 1e9
+    upd_rate = w.updates / (kmean / 1e3) / 1e9
+    alu_peak = ALU_UPDATES_PER_SM_CLK * SM_COUNT * sm_max * 1e6 / 1e9
+    traffic = None
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            tr = json.load(f).get(args.workload)
+            traffic = tr if isinstance(tr, (int, float)) else None
+    except Exception:
+        pass
+    cpu_value, cores, sample = cpu_oracle_rate(g, w, args.cpu_seconds, 3 * args.cpu_seconds)
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"{w.name}: B={w.B} L={w.L} D={w.D} N={w.N} io={w.dtype} "
+                               f"{'ZOH' if w.zoh else 'Euler'} h0={'yes' if w.h0_std else 'no'}",
+                   "B": w.B, "L": w.L, "D": w.D, "N": w.N, "io_dtype": w.dtype,
+                   "parallelism": f"dp{world} (independent batch-row shards, no collective)",
+                   "l2": f"inputs larger than L2 ({alg_bytes / 1e6:.0f} MB per step vs "
+                         f"{L2_BYTES / 2**20:.0f} MiB L2); no flush"},
+        "roofline": {"bound": "alu", "achieved": upd_rate, "peak": alu_peak,
+                     "unit": "Gupdates/s", "frac": upd_rate / alu_peak, "traffic": traffic,
+                     "kernel": "sscan_fwd_kernel",
+                     "peak_basis": f"{ALU_UPDATES_PER_SM_CLK:.1f} state updates/SM/clk "
+                                   f"(16 MUFU + 128 FMA lanes) x {SM_COUNT} SMs x {sm_max:.0f} MHz"},
+        "hbm": {"achieved": hbm_achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": hbm_achieved / hbm_peak, "peak_source": peak_src,
+                "algorithmic_bytes_per_step": alg_bytes},
+        "kernel_ms": {"mean": kmean, "min": min(kern_ms), "max": max(kern_ms)},
+        "e2e": {"value": w.elements * e2e_steps * world / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+        "cpu_baseline": {"value": cpu_value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+    }
+    plan.close()
+    return out
+
+
+# -------------------------------------------------------- reference arm --
+
+def run_reference(args):
+    w = W.WORKLOADS[args.workload]
+    g = W.make_inputs(w)
+    from oracle import oracle as O
+    v = {k: W.as_f32(g[k], g["dtype"]).astype(np.float64) for k in ("u", "delta", "B", "C")}
+    A = g["A"].astype(np.float64)
+    h0 = None if g["h0"] is None else g["h0"].astype(np.float64)
+    cores = O.host_threads()
+    # each step: a bounded sample of the workload's rows (rows are independent)
+    target = max(1.0, args.ref_step_seconds)
+    rows_all = [(b, d) for b in range(w.B) for d in range(w.D)]
+    probe = rows_all[: max(1, len(rows_all) // 64)]
+    t0 = time.perf_counter()
+    O.forward_rows(probe, v["u"], v["delta"], A, v["B"], v["C"], h0, w.zoh, nthreads=cores)
+    per_row = (time.perf_counter() - t0) / len(probe)
+    nrows = int(min(len(rows_all), max(1, target / max(per_row, 1e-9))))
+    rng = np.random.default_rng(0)
+    sel = [rows_all[i] for i in sorted(rng.choice(len(rows_all), nrows, replace=False))]
+    for _ in range(args.warmup):
+        O.forward_rows(sel[: max(1, nrows // 8)], v["u"], v["delta"], A, v["B"], v["C"], h0,
+                       w.zoh, nthreads=cores)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        O.forward_rows(sel, v["u"], v["delta"], A, v["B"], v["C"], h0, w.zoh, nthreads=cores)
+        times.append(time.perf_counter() - t0)
+    tot = sum(times)
+    value = nrows * w.L * args.steps / tot
+    sample = f"{nrows} of {len(rows_all)} (b,d) rows x {w.L} tokens per step"
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{w.name}: B={w.B} L={w.L} D={w.D} N={w.N} io={w.dtype} "
+                               f"{'ZOH' if w.zoh else 'Euler'} h0={'yes' if w.h0_std else 'no'}",
+                   "B": w.B, "L": w.L, "D": w.D, "N": w.N, "io_dtype": w.dtype},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="mamba130m_f32", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="minimum host time spent timing the CPU oracle baseline")
+    ap.add_argument("--ref-step-seconds", type=float, default=2.0,
+                    help="host time per step of the reference (oracle) arm")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            ap.error("--gpus > 1 needs one process per GPU (torch.distributed.run)")
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,139 @@
+/*
+ * sscan.h -- C ABI of the B200 (sm_100a) selective-scan forward library
+ * (libsscan.so).
+ *
+ * The operation ("tm_ssm_selective" (Transformer Math page on selective
+ * SSMs), section "Discretization becomes a per-token operation"; the
+ * selective_scan reference loop of "12. Selective State Space"; shapes from
+ * "Mamba & Mamba-2 Architecture", section 1): for every batch row b, channel
+ * d and state n, with the step delta = delta[b,t,d] and x = u[b,t,d],
+ *
+ *     Abar       = exp(delta * A[d,n])                     (zero-order hold of A)
+ *     Bbar u     = delta * B[b,t,n] * x                    (Euler, the default)
+ *                | (exp(delta*A[d,n]) - 1) / A[d,n] * B[b,t,n] * x   (SSCAN_ZOH)
+ *     h[b,d,n]   = Abar * h[b,d,n] + Bbar u                (h before t = 0: h0, or 0)
+ *     y[b,t,d]   = sum_n C[b,t,n] * h[b,d,n]               (state after token t)
+ *     h_final[b,d,n] = h after the last token
+ *
+ * The [B,L,D,N] state sequence is never written to memory: each (b,d) state
+ * row lives in registers ("Selective State-Space Models (Mamba) and
+ * Hardware-Aware Scans", section 3, kernel fusion and SRAM residency).
+ *
+ * Layout.  Every tensor is dense row-major (C order), in device memory:
+ *     u, delta, y : [B][L][D]   dtype of the plan (fp32 or bf16)
+ *     B, C        : [B][L][N]   dtype of the plan
+ *     A           : [D][N]      fp32 (the pages' A = -exp(A_log), diagonal)
+ *     h0, h_final : [B][D][N]   fp32 (the state is always kept in fp32)
+ * Every pointer must be 16-byte aligned.  The state and all arithmetic are
+ * fp32; a bf16 plan widens its inputs exactly and rounds y to nearest-even.
+ *
+ * Ownership.  The caller owns every buffer passed in (inputs, outputs and
+ * the workspace).  A plan owns its host-side description and one 4-byte
+ * device status word that it allocates at creation and frees on destroy.
+ *
+ * Streams and errors.  sscan_forward enqueues its work on the caller's
+ * stream and returns without synchronising.  Every entry point returns an
+ * SSCAN_* status: argument problems are reported before anything is
+ * launched; a failed launch gives SSCAN_ERR_CUDA.  Conditions only the
+ * device can see (a bounded wait that gave up) are latched in the plan's
+ * status word and read back with sscan_get_status.
+ *
+ * Aliasing.  y must not overlap any input.  h_final may be the same buffer
+ * as h0 (each state row is read before it is written, by the same thread).
+ *
+ * Thread safety.  A plan may be used from one host thread at a time; calls
+ * with distinct plans are independent.
+ */
+#ifndef SSCAN_H
+#define SSCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SSCAN_API __attribute__((visibility("default")))
+#else
+#define SSCAN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct sscan_plan *sscan_plan_t;
+
+/* dtype of u, delta, B, C and y */
+enum { SSCAN_F32 = 0, SSCAN_BF16 = 1 };
+
+/* flags */
+enum {
+    /* exact zero-order-hold input term (exp(delta*A)-1)/A * B * u instead of
+     * the Euler term delta * B * u ("tm_ssm_selective", section
+     * "Discretization becomes a per-token operation") */
+    SSCAN_ZOH = 1u << 0
+};
+
+/* status codes */
+enum {
+    SSCAN_OK = 0,
+    SSCAN_ERR_INVALID = 1,      /* bad size, null pointer, overlapping output, bad flag */
+    SSCAN_ERR_UNSUPPORTED = 2,  /* N outside {16, 32, 64}, or no usable CUDA device */
+    SSCAN_ERR_ALIGN = 3,        /* a pointer is not 16-byte aligned */
+    SSCAN_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+    SSCAN_ERR_TIMEOUT = 5,      /* device side: a bounded wait for another block gave up */
+    SSCAN_ERR_WORKSPACE = 6     /* workspace missing, misaligned or too small */
+};
+
+/* Create a plan for one problem shape on the current CUDA device.
+ *   B, L, D  batch rows, tokens, channels (B, D >= 1; L >= 0)
+ *   N        state size per channel, one of 16, 32, 64 (the pages use 16;
+ *            "12. Selective State Space" discusses 64 and 128)
+ *   dtype    SSCAN_F32 or SSCAN_BF16
+ *   flags    0 or SSCAN_ZOH
+ * On success *plan receives the plan and SSCAN_OK is returned; otherwise
+ * *plan is set to NULL.  Sizes are validated before any CUDA call, so
+ * SSCAN_ERR_INVALID / SSCAN_ERR_UNSUPPORTED come back without a device. */
+SSCAN_API int sscan_plan_create(sscan_plan_t *plan, int64_t B, int64_t L, int64_t D, int64_t N,
+                      int dtype, uint32_t flags);
+
+/* Release a plan (NULL is ignored).  Not stream-ordered: no forward call of
+ * this plan may still be running. */
+SSCAN_API void sscan_plan_destroy(sscan_plan_t plan);
+
+/* Bytes of device workspace sscan_forward needs for this plan (0 when the
+ * chosen schedule needs none).  The workspace must be 256-byte aligned. */
+SSCAN_API size_t sscan_workspace_bytes(sscan_plan_t plan);
+
+/* Enqueue the forward pass on `stream` (a cudaStream_t; NULL = legacy default).
+ *   u, delta        [B][L][D], plan dtype
+ *   A               [D][N] fp32
+ *   B, C            [B][L][N], plan dtype
+ *   h0              [B][D][N] fp32, or NULL for a zero initial state
+ *   y               [B][L][D], plan dtype (output)
+ *   h_final         [B][D][N] fp32 (output), or NULL to skip it
+ *   workspace       sscan_workspace_bytes(plan) bytes, or NULL when that is 0
+ * Returns SSCAN_OK once the work is enqueued. */
+SSCAN_API int sscan_forward(sscan_plan_t plan, const void *u, const void *delta, const float *A,
+                  const void *B, const void *C, const float *h0, void *y, float *h_final,
+                  void *workspace, void *stream);
+
+/* Wait for `stream`, then read and clear the plan's device status word.
+ * Returns SSCAN_OK, SSCAN_ERR_TIMEOUT, or SSCAN_ERR_CUDA. */
+SSCAN_API int sscan_get_status(sscan_plan_t plan, void *stream);
+
+/* Static description of a status code. */
+SSCAN_API const char *sscan_status_string(int status);
+
+/* Describe the schedule the plan chose (states per thread, threads per
+ * channel, time chunks, grid) into buf (NUL-terminated, truncated to len).
+ * Returns the number of characters the full description needs. */
+SSCAN_API int sscan_plan_describe(sscan_plan_t plan, char *buf, size_t len);
+
+/* Library version, major*10000 + minor*100 + patch. */
+SSCAN_API int sscan_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSCAN_H */

@@ -1,0 +1,198 @@
+"""Thin ctypes binding of the C ABI in ``include/sscan.h`` (libsscan.so).
+
+Argument marshalling only: every step of the selective-scan forward runs in the
+CUDA library.  PyTorch supplies device memory and the current stream.  There is
+no fallback: if the library is missing or the call fails, this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsscan.so")
+
+F32, BF16 = 0, 1
+ZOH = 1
+OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(7)
+
+SYMBOLS = ("sscan_plan_create", "sscan_plan_destroy", "sscan_workspace_bytes", "sscan_forward",
+           "sscan_get_status", "sscan_status_string", "sscan_plan_describe", "sscan_version")
+
+
+class SscanError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {status_string(code)} (code {code})")
+        self.code = code
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Open libsscan.so (built in-tree by ``python -m selective_state_space_32_b200.build``)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                                   "`python -m selective_state_space_32_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, i64, ip, u32, sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                                    ctypes.c_uint32, ctypes.c_size_t)
+            L.sscan_plan_create.argtypes = [ctypes.POINTER(vp), i64, i64, i64, i64, ip, u32]
+            L.sscan_plan_create.restype = ip
+            L.sscan_plan_destroy.argtypes = [vp]
+            L.sscan_plan_destroy.restype = None
+            L.sscan_workspace_bytes.argtypes = [vp]
+            L.sscan_workspace_bytes.restype = sz
+            L.sscan_forward.argtypes = [vp] * 11
+            L.sscan_forward.restype = ip
+            L.sscan_get_status.argtypes = [vp, vp]
+            L.sscan_get_status.restype = ip
+            L.sscan_status_string.argtypes = [ip]
+            L.sscan_status_string.restype = ctypes.c_char_p
+            L.sscan_plan_describe.argtypes = [vp, ctypes.c_char_p, sz]
+            L.sscan_plan_describe.restype = ip
+            L.sscan_version.argtypes = []
+            L.sscan_version.restype = ip
+            _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().sscan_status_string(int(code)).decode()
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return F32
+    if dt == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {dt} (float32 or bfloat16)")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+class Plan:
+    """A sscan_plan for one (B, L, D, N, dtype, zoh) shape on the current device."""
+
+    def __init__(self, B: int, L: int, D: int, N: int, dtype: torch.dtype = torch.float32,
+                 zoh: bool = False):
+        self.shape = (int(B), int(L), int(D), int(N))
+        self.dtype = dtype
+        self.zoh = bool(zoh)
+        h = ctypes.c_void_p()
+        rc = lib().sscan_plan_create(ctypes.byref(h), *self.shape, _dtype_code(dtype),
+                                     ZOH if zoh else 0)
+        if rc != OK:
+            raise SscanError(rc, "sscan_plan_create")
+        self._h = h
+        self.workspace_bytes = int(lib().sscan_workspace_bytes(h))
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().sscan_plan_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def describe(self) -> str:
+        buf = ctypes.create_string_buffer(512)
+        lib().sscan_plan_describe(self._h, buf, 512)
+        return buf.value.decode()
+
+    def new_workspace(self, device=None) -> Optional[torch.Tensor]:
+        if self.workspace_bytes == 0:
+            return None
+        return torch.empty(self.workspace_bytes, dtype=torch.uint8, device=device or "cuda")
+
+    def forward(self, u, delta, A, B, C, h0=None, y=None, h_final=None, workspace=None,
+                want_final: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+        """Enqueue the forward on ``stream`` (default: torch's current stream)."""
+        Bt, L, D, N = self.shape
+        if y is None:
+            y = torch.empty((Bt, L, D), dtype=self.dtype, device=u.device)
+        if h_final is None and want_final:
+            h_final = torch.empty((Bt, D, N), dtype=torch.float32, device=u.device)
+        for name, t, shape, dt in (("u", u, (Bt, L, D), self.dtype),
+                                   ("delta", delta, (Bt, L, D), self.dtype),
+                                   ("A", A, (D, N), torch.float32),
+                                   ("B", B, (Bt, L, N), self.dtype),
+                                   ("C", C, (Bt, L, N), self.dtype),
+                                   ("h0", h0, (Bt, D, N), torch.float32),
+                                   ("y", y, (Bt, L, D), self.dtype),
+                                   ("h_final", h_final, (Bt, D, N), torch.float32)):
+            if t is None:
+                continue
+            if tuple(t.shape) != shape or t.dtype != dt or not t.is_cuda or not t.is_contiguous():
+                raise ValueError(f"{name}: want contiguous CUDA {dt} {shape}, got "
+                                 f"{t.dtype} {tuple(t.shape)} on {t.device}")
+        if workspace is None and self.workspace_bytes:
+            workspace = self.new_workspace(u.device)
+        if stream is None:
+            stream = torch.cuda.current_stream(u.device)
+        rc = lib().sscan_forward(self._h, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+                                 _ptr(h0), _ptr(y), _ptr(h_final), _ptr(workspace),
+                                 ctypes.c_void_p(stream.cuda_stream))
+        if rc != OK:
+            raise SscanError(rc, "sscan_forward")
+        return y, h_final
+
+    def status(self, stream=None) -> int:
+        """Synchronise ``stream`` and read (and clear) the plan's device status word."""
+        if stream is None:
+            stream = torch.cuda.current_stream()
+        return int(lib().sscan_get_status(self._h, ctypes.c_void_p(stream.cuda_stream)))
+
+
+_plans: dict = {}
+
+
+def get_plan(B, L, D, N, dtype=torch.float32, zoh=False) -> Plan:
+    key = (int(B), int(L), int(D), int(N), dtype, bool(zoh), torch.cuda.current_device())
+    p = _plans.get(key)
+    if p is None:
+        p = _plans[key] = Plan(B, L, D, N, dtype, zoh)
+    return p
+
+
+def forward(u, delta, A, B, C, h0=None, zoh: bool = False, want_final: bool = True):
+    """Selective-scan forward on CUDA tensors: returns (y [B,L,D], h_final [B,D,N] or None).
+
+    u, delta: [B, L, D] float32 or bfloat16; A: [D, N] float32; B, C: [B, L, N]
+    (dtype of u); h0: [B, D, N] float32 or None.
+    """
+    Bt, L, D = u.shape
+    N = A.shape[1]
+    return get_plan(Bt, L, D, N, u.dtype, zoh).forward(u, delta, A, B, C, h0,
+                                                        want_final=want_final)
+
+
+def forward_host(u, delta, A, B, C, h0=None, zoh: bool = False, device="cuda", out=None):
+    """Forward on host (CPU) tensors: copies the inputs to the device, runs the scan
+    and copies y and h_final back, then waits for the copies.  Pinned host tensors
+    give asynchronous copies; ``out`` = (y_host, h_final_host) reuses output buffers.
+    Returns (y_host, h_final_host)."""
+    dev = torch.device(device)
+    dv = [None if t is None else t.to(dev, non_blocking=True) for t in (u, delta, A, B, C, h0)]
+    y, hf = forward(*dv[:5], h0=dv[5], zoh=zoh)
+    if out is None:
+        pin = u.is_pinned()
+        out = (torch.empty(y.shape, dtype=y.dtype, pin_memory=pin),
+               torch.empty(hf.shape, dtype=hf.dtype, pin_memory=pin))
+    out[0].copy_(y, non_blocking=True)
+    out[1].copy_(hf, non_blocking=True)
+    torch.cuda.current_stream(dev).synchronize()
+    return out

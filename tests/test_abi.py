@@ -1,0 +1,65 @@
+"""The C-ABI library builds, loads and exports every entry point include/sscan.h declares.
+
+These run without a GPU: no compute call is made.  Argument checks that the ABI
+promises to perform before touching the device are exercised here too.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from selective_state_space_32_b200 import build as B
+from selective_state_space_32_b200 import sscan as S
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                      "include", "sscan.h")
+
+
+def declared_symbols():
+    with open(HEADER) as f:
+        text = f.read()
+    return re.findall(r"SSCAN_API\s+[\w\s\*]+?\b(sscan_\w+)\s*\(", text)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return S.lib()
+
+
+def test_header_declares_the_binding_symbols():
+    assert sorted(declared_symbols()) == sorted(S.SYMBOLS)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_status_strings(lib):
+    assert lib.sscan_version() >= 100
+    for code in range(7):
+        assert S.status_string(code)
+    assert S.status_string(S.ERR_ALIGN) == "pointer not 16-byte aligned"
+
+
+@pytest.mark.parametrize("args,want", [
+    ((0, 16, 64, 16, S.F32, 0), S.ERR_INVALID),        # B = 0
+    ((1, -1, 64, 16, S.F32, 0), S.ERR_INVALID),        # L < 0
+    ((1, 16, 0, 16, S.F32, 0), S.ERR_INVALID),         # D = 0
+    ((1, 16, 64, 16, 7, 0), S.ERR_INVALID),            # unknown dtype
+    ((1, 16, 64, 16, S.F32, 1 << 5), S.ERR_INVALID),   # unknown flag
+    ((1, 16, 64, 24, S.F32, 0), S.ERR_UNSUPPORTED),    # N not in {16, 32, 64}
+    ((1, 16, 64, 128, S.BF16, 1), S.ERR_UNSUPPORTED),
+])
+def test_plan_create_rejects_bad_sizes_without_a_device(lib, args, want):
+    h = ctypes.c_void_p(123)
+    assert lib.sscan_plan_create(ctypes.byref(h), *args) == want
+    assert not h.value
+
+
+def test_null_plan_is_rejected(lib):
+    assert lib.sscan_forward(None, *([None] * 10)) == S.ERR_INVALID
+    assert lib.sscan_get_status(None, None) == S.ERR_INVALID
+    lib.sscan_plan_destroy(None)

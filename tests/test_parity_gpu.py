@@ -1,0 +1,146 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small cases compare every element and span several blocks plus ragged tails;
+the full-size workloads run the exact launch the benchmark times and compare a
+seeded sample of (b, d) rows, each recomputed by the oracle row by row (rows
+are independent, so a sampled row is an exact reference).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from selective_state_space_32_b200 import sscan as S
+from selective_state_space_32_b200 import workloads as W
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from selective_state_space_32_b200 import build
+    build.build()
+    S.lib()
+
+
+SMALL = [
+    # (B, L, D, N, dtype, h0, zoh, A_jitter)
+    (1, 256, 64, 16, "f32", False, False, 0.0),     # the tiny workload's shape
+    (2, 257, 130, 16, "f32", True, False, 0.3),     # ragged L and D, 3 blocks
+    (3, 1, 7, 16, "f32", True, True, 0.3),          # one token, D below a warp
+    (1, 255, 65, 32, "f32", True, False, 0.3),
+    (2, 129, 33, 64, "f32", True, True, 0.3),
+    (2, 300, 96, 16, "bf16", True, False, 0.0),
+    (1, 200, 40, 64, "bf16", False, True, 0.0),
+    (2, 64, 200, 32, "bf16", True, True, 0.5),
+    (1, 1000, 64, 16, "f32", True, True, 0.0),      # long-ish horizon, exact ZOH in fp32
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[f"B{c[0]}L{c[1]}D{c[2]}N{c[3]}{c[4]}"
+                                              f"{'_h0' if c[5] else ''}{'_zoh' if c[6] else ''}"
+                                              for c in SMALL])
+def test_small_cases_elementwise(case):
+    Bt, L, D, N, dt, with_h0, zoh, jit = case
+    g = W.generate(Bt, L, D, N, dt, 0.1 if with_h0 else 0.0, 0.0, seed=1000 + L + D + N,
+                   A_jitter=jit)
+    y, hf = P.run_gpu(g, zoh)
+    yr, hr = P.run_oracle(g, zoh)
+    P.check(y, yr, dt, "y")
+    P.check(hf, hr, dt, "h_final")
+
+
+def test_tiny_workload_full():
+    w = W.WORKLOADS["tiny_f32"]
+    g = W.make_inputs(w)
+    y, hf = P.run_gpu(g, w.zoh)
+    yr, hr = P.run_oracle(g, w.zoh)
+    P.check(y, yr, "f32", "y")
+    P.check(hf, hr, "f32", "h_final")
+
+
+def test_empty_sequence_keeps_h0():
+    g = W.generate(2, 0, 70, 16, "f32", 0.1, seed=5)
+    y, hf = P.run_gpu(g)
+    assert y.shape == (2, 0, 70)
+    assert np.array_equal(hf, g["h0"])
+
+
+def test_split_call_resume_matches_one_call():
+    g = W.generate(2, 700, 96, 16, "f32", 0.1, seed=6, A_jitter=0.2)
+    d = P.to_device(g)
+    y, hf = S.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"])
+    c = 333
+    y1, h1 = S.forward(d["u"][:, :c].contiguous(), d["delta"][:, :c].contiguous(), d["A"],
+                       d["B"][:, :c].contiguous(), d["C"][:, :c].contiguous(), d["h0"])
+    y2, h2 = S.forward(d["u"][:, c:].contiguous(), d["delta"][:, c:].contiguous(), d["A"],
+                       d["B"][:, c:].contiguous(), d["C"][:, c:].contiguous(), h1)
+    torch.cuda.synchronize()
+    yr, hr = P.run_oracle(g)
+    P.check(torch.cat([y1, y2], 1).cpu().numpy(), yr, "f32", "y split")
+    P.check(h2.cpu().numpy(), hr, "f32", "h_final split")
+    # the schedule does not depend on where the sequence was cut
+    assert torch.allclose(torch.cat([y1, y2], 1), y, rtol=1e-5, atol=1e-6)
+
+
+def test_h_final_may_alias_h0():
+    g = W.generate(1, 100, 64, 16, "f32", 0.1, seed=7)
+    d = P.to_device(g)
+    plan = S.get_plan(1, 100, 64, 16, torch.float32)
+    h = d["h0"].clone()
+    y, hf = plan.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], h0=h, h_final=h)
+    torch.cuda.synchronize()
+    yr, hr = P.run_oracle(g)
+    P.check(y.cpu().numpy(), yr, "f32", "y")
+    P.check(h.cpu().numpy(), hr, "f32", "h_final in place")
+
+
+def test_argument_errors_are_reported_before_launch():
+    g = W.generate(1, 32, 64, 16, "f32", 0.0, seed=8)
+    d = P.to_device(g)
+    plan = S.get_plan(1, 32, 64, 16, torch.float32)
+    lib = S.lib()
+    import ctypes
+    p = lambda t, off=0: ctypes.c_void_p(t.data_ptr() + off)
+    y = torch.empty(1, 32, 64, device="cuda")
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    # misaligned u
+    assert lib.sscan_forward(plan._h, p(d["u"], 4), p(d["delta"]), p(d["A"]), p(d["B"]),
+                             p(d["C"]), None, p(y), None, None, s) == S.ERR_ALIGN
+    # y overlapping an input
+    assert lib.sscan_forward(plan._h, p(d["u"]), p(d["delta"]), p(d["A"]), p(d["B"]),
+                             p(d["C"]), None, p(d["u"]), None, None, s) == S.ERR_INVALID
+    # missing B
+    assert lib.sscan_forward(plan._h, p(d["u"]), p(d["delta"]), p(d["A"]), None,
+                             p(d["C"]), None, p(y), None, None, s) == S.ERR_INVALID
+    assert plan.status() == S.OK
+
+
+# ------------------------------------------------------------- full sizes --
+
+def _sample_rows(w, k, seed):
+    rng = np.random.default_rng(seed)
+    rows = {(0, 0), (w.B - 1, w.D - 1), (0, w.D - 1), (w.B - 1, 0)}
+    while len(rows) < k:
+        rows.add((int(rng.integers(w.B)), int(rng.integers(w.D))))
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("name,k", [("mamba130m_f32", 256), ("mamba1p4b_bf16", 128),
+                                    ("longseq_bf16", 48), ("zoh_n64_bf16", 192)])
+def test_full_workload_sampled_rows(name, k):
+    w = W.WORKLOADS[name]
+    g = W.make_inputs(w)
+    y, hf = P.run_gpu(g, w.zoh)
+    rows = _sample_rows(w, k, w.index)
+    v = P.host_values(g)
+    yr, hr = O.forward_rows(rows, v["u"], v["delta"], v["A"], v["B"], v["C"], v["h0"], w.zoh)
+    rb = np.array([r[0] for r in rows])
+    rd = np.array([r[1] for r in rows])
+    P.check(y[rb, :, rd], yr, w.dtype, f"{name} y rows")
+    P.check(hf[rb, rd], hr, w.dtype, f"{name} h_final rows")
+    # whole-output properties that hold at any size
+    assert np.all(np.isfinite(y)) and np.all(np.isfinite(hf))
