@@ -135,6 +135,23 @@ def cpu_oracle_rate(g, w, min_seconds=10.0, max_seconds=30.0):
     return n * w.elements / el, cores, f"{n} full pass(es) over the workload ({w.elements} elements each) in {el:.2f} s"
 
 
+# ------------------------------------------------------- multi-rank logic --
+
+def shard_seed(w, rank: int) -> int:
+    """Seed of rank r's shard: batch rows [r*B, (r+1)*B) of an N*B-row job."""
+    return W.SEED_BASE + w.index + 1000 * rank
+
+
+def max_over_ranks(values, world: int, device=None):
+    """Element-wise maximum of a list of floats over all ranks (timings)."""
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 # -------------------------------------------------------------- our arm --
 
 def run_ours(args, rank, world, local_rank):
@@ -147,7 +164,7 @@ def run_ours(args, rank, world, local_rank):
     w = W.WORKLOADS[args.workload]
     # shard: rank r owns batch rows [r*B, (r+1)*B) of an N*B-row job (own seed)
     g = W.generate(w.B, w.L, w.D, w.N, w.dtype, w.h0_std, w.reset_frac,
-                   seed=W.SEED_BASE + w.index + 1000 * rank)
+                   seed=shard_seed(w, rank))
     tdt = torch.float32 if w.dtype == "f32" else torch.bfloat16
 
     def host(x, dt):
@@ -226,10 +243,7 @@ def run_ours(args, rank, world, local_rank):
     d2h = sum(v.numel() * v.element_size() for v in out_h)
 
     # ---- max over ranks ----
-    t = torch.tensor([elapsed_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_ms, e2e_ms = float(t[0]), float(t[1])
+    elapsed_ms, e2e_ms = max_over_ranks([elapsed_ms, e2e_ms], world, dev)
 
     if rank != 0:
         return None

@@ -1,0 +1,219 @@
+// device_utils.cuh -- device helpers shared by the selective-scan kernels:
+// packed f32x2 arithmetic, 2^x on the MUFU and on the FMA pipe, storage-type
+// conversion, and the mbarrier / TMA / flag primitives of the chained kernel.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace sscan {
+
+// ------------------------------------------------------------ packed fp32 pairs
+
+typedef unsigned long long f2;  // two fp32 values in one 64-bit register pair
+
+__device__ __forceinline__ f2 pack2(float lo, float hi) {
+    f2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpack2(f2 v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+    f2 r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+    f2 r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+    f2 r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f2 splat2(float v) { return pack2(v, v); }
+
+// 2^x on the MUFU pipe (ex2.approx; results below 2^-126 flush to zero)
+__device__ __forceinline__ float ex2(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// 2^(d*a) for a pair on the FMA pipe, |d*a| <= 125 (the caller clamps d).
+// Range reduction: t = d*a + 1.5*2^23 leaves j = round(d*a) in the low
+// mantissa bits; f = d*a - j in [-1/2, 1/2]; 2^f = 1 + f*q(f) with q of degree
+// 4 fitted for minimax relative error on [-1/2, 1/2] (csrc/gen_exp2_poly.py,
+// max relative error 1.7e-7 in fp32); the result's exponent is then raised by
+// j with one integer add of j << 23 (t's low bits shifted into the exponent).
+__device__ __forceinline__ f2 exp2_fma_pair(f2 dd, f2 a) {
+    const f2 kShift = splat2(12582912.0f);  // 1.5 * 2^23
+    const f2 kNeg1 = splat2(-1.0f);
+    const f2 t = fma2(dd, a, kShift);
+    const f2 jn = fma2(t, kNeg1, kShift);   // -round(d*a), exact
+    const f2 f = fma2(dd, a, jn);           // d*a - round(d*a)
+    f2 q = fma2(splat2(1.326472731307149e-03f), f, splat2(9.671512991189957e-03f));
+    q = fma2(q, f, splat2(5.550733581185341e-02f));
+    q = fma2(q, f, splat2(2.402224242687225e-01f));
+    q = fma2(q, f, splat2(6.931470036506653e-01f));
+    q = fma2(q, f, splat2(1.0f));
+    float t0, t1, q0, q1;
+    unpack2(t, t0, t1);
+    unpack2(q, q0, q1);
+    const uint32_t r0 = __float_as_uint(q0) + (__float_as_uint(t0) << 23);
+    const uint32_t r1 = __float_as_uint(q1) + (__float_as_uint(t1) << 23);
+    return pack2(__uint_as_float(r0), __uint_as_float(r1));
+}
+
+// phi(z) = (exp(z) - 1) / z = sum_k z^k / (k+1)!, truncated after z^7; for
+// |z| <= 1/2 the first omitted term is below 1.1e-8 relative.  Coefficients
+// are the Taylor series 1/(k+1)!, highest first.
+__device__ __forceinline__ f2 phi2(f2 z) {
+    f2 q = fma2(splat2(1.0f / 40320.0f), z, splat2(1.0f / 5040.0f));
+    q = fma2(q, z, splat2(1.0f / 720.0f));
+    q = fma2(q, z, splat2(1.0f / 120.0f));
+    q = fma2(q, z, splat2(1.0f / 24.0f));
+    q = fma2(q, z, splat2(1.0f / 6.0f));
+    q = fma2(q, z, splat2(0.5f));
+    return fma2(q, z, splat2(1.0f));
+}
+
+// Exact ZOH coefficient (exp(z) - 1) / A for a pair, z = d*A: d*phi(z) when
+// |z| <= 1/2 (also exact at A = 0), (abar - 1) * (1/A) otherwise.
+__device__ __forceinline__ f2 zoh_coef_pair(f2 dd, f2 a1, f2 ia, f2 abar) {
+    const f2 z = mul2(dd, a1);
+    const f2 small = mul2(dd, phi2(z));
+    const f2 big = mul2(add2(abar, splat2(-1.0f)), ia);
+    float z0, z1, s0, s1, g0, g1;
+    unpack2(z, z0, z1);
+    unpack2(small, s0, s1);
+    unpack2(big, g0, g1);
+    return pack2(fabsf(z0) <= 0.5f ? s0 : g0, fabsf(z1) <= 0.5f ? s1 : g1);
+}
+
+// ------------------------------------------------------------- storage types
+
+template <class IO> struct Io;
+template <> struct Io<float> {
+    static constexpr int kBytes = 4;
+    static __device__ __forceinline__ float ld(const float *p) { return __ldg(p); }
+    static __device__ __forceinline__ float widen(float v) { return v; }
+    static __device__ __forceinline__ void st(float *p, float v) { *p = v; }
+    // NP consecutive pairs (2*NP values) starting at a 16-byte aligned p
+    template <int NP>
+    static __device__ __forceinline__ void ld_pairs(const float *p, f2 (&out)[NP]) {
+#pragma unroll
+        for (int i = 0; i < NP / 2; ++i) {
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(p) + i);
+            out[2 * i] = pack2(v.x, v.y);
+            out[2 * i + 1] = pack2(v.z, v.w);
+        }
+    }
+};
+template <> struct Io<uint16_t> {  // bf16 bit patterns
+    static constexpr int kBytes = 2;
+    static __device__ __forceinline__ uint16_t ld(const uint16_t *p) { return __ldg(p); }
+    static __device__ __forceinline__ float widen(uint16_t v) {
+        return __uint_as_float(static_cast<uint32_t>(v) << 16);
+    }
+    static __device__ __forceinline__ void st(uint16_t *p, float v) {
+        uint16_t r;
+        asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(v));
+        *p = r;
+    }
+    template <int NP>
+    static __device__ __forceinline__ void ld_pairs(const uint16_t *p, f2 (&out)[NP]) {
+#pragma unroll
+        for (int i = 0; i < NP / 4; ++i) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p) + i);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)  // low half = even state, high half = odd state
+                out[4 * i + j] = pack2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xffff0000u));
+        }
+    }
+};
+
+// ------------------------------------------------- mbarrier / TMA / flag wait
+
+constexpr uint32_t kSpinLimit = 1u << 22;  // bound on every device-side wait loop
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Wait for the phase with the given parity to complete; false if the bound ran out.
+// A non-blocking test first: a stage loaded well ahead is normally complete already.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+    if (mbar_test_wait(bar, parity)) return true;
+    for (uint32_t i = 0; i < kSpinLimit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+// 2-D tiled TMA load (no multicast) of box {x, y} into shared memory, completing on bar.
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+// Order this thread's (and, after a warp/CTA barrier, its peers') generic-proxy
+// shared-memory accesses before later async-proxy (TMA) accesses.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+}  // namespace sscan

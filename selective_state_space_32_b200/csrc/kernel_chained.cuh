@@ -1,0 +1,713 @@
+// kernel_chained.cuh -- persistent selective-scan forward with TMA-staged
+// inputs and a static, exactly balanced schedule of chain segments.
+//
+// Work unit.  A "chain" is one batch row b and CPW = 32/LPC consecutive
+// channels over the whole sequence; one warp runs a chain with lane
+// (c, g) = (channel c of the chain, state group g) owning NL = N/LPC states of
+// channel c in registers.  The recurrence h = Abar*h + Bbar u is sequential in
+// time ("Selective State-Space Models (Mamba) and Hardware-Aware Scans",
+// section 2), so a chain's steps must run in order; chains are independent.
+//
+// Schedule.  The B*ceil(D/CPW) chains are laid end to end (chain-major, then
+// time) and cut into W equal segments of S = ceil(chains*L / W) chain-steps,
+// one per warp of a persistent grid, so every warp does the same number of
+// state updates.  With S >= L a chain is cut at most once, between two
+// consecutive warps: the earlier warp runs the chain's head (from t = 0) FIRST
+// and publishes the state at the cut; the later warp runs its own head and
+// whole chains first and the chain's tail LAST, after reading that state.
+// This is "scan within a block, carry the block's state forward"
+// ("tm_ssm_selective", section "What it costs at inference, and on a CPU"):
+// the carry is the exact state, so there is no fix-up pass and no exponent is
+// computed twice.  The wait cannot deadlock (the grid is launched
+// cooperatively, so all warps are resident, and a warp only waits for a head
+// that its predecessor runs before anything else) and is bounded anyway.
+//
+// Pipeline.  Each warp owns a ring of STAGES shared-memory stages of T tokens:
+// u and delta tiles [T][CPW] and B, C tiles [T][N], loaded by lane 0 with 2-D
+// TMA (no multicast) on an mbarrier; once the whole warp is past a stage
+// (__syncwarp plus an async-proxy fence), lane 0 refills its slot.  The compute
+// loop therefore only reads shared memory.  bf16 B/C tiles are widened once per stage by the warp.
+//
+// Arithmetic per state update: Abar = 2^(delta*A*log2 e) on the MUFU pipe, or
+// for a quarter of the states on the FMA pipe (exp2_fma_pair) to balance the
+// two pipes; Bbar u (Euler or exact ZOH), h = Abar*h + Bbar u and y += C*h on
+// packed f32x2 instructions.  y is reduced over the LPC lanes of a channel
+// with shuffles and stored directly.
+#pragma once
+
+#include "device_utils.cuh"
+
+namespace sscan {
+
+struct ChainedParams {
+    const float *A;                // [D][N]
+    const float *h0;               // [B][D][N] or null
+    void *y;                       // [B][L][D]
+    float *h_final;                // [B][D][N] or null
+    float *carry;                  // [chains][32][NL] state at a cut
+    unsigned long long *flags;     // [chains] (epoch << 32) | cut position
+    int *status;                   // device status word
+    unsigned long long epoch_hi;   // this launch's epoch << 32
+    int64_t L, D;
+    int64_t chains_per_row;        // ceil(D / CPW)
+    int64_t chains;                // B * chains_per_row
+    int64_t seg;                   // chain-steps per warp (S)
+    // split mode (chains cut into several pieces that are scanned concurrently)
+    const void *delta;             // [B][L][D], read again by the fix-up
+    const void *Cm;                // [B][L][N], read again by the fix-up
+    float *rec_h;                  // [chains][max_pieces][32][NL] local end state of a piece
+    float *rec_s;                  // [chains][max_pieces][32] sum of delta over the piece
+    int *rec_mono;                 // [chains][max_pieces] delta >= 0 over the piece and A <= 0
+    unsigned long long *rec_flags; // [chains][max_pieces] (epoch << 32) | 1 once published
+    int64_t max_pieces;
+};
+
+template <class IO, int N_, int NL_, int T_, int STAGES_, int WPC_>
+struct ChainedCfg {
+    static constexpr int N = N_, NL = NL_, T = T_, STAGES = STAGES_, WPC = WPC_;
+    static constexpr int LPC = N / NL;      // lanes per channel
+    static constexpr int CPW = 32 / LPC;    // channels per warp (chain width)
+    static constexpr int NP = NL / 2;       // packed pairs per lane
+    static constexpr int G = NL >= 16 ? 2 : (NL >= 8 ? 4 : 8);  // tokens per discretize group
+    static constexpr int ES = sizeof(IO);
+    static constexpr int kU = T * CPW * ES;                 // one u or delta tile
+    static constexpr int kB = T * N * ES;                   // one B or C tile
+    static constexpr int kStage = 2 * kU + 2 * kB;          // TMA bytes per stage
+    static constexpr int kConv = ES == 2 ? 2 * T * N * 4 : 0;  // widened B, C (bf16 I/O)
+    static constexpr int kBar = STAGES * 8;
+    static constexpr int kWarp = ((STAGES * kStage + kConv + kBar) + 127) / 128 * 128;
+    static constexpr int kSmem = WPC * kWarp;
+    static_assert(LPC >= 1 && LPC <= 8 && N % NL == 0 && NL % 4 == 0, "bad split");
+    static_assert(CPW * ES % 16 == 0 && N * ES % 16 == 0, "TMA rows must be 16-byte multiples");
+    static_assert(kU % 128 == 0 && kB % 128 == 0, "tile alignment");
+    static_assert(ES == 4 || (T * N) % 256 == 0, "bf16 widening splits the tile in 8-value chunks");
+};
+
+// Discretize one token for one lane: Abar and Bbar u for the lane's NL states.
+// Independent of the state, so a group of tokens is discretized ahead of the
+// (sequential) state updates and the MUFU latency overlaps them.  PAR is the
+// token's parity; it selects which pairs take 2^x on the FMA pipe (a quarter
+// of all pairs across two tokens).
+template <int NP, bool ZOH, bool POLY, int PAR>
+__device__ __forceinline__ void discretize(f2 (&ab)[NP], f2 (&bu)[NP], const f2 (&A2)[NP], const f2 (&A1)[NP],
+                                           const f2 (&iA)[NP], float cap, float x, float dl,
+                                           const float *Bs) {
+    const f2 dd = splat2(dl);
+    f2 du2, xx, ddc;
+    if (ZOH)
+        xx = splat2(x);
+    else
+        du2 = splat2(dl * x);
+    if (POLY) ddc = splat2(fminf(dl, cap));
+#pragma unroll
+    for (int i = 0; i < NP / 2; ++i) {
+        const float4 bv = reinterpret_cast<const float4 *>(Bs)[i];
+        const f2 b01 = pack2(bv.x, bv.y), b23 = pack2(bv.z, bv.w);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int p = 2 * i + q;
+            const f2 bp = q ? b23 : b01;
+            if (POLY && ((PAR * NP + p) % 4 == 3)) {
+                ab[p] = exp2_fma_pair(ddc, A2[p]);
+            } else {
+                float e0, e1;
+                unpack2(mul2(dd, A2[p]), e0, e1);
+                ab[p] = pack2(ex2(e0), ex2(e1));
+            }
+            if (ZOH)
+                bu[p] = mul2(zoh_coef_pair(dd, A1[p], iA[p], ab[p]), mul2(bp, xx));
+            else
+                bu[p] = mul2(bp, du2);
+        }
+    }
+}
+
+// The state update and readout of one token: h = Abar*h + Bbar u, partial y = C.h.
+template <int NP>
+__device__ __forceinline__ float advance(f2 (&h)[NP], const f2 (&ab)[NP], const f2 (&bu)[NP], const float *Cs) {
+    f2 ya = splat2(0.0f);
+#pragma unroll
+    for (int i = 0; i < NP / 2; ++i) {
+        const float4 cv = reinterpret_cast<const float4 *>(Cs)[i];
+        h[2 * i] = fma2(ab[2 * i], h[2 * i], bu[2 * i]);
+        ya = fma2(pack2(cv.x, cv.y), h[2 * i], ya);
+        h[2 * i + 1] = fma2(ab[2 * i + 1], h[2 * i + 1], bu[2 * i + 1]);
+        ya = fma2(pack2(cv.z, cv.w), h[2 * i + 1], ya);
+    }
+    float y0, y1;
+    unpack2(ya, y0, y1);
+    return y0 + y1;
+}
+
+// Sum G per-token partial outputs over the LPC lanes of a channel and scatter
+// the totals: afterwards this lane holds the full y of tokens
+// base .. base + cnt - 1 in v[0 .. cnt), cnt = max(1, G / LPC).  Each level
+// halves the token set a lane keeps and sends the other half to its partner.
+template <int LPC, int G>
+__device__ __forceinline__ int reduce_scatter(float (&v)[G], int g) {
+    int base = 0;
+#pragma unroll
+    for (int m = LPC / 2, cnt = G; m >= 1; m >>= 1) {
+        if (cnt >= 2) {
+            const bool up = (g & m) != 0;
+#pragma unroll
+            for (int i = 0; i < cnt / 2; ++i) {
+                const float send = up ? v[i] : v[i + cnt / 2];
+                const float keep = up ? v[i + cnt / 2] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+            }
+            if (up) base += cnt / 2;
+            cnt /= 2;
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
+        }
+    }
+    return base;
+}
+
+// Split mode, second phase for one piece [ts, te) of chain c (ts > 0) that was
+// scanned from a zero state.  Its carried-in state is the inclusive state of
+// the previous pieces: h_in = sum_i (prod_{k>i} P_k) hloc_i over the earlier
+// pieces i, where P_k = prod Abar over piece k = 2^(A*log2e * sum delta) (one
+// exponent per state and piece).  The records are published at the end of
+// every piece's local scan, so the look-back never waits for another fix-up.
+// The exact output is y_t = y_local,t + C_t . z_t with z_t = Abar_t z_{t-1},
+// z = h_in before ts; the loop stops once every |z| has fallen below
+// 2^-40 max(1, |h_in|) and delta >= 0, A <= 0 over the piece guarantee that
+// it can only shrink further ("Delta is a gate": large steps reset the state,
+// "tm_ssm_selective").  The piece's final state is hloc + P_piece h_in.
+template <class IO, class Cfg>
+__device__ __noinline__ void split_fixup(const ChainedParams &P, int64_t c, int64_t ts, int64_t te,
+                                         int64_t wk, int lane) {
+    constexpr int N = Cfg::N, NL = Cfg::NL, LPC = Cfg::LPC, CPW = Cfg::CPW, NP = Cfg::NP;
+    constexpr int FB = NL <= 8 ? 8 : 4;  // tokens per block of loads
+    const int64_t L = P.L, D = P.D;
+    const int cl = lane / LPC, g = lane % LPC, n0 = g * NL;
+    const int64_t b = c / P.chains_per_row, cw = c - b * P.chains_per_row;
+    const int64_t d = cw * CPW + cl;
+    const bool valid = d < D;
+    const int64_t dcl = valid ? d : D - 1;
+    f2 A2[NP];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+        const float a0 = __ldg(P.A + dcl * N + n0 + 2 * p), a1 = __ldg(P.A + dcl * N + n0 + 2 * p + 1);
+        A2[p] = pack2(static_cast<float>(static_cast<double>(a0) * 1.4426950408889634),
+                      static_cast<float>(static_cast<double>(a1) * 1.4426950408889634));
+    }
+    const int64_t jp = wk - (c * L) / P.seg;  // index of this piece within chain c
+    f2 acc_h[NP], acc_p[NP];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+        acc_h[p] = splat2(0.0f);
+        acc_p[p] = splat2(1.0f);
+    }
+    for (int64_t i = jp - 1; i >= 0; --i) {
+        const int64_t r = c * P.max_pieces + i;
+        int bad = 0;
+        if (lane == 0) {
+            uint32_t it = 0;
+            while (ld_acquire_u64(P.rec_flags + r) != (P.epoch_hi | 1ull)) {
+                if (++it > (kSpinLimit >> 2)) {
+                    bad = 1;
+                    atomicOr(P.status, 1);
+                    break;
+                }
+                __nanosleep(128);
+            }
+        }
+        bad = __shfl_sync(0xffffffffu, bad, 0);
+        __syncwarp();
+        if (bad) break;
+        const float sd = __ldcg(P.rec_s + r * 32 + lane);
+        const float *src = P.rec_h + (r * 32 + lane) * NL;
+        bool all_zero = true;
+#pragma unroll
+        for (int p = 0; p < NP; p += 2) {
+            const float4 v = __ldcg(reinterpret_cast<const float4 *>(src + 2 * p));
+            const f2 hl[2] = {pack2(v.x, v.y), pack2(v.z, v.w)};
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                float e0, e1;
+                unpack2(mul2(splat2(sd), A2[p + q]), e0, e1);
+                acc_h[p + q] = fma2(acc_p[p + q], hl[q], acc_h[p + q]);
+                acc_p[p + q] = mul2(acc_p[p + q], pack2(ex2(e0), ex2(e1)));
+                float p0, p1;
+                unpack2(acc_p[p + q], p0, p1);
+                all_zero = all_zero && p0 == 0.0f && p1 == 0.0f;
+            }
+        }
+        if (__all_sync(0xffffffffu, all_zero)) break;  // older pieces are multiplied by exact zeros
+    }
+    // this piece's own record: local end state, sum of delta, monotone flag
+    const int64_t ro = c * P.max_pieces + jp;
+    const bool mono = __ldcg(P.rec_mono + ro) != 0;
+    float hmax = 0.0f;
+    f2 z[NP];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+        z[p] = acc_h[p];
+        float a, bq;
+        unpack2(z[p], a, bq);
+        hmax = fmaxf(hmax, fmaxf(fabsf(a), fabsf(bq)));
+    }
+    const float tau = ldexpf(fmaxf(1.0f, hmax), -40);
+    const IO *dptr = static_cast<const IO *>(P.delta) + b * L * D + dcl;
+    const IO *cptr = static_cast<const IO *>(P.Cm) + b * L * N + n0;
+    IO *yptr = static_cast<IO *>(P.y) + b * L * D + dcl;
+    const bool writer = valid && g == 0;
+    for (int64_t tb = ts; tb < te; tb += FB) {
+        const int nb = static_cast<int>(te - tb < FB ? te - tb : FB);
+        float dl[FB], yo[FB];
+        f2 cv[FB][NP];
+#pragma unroll
+        for (int q = 0; q < FB; ++q) {
+            const int64_t t = tb + (q < nb ? q : 0);
+            dl[q] = Io<IO>::widen(Io<IO>::ld(dptr + t * D));
+            Io<IO>::template ld_pairs<NP>(cptr + t * N, cv[q]);
+            yo[q] = writer ? Io<IO>::widen(__ldcg(yptr + t * D)) : 0.0f;
+        }
+#pragma unroll
+        for (int q = 0; q < FB; ++q) {
+            if (q < nb) {
+                f2 ya = splat2(0.0f);
+#pragma unroll
+                for (int p = 0; p < NP; ++p) {
+                    float e0, e1;
+                    unpack2(mul2(splat2(dl[q]), A2[p]), e0, e1);
+                    z[p] = mul2(pack2(ex2(e0), ex2(e1)), z[p]);
+                    ya = fma2(cv[q][p], z[p], ya);
+                }
+                float y0, y1;
+                unpack2(ya, y0, y1);
+                float corr = y0 + y1;
+#pragma unroll
+                for (int o = 1; o < LPC; o <<= 1) corr += __shfl_xor_sync(0xffffffffu, corr, o);
+                if (writer) Io<IO>::st(yptr + (tb + q) * D, yo[q] + corr);
+            }
+        }
+        if (mono) {
+            float zmax = 0.0f;
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+                float a, bq;
+                unpack2(z[p], a, bq);
+                zmax = fmaxf(zmax, fmaxf(fabsf(a), fabsf(bq)));
+            }
+            if (__all_sync(0xffffffffu, zmax <= tau)) break;
+        }
+    }
+    if (te == L && P.h_final != nullptr) {
+        const float sd = __ldcg(P.rec_s + ro * 32 + lane);
+        const float *src = P.rec_h + (ro * 32 + lane) * NL;
+        float *dst = P.h_final + (b * D + d) * N + n0;
+#pragma unroll
+        for (int p = 0; p < NP; p += 2) {
+            const float4 v = __ldcg(reinterpret_cast<const float4 *>(src + 2 * p));
+            float o[4];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                float e0, e1;
+                unpack2(mul2(splat2(sd), A2[p + q]), e0, e1);
+                float h0v, h1v;
+                unpack2(acc_h[p + q], h0v, h1v);
+                o[2 * q] = (q ? v.z : v.x) + ex2(e0) * h0v;
+                o[2 * q + 1] = (q ? v.w : v.y) + ex2(e1) * h1v;
+            }
+            if (valid) *reinterpret_cast<float4 *>(dst + 2 * p) = make_float4(o[0], o[1], o[2], o[3]);
+        }
+    }
+}
+
+template <class IO, class Cfg, bool ZOH, bool POLY, bool SPLIT>
+__global__ void __launch_bounds__(Cfg::WPC * 32, 1)
+sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_d,
+                     const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
+                     const ChainedParams P) {
+    constexpr int N = Cfg::N, NL = Cfg::NL, T = Cfg::T, STAGES = Cfg::STAGES;
+    constexpr int LPC = Cfg::LPC, CPW = Cfg::CPW, NP = Cfg::NP;
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    unsigned char *wbase = smem + warp * Cfg::kWarp;
+    float *convB = reinterpret_cast<float *>(wbase + STAGES * Cfg::kStage);
+    float *convC = convB + T * N;
+    uint64_t *full = reinterpret_cast<uint64_t *>(wbase + STAGES * Cfg::kStage + Cfg::kConv);
+
+    const int64_t L = P.L, D = P.D;
+    const int64_t Q = P.chains * L;
+    const int64_t wk = static_cast<int64_t>(blockIdx.x) * Cfg::WPC + warp;  // this warp's segment
+    const int64_t q0 = wk * P.seg;
+    if (q0 >= Q) return;  // this warp has no work (whole warp leaves; no block barrier follows)
+    const int64_t q1 = q0 + P.seg < Q ? q0 + P.seg : Q;
+
+    // ---- this warp's parts: [head of the last chain] [whole chains] [tail of the first chain]
+    const int64_t c_first = q0 / L, t_first = q0 - c_first * L;
+    const int64_t c_last = (q1 - 1) / L, t_last = q1 - c_last * L;  // t_last in [1, L]
+    const bool single = c_first == c_last;
+    const int n_head = (!single && t_last < L) ? 1 : 0;
+    const int n_tail = (!single && t_first > 0) ? 1 : 0;
+    const int64_t f_lo = t_first == 0 ? c_first : c_first + 1;
+    const int64_t f_hi = t_last == L ? c_last : c_last - 1;
+    const int64_t n_full = single ? 0 : (f_hi >= f_lo ? f_hi - f_lo + 1 : 0);
+    const int64_t n_parts = single ? 1 : n_head + n_full + n_tail;
+    auto part = [&](int64_t k, int64_t &c, int64_t &ts, int64_t &te) {
+        if (single) {
+            c = c_first; ts = t_first; te = t_last;
+        } else if (k < n_head) {
+            c = c_last; ts = 0; te = t_last;
+        } else if (k < n_head + n_full) {
+            c = f_lo + (k - n_head); ts = 0; te = L;
+        } else {
+            c = c_first; ts = t_first; te = L;
+        }
+    };
+
+    auto tile_u = [&](int s) { return reinterpret_cast<IO *>(wbase + s * Cfg::kStage); };
+    auto tile_d = [&](int s) { return reinterpret_cast<IO *>(wbase + s * Cfg::kStage + Cfg::kU); };
+    auto tile_b = [&](int s) { return reinterpret_cast<IO *>(wbase + s * Cfg::kStage + 2 * Cfg::kU); };
+    auto tile_c = [&](int s) {
+        return reinterpret_cast<IO *>(wbase + s * Cfg::kStage + 2 * Cfg::kU + Cfg::kB);
+    };
+
+    if (lane == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+        }
+        mbar_fence_init();
+        tma_prefetch_desc(&tm_u);
+        tma_prefetch_desc(&tm_d);
+        tma_prefetch_desc(&tm_b);
+        tma_prefetch_desc(&tm_c);
+    }
+    __syncwarp();
+
+    // ---- producer cursor (lane 0 only): which stage to load next
+    int64_t pk = 0, pc = 0, pts = 0, pte = 0, pt = 0;
+    int64_t issued = 0;
+    bool p_done = false;
+    int px = 0, prow = 0;  // TMA coordinates of the cursor's chain: channel, row of t = 0
+    auto p_begin_part = [&]() {
+        if (pk >= n_parts) { p_done = true; return; }
+        part(pk, pc, pts, pte);
+        pt = pts;
+        const int64_t b = pc / P.chains_per_row;
+        px = static_cast<int>((pc - b * P.chains_per_row) * CPW);
+        prow = static_cast<int>(b * L);
+    };
+    auto p_issue = [&]() {  // load the stage at the cursor into slot issued % STAGES, advance
+        const int s = static_cast<int>(issued % STAGES);
+        const int x = px;
+        const int yrow = prow + static_cast<int>(pt);
+        mbar_expect_tx(&full[s], Cfg::kStage);
+        tma_load_2d(tile_u(s), &tm_u, x, yrow, &full[s]);
+        tma_load_2d(tile_d(s), &tm_d, x, yrow, &full[s]);
+        tma_load_2d(tile_b(s), &tm_b, 0, yrow, &full[s]);
+        tma_load_2d(tile_c(s), &tm_c, 0, yrow, &full[s]);
+        ++issued;
+        pt += T;
+        if (pt >= pte) {
+            ++pk;
+            p_begin_part();
+        }
+    };
+    if (lane == 0) {
+        p_begin_part();
+        for (int s = 0; s < STAGES && !p_done; ++s) p_issue();
+    }
+
+    const int cl = lane / LPC;   // channel within the chain
+    const int g = lane % LPC;    // state group
+    const int n0 = g * NL;
+    int64_t consumed = 0;
+    bool failed = false;
+
+    for (int64_t k = 0; k < n_parts && !failed; ++k) {
+        int64_t c, ts, te;
+        part(k, c, ts, te);
+        const int64_t b = c / P.chains_per_row, cw = c - b * P.chains_per_row;
+        const int64_t d = cw * CPW + cl;
+        const bool valid = d < D;
+        const int64_t dcl = valid ? d : D - 1;
+
+        f2 A2[NP], A1[NP], iA[NP], h[NP];
+        float amax = 0.0f;
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+            const float a0 = __ldg(P.A + dcl * N + n0 + 2 * p);
+            const float a1 = __ldg(P.A + dcl * N + n0 + 2 * p + 1);
+            A2[p] = pack2(static_cast<float>(static_cast<double>(a0) * 1.4426950408889634),
+                          static_cast<float>(static_cast<double>(a1) * 1.4426950408889634));
+            if (ZOH) {
+                A1[p] = pack2(a0, a1);
+                iA[p] = pack2(1.0f / a0, 1.0f / a1);
+            }
+            if (POLY && (p % 2 == 1)) {  // pairs that may take the FMA-pipe exponent
+                float x0, x1;
+                unpack2(A2[p], x0, x1);
+                amax = fmaxf(amax, fmaxf(fabsf(x0), fabsf(x1)));
+            }
+        }
+        // |delta * A2| <= 125 on the FMA-pipe pairs keeps 2^x in the normal range;
+        // clamping delta there changes nothing visible (2^-125 vs 0 in Abar).
+        const float cap = amax > 0.0f ? 125.0f / amax : 3.0e38f;
+
+        if (ts == 0) {
+            if (P.h0 != nullptr) {
+                const float *src = P.h0 + (b * D + dcl) * N + n0;
+#pragma unroll
+                for (int p = 0; p < NP; p += 2) {
+                    const float4 v = *reinterpret_cast<const float4 *>(src + 2 * p);
+                    h[p] = pack2(v.x, v.y);
+                    h[p + 1] = pack2(v.z, v.w);
+                }
+            } else {
+#pragma unroll
+                for (int p = 0; p < NP; ++p) h[p] = splat2(0.0f);
+            }
+        } else if (SPLIT) {
+#pragma unroll
+            for (int p = 0; p < NP; ++p) h[p] = splat2(0.0f);  // local scan; carried in later
+        } else {
+            // the state at the cut, published by the previous warp
+            int bad = 0;
+            if (lane == 0) {
+                const unsigned long long want = P.epoch_hi | static_cast<unsigned long long>(ts);
+                uint32_t it = 0;
+                while (ld_acquire_u64(P.flags + c) != want) {
+                    if (++it > (kSpinLimit >> 2)) {
+                        bad = 1;
+                        atomicOr(P.status, 1);
+                        break;
+                    }
+                    __nanosleep(128);
+                }
+            }
+            bad = __shfl_sync(0xffffffffu, bad, 0);
+            __syncwarp();  // order every lane's reads after lane 0's acquire
+            const float *src = P.carry + (c * 32 + lane) * NL;
+#pragma unroll
+            for (int p = 0; p < NP; p += 2) {
+                const float4 v = bad ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                     : __ldcg(reinterpret_cast<const float4 *>(src + 2 * p));
+                h[p] = pack2(v.x, v.y);
+                h[p + 1] = pack2(v.z, v.w);
+            }
+        }
+
+        double dsum = 0.0;      // split mode: sum of delta over the part (for prod Abar)
+        float dmin = 3.0e38f;   // split mode: smallest delta of the part
+        IO *ybase = static_cast<IO *>(P.y) + b * L * D + d;
+        for (int64_t t0 = ts; t0 < te; t0 += T) {
+            const int s = static_cast<int>(consumed % STAGES);
+            const uint32_t par = static_cast<uint32_t>((consumed / STAGES) & 1);
+            const bool landed = mbar_wait(&full[s], par);
+            if (!__all_sync(0xffffffffu, landed)) {
+                if (lane == 0) atomicOr(P.status, 2);
+                failed = true;
+                break;
+            }
+            const IO *us = tile_u(s);
+            const IO *dsm = tile_d(s);
+            const float *Bs;
+            const float *Cs;
+            if (Cfg::ES == 4) {
+                Bs = reinterpret_cast<const float *>(tile_b(s));
+                Cs = reinterpret_cast<const float *>(tile_c(s));
+            } else {
+                // widen the stage's B and C tiles to fp32 once for all lanes
+                constexpr int kChunks = T * N / 8;  // 8 bf16 per 16-byte chunk
+                const uint4 *rb = reinterpret_cast<const uint4 *>(tile_b(s));
+                const uint4 *rc = reinterpret_cast<const uint4 *>(tile_c(s));
+#pragma unroll
+                for (int q = lane; q < kChunks; q += 32) {
+                    const uint4 vb = rb[q], vc = rc[q];
+                    const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
+                    const uint32_t wc[4] = {vc.x, vc.y, vc.z, vc.w};
+                    float4 *ob = reinterpret_cast<float4 *>(convB + 8 * q);
+                    float4 *oc = reinterpret_cast<float4 *>(convC + 8 * q);
+                    ob[0] = make_float4(__uint_as_float(wb[0] << 16), __uint_as_float(wb[0] & 0xffff0000u),
+                                        __uint_as_float(wb[1] << 16), __uint_as_float(wb[1] & 0xffff0000u));
+                    ob[1] = make_float4(__uint_as_float(wb[2] << 16), __uint_as_float(wb[2] & 0xffff0000u),
+                                        __uint_as_float(wb[3] << 16), __uint_as_float(wb[3] & 0xffff0000u));
+                    oc[0] = make_float4(__uint_as_float(wc[0] << 16), __uint_as_float(wc[0] & 0xffff0000u),
+                                        __uint_as_float(wc[1] << 16), __uint_as_float(wc[1] & 0xffff0000u));
+                    oc[1] = make_float4(__uint_as_float(wc[2] << 16), __uint_as_float(wc[2] & 0xffff0000u),
+                                        __uint_as_float(wc[3] << 16), __uint_as_float(wc[3] & 0xffff0000u));
+                }
+                __syncwarp();
+                Bs = convB;
+                Cs = convC;
+            }
+            const int nsteps = static_cast<int>(te - t0 < T ? te - t0 : T);
+            IO *yp = ybase + t0 * D;
+            int j = 0;
+            float ssum = 0.0f;  // split mode: this stage's share of dsum
+            // Groups of G tokens: discretize the whole group first (independent of h),
+            // then its sequential state updates, then one reduce-scatter of the G
+            // partial outputs over the channel's lanes, so every lane stores.
+            constexpr int G = Cfg::G;
+            constexpr int KEEP = G / LPC > 0 ? G / LPC : 1;
+            const bool g_store = valid && (LPC <= G || (g & (LPC / G - 1)) == 0);
+            auto group = [&](int j0) {
+                f2 ab[G][NP], bu[G][NP];
+#pragma unroll
+                for (int q = 0; q < G; ++q) {
+                    const float x = Io<IO>::widen(us[(j0 + q) * CPW + cl]);
+                    const float dl = Io<IO>::widen(dsm[(j0 + q) * CPW + cl]);
+                    if (SPLIT) {
+                        ssum += dl;
+                        dmin = fminf(dmin, dl);
+                    }
+                    if (q & 1)
+                        discretize<NP, ZOH, POLY, 1>(ab[q], bu[q], A2, A1, iA, cap, x, dl, Bs + (j0 + q) * N + n0);
+                    else
+                        discretize<NP, ZOH, POLY, 0>(ab[q], bu[q], A2, A1, iA, cap, x, dl, Bs + (j0 + q) * N + n0);
+                }
+                float yv[G];
+#pragma unroll
+                for (int q = 0; q < G; ++q) yv[q] = advance<NP>(h, ab[q], bu[q], Cs + (j0 + q) * N + n0);
+                const int base = reduce_scatter<LPC, G>(yv, g);
+                if (g_store) {
+#pragma unroll
+                    for (int q = 0; q < KEEP; ++q) Io<IO>::st(yp + (j0 + base + q) * D, yv[q]);
+                }
+            };
+            if (nsteps == T && NP <= 4) {
+                // A full stage as one straight-line block with a per-token software
+                // pipeline: token q+PD is discretized (MUFU exponents, independent of h)
+                // right before token q's state update, so in program order every burst
+                // of exponents sits next to FMA-pipe work that does not depend on it.
+                constexpr int PD = 2;  // pipeline distance in tokens
+                f2 ab[PD + 1][NP], bu[PD + 1][NP];
+                auto disc_tok = [&](int q, f2 (&a)[NP], f2 (&b2)[NP]) {
+                    const float x = Io<IO>::widen(us[q * CPW + cl]);
+                    const float dl = Io<IO>::widen(dsm[q * CPW + cl]);
+                    if (SPLIT) {
+                        ssum += dl;
+                        dmin = fminf(dmin, dl);
+                    }
+                    if (q & 1)
+                        discretize<NP, ZOH, POLY, 1>(a, b2, A2, A1, iA, cap, x, dl, Bs + q * N + n0);
+                    else
+                        discretize<NP, ZOH, POLY, 0>(a, b2, A2, A1, iA, cap, x, dl, Bs + q * N + n0);
+                };
+#pragma unroll
+                for (int q = 0; q < PD; ++q) disc_tok(q, ab[q], bu[q]);
+                float yv[G];
+#pragma unroll
+                for (int q = 0; q < T; ++q) {
+                    if (q + PD < T) disc_tok(q + PD, ab[(q + PD) % (PD + 1)], bu[(q + PD) % (PD + 1)]);
+                    yv[q % G] = advance<NP>(h, ab[q % (PD + 1)], bu[q % (PD + 1)], Cs + q * N + n0);
+                    if (q % G == G - 1) {
+                        const int base = reduce_scatter<LPC, G>(yv, g);
+                        if (g_store) {
+#pragma unroll
+                            for (int r = 0; r < KEEP; ++r) Io<IO>::st(yp + (q - (G - 1) + base + r) * D, yv[r]);
+                        }
+                    }
+                }
+                j = T;
+            } else if (nsteps == T) {
+#pragma unroll
+                for (int j0 = 0; j0 < T; j0 += G) group(j0);
+                j = T;
+            } else {
+                for (; j + G <= nsteps; j += G) group(j);
+            }
+            for (; j < nsteps; ++j) {  // ragged end of a part
+                f2 ab[NP], bu[NP];
+                const float x = Io<IO>::widen(us[j * CPW + cl]);
+                const float dl = Io<IO>::widen(dsm[j * CPW + cl]);
+                if (SPLIT) {
+                    ssum += dl;
+                    dmin = fminf(dmin, dl);
+                }
+                discretize<NP, ZOH, POLY, 0>(ab, bu, A2, A1, iA, cap, x, dl, Bs + j * N + n0);
+                float yv = advance<NP>(h, ab, bu, Cs + j * N + n0);
+#pragma unroll
+                for (int o = 1; o < LPC; o <<= 1) yv += __shfl_xor_sync(0xffffffffu, yv, o);
+                if (valid && g == 0) Io<IO>::st(yp + j * D, yv);
+            }
+            if (SPLIT) dsum += static_cast<double>(ssum);
+            // Every lane of this warp is done reading the slot (the warp that consumes a
+            // slot is the one that refills it): order those shared-memory reads before
+            // the TMA write that reuses the slot, then load the stage STAGES ahead.
+            __syncwarp();
+            if (lane == 0 && !p_done) {
+                fence_proxy_async_smem();
+                p_issue();
+            }
+            ++consumed;
+        }
+        if (failed) break;
+
+        if (SPLIT && (ts > 0 || te < L)) {
+            // publish this piece's record: local end state, sum of delta, monotone flag
+            const int64_t r = c * P.max_pieces + (wk - (c * L) / P.seg);
+            float *dst = P.rec_h + (r * 32 + lane) * NL;
+            bool a_nonpos = true;
+#pragma unroll
+            for (int p = 0; p < NP; p += 2) {
+                float a, bq, cq, e;
+                unpack2(h[p], a, bq);
+                unpack2(h[p + 1], cq, e);
+                __stcg(reinterpret_cast<float4 *>(dst + 2 * p), make_float4(a, bq, cq, e));
+            }
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+                float x0, x1;
+                unpack2(A2[p], x0, x1);
+                a_nonpos = a_nonpos && x0 <= 0.0f && x1 <= 0.0f;
+            }
+            __stcg(P.rec_s + r * 32 + lane, static_cast<float>(dsum));
+            const bool mono = __all_sync(0xffffffffu, a_nonpos && dmin >= 0.0f);
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) {
+                __stcg(P.rec_mono + r, mono ? 1 : 0);
+                __threadfence();
+                st_release_u64(P.rec_flags + r, P.epoch_hi | 1ull);
+            }
+        } else if (te < L) {
+            // publish the state at the cut for the warp that runs the rest of this chain
+            float *dst = P.carry + (c * 32 + lane) * NL;
+#pragma unroll
+            for (int p = 0; p < NP; p += 2) {
+                float a, bq, cq, e;
+                unpack2(h[p], a, bq);
+                unpack2(h[p + 1], cq, e);
+                __stcg(reinterpret_cast<float4 *>(dst + 2 * p), make_float4(a, bq, cq, e));
+            }
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) st_release_u64(P.flags + c, P.epoch_hi | static_cast<unsigned long long>(te));
+        } else if (P.h_final != nullptr && valid) {
+            float *dst = P.h_final + (b * D + d) * N + n0;
+#pragma unroll
+            for (int p = 0; p < NP; p += 2) {
+                float a, bq, cq, e;
+                unpack2(h[p], a, bq);
+                unpack2(h[p + 1], cq, e);
+                *reinterpret_cast<float4 *>(dst + 2 * p) = make_float4(a, bq, cq, e);
+            }
+        }
+    }
+    if (SPLIT && !failed) {
+        __syncwarp();
+        __threadfence_block();  // phase-1 y stores of every lane before the fix-up reads them
+        for (int64_t k = 0; k < n_parts; ++k) {
+            int64_t c, ts, te;
+            part(k, c, ts, te);
+            if (ts == 0) continue;
+            split_fixup<IO, Cfg>(P, c, ts, te, wk, lane);
+        }
+    }
+    if (failed) {
+        // drain loads still in flight into this warp's ring before leaving (bounded)
+        if (lane == 0)
+            for (int64_t i = consumed; i < issued; ++i)
+                mbar_wait(&full[i % STAGES], static_cast<uint32_t>((i / STAGES) & 1));
+        __syncwarp();
+    }
+}
+
+}  // namespace sscan

@@ -1,0 +1,138 @@
+// kernel_generic.cuh -- the generic selective-scan forward kernel.
+//
+// One thread owns NL of the N states of one (b,d) channel in registers for the
+// whole sequence; LPC = N/NL neighbouring lanes share a channel and combine
+// their partial y with shuffles.  u/delta are read with plain loads (adjacent
+// lanes -> adjacent channels) through an 8-token register prefetch ring; B/C
+// rows come from L1.  It accepts any D and any 16-byte aligned pointers and
+// is used where the chained TMA kernel does not apply (D*element size not a
+// multiple of 16 bytes, an empty sequence, or too few channels to fill the GPU
+// without splitting the sequence).
+#pragma once
+
+#include "device_utils.cuh"
+
+namespace sscan {
+
+constexpr int kGenericThreads = 128;  // threads per block
+constexpr int kPrefetch = 8;          // tokens of u/delta kept in flight per thread
+
+
+// One block: kGenericThreads/LPC channels of batch row blockIdx.y, channels
+// blockIdx.x*(kGenericThreads/LPC) ...; thread (channel c, group g) owns states
+// [g*NL, (g+1)*NL).  Lanes of one channel are adjacent (g fastest).
+template <class IO, int NL, int LPC, bool ZOH>
+__global__ void __launch_bounds__(kGenericThreads)
+sscan_generic_kernel(const IO *__restrict__ u, const IO *__restrict__ delta,
+                 const float *__restrict__ A, const IO *__restrict__ Bm,
+                 const IO *__restrict__ Cm, const float *h0, IO *__restrict__ y,
+                 float *h_final, int64_t L, int64_t D) {
+    constexpr int N = NL * LPC;
+    constexpr int NP = NL / 2;  // packed pairs per thread
+    constexpr int CPB = kGenericThreads / LPC;
+    const int g = threadIdx.x % LPC;
+    const int64_t b = blockIdx.y;
+    const int64_t d = static_cast<int64_t>(blockIdx.x) * CPB + threadIdx.x / LPC;
+    const bool valid = d < D;
+    const int64_t dc = valid ? d : D - 1;  // ragged tail: read a real channel, store nothing
+    const int n0 = g * NL;
+
+    // per-thread constants: A*log2(e) (Abar = 2^(delta*A2)); ZOH also needs A and 1/A
+    f2 A2[NP], A1[NP], iA[NP];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+        const float a0 = __ldg(A + dc * N + n0 + 2 * p), a1 = __ldg(A + dc * N + n0 + 2 * p + 1);
+        A2[p] = pack2(static_cast<float>(static_cast<double>(a0) * 1.4426950408889634),
+                      static_cast<float>(static_cast<double>(a1) * 1.4426950408889634));
+        if (ZOH) {
+            A1[p] = pack2(a0, a1);
+            iA[p] = pack2(1.0f / a0, 1.0f / a1);
+        }
+    }
+    f2 h[NP];
+    const int64_t srow = (b * D + dc) * N + n0;
+    if (h0 != nullptr) {
+#pragma unroll
+        for (int p = 0; p < NP; p += 2) {
+            const float4 v = *reinterpret_cast<const float4 *>(h0 + srow + 2 * p);
+            h[p] = pack2(v.x, v.y);
+            h[p + 1] = pack2(v.z, v.w);
+        }
+    } else {
+#pragma unroll
+        for (int p = 0; p < NP; ++p) h[p] = pack2(0.0f, 0.0f);
+    }
+
+    const IO *up = u + b * L * D + dc;
+    const IO *dp = delta + b * L * D + dc;
+    const IO *bp = Bm + b * L * N + n0;
+    const IO *cp = Cm + b * L * N + n0;
+    IO *yp = y + b * L * D + dc;
+    const bool writer = valid && g == 0;
+
+    IO ubuf[kPrefetch], dbuf[kPrefetch];
+#pragma unroll
+    for (int k = 0; k < kPrefetch; ++k)
+        if (k < L) {
+            ubuf[k] = Io<IO>::ld(up + k * D);
+            dbuf[k] = Io<IO>::ld(dp + k * D);
+        }
+
+    for (int64_t t0 = 0; t0 < L; t0 += kPrefetch) {
+#pragma unroll
+        for (int k = 0; k < kPrefetch; ++k) {
+            const int64_t t = t0 + k;
+            if (t < L) {
+                const float x = Io<IO>::widen(ubuf[k]);
+                const float dl = Io<IO>::widen(dbuf[k]);
+                if (t + kPrefetch < L) {
+                    ubuf[k] = Io<IO>::ld(up + (t + kPrefetch) * D);
+                    dbuf[k] = Io<IO>::ld(dp + (t + kPrefetch) * D);
+                }
+                f2 Bp[NP], Cp[NP];
+                Io<IO>::template ld_pairs<NP>(bp + t * N, Bp);
+                Io<IO>::template ld_pairs<NP>(cp + t * N, Cp);
+
+                const f2 dd = pack2(dl, dl);
+                const float du = dl * x;
+                const f2 du2 = pack2(du, du);
+                const f2 xx = pack2(x, x);
+                f2 ya = pack2(0.0f, 0.0f), yb = pack2(0.0f, 0.0f);
+#pragma unroll
+                for (int p = 0; p < NP; ++p) {
+                    float e0, e1;
+                    unpack2(mul2(dd, A2[p]), e0, e1);
+                    const f2 abar = pack2(ex2(e0), ex2(e1));
+                    f2 bu;
+                    if (!ZOH) {
+                        bu = mul2(Bp[p], du2);
+                    } else {
+                        bu = mul2(zoh_coef_pair(dd, A1[p], iA[p], abar), mul2(Bp[p], xx));
+                    }
+                    h[p] = fma2(abar, h[p], bu);
+                    if (p & 1)
+                        yb = fma2(Cp[p], h[p], yb);
+                    else
+                        ya = fma2(Cp[p], h[p], ya);
+                }
+                float y0, y1;
+                unpack2(add2(ya, yb), y0, y1);
+                float yv = y0 + y1;
+#pragma unroll
+                for (int o = 1; o < LPC; o <<= 1) yv += __shfl_xor_sync(0xffffffffu, yv, o);
+                if (writer) Io<IO>::st(yp + t * D, yv);
+            }
+        }
+    }
+    if (h_final != nullptr && valid) {
+#pragma unroll
+        for (int p = 0; p < NP; p += 2) {
+            float a, bq, c, e;
+            unpack2(h[p], a, bq);
+            unpack2(h[p + 1], c, e);
+            *reinterpret_cast<float4 *>(h_final + (b * D + d) * N + n0 + 2 * p) = make_float4(a, bq, c, e);
+        }
+    }
+}
+
+}  // namespace sscan

@@ -1,5 +1,6 @@
-// sscan.cu -- selective-scan (Mamba / S6) forward for B200 (sm_100a), and the
-// C ABI declared in include/sscan.h.
+// sscan.cu -- host side of the B200 (sm_100a) selective-scan forward library:
+// plans, schedule choice, TMA descriptors, launches, and the C ABI declared in
+// include/sscan.h.
 //
 // What is computed ("tm_ssm_selective" (Transformer Math page on selective
 // SSMs), section "Discretization becomes a per-token operation"; the
@@ -7,265 +8,72 @@
 //     Abar = exp(delta*A[d,n]);   Bbar u = delta*B[n]*u  (Euler) or
 //     (exp(delta*A)-1)/A*B[n]*u (ZOH);   h = Abar*h + Bbar u;   y = sum_n C[n]*h.
 //
-// Design (B200-first; the pages' SRAM-fused kernel for older GPUs is prior art):
-//  * Each thread owns NL of the N states of one (b,d) channel in registers
-//    for the whole sequence; LPC = N/NL neighbouring lanes share a channel and
-//    combine their partial y with warp shuffles.  The [B,L,D,N] tensors
-//    (Abar, Bbar u, h over time) never exist outside registers.
-//  * fp32 arithmetic throughout, on packed f32x2 FMA/MUL/ADD (two states per
-//    instruction) to halve the issue slots; exp through ex2.approx on the
-//    MUFU pipe with the log2(e) factor folded into A once per thread.
-//  * u/delta are streamed along D (adjacent lanes -> adjacent channels, so
-//    loads coalesce) with an 8-token register prefetch ring; B/C rows are
-//    shared by every channel of a batch row and come from L1.
-//  * The path is ALU bound on B200 (one exp and four FMA-pipe operations per
-//    state update against 1-3 bytes of HBM traffic), so no tensor cores.
+// Two kernels:
+//  * chained (kernel_chained.cuh): persistent, cooperative, one warp per
+//    chain segment, TMA-staged inputs, exactly balanced work per warp;
+//  * generic (kernel_generic.cuh): one thread per (channel, state group),
+//    plain loads; for shapes the chained kernel cannot take.
+// Both keep every (b,d) state row in registers; the [B,L,D,N] tensors never
+// reach memory.  The path is ALU bound on B200 (one 2^x and four FMA-pipe
+// operations per state update against 1-3 bytes of HBM traffic), so there are
+// no tensor-core stages.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 
+#include "device_utils.cuh"
+#include "kernel_chained.cuh"
+#include "kernel_generic.cuh"
 #include "sscan.h"
 
-#define SSCAN_VERSION 100  // 0.1.0
+#define SSCAN_VERSION 200  // 0.2.0
+
+using namespace sscan;
 
 namespace {
 
-// ---------------------------------------------------------------- device utils
+enum Mode { kGeneric = 0, kChained = 1 };
 
-typedef unsigned long long f2;  // two fp32 values in one 64-bit register pair
-
-__device__ __forceinline__ f2 pack2(float lo, float hi) {
-    f2 r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ void unpack2(f2 v, float &lo, float &hi) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
-    f2 r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
-__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
-    f2 r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ f2 add2(f2 a, f2 b) {
-    f2 r;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-// 2^x on the MUFU pipe (flushes results below 2^-126 to zero)
-__device__ __forceinline__ float ex2(float x) {
-    float r;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-    return r;
-}
-
-// Storage types: fp32 as float, bf16 as its 16-bit pattern.
-template <class IO> struct Io;
-template <> struct Io<float> {
-    static __device__ __forceinline__ float ld(const float *p) { return __ldg(p); }
-    static __device__ __forceinline__ float widen(float v) { return v; }
-    static __device__ __forceinline__ void st(float *p, float v) { *p = v; }
-    // NP consecutive pairs (2*NP values) starting at p (16-byte aligned)
-    template <int NP>
-    static __device__ __forceinline__ void ld_pairs(const float *p, f2 (&out)[NP]) {
-#pragma unroll
-        for (int i = 0; i < NP / 2; ++i) {
-            const float4 v = __ldg(reinterpret_cast<const float4 *>(p) + i);
-            out[2 * i] = pack2(v.x, v.y);
-            out[2 * i + 1] = pack2(v.z, v.w);
-        }
-    }
+// Chained-kernel shapes compiled into the library.  NL states per lane, T
+// tokens per pipeline stage, STAGES stages per warp, WPC warps per block.
+struct KCfg {
+    int N, NL, T, STAGES, WPC;
 };
-template <> struct Io<uint16_t> {
-    static __device__ __forceinline__ uint16_t ld(const uint16_t *p) { return __ldg(p); }
-    static __device__ __forceinline__ float widen(uint16_t v) {
-        return __uint_as_float(static_cast<uint32_t>(v) << 16);
-    }
-    static __device__ __forceinline__ void st(uint16_t *p, float v) {
-        uint16_t r;
-        asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(v));
-        *p = r;
-    }
-    template <int NP>
-    static __device__ __forceinline__ void ld_pairs(const uint16_t *p, f2 (&out)[NP]) {
-#pragma unroll
-        for (int i = 0; i < NP / 4; ++i) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p) + i);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j)  // low half = even state, high half = odd state
-                out[4 * i + j] = pack2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xffff0000u));
-        }
-    }
+// In order of preference for a shape; a shape is taken when the problem has at
+// least one chain per warp of the persistent grid (148 blocks x WPC warps).
+// Measured on B200: the MUFU pipe saturates from 2 warps per SM sub-partition
+// at 8 states per lane and from ~4 at 4 states per lane.
+constexpr KCfg kChainedCfgs[] = {
+    {16, 8, 32, 4, 8},   // 16 channels per warp, 2 warps per SM sub-partition (bf16 only: smem)
+    {16, 4, 16, 4, 12},  // 8 channels per warp, 3 warps per sub-partition
+    {16, 4, 16, 4, 8},   // 8 channels per warp, 2 warps per sub-partition
+    {16, 8, 32, 4, 4},   // 16 channels per warp, 1 warp per sub-partition
+    {16, 4, 16, 4, 4},   // 8 channels per warp, 1 warp per sub-partition
+    {32, 8, 32, 4, 4},   // 8 channels per warp
+    {64, 16, 16, 3, 8},  // 8 channels per warp, 2 warps per sub-partition
 };
+constexpr int kNumCfgs = sizeof(kChainedCfgs) / sizeof(kChainedCfgs[0]);
 
-constexpr int kThreads = 128;  // threads per block
-constexpr int kPrefetch = 8;   // tokens of u/delta kept in flight per thread
+std::atomic<uint32_t> g_epoch{1};  // launch tags of the chained kernel (unique per process)
 
-// phi(z) = (exp(z) - 1) / z = sum_k z^k / (k+1)!, truncated after z^7; for
-// |z| <= 1/2 the first omitted term is below 1.1e-8 relative.  Coefficients
-// are the Taylor series 1/(k+1)!, highest first.
-__device__ __forceinline__ f2 phi2(f2 z) {
-    const f2 c7 = pack2(1.0f / 40320.0f, 1.0f / 40320.0f);
-    const f2 c6 = pack2(1.0f / 5040.0f, 1.0f / 5040.0f);
-    const f2 c5 = pack2(1.0f / 720.0f, 1.0f / 720.0f);
-    const f2 c4 = pack2(1.0f / 120.0f, 1.0f / 120.0f);
-    const f2 c3 = pack2(1.0f / 24.0f, 1.0f / 24.0f);
-    const f2 c2 = pack2(1.0f / 6.0f, 1.0f / 6.0f);
-    const f2 c1 = pack2(0.5f, 0.5f);
-    const f2 c0 = pack2(1.0f, 1.0f);
-    f2 q = fma2(c7, z, c6);
-    q = fma2(q, z, c5);
-    q = fma2(q, z, c4);
-    q = fma2(q, z, c3);
-    q = fma2(q, z, c2);
-    q = fma2(q, z, c1);
-    return fma2(q, z, c0);
+constexpr int kMaxSmem = 227 * 1024;  // dynamic shared memory per block on B200
+
+// Shared memory of a chained-kernel shape (mirrors ChainedCfg::kSmem).
+int chained_smem_bytes(const KCfg &k, int es) {
+    const int lpc = k.N / k.NL, cpw = 32 / lpc;
+    const int kU = k.T * cpw * es, kB = k.T * k.N * es;
+    const int stage = 2 * kU + 2 * kB, conv = es == 2 ? 2 * k.T * k.N * 4 : 0, bar = k.STAGES * 8;
+    const int warp = (k.STAGES * stage + conv + bar + 127) / 128 * 128;
+    return k.WPC * warp;
 }
-
-// ------------------------------------------------------------------ kernel
-
-// One block: kThreads/LPC channels of batch row blockIdx.y, channels
-// blockIdx.x*(kThreads/LPC) ...; thread (channel c, group g) owns states
-// [g*NL, (g+1)*NL).  Lanes of one channel are adjacent (g fastest).
-template <class IO, int NL, int LPC, bool ZOH>
-__global__ void __launch_bounds__(kThreads)
-sscan_fwd_kernel(const IO *__restrict__ u, const IO *__restrict__ delta,
-                 const float *__restrict__ A, const IO *__restrict__ Bm,
-                 const IO *__restrict__ Cm, const float *h0, IO *__restrict__ y,
-                 float *h_final, int64_t L, int64_t D) {
-    constexpr int N = NL * LPC;
-    constexpr int NP = NL / 2;  // packed pairs per thread
-    constexpr int CPB = kThreads / LPC;
-    const int g = threadIdx.x % LPC;
-    const int64_t b = blockIdx.y;
-    const int64_t d = static_cast<int64_t>(blockIdx.x) * CPB + threadIdx.x / LPC;
-    const bool valid = d < D;
-    const int64_t dc = valid ? d : D - 1;  // ragged tail: read a real channel, store nothing
-    const int n0 = g * NL;
-
-    // per-thread constants: A*log2(e) (Abar = 2^(delta*A2)); ZOH also needs A and 1/A
-    f2 A2[NP], A1[NP], iA[NP];
-#pragma unroll
-    for (int p = 0; p < NP; ++p) {
-        const float a0 = __ldg(A + dc * N + n0 + 2 * p), a1 = __ldg(A + dc * N + n0 + 2 * p + 1);
-        A2[p] = pack2(static_cast<float>(static_cast<double>(a0) * 1.4426950408889634),
-                      static_cast<float>(static_cast<double>(a1) * 1.4426950408889634));
-        if (ZOH) {
-            A1[p] = pack2(a0, a1);
-            iA[p] = pack2(1.0f / a0, 1.0f / a1);
-        }
-    }
-    f2 h[NP];
-    const int64_t srow = (b * D + dc) * N + n0;
-    if (h0 != nullptr) {
-#pragma unroll
-        for (int p = 0; p < NP; p += 2) {
-            const float4 v = *reinterpret_cast<const float4 *>(h0 + srow + 2 * p);
-            h[p] = pack2(v.x, v.y);
-            h[p + 1] = pack2(v.z, v.w);
-        }
-    } else {
-#pragma unroll
-        for (int p = 0; p < NP; ++p) h[p] = pack2(0.0f, 0.0f);
-    }
-
-    const IO *up = u + b * L * D + dc;
-    const IO *dp = delta + b * L * D + dc;
-    const IO *bp = Bm + b * L * N + n0;
-    const IO *cp = Cm + b * L * N + n0;
-    IO *yp = y + b * L * D + dc;
-    const bool writer = valid && g == 0;
-
-    IO ubuf[kPrefetch], dbuf[kPrefetch];
-#pragma unroll
-    for (int k = 0; k < kPrefetch; ++k)
-        if (k < L) {
-            ubuf[k] = Io<IO>::ld(up + k * D);
-            dbuf[k] = Io<IO>::ld(dp + k * D);
-        }
-
-    for (int64_t t0 = 0; t0 < L; t0 += kPrefetch) {
-#pragma unroll
-        for (int k = 0; k < kPrefetch; ++k) {
-            const int64_t t = t0 + k;
-            if (t < L) {
-                const float x = Io<IO>::widen(ubuf[k]);
-                const float dl = Io<IO>::widen(dbuf[k]);
-                if (t + kPrefetch < L) {
-                    ubuf[k] = Io<IO>::ld(up + (t + kPrefetch) * D);
-                    dbuf[k] = Io<IO>::ld(dp + (t + kPrefetch) * D);
-                }
-                f2 Bp[NP], Cp[NP];
-                Io<IO>::template ld_pairs<NP>(bp + t * N, Bp);
-                Io<IO>::template ld_pairs<NP>(cp + t * N, Cp);
-
-                const f2 dd = pack2(dl, dl);
-                const float du = dl * x;
-                const f2 du2 = pack2(du, du);
-                const f2 xx = pack2(x, x);
-                f2 ya = pack2(0.0f, 0.0f), yb = pack2(0.0f, 0.0f);
-#pragma unroll
-                for (int p = 0; p < NP; ++p) {
-                    float e0, e1;
-                    unpack2(mul2(dd, A2[p]), e0, e1);
-                    const f2 abar = pack2(ex2(e0), ex2(e1));
-                    f2 bu;
-                    if (!ZOH) {
-                        bu = mul2(Bp[p], du2);
-                    } else {
-                        // (exp(z)-1)/A * B*u with z = delta*A: delta*phi(z) for |z| <= 1/2
-                        // (exact at A = 0), (Abar - 1) * (1/A) otherwise.
-                        const f2 z = mul2(dd, A1[p]);
-                        const f2 small = mul2(dd, phi2(z));
-                        const f2 big = mul2(add2(abar, pack2(-1.0f, -1.0f)), iA[p]);
-                        float z0, z1, s0, s1, g0, g1;
-                        unpack2(z, z0, z1);
-                        unpack2(small, s0, s1);
-                        unpack2(big, g0, g1);
-                        const f2 coef = pack2(fabsf(z0) <= 0.5f ? s0 : g0, fabsf(z1) <= 0.5f ? s1 : g1);
-                        bu = mul2(coef, mul2(Bp[p], xx));
-                    }
-                    h[p] = fma2(abar, h[p], bu);
-                    if (p & 1)
-                        yb = fma2(Cp[p], h[p], yb);
-                    else
-                        ya = fma2(Cp[p], h[p], ya);
-                }
-                float y0, y1;
-                unpack2(add2(ya, yb), y0, y1);
-                float yv = y0 + y1;
-#pragma unroll
-                for (int o = 1; o < LPC; o <<= 1) yv += __shfl_xor_sync(0xffffffffu, yv, o);
-                if (writer) Io<IO>::st(yp + t * D, yv);
-            }
-        }
-    }
-    if (h_final != nullptr && valid) {
-#pragma unroll
-        for (int p = 0; p < NP; p += 2) {
-            float a, bq, c, e;
-            unpack2(h[p], a, bq);
-            unpack2(h[p + 1], c, e);
-            *reinterpret_cast<float4 *>(h_final + (b * D + d) * N + n0 + 2 * p) = make_float4(a, bq, c, e);
-        }
-    }
-}
-
-// ------------------------------------------------------------------- host side
-
-struct Schedule {
-    int nl;   // states per thread
-    int lpc;  // threads per channel
-};
 
 }  // namespace
 
@@ -275,8 +83,22 @@ struct sscan_plan {
     uint32_t flags;
     int device;
     int sm_count;
-    Schedule sched;
-    int *d_status;  // device status word
+    int *d_status;
+    Mode mode;
+    // chained kernel
+    int cfg;           // index into kChainedCfgs
+    bool poly;         // part of the exponents on the FMA pipe
+    bool split;        // chains cut into concurrently scanned pieces + look-back fix-up
+    int64_t chains_per_row, chains, workers, seg, max_pieces;
+    size_t flag_off, flag_bytes;                // flags cleared on a workspace's first use
+    size_t rec_s_off, rec_mono_off, ws_bytes;   // split-mode record arrays (rec_h at 0)
+    const void *last_ws;  // workspace whose flags were last cleared
+    // tensor-map cache
+    const void *tm_ptr[4];
+    CUtensorMap tm[4];
+    bool tm_valid;
+    // generic kernel
+    int g_nl, g_lpc;
 };
 
 namespace {
@@ -289,37 +111,239 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
     return a0 < b0 + nb && b0 < a0 + na;
 }
 
-Schedule choose_schedule(int64_t N) {
-    if (N == 16) return {8, 2};
-    if (N == 32) return {16, 2};
-    return {16, 4};  // N == 64
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
 }
 
+// Optional tuning override read at plan creation, e.g. SSCAN_TUNE="cfg=1,poly=0,sms=4":
+// cfg indexes the chained shapes above (-1 forces the generic kernel), poly=0
+// keeps every exponent on the MUFU pipe, sms limits the chained grid to that
+// many blocks, split=1 forces the split mode (tests use the last two to cut
+// chains on small problems).
+void read_tune(int &cfg, int &poly, int &sms, int &split) {
+    cfg = -2;
+    poly = -1;
+    sms = 0;
+    split = 0;
+    const char *s = getenv("SSCAN_TUNE");
+    if (!s) return;
+    if (const char *c = strstr(s, "cfg=")) cfg = atoi(c + 4);
+    if (const char *c = strstr(s, "poly=")) poly = atoi(c + 5);
+    if (const char *c = strstr(s, "sms=")) sms = atoi(c + 4);
+    if (const char *c = strstr(s, "split=")) split = atoi(c + 6);
+}
+
+void choose_schedule(sscan_plan *p) {
+    const int es = p->dtype == SSCAN_F32 ? 4 : 2;
+    p->mode = kGeneric;
+    p->g_nl = p->N == 16 ? 8 : 16;
+    p->g_lpc = static_cast<int>(p->N) / p->g_nl;
+    int want = -2, poly = -1, sms = 0, force_split = 0;
+    read_tune(want, poly, sms, force_split);
+    const int blocks = (sms > 0 && sms < p->sm_count) ? sms : p->sm_count;
+    // the FMA-pipe exponent measured slower than MUFU alone at every occupancy: off unless asked
+    p->poly = (p->flags & SSCAN_ZOH) ? false : (poly == 1);
+    if (want == -1) return;
+    // the chained kernel needs TMA-compatible rows and int32 TMA row coordinates
+    if (p->L == 0 || (p->D * es) % 16 != 0 || p->B * p->L >= (int64_t(1) << 31) ||
+        p->L >= (int64_t(1) << 32))
+        return;
+    // 1) chained: enough chains that each is cut at most once (segment >= L)
+    // 2) split: fewer chains than warps; cut them into pieces scanned concurrently
+    for (int pass = force_split ? 1 : 0; pass < 2; ++pass) {
+        for (int i = 0; i < kNumCfgs; ++i) {
+            const KCfg &k = kChainedCfgs[i];
+            if (k.N != p->N) continue;
+            if (want >= 0 && want != i) continue;
+            const int lpc = k.N / k.NL, cpw = 32 / lpc;
+            if ((cpw * es) % 16 != 0) continue;
+            if (chained_smem_bytes(k, es) > kMaxSmem) continue;
+            const int64_t cpr = ceil_div(p->D, cpw);
+            const int64_t chains = p->B * cpr;
+            int64_t workers = int64_t(blocks) * k.WPC;
+            const bool split = pass == 1;
+            // segments somewhat shorter than L cut a few chains twice (a short wait for the
+            // middle piece); measured cheaper than fewer warps down to ~0.85 L
+            if (!split && chains * 20 < workers * 17 && want < 0) continue;
+            if (split && !force_split) {  // at least 256 tokens per warp; whole blocks
+                const int64_t cap = (chains * p->L / 256) / k.WPC * k.WPC;
+                if (cap < workers) workers = cap > k.WPC ? cap : k.WPC;
+            }
+            p->mode = kChained;
+            p->split = split && chains < workers;  // else the capped grid already fits whole chains
+            p->cfg = i;
+            p->chains_per_row = cpr;
+            p->chains = chains;
+            p->workers = workers;
+            p->seg = ceil_div(chains * p->L, workers);
+            if (p->split) {
+                p->max_pieces = p->L / p->seg + 2;
+                const size_t recs = size_t(chains) * size_t(p->max_pieces);
+                p->rec_s_off = align_up(recs * 32 * k.NL * sizeof(float), 256);
+                p->rec_mono_off = p->rec_s_off + align_up(recs * 32 * sizeof(float), 256);
+                p->flag_off = p->rec_mono_off + align_up(recs * sizeof(int), 256);
+                p->flag_bytes = recs * sizeof(unsigned long long);
+            } else {
+                p->max_pieces = 0;
+                p->rec_s_off = p->rec_mono_off = 0;
+                p->flag_off = align_up(size_t(chains) * 32 * k.NL * sizeof(float), 256);
+                p->flag_bytes = size_t(chains) * sizeof(unsigned long long);
+            }
+            p->ws_bytes = p->flag_off + align_up(p->flag_bytes, 256);
+            return;
+        }
+    }
+}
+
+// ------------------------------------------------------------ generic launch
+
 template <class IO, int NL, int LPC>
-cudaError_t launch_t(const sscan_plan *p, const void *u, const void *dl, const float *A,
-                     const void *Bm, const void *Cm, const float *h0, void *y, float *hf,
-                     cudaStream_t s) {
-    const dim3 grid(static_cast<unsigned>((p->D + kThreads / LPC - 1) / (kThreads / LPC)),
-                    static_cast<unsigned>(p->B));
+cudaError_t launch_generic_t(const sscan_plan *p, const void *u, const void *dl, const float *A,
+                             const void *Bm, const void *Cm, const float *h0, void *y, float *hf,
+                             cudaStream_t s) {
+    const dim3 grid(static_cast<unsigned>(ceil_div(p->D, kGenericThreads / LPC)), static_cast<unsigned>(p->B));
     if (p->flags & SSCAN_ZOH)
-        sscan_fwd_kernel<IO, NL, LPC, true><<<grid, kThreads, 0, s>>>(
+        sscan_generic_kernel<IO, NL, LPC, true><<<grid, kGenericThreads, 0, s>>>(
             static_cast<const IO *>(u), static_cast<const IO *>(dl), A, static_cast<const IO *>(Bm),
             static_cast<const IO *>(Cm), h0, static_cast<IO *>(y), hf, p->L, p->D);
     else
-        sscan_fwd_kernel<IO, NL, LPC, false><<<grid, kThreads, 0, s>>>(
+        sscan_generic_kernel<IO, NL, LPC, false><<<grid, kGenericThreads, 0, s>>>(
             static_cast<const IO *>(u), static_cast<const IO *>(dl), A, static_cast<const IO *>(Bm),
             static_cast<const IO *>(Cm), h0, static_cast<IO *>(y), hf, p->L, p->D);
     return cudaGetLastError();
 }
 
 template <class IO>
-cudaError_t launch_io(const sscan_plan *p, const void *u, const void *dl, const float *A,
-                      const void *Bm, const void *Cm, const float *h0, void *y, float *hf,
-                      cudaStream_t s) {
+cudaError_t launch_generic(const sscan_plan *p, const void *u, const void *dl, const float *A,
+                           const void *Bm, const void *Cm, const float *h0, void *y, float *hf,
+                           cudaStream_t s) {
     switch (p->N) {
-        case 16: return launch_t<IO, 8, 2>(p, u, dl, A, Bm, Cm, h0, y, hf, s);
-        case 32: return launch_t<IO, 16, 2>(p, u, dl, A, Bm, Cm, h0, y, hf, s);
-        default: return launch_t<IO, 16, 4>(p, u, dl, A, Bm, Cm, h0, y, hf, s);
+        case 16: return launch_generic_t<IO, 8, 2>(p, u, dl, A, Bm, Cm, h0, y, hf, s);
+        case 32: return launch_generic_t<IO, 16, 2>(p, u, dl, A, Bm, Cm, h0, y, hf, s);
+        default: return launch_generic_t<IO, 16, 4>(p, u, dl, A, Bm, Cm, h0, y, hf, s);
+    }
+}
+
+// ------------------------------------------------------------ chained launch
+
+bool encode_map(CUtensorMap *m, const void *ptr, int es, uint64_t inner, uint64_t rows, uint32_t box_inner,
+                uint32_t box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {inner * static_cast<uint64_t>(es)};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(m, es == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                           const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <class IO, int CFG, bool ZOH, bool POLY, bool SPLIT>
+int launch_chained_t(sscan_plan *p, const void *u, const void *dl, const float *A, const void *Bm,
+                     const void *Cm, const float *h0, void *y, float *hf, void *ws, cudaStream_t s) {
+    constexpr KCfg k = kChainedCfgs[CFG];
+    using Cfg = ChainedCfg<IO, k.N, k.NL, k.T, k.STAGES, k.WPC>;
+    auto kern = sscan_chained_kernel<IO, Cfg, ZOH, POLY, SPLIT>;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [&] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+    });
+    if (attr_err != cudaSuccess) return SSCAN_ERR_CUDA;
+
+    const int es = sizeof(IO);
+    const void *ptrs[4] = {u, dl, Bm, Cm};
+    if (!p->tm_valid || memcmp(ptrs, p->tm_ptr, sizeof ptrs) != 0) {
+        const uint64_t rows = static_cast<uint64_t>(p->B * p->L);
+        if (!encode_map(&p->tm[0], u, es, p->D, rows, Cfg::CPW, Cfg::T) ||
+            !encode_map(&p->tm[1], dl, es, p->D, rows, Cfg::CPW, Cfg::T) ||
+            !encode_map(&p->tm[2], Bm, es, p->N, rows, p->N, Cfg::T) ||
+            !encode_map(&p->tm[3], Cm, es, p->N, rows, p->N, Cfg::T)) {
+            p->tm_valid = false;
+            return SSCAN_ERR_CUDA;
+        }
+        memcpy(p->tm_ptr, ptrs, sizeof ptrs);
+        p->tm_valid = true;
+    }
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    unsigned long long *flags = reinterpret_cast<unsigned long long *>(w + p->flag_off);
+    if (ws != p->last_ws) {  // a workspace seen for the first time: clear its flags once
+        if (cudaMemsetAsync(flags, 0, p->flag_bytes, s) != cudaSuccess) return SSCAN_ERR_CUDA;
+        p->last_ws = ws;
+    }
+    uint32_t ep = g_epoch.fetch_add(1);
+    if (ep == 0) ep = g_epoch.fetch_add(1);
+    ChainedParams prm;
+    prm.A = A;
+    prm.h0 = h0;
+    prm.y = y;
+    prm.h_final = hf;
+    prm.carry = reinterpret_cast<float *>(w);
+    prm.flags = flags;
+    prm.delta = dl;
+    prm.Cm = Cm;
+    prm.rec_h = reinterpret_cast<float *>(w);
+    prm.rec_s = reinterpret_cast<float *>(w + p->rec_s_off);
+    prm.rec_mono = reinterpret_cast<int *>(w + p->rec_mono_off);
+    prm.rec_flags = flags;
+    prm.max_pieces = p->max_pieces;
+    prm.status = p->d_status;
+    prm.epoch_hi = static_cast<unsigned long long>(ep) << 32;
+    prm.L = p->L;
+    prm.D = p->D;
+    prm.chains_per_row = p->chains_per_row;
+    prm.chains = p->chains;
+    prm.seg = p->seg;
+    void *args[] = {&p->tm[0], &p->tm[1], &p->tm[2], &p->tm[3], &prm};
+    const dim3 grid(static_cast<unsigned>(p->workers / k.WPC)), block(k.WPC * 32);
+    const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kern), grid, block, args,
+                                                      Cfg::kSmem, s);
+    return e == cudaSuccess ? SSCAN_OK : SSCAN_ERR_CUDA;
+}
+
+template <class IO, int CFG, bool SPLIT>
+int launch_chained_mode(sscan_plan *p, const void *u, const void *dl, const float *A, const void *Bm,
+                        const void *Cm, const float *h0, void *y, float *hf, void *ws, cudaStream_t s) {
+    if (p->flags & SSCAN_ZOH)
+        return launch_chained_t<IO, CFG, true, false, SPLIT>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
+    if (p->poly) return launch_chained_t<IO, CFG, false, true, SPLIT>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
+    return launch_chained_t<IO, CFG, false, false, SPLIT>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
+}
+
+template <class IO, int CFG>
+int launch_chained_cfg(sscan_plan *p, const void *u, const void *dl, const float *A, const void *Bm,
+                       const void *Cm, const float *h0, void *y, float *hf, void *ws, cudaStream_t s) {
+    return p->split ? launch_chained_mode<IO, CFG, true>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s)
+                    : launch_chained_mode<IO, CFG, false>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
+}
+
+template <class IO>
+int launch_chained(sscan_plan *p, const void *u, const void *dl, const float *A, const void *Bm,
+                   const void *Cm, const float *h0, void *y, float *hf, void *ws, cudaStream_t s) {
+    switch (p->cfg) {
+        case 0: return launch_chained_cfg<IO, 0>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
+        case 1: return launch_chained_cfg<IO, 1>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
+        case 2: return launch_chained_cfg<IO, 2>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
+        case 3: return launch_chained_cfg<IO, 3>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
+        case 4: return launch_chained_cfg<IO, 4>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
+        case 5: return launch_chained_cfg<IO, 5>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
+        case 6: return launch_chained_cfg<IO, 6>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
+        default: return SSCAN_ERR_UNSUPPORTED;
     }
 }
 
@@ -356,7 +380,7 @@ int sscan_plan_create(sscan_plan_t *plan, int64_t B, int64_t L, int64_t D, int64
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return SSCAN_ERR_CUDA;
-    sscan_plan *p = new (std::nothrow) sscan_plan;
+    sscan_plan *p = new (std::nothrow) sscan_plan();
     if (!p) return SSCAN_ERR_INVALID;
     p->B = B;
     p->L = L;
@@ -366,8 +390,11 @@ int sscan_plan_create(sscan_plan_t *plan, int64_t B, int64_t L, int64_t D, int64
     p->flags = flags;
     p->device = dev;
     p->sm_count = sms;
-    p->sched = choose_schedule(N);
     p->d_status = nullptr;
+    p->last_ws = nullptr;
+    p->tm_valid = false;
+    p->ws_bytes = 0;
+    choose_schedule(p);
     if (cudaMalloc(&p->d_status, sizeof(int)) != cudaSuccess ||
         cudaMemset(p->d_status, 0, sizeof(int)) != cudaSuccess) {
         if (p->d_status) cudaFree(p->d_status);
@@ -384,21 +411,33 @@ void sscan_plan_destroy(sscan_plan_t plan) {
     delete plan;
 }
 
-size_t sscan_workspace_bytes(sscan_plan_t plan) {
-    (void)plan;
-    return 0;
-}
+size_t sscan_workspace_bytes(sscan_plan_t plan) { return plan ? plan->ws_bytes : 0; }
 
 int sscan_plan_describe(sscan_plan_t plan, char *buf, size_t len) {
     if (!plan) return -1;
-    char tmp[256];
-    const int n = snprintf(tmp, sizeof tmp,
-                           "B=%lld L=%lld D=%lld N=%lld dtype=%s zoh=%d states_per_thread=%d "
-                           "threads_per_channel=%d block=%d sms=%d",
-                           (long long)plan->B, (long long)plan->L, (long long)plan->D,
-                           (long long)plan->N, plan->dtype == SSCAN_F32 ? "f32" : "bf16",
-                           (plan->flags & SSCAN_ZOH) ? 1 : 0, plan->sched.nl, plan->sched.lpc,
-                           kThreads, plan->sm_count);
+    char tmp[512];
+    int n;
+    if (plan->mode == kChained) {
+        const KCfg &k = kChainedCfgs[plan->cfg];
+        n = snprintf(tmp, sizeof tmp,
+                     "kernel=chained B=%lld L=%lld D=%lld N=%lld dtype=%s zoh=%d states_per_thread=%d "
+                     "threads_per_channel=%d channels_per_warp=%d warps_per_block=%d tokens_per_stage=%d "
+                     "stages=%d fma_pipe_exp=%d split=%d chains=%lld warps=%lld segment=%lld workspace=%zu "
+                     "sms=%d",
+                     (long long)plan->B, (long long)plan->L, (long long)plan->D, (long long)plan->N,
+                     plan->dtype == SSCAN_F32 ? "f32" : "bf16", (plan->flags & SSCAN_ZOH) ? 1 : 0, k.NL,
+                     k.N / k.NL, 32 / (k.N / k.NL), k.WPC, k.T, k.STAGES, plan->poly ? 1 : 0,
+                     plan->split ? 1 : 0,
+                     (long long)plan->chains, (long long)plan->workers, (long long)plan->seg, plan->ws_bytes,
+                     plan->sm_count);
+    } else {
+        n = snprintf(tmp, sizeof tmp,
+                     "kernel=generic B=%lld L=%lld D=%lld N=%lld dtype=%s zoh=%d states_per_thread=%d "
+                     "threads_per_channel=%d block=%d sms=%d",
+                     (long long)plan->B, (long long)plan->L, (long long)plan->D, (long long)plan->N,
+                     plan->dtype == SSCAN_F32 ? "f32" : "bf16", (plan->flags & SSCAN_ZOH) ? 1 : 0,
+                     plan->g_nl, plan->g_lpc, kGenericThreads, plan->sm_count);
+    }
     if (buf && len) {
         strncpy(buf, tmp, len - 1);
         buf[len - 1] = '\0';
@@ -409,9 +448,8 @@ int sscan_plan_describe(sscan_plan_t plan, char *buf, size_t len) {
 int sscan_forward(sscan_plan_t plan, const void *u, const void *delta, const float *A,
                   const void *B, const void *C, const float *h0, void *y, float *h_final,
                   void *workspace, void *stream) {
-    (void)workspace;
     if (!plan) return SSCAN_ERR_INVALID;
-    const sscan_plan *p = plan;
+    sscan_plan *p = plan;
     const size_t es = p->dtype == SSCAN_F32 ? 4 : 2;
     const size_t n_bld = static_cast<size_t>(p->B * p->L * p->D);
     const size_t n_bln = static_cast<size_t>(p->B * p->L * p->N);
@@ -435,10 +473,19 @@ int sscan_forward(sscan_plan_t plan, const void *u, const void *delta, const flo
     if (overlaps(h_final, n_bdn * 4, y, n_bld * es)) return SSCAN_ERR_INVALID;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (p->mode == kChained) {
+        if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SSCAN_ERR_WORKSPACE;
+        const size_t sz[8] = {n_bld * es, n_bld * es, n_dn * 4, n_bln * es,
+                              n_bln * es, n_bdn * 4, n_bld * es, n_bdn * 4};
+        for (int i = 0; i < 8; ++i)
+            if (overlaps(workspace, p->ws_bytes, ptrs[i], sz[i])) return SSCAN_ERR_WORKSPACE;
+        return p->dtype == SSCAN_F32
+                   ? launch_chained<float>(p, u, delta, A, B, C, h0, y, h_final, workspace, s)
+                   : launch_chained<uint16_t>(p, u, delta, A, B, C, h0, y, h_final, workspace, s);
+    }
     const cudaError_t e =
-        p->dtype == SSCAN_F32
-            ? launch_io<float>(p, u, delta, A, B, C, h0, y, h_final, s)
-            : launch_io<uint16_t>(p, u, delta, A, B, C, h0, y, h_final, s);
+        p->dtype == SSCAN_F32 ? launch_generic<float>(p, u, delta, A, B, C, h0, y, h_final, s)
+                              : launch_generic<uint16_t>(p, u, delta, A, B, C, h0, y, h_final, s);
     return e == cudaSuccess ? SSCAN_OK : SSCAN_ERR_CUDA;
 }
 
@@ -450,7 +497,7 @@ int sscan_get_status(sscan_plan_t plan, void *stream) {
         cudaMemsetAsync(plan->d_status, 0, sizeof(int), s) != cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess)
         return SSCAN_ERR_CUDA;
-    return v;
+    return v == 0 ? SSCAN_OK : SSCAN_ERR_TIMEOUT;
 }
 
 }  // extern "C"

@@ -53,6 +53,91 @@ def test_small_cases_elementwise(case):
     P.check(hf, hr, dt, "h_final")
 
 
+CHAINED = [
+    # (B, L, D, N, dtype, h0, zoh, cfg, blocks, poly): the chained kernel forced onto a
+    # small grid so that chains are cut between warps (head published, tail resumed).
+    # cfg indexes the library's shape table (see csrc/sscan.cu).
+    (2, 300, 128, 16, "f32", True, False, 3, 3, 1),     # 8 states/lane, FMA-pipe exp on
+    (2, 300, 128, 16, "f32", True, False, 3, 3, 0),
+    (2, 300, 136, 16, "f32", True, False, 2, 2, 0),     # 4 states/lane; ragged last chain
+    (1, 517, 64, 16, "bf16", True, False, 4, 1, 1),
+    (2, 200, 64, 32, "f32", True, True, 5, 2, 0),
+    (2, 100, 72, 64, "bf16", True, True, 6, 1, 0),
+    (3, 37, 128, 16, "f32", False, False, 3, 2, 1),     # L shorter than two stages
+    (2, 300, 128, 16, "f32", True, False, 3, 20, 1),    # segment < L: chains cut many times
+    (2, 300, 256, 16, "bf16", True, False, 0, 1, 0),    # 8 states/lane, 8 warps/block
+    (2, 300, 128, 16, "bf16", True, False, 1, 1, 0),    # 4 states/lane, 12 warps/block
+]
+
+
+@pytest.mark.parametrize("case", CHAINED, ids=[f"cfg{c[7]}_B{c[0]}L{c[1]}D{c[2]}N{c[3]}{c[4]}_blk{c[8]}"
+                                                f"{'_zoh' if c[6] else ''}_poly{c[9]}" for c in CHAINED])
+def test_chained_kernel_forced(case, monkeypatch):
+    Bt, L, D, N, dt, with_h0, zoh, cfg, blocks, poly = case
+    g = W.generate(Bt, L, D, N, dt, 0.1 if with_h0 else 0.0, seed=2000 + L + D, A_jitter=0.3)
+    monkeypatch.setenv("SSCAN_TUNE", f"cfg={cfg},sms={blocks},poly={poly}")
+    plan = S.Plan(Bt, L, D, N, torch.float32 if dt == "f32" else torch.bfloat16, zoh)
+    assert "kernel=chained" in plan.describe(), plan.describe()
+    d = P.to_device(g)
+    y, hf = plan.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"])
+    assert plan.status() == S.OK
+    yr, hr = P.run_oracle(g, zoh)
+    P.check(y.float().cpu().numpy(), yr, dt, "y")
+    P.check(hf.cpu().numpy(), hr, dt, "h_final")
+    # a second call through the same plan and workspace (new launch epoch) is identical
+    y2, hf2 = plan.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"])
+    assert plan.status() == S.OK
+    assert torch.equal(y, y2) and torch.equal(hf, hf2)
+    plan.close()
+
+
+SPLIT = [
+    # (B, L, D, N, dtype, h0, zoh, reset_frac, blocks, negate): split mode forced on a small
+    # grid: pieces scanned from zero, exact carry-in by look-back, bounded fix-up of y
+    (1, 4096, 64, 16, "bf16", True, False, 0.32, 8, False),   # resets: short fix-up windows
+    (1, 4096, 64, 16, "f32", True, False, 0.32, 8, False),
+    (2, 3000, 64, 16, "f32", True, False, 0.0, 8, False),     # slow decay: long windows
+    (1, 2050, 128, 16, "f32", True, True, 0.0, 6, False),     # exact ZOH, ragged pieces
+    (1, 1500, 64, 16, "f32", True, False, 0.32, 4, True),     # some delta < 0: no early exit
+    (2, 700, 72, 64, "bf16", True, True, 0.32, 4, False),     # N = 64 (32 warps > 18 chains)
+]
+
+
+@pytest.mark.parametrize("case", SPLIT, ids=[f"B{c[0]}L{c[1]}D{c[2]}N{c[3]}{c[4]}_r{c[7]}_blk{c[8]}"
+                                              f"{'_zoh' if c[6] else ''}{'_neg' if c[9] else ''}"
+                                              for c in SPLIT])
+def test_split_mode_forced(case, monkeypatch):
+    Bt, L, D, N, dt, with_h0, zoh, rf, blocks, negate = case
+    g = W.generate(Bt, L, D, N, dt, 0.1 if with_h0 else 0.0, rf, seed=3000 + L + D,
+                   A_jitter=0.2)
+    if negate:  # a few negative steps (outside the softplus range) disable the early exit
+        v = W.as_f32(g["delta"], dt).copy()
+        v[:, 100:103, :] *= -0.5
+        g["delta"] = v if dt == "f32" else W.f32_to_bf16_bits(v)
+    monkeypatch.setenv("SSCAN_TUNE", f"split=1,sms={blocks}")
+    plan = S.Plan(Bt, L, D, N, torch.float32 if dt == "f32" else torch.bfloat16, zoh)
+    desc = plan.describe()
+    assert "kernel=chained" in desc and "split=1" in desc, desc
+    d = P.to_device(g)
+    y, hf = plan.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"])
+    assert plan.status() == S.OK
+    yr, hr = P.run_oracle(g, zoh)
+    P.check(y.float().cpu().numpy(), yr, dt, "y")
+    P.check(hf.cpu().numpy(), hr, dt, "h_final")
+    plan.close()
+
+
+def test_default_schedules():
+    """The full-size workloads get the chained kernel; the 2048-channel long sequence is split."""
+    for name, want in [("mamba130m_f32", "split=0"), ("mamba1p4b_bf16", "split=0"),
+                       ("zoh_n64_bf16", "split=0"), ("longseq_bf16", "split=1")]:
+        w = W.WORKLOADS[name]
+        plan = S.Plan(w.B, w.L, w.D, w.N, torch.float32 if w.dtype == "f32" else torch.bfloat16,
+                      w.zoh)
+        assert "kernel=chained" in plan.describe() and want in plan.describe(), (name, plan.describe())
+        plan.close()
+
+
 def test_tiny_workload_full():
     w = W.WORKLOADS["tiny_f32"]
     g = W.make_inputs(w)
