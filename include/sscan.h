@@ -132,6 +132,35 @@ SSCAN_API int sscan_plan_describe(sscan_plan_t plan, char *buf, size_t len);
 /* Library version, major*10000 + minor*100 + patch. */
 SSCAN_API int sscan_version(void);
 
+/* The forward pass for callers that must not allocate device memory.  There is
+ * no counterpart in the pages: this is a deployment convenience.
+ *
+ * Who needs it: code that runs where cudaMalloc is unavailable or unwelcome,
+ * e.g. a host that has handed all device memory to its own pool, or a
+ * latency-critical call site that cannot afford an allocation (which may
+ * synchronise the device).  Such callers still own and pass every input and
+ * output buffer; what they cannot provide is the plan (its status word) and
+ * the scratch workspace that sscan_forward needs for some shapes.
+ *
+ * This entry point allocates nothing.  It takes the shape directly (same
+ * meaning and limits as sscan_plan_create), the same buffers as sscan_forward
+ * and a stream, chooses the same schedule a plan would, and uses as scratch a
+ * fixed 32 MiB array compiled into the library (every GPU that loads the
+ * library holds it until the process exits).  Shapes whose workspace does not
+ * fit return SSCAN_ERR_WORKSPACE without launching.
+ *
+ * The first call on a device looks up the array's device address on that
+ * device (the current one); make that first call before capturing any stream
+ * work.  Every call shares the one array: its contents persist between calls,
+ * the parts that must start at zero are cleared on the caller's stream at the
+ * start of each call, and calls whose work overlaps on the GPU (other streams,
+ * other host threads) race on it.  The return value reports argument and
+ * launch errors; the device status word is reset per call and not returned. */
+SSCAN_API int sscan_forward_noalloc(int64_t B, int64_t L, int64_t D, int64_t N, int dtype,
+                                    uint32_t flags, const void *u, const void *delta, const float *A,
+                                    const void *B_in, const void *C_in, const float *h0, void *y,
+                                    float *h_final, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -349,6 +349,39 @@ int launch_chained(sscan_plan *p, const void *u, const void *dl, const float *A,
 
 }  // namespace
 
+// ------------------------------------------------ allocation-free entry point
+
+namespace {
+
+// Scratch for sscan_forward_noalloc: a fixed array in the library's own device
+// image instead of a caller- or library-allocated buffer.  Every device that
+// loads the library holds these bytes until the process exits.  Layout: the
+// 4-byte device status word at offset 0, the kernel's workspace from offset 256.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+constexpr size_t kNoAllocWorkspaceOffset = 256;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_addr[kMaxDevices] = {};
+
+// The scratch array's device address on device `dev` (the current device).  In
+// host code the symbol itself is only a host-side stand-in, so the address is
+// looked up once per device and cached.
+int noalloc_scratch(int dev, unsigned char **out) {
+    if (dev < 0 || dev >= kMaxDevices) return SSCAN_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return SSCAN_ERR_CUDA;
+        g_noalloc_addr[dev] = ptr;
+    }
+    *out = static_cast<unsigned char *>(g_noalloc_addr[dev]);
+    return SSCAN_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int sscan_version(void) { return SSCAN_VERSION; }
@@ -498,6 +531,42 @@ int sscan_get_status(sscan_plan_t plan, void *stream) {
         cudaStreamSynchronize(s) != cudaSuccess)
         return SSCAN_ERR_CUDA;
     return v == 0 ? SSCAN_OK : SSCAN_ERR_TIMEOUT;
+}
+
+int sscan_forward_noalloc(int64_t B, int64_t L, int64_t D, int64_t N, int dtype, uint32_t flags,
+                          const void *u, const void *delta, const float *A, const void *Bm, const void *Cm,
+                          const float *h0, void *y, float *h_final, void *stream) {
+    // the same size checks as sscan_plan_create, without allocating a plan
+    if (B < 1 || D < 1 || L < 0) return SSCAN_ERR_INVALID;
+    if (B > 65535 || D > (int64_t(1) << 31) || L > (int64_t(1) << 40)) return SSCAN_ERR_UNSUPPORTED;
+    if (dtype != SSCAN_F32 && dtype != SSCAN_BF16) return SSCAN_ERR_INVALID;
+    if (flags & ~static_cast<uint32_t>(SSCAN_ZOH)) return SSCAN_ERR_INVALID;
+    if (N != 16 && N != 32 && N != 64) return SSCAN_ERR_UNSUPPORTED;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SSCAN_ERR_UNSUPPORTED;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return SSCAN_ERR_CUDA;
+    unsigned char *scratch = nullptr;
+    const int rc = noalloc_scratch(dev, &scratch);
+    if (rc != SSCAN_OK) return rc;
+    sscan_plan p{};  // on the stack: same schedule as a plan for this shape
+    p.B = B;
+    p.L = L;
+    p.D = D;
+    p.N = N;
+    p.dtype = dtype;
+    p.flags = flags;
+    p.device = dev;
+    p.sm_count = sms;
+    p.last_ws = nullptr;  // the launch clears the workspace flags it uses
+    p.tm_valid = false;
+    p.ws_bytes = 0;
+    choose_schedule(&p);
+    if (p.ws_bytes > kNoAllocScratchBytes - kNoAllocWorkspaceOffset) return SSCAN_ERR_WORKSPACE;
+    p.d_status = reinterpret_cast<int *>(scratch);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(p.d_status, 0, sizeof(int), s) != cudaSuccess) return SSCAN_ERR_CUDA;
+    return sscan_forward(&p, u, delta, A, Bm, Cm, h0, y, h_final,
+                         p.ws_bytes ? scratch + kNoAllocWorkspaceOffset : nullptr, stream);
 }
 
 }  // extern "C"

@@ -21,7 +21,8 @@ ZOH = 1
 OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(7)
 
 SYMBOLS = ("sscan_plan_create", "sscan_plan_destroy", "sscan_workspace_bytes", "sscan_forward",
-           "sscan_get_status", "sscan_status_string", "sscan_plan_describe", "sscan_version")
+           "sscan_get_status", "sscan_status_string", "sscan_plan_describe", "sscan_version",
+           "sscan_forward_noalloc")
 
 
 class SscanError(RuntimeError):
@@ -61,6 +62,8 @@ def lib() -> ctypes.CDLL:
             L.sscan_plan_describe.restype = ip
             L.sscan_version.argtypes = []
             L.sscan_version.restype = ip
+            L.sscan_forward_noalloc.argtypes = [i64, i64, i64, i64, ip, u32] + [vp] * 9
+            L.sscan_forward_noalloc.restype = ip
             _lib = L
     return _lib
 
