@@ -55,6 +55,32 @@ def load_peaks():
         return FALLBACK_HBM_GBS, SM_MAX_MHZ, "fallback"
 
 
+def kernel_sources_hash() -> str:
+    """sha256 over the CUDA sources, to tell whether a stored ncu figure is current."""
+    import hashlib
+    h = hashlib.sha256()
+    cdir = os.path.join(ROOT, "selective_state_space_32_b200", "csrc")
+    for name in sorted(os.listdir(cdir)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(cdir, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload: str):
+    """DRAM bytes (read + write) per launch of the dominant kernel from the committed
+    ncu capture (profiles/traffic.json), or None if absent or taken on other sources."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+        if t.get("kernel_sources_sha256") != kernel_sources_hash():
+            return None
+        v = t["workloads"][workload]["dram_bytes_per_launch"]
+        return float(v)
+    except Exception:
+        return None
+
+
 # ---------------------------------------------------------------- clocks --
 
 class ClockSampler:
@@ -254,13 +280,7 @@ def run_ours(args, rank, world, local_rank):
     hbm_achieved = alg_bytes / (kmean / 1e3) / 1e9
     upd_rate = w.updates / (kmean / 1e3) / 1e9
     alu_peak = ALU_UPDATES_PER_SM_CLK * SM_COUNT * sm_max * 1e6 / 1e9
-    traffic = None
-    try:
-        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            tr = json.load(f).get(args.workload)
-            traffic = tr if isinstance(tr, (int, float)) else None
-    except Exception:
-        pass
+    traffic = measured_traffic(args.workload)
     cpu_value, cores, sample = cpu_oracle_rate(g, w, args.cpu_seconds, 3 * args.cpu_seconds)
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -22,11 +22,12 @@
 // cooperatively, so all warps are resident, and a warp only waits for a head
 // that its predecessor runs before anything else) and is bounded anyway.
 //
-// Pipeline.  Each warp owns a ring of STAGES shared-memory stages of T tokens:
-// u and delta tiles [T][CPW] and B, C tiles [T][N], loaded by lane 0 with 2-D
-// TMA (no multicast) on an mbarrier; once the whole warp is past a stage
-// (__syncwarp plus an async-proxy fence), lane 0 refills its slot.  The compute
-// loop therefore only reads shared memory.  bf16 B/C tiles are widened once per stage by the warp.
+// Pipeline.  Each consumer warp owns a ring of STAGES shared-memory stages of T
+// tokens: u and delta tiles [T][CPW] and B, C tiles [T][N].  A producer warp per
+// block loads them with 2-D TMA (no multicast) on a "full" mbarrier per slot and
+// refills a slot after its consumer releases it on an "empty" mbarrier, so the
+// (slow) TMA issue never stalls a consumer and the compute loop only reads
+// shared memory.  bf16 B/C tiles are widened once per stage by the warp.
 //
 // Arithmetic per state update: Abar = 2^(delta*A*log2 e) on the MUFU pipe, or
 // for a quarter of the states on the FMA pipe (exp2_fma_pair) to balance the
@@ -74,9 +75,10 @@ struct ChainedCfg {
     static constexpr int kB = T * N * ES;                   // one B or C tile
     static constexpr int kStage = 2 * kU + 2 * kB;          // TMA bytes per stage
     static constexpr int kConv = ES == 2 ? 2 * T * N * 4 : 0;  // widened B, C (bf16 I/O)
-    static constexpr int kBar = STAGES * 8;
-    static constexpr int kWarp = ((STAGES * kStage + kConv + kBar) + 127) / 128 * 128;
-    static constexpr int kSmem = WPC * kWarp;
+    static constexpr int kWarp = ((STAGES * kStage + kConv) + 127) / 128 * 128;
+    static constexpr int kBars = (2 * WPC * STAGES * 8 + 127) / 128 * 128;  // full + empty per slot
+    static constexpr int kSmem = WPC * kWarp + kBars;
+    static constexpr int kThreads = (WPC + 1) * 32;  // WPC consumer warps + 1 producer warp
     static_assert(LPC >= 1 && LPC <= 8 && N % NL == 0 && NL % 4 == 0, "bad split");
     static_assert(CPW * ES % 16 == 0 && N * ES % 16 == 0, "TMA rows must be 16-byte multiples");
     static_assert(kU % 128 == 0 && kB % 128 == 0, "tile alignment");
@@ -164,6 +166,48 @@ __device__ __forceinline__ int reduce_scatter(float (&v)[G], int g) {
     }
     return base;
 }
+
+// The chain-steps [q0, q1) of one warp's segment, as parts: [head of the last
+// chain] [whole chains] [tail of the first chain], in that order of processing.
+struct Segment {
+    int64_t c_first, t_first, c_last, t_last, f_lo, n_full, n_parts;
+    int n_head;
+    bool single;
+    __device__ __forceinline__ Segment(int64_t wk, const ChainedParams &P) {
+        const int64_t L = P.L, Q = P.chains * L;
+        const int64_t q0 = wk * P.seg;
+        if (q0 >= Q) {
+            n_parts = 0;
+            c_first = t_first = c_last = t_last = f_lo = n_full = 0;
+            n_head = 0;
+            single = true;
+            return;
+        }
+        const int64_t q1 = q0 + P.seg < Q ? q0 + P.seg : Q;
+        c_first = q0 / L;
+        t_first = q0 - c_first * L;
+        c_last = (q1 - 1) / L;
+        t_last = q1 - c_last * L;  // in [1, L]
+        single = c_first == c_last;
+        n_head = (!single && t_last < L) ? 1 : 0;
+        const int n_tail = (!single && t_first > 0) ? 1 : 0;
+        f_lo = t_first == 0 ? c_first : c_first + 1;
+        const int64_t f_hi = t_last == L ? c_last : c_last - 1;
+        n_full = single ? 0 : (f_hi >= f_lo ? f_hi - f_lo + 1 : 0);
+        n_parts = single ? 1 : n_head + n_full + n_tail;
+    }
+    __device__ __forceinline__ void part(int64_t k, int64_t L, int64_t &c, int64_t &ts, int64_t &te) const {
+        if (single) {
+            c = c_first; ts = t_first; te = t_last;
+        } else if (k < n_head) {
+            c = c_last; ts = 0; te = t_last;
+        } else if (k < n_head + n_full) {
+            c = f_lo + (k - n_head); ts = 0; te = L;
+        } else {
+            c = c_first; ts = t_first; te = L;
+        }
+    }
+};
 
 // Split mode, second phase for one piece [ts, te) of chain c (ts > 0) that was
 // scanned from a zero state.  Its carried-in state is the inclusive state of
@@ -318,8 +362,79 @@ __device__ __noinline__ void split_fixup(const ChainedParams &P, int64_t c, int6
     }
 }
 
+// The producer: the block's last warp keeps every consumer warp's ring filled,
+// lane i serving consumer warp i, all lanes in lockstep so that one TMA
+// instruction issues the loads of every consumer that has a free slot (issuing
+// a TMA load costs the issuing warp on the order of a hundred cycles).
+// Consumer i's stages are loaded in its processing order (the same Segment walk
+// the consumer does) into slot r % STAGES once the consumer has released the
+// stage that used the slot before.  No lane ever blocks on one consumer (a
+// consumer may be waiting for another warp's carry): each lane tests its
+// consumer's barrier, and the warp backs off briefly when no lane could issue.
+template <class IO, class Cfg>
+__device__ __forceinline__ void produce(const CUtensorMap *tm_u, const CUtensorMap *tm_d, const CUtensorMap *tm_b,
+                                        const CUtensorMap *tm_c, const ChainedParams &P, unsigned char *smem,
+                                        uint64_t *full, uint64_t *empty, int lane) {
+    constexpr int WPC = Cfg::WPC, T = Cfg::T, STAGES = Cfg::STAGES, CPW = Cfg::CPW;
+    if (lane == 0) {
+        tma_prefetch_desc(tm_u);
+        tma_prefetch_desc(tm_d);
+        tma_prefetch_desc(tm_b);
+        tma_prefetch_desc(tm_c);
+    }
+    const int64_t L = P.L;
+    const int i = lane;  // the consumer this lane serves
+    const Segment sg(static_cast<int64_t>(blockIdx.x) * WPC + (i < WPC ? i : 0), P);
+    int64_t k = (i < WPC && sg.n_parts > 0) ? 0 : -1;
+    int64_t te = 0, t = 0, r = 0;
+    int x = 0, row = 0;
+    auto begin_part = [&]() {
+        int64_t c, ts;
+        sg.part(k, L, c, ts, te);
+        t = ts;
+        const int64_t b = c / P.chains_per_row;
+        x = static_cast<int>((c - b * P.chains_per_row) * CPW);
+        row = static_cast<int>(b * L);
+    };
+    if (k >= 0) begin_part();
+    unsigned char *ring = smem + (i < WPC ? i : 0) * Cfg::kWarp;
+    uint32_t idle = 0;
+    while (__any_sync(0xffffffffu, k >= 0)) {
+        const int s = static_cast<int>(r % STAGES);
+        const bool ready = k >= 0 && (r < STAGES || mbar_test_wait(&empty[i * STAGES + s],
+                                                                   static_cast<uint32_t>((r / STAGES - 1) & 1)));
+        if (ready) {
+            unsigned char *slot = ring + s * Cfg::kStage;
+            uint64_t *bar = &full[i * STAGES + s];
+            const int yrow = row + static_cast<int>(t);
+            mbar_expect_tx(bar, Cfg::kStage);
+            tma_load_2d(slot, tm_u, x, yrow, bar);
+            tma_load_2d(slot + Cfg::kU, tm_d, x, yrow, bar);
+            tma_load_2d(slot + 2 * Cfg::kU, tm_b, 0, yrow, bar);
+            tma_load_2d(slot + 2 * Cfg::kU + Cfg::kB, tm_c, 0, yrow, bar);
+            ++r;
+            t += T;
+            if (t >= te) {
+                if (++k < sg.n_parts)
+                    begin_part();
+                else
+                    k = -1;
+            }
+        }
+        if (__any_sync(0xffffffffu, ready)) {
+            idle = 0;
+        } else {
+            if (++idle > (kSpinLimit << 2)) {  // consumers stopped releasing slots
+                if (lane == 0) atomicOr(P.status, 4);
+                return;
+            }
+            __nanosleep(64);
+        }
+    }
+}
+
 template <class IO, class Cfg, bool ZOH, bool POLY, bool SPLIT>
-__global__ void __launch_bounds__(Cfg::WPC * 32, 1)
+__global__ void __launch_bounds__(Cfg::kThreads, 1)
 sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_d,
                      const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
                      const ChainedParams P) {
@@ -327,39 +442,28 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
     constexpr int LPC = Cfg::LPC, CPW = Cfg::CPW, NP = Cfg::NP;
     extern __shared__ __align__(128) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::WPC * Cfg::kWarp);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2 * Cfg::WPC * STAGES; ++i) mbar_init(&bars[i], 1);
+        mbar_fence_init();
+    }
+    __syncthreads();  // the only block-wide barrier
+    if (warp == Cfg::WPC) {
+        produce<IO, Cfg>(&tm_u, &tm_d, &tm_b, &tm_c, P, smem, bars, bars + Cfg::WPC * STAGES, lane);
+        return;
+    }
     unsigned char *wbase = smem + warp * Cfg::kWarp;
     float *convB = reinterpret_cast<float *>(wbase + STAGES * Cfg::kStage);
     float *convC = convB + T * N;
-    uint64_t *full = reinterpret_cast<uint64_t *>(wbase + STAGES * Cfg::kStage + Cfg::kConv);
+    uint64_t *full = bars + warp * STAGES;
+    uint64_t *empty = bars + (Cfg::WPC + warp) * STAGES;
 
     const int64_t L = P.L, D = P.D;
-    const int64_t Q = P.chains * L;
     const int64_t wk = static_cast<int64_t>(blockIdx.x) * Cfg::WPC + warp;  // this warp's segment
-    const int64_t q0 = wk * P.seg;
-    if (q0 >= Q) return;  // this warp has no work (whole warp leaves; no block barrier follows)
-    const int64_t q1 = q0 + P.seg < Q ? q0 + P.seg : Q;
-
-    // ---- this warp's parts: [head of the last chain] [whole chains] [tail of the first chain]
-    const int64_t c_first = q0 / L, t_first = q0 - c_first * L;
-    const int64_t c_last = (q1 - 1) / L, t_last = q1 - c_last * L;  // t_last in [1, L]
-    const bool single = c_first == c_last;
-    const int n_head = (!single && t_last < L) ? 1 : 0;
-    const int n_tail = (!single && t_first > 0) ? 1 : 0;
-    const int64_t f_lo = t_first == 0 ? c_first : c_first + 1;
-    const int64_t f_hi = t_last == L ? c_last : c_last - 1;
-    const int64_t n_full = single ? 0 : (f_hi >= f_lo ? f_hi - f_lo + 1 : 0);
-    const int64_t n_parts = single ? 1 : n_head + n_full + n_tail;
-    auto part = [&](int64_t k, int64_t &c, int64_t &ts, int64_t &te) {
-        if (single) {
-            c = c_first; ts = t_first; te = t_last;
-        } else if (k < n_head) {
-            c = c_last; ts = 0; te = t_last;
-        } else if (k < n_head + n_full) {
-            c = f_lo + (k - n_head); ts = 0; te = L;
-        } else {
-            c = c_first; ts = t_first; te = L;
-        }
-    };
+    const Segment seg(wk, P);
+    if (seg.n_parts == 0) return;  // this warp has no work
+    const int64_t n_parts = seg.n_parts;
+    auto part = [&](int64_t k, int64_t &c, int64_t &ts, int64_t &te) { seg.part(k, L, c, ts, te); };
 
     auto tile_u = [&](int s) { return reinterpret_cast<IO *>(wbase + s * Cfg::kStage); };
     auto tile_d = [&](int s) { return reinterpret_cast<IO *>(wbase + s * Cfg::kStage + Cfg::kU); };
@@ -367,52 +471,6 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
     auto tile_c = [&](int s) {
         return reinterpret_cast<IO *>(wbase + s * Cfg::kStage + 2 * Cfg::kU + Cfg::kB);
     };
-
-    if (lane == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
-        }
-        mbar_fence_init();
-        tma_prefetch_desc(&tm_u);
-        tma_prefetch_desc(&tm_d);
-        tma_prefetch_desc(&tm_b);
-        tma_prefetch_desc(&tm_c);
-    }
-    __syncwarp();
-
-    // ---- producer cursor (lane 0 only): which stage to load next
-    int64_t pk = 0, pc = 0, pts = 0, pte = 0, pt = 0;
-    int64_t issued = 0;
-    bool p_done = false;
-    int px = 0, prow = 0;  // TMA coordinates of the cursor's chain: channel, row of t = 0
-    auto p_begin_part = [&]() {
-        if (pk >= n_parts) { p_done = true; return; }
-        part(pk, pc, pts, pte);
-        pt = pts;
-        const int64_t b = pc / P.chains_per_row;
-        px = static_cast<int>((pc - b * P.chains_per_row) * CPW);
-        prow = static_cast<int>(b * L);
-    };
-    auto p_issue = [&]() {  // load the stage at the cursor into slot issued % STAGES, advance
-        const int s = static_cast<int>(issued % STAGES);
-        const int x = px;
-        const int yrow = prow + static_cast<int>(pt);
-        mbar_expect_tx(&full[s], Cfg::kStage);
-        tma_load_2d(tile_u(s), &tm_u, x, yrow, &full[s]);
-        tma_load_2d(tile_d(s), &tm_d, x, yrow, &full[s]);
-        tma_load_2d(tile_b(s), &tm_b, 0, yrow, &full[s]);
-        tma_load_2d(tile_c(s), &tm_c, 0, yrow, &full[s]);
-        ++issued;
-        pt += T;
-        if (pt >= pte) {
-            ++pk;
-            p_begin_part();
-        }
-    };
-    if (lane == 0) {
-        p_begin_part();
-        for (int s = 0; s < STAGES && !p_done; ++s) p_issue();
-    }
 
     const int cl = lane / LPC;   // channel within the chain
     const int g = lane % LPC;    // state group
@@ -628,14 +686,9 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
                 if (valid && g == 0) Io<IO>::st(yp + j * D, yv);
             }
             if (SPLIT) dsum += static_cast<double>(ssum);
-            // Every lane of this warp is done reading the slot (the warp that consumes a
-            // slot is the one that refills it): order those shared-memory reads before
-            // the TMA write that reuses the slot, then load the stage STAGES ahead.
+            // every lane is done reading the slot: release it to the producer
             __syncwarp();
-            if (lane == 0 && !p_done) {
-                fence_proxy_async_smem();
-                p_issue();
-            }
+            if (lane == 0) mbar_arrive(&empty[s]);
             ++consumed;
         }
         if (failed) break;
@@ -702,9 +755,10 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
         }
     }
     if (failed) {
-        // drain loads still in flight into this warp's ring before leaving (bounded)
+        // drain loads that may still be in flight into this warp's ring (the producer
+        // refills only released slots, so at most STAGES) before leaving; bounded
         if (lane == 0)
-            for (int64_t i = consumed; i < issued; ++i)
+            for (int64_t i = consumed; i < consumed + STAGES; ++i)
                 mbar_wait(&full[i % STAGES], static_cast<uint32_t>((i / STAGES) & 1));
         __syncwarp();
     }

@@ -52,14 +52,19 @@ struct KCfg {
 // Measured on B200: the MUFU pipe saturates from 2 warps per SM sub-partition
 // at 8 states per lane and from ~4 at 4 states per lane.
 constexpr KCfg kChainedCfgs[] = {
-    {16, 8, 32, 4, 8},   // 16 channels per warp, 2 warps per SM sub-partition (bf16 only: smem)
-    {16, 4, 16, 4, 12},  // 8 channels per warp, 3 warps per sub-partition
-    {16, 4, 16, 4, 8},   // 8 channels per warp, 2 warps per sub-partition
-    {16, 8, 32, 4, 4},   // 16 channels per warp, 1 warp per sub-partition
-    {16, 4, 16, 4, 4},   // 8 channels per warp, 1 warp per sub-partition
-    {32, 8, 32, 4, 4},   // 8 channels per warp
-    {64, 16, 16, 3, 8},  // 8 channels per warp, 2 warps per sub-partition
+    {16, 8, 32, 4, 8},   // 0: 16 channels per warp, 2 warps per SM sub-partition (bf16 only: smem)
+    {16, 4, 16, 4, 12},  // 1: 8 channels per warp, 3 warps per sub-partition
+    {16, 4, 16, 4, 8},   // 2: 8 channels per warp, 2 warps per sub-partition
+    {16, 8, 32, 4, 4},   // 3: 16 channels per warp, 1 warp per sub-partition
+    {16, 4, 16, 4, 4},   // 4: 8 channels per warp, 1 warp per sub-partition
+    {32, 8, 32, 4, 4},   // 5: 8 channels per warp
+    {64, 16, 16, 3, 8},  // 6: 8 channels per warp, 2 warps per sub-partition
 };
+// Order in which the shapes are tried (measured on B200: for N = 16, fp32 I/O
+// runs fastest at 8 states per lane and one consumer warp per sub-partition,
+// bf16 I/O at 4 states per lane and two).
+constexpr int kPrefF32[] = {3, 2, 1, 4, 5, 6, 0};
+constexpr int kPrefBF16[] = {0, 2, 3, 1, 4, 5, 6};
 constexpr int kNumCfgs = sizeof(kChainedCfgs) / sizeof(kChainedCfgs[0]);
 
 std::atomic<uint32_t> g_epoch{1};  // launch tags of the chained kernel (unique per process)
@@ -70,9 +75,10 @@ constexpr int kMaxSmem = 227 * 1024;  // dynamic shared memory per block on B200
 int chained_smem_bytes(const KCfg &k, int es) {
     const int lpc = k.N / k.NL, cpw = 32 / lpc;
     const int kU = k.T * cpw * es, kB = k.T * k.N * es;
-    const int stage = 2 * kU + 2 * kB, conv = es == 2 ? 2 * k.T * k.N * 4 : 0, bar = k.STAGES * 8;
-    const int warp = (k.STAGES * stage + conv + bar + 127) / 128 * 128;
-    return k.WPC * warp;
+    const int stage = 2 * kU + 2 * kB, conv = es == 2 ? 2 * k.T * k.N * 4 : 0;
+    const int warp = (k.STAGES * stage + conv + 127) / 128 * 128;
+    const int bars = (2 * k.WPC * k.STAGES * 8 + 127) / 128 * 128;
+    return k.WPC * warp + bars;
 }
 
 }  // namespace
@@ -163,7 +169,8 @@ void choose_schedule(sscan_plan *p) {
     // 1) chained: enough chains that each is cut at most once (segment >= L)
     // 2) split: fewer chains than warps; cut them into pieces scanned concurrently
     for (int pass = force_split ? 1 : 0; pass < 2; ++pass) {
-        for (int i = 0; i < kNumCfgs; ++i) {
+        for (int oi = 0; oi < kNumCfgs; ++oi) {
+            const int i = es == 4 ? kPrefF32[oi] : kPrefBF16[oi];
             const KCfg &k = kChainedCfgs[i];
             if (k.N != p->N) continue;
             if (want >= 0 && want != i) continue;
@@ -310,7 +317,7 @@ int launch_chained_t(sscan_plan *p, const void *u, const void *dl, const float *
     prm.chains = p->chains;
     prm.seg = p->seg;
     void *args[] = {&p->tm[0], &p->tm[1], &p->tm[2], &p->tm[3], &prm};
-    const dim3 grid(static_cast<unsigned>(p->workers / k.WPC)), block(k.WPC * 32);
+    const dim3 grid(static_cast<unsigned>(p->workers / k.WPC)), block(Cfg::kThreads);
     const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kern), grid, block, args,
                                                       Cfg::kSmem, s);
     return e == cudaSuccess ? SSCAN_OK : SSCAN_ERR_CUDA;

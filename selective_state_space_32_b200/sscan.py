@@ -183,19 +183,44 @@ def forward(u, delta, A, B, C, h0=None, zoh: bool = False, want_final: bool = Tr
                                                         want_final=want_final)
 
 
-def forward_host(u, delta, A, B, C, h0=None, zoh: bool = False, device="cuda", out=None):
+def forward_host(u, delta, A, B, C, h0=None, zoh: bool = False, device="cuda", out=None,
+                 chunks: int = 4):
     """Forward on host (CPU) tensors: copies the inputs to the device, runs the scan
-    and copies y and h_final back, then waits for the copies.  Pinned host tensors
-    give asynchronous copies; ``out`` = (y_host, h_final_host) reuses output buffers.
+    and copies y and h_final back, then waits for the copies.
+
+    Batch rows are independent, so the batch is cut into ``chunks`` pieces that
+    flow through two streams: a piece's host-to-device copy overlaps the previous
+    piece's scan and device-to-host copy (the transfer, not the scan, bounds this
+    path).  Pinned host tensors are needed for the copies to be asynchronous;
+    ``out`` = (y_host, h_final_host) reuses output buffers.
     Returns (y_host, h_final_host)."""
     dev = torch.device(device)
-    dv = [None if t is None else t.to(dev, non_blocking=True) for t in (u, delta, A, B, C, h0)]
-    y, hf = forward(*dv[:5], h0=dv[5], zoh=zoh)
+    Bt, L, D = u.shape
+    N = A.shape[1]
     if out is None:
         pin = u.is_pinned()
-        out = (torch.empty(y.shape, dtype=y.dtype, pin_memory=pin),
-               torch.empty(hf.shape, dtype=hf.dtype, pin_memory=pin))
-    out[0].copy_(y, non_blocking=True)
-    out[1].copy_(hf, non_blocking=True)
-    torch.cuda.current_stream(dev).synchronize()
+        out = (torch.empty((Bt, L, D), dtype=u.dtype, pin_memory=pin),
+               torch.empty((Bt, D, N), dtype=torch.float32, pin_memory=pin))
+    n = max(1, min(int(chunks), Bt))
+    bounds = [Bt * i // n for i in range(n + 1)]
+    main = torch.cuda.current_stream(dev)
+    streams = [torch.cuda.Stream(dev) for _ in range(min(2, n))]
+    A_d = A.to(dev, non_blocking=True)
+    for st in streams:
+        st.wait_stream(main)
+    for i in range(n):
+        b0, b1 = bounds[i], bounds[i + 1]
+        st = streams[i % len(streams)]
+        with torch.cuda.stream(st):
+            dv = [None if t is None else t[b0:b1].to(dev, non_blocking=True)
+                  for t in (u, delta, B, C, h0)]
+            plan = get_plan(b1 - b0, L, D, N, u.dtype, zoh)
+            y, hf = plan.forward(dv[0], dv[1], A_d, dv[2], dv[3], dv[4], stream=st)
+            out[0][b0:b1].copy_(y, non_blocking=True)
+            out[1][b0:b1].copy_(hf, non_blocking=True)
+            for t in (*dv, y, hf):  # keep the caching allocator from reusing them early
+                if t is not None:
+                    t.record_stream(st)
+    for st in streams:
+        st.synchronize()
     return out

@@ -171,6 +171,21 @@ def test_split_call_resume_matches_one_call():
     assert torch.allclose(torch.cat([y1, y2], 1), y, rtol=1e-5, atol=1e-6)
 
 
+def test_forward_host_chunked_matches_device_path():
+    g = W.generate(6, 300, 256, 16, "bf16", 0.1, seed=9)
+    d = P.to_device(g)
+    y_dev, hf_dev = S.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"])
+    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in d.items()}
+    for chunks in (1, 4):
+        y_h, hf_h = S.forward_host(host["u"], host["delta"], host["A"], host["B"], host["C"],
+                                   host["h0"], chunks=chunks)
+        assert y_h.dtype == torch.bfloat16 and not y_h.is_cuda
+        yr, hr = P.run_oracle(g)
+        P.check(y_h.float().numpy(), yr, "bf16", f"y host chunks={chunks}")
+        P.check(hf_h.numpy(), hr, "bf16", f"h_final host chunks={chunks}")
+        assert torch.allclose(hf_h, hf_dev.cpu(), rtol=1e-5, atol=1e-6)
+
+
 def test_h_final_may_alias_h0():
     g = W.generate(1, 100, 64, 16, "f32", 0.1, seed=7)
     d = P.to_device(g)
