@@ -71,21 +71,19 @@ __device__ __forceinline__ f2 exp2_fma_pair(f2 dd, f2 a) {
     return pack2(__uint_as_float(r0), __uint_as_float(r1));
 }
 
-// phi(z) = (exp(z) - 1) / z = sum_k z^k / (k+1)!, truncated after z^7; for
-// |z| <= 1/2 the first omitted term is below 1.1e-8 relative.  Coefficients
-// are the Taylor series 1/(k+1)!, highest first.
+// phi(z) = (exp(z) - 1) / z for |z| <= 1/4: degree-4 polynomial fitted for
+// minimax relative error (csrc/gen_phi_poly.py; 1.5e-7 max relative error in
+// fp32), constant term exactly 1 so that phi(0) = 1.
 __device__ __forceinline__ f2 phi2(f2 z) {
-    f2 q = fma2(splat2(1.0f / 40320.0f), z, splat2(1.0f / 5040.0f));
-    q = fma2(q, z, splat2(1.0f / 720.0f));
-    q = fma2(q, z, splat2(1.0f / 120.0f));
-    q = fma2(q, z, splat2(1.0f / 24.0f));
-    q = fma2(q, z, splat2(1.0f / 6.0f));
-    q = fma2(q, z, splat2(0.5f));
+    f2 q = fma2(splat2(8.333330042660236e-03f), z, splat2(4.177515208721161e-02f));
+    q = fma2(q, z, splat2(1.666673868894577e-01f));
+    q = fma2(q, z, splat2(4.999983012676239e-01f));
     return fma2(q, z, splat2(1.0f));
 }
 
 // Exact ZOH coefficient (exp(z) - 1) / A for a pair, z = d*A: d*phi(z) when
-// |z| <= 1/2 (also exact at A = 0), (abar - 1) * (1/A) otherwise.
+// |z| <= 1/4 (also exact at A = 0), (abar - 1) * (1/A) otherwise (there
+// |abar - 1| >= 0.22, so the 2^-22 relative error of abar stays below ~1.1e-6).
 __device__ __forceinline__ f2 zoh_coef_pair(f2 dd, f2 a1, f2 ia, f2 abar) {
     const f2 z = mul2(dd, a1);
     const f2 small = mul2(dd, phi2(z));
@@ -94,7 +92,7 @@ __device__ __forceinline__ f2 zoh_coef_pair(f2 dd, f2 a1, f2 ia, f2 abar) {
     unpack2(z, z0, z1);
     unpack2(small, s0, s1);
     unpack2(big, g0, g1);
-    return pack2(fabsf(z0) <= 0.5f ? s0 : g0, fabsf(z1) <= 0.5f ? s1 : g1);
+    return pack2(fabsf(z0) <= 0.25f ? s0 : g0, fabsf(z1) <= 0.25f ? s1 : g1);
 }
 
 // ------------------------------------------------------------- storage types

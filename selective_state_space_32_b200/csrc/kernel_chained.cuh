@@ -69,7 +69,7 @@ struct ChainedCfg {
     static constexpr int LPC = N / NL;      // lanes per channel
     static constexpr int CPW = 32 / LPC;    // channels per warp (chain width)
     static constexpr int NP = NL / 2;       // packed pairs per lane
-    static constexpr int G = NL >= 16 ? 2 : (NL >= 8 ? 4 : 8);  // tokens per discretize group
+    static constexpr int G = NL >= 16 ? 2 : 8;  // tokens per discretize group (measured best)
     static constexpr int ES = sizeof(IO);
     static constexpr int kU = T * CPW * ES;                 // one u or delta tile
     static constexpr int kB = T * N * ES;                   // one B or C tile
@@ -629,42 +629,7 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
                     for (int q = 0; q < KEEP; ++q) Io<IO>::st(yp + (j0 + base + q) * D, yv[q]);
                 }
             };
-            if (nsteps == T && NP <= 4) {
-                // A full stage as one straight-line block with a per-token software
-                // pipeline: token q+PD is discretized (MUFU exponents, independent of h)
-                // right before token q's state update, so in program order every burst
-                // of exponents sits next to FMA-pipe work that does not depend on it.
-                constexpr int PD = 2;  // pipeline distance in tokens
-                f2 ab[PD + 1][NP], bu[PD + 1][NP];
-                auto disc_tok = [&](int q, f2 (&a)[NP], f2 (&b2)[NP]) {
-                    const float x = Io<IO>::widen(us[q * CPW + cl]);
-                    const float dl = Io<IO>::widen(dsm[q * CPW + cl]);
-                    if (SPLIT) {
-                        ssum += dl;
-                        dmin = fminf(dmin, dl);
-                    }
-                    if (q & 1)
-                        discretize<NP, ZOH, POLY, 1>(a, b2, A2, A1, iA, cap, x, dl, Bs + q * N + n0);
-                    else
-                        discretize<NP, ZOH, POLY, 0>(a, b2, A2, A1, iA, cap, x, dl, Bs + q * N + n0);
-                };
-#pragma unroll
-                for (int q = 0; q < PD; ++q) disc_tok(q, ab[q], bu[q]);
-                float yv[G];
-#pragma unroll
-                for (int q = 0; q < T; ++q) {
-                    if (q + PD < T) disc_tok(q + PD, ab[(q + PD) % (PD + 1)], bu[(q + PD) % (PD + 1)]);
-                    yv[q % G] = advance<NP>(h, ab[q % (PD + 1)], bu[q % (PD + 1)], Cs + q * N + n0);
-                    if (q % G == G - 1) {
-                        const int base = reduce_scatter<LPC, G>(yv, g);
-                        if (g_store) {
-#pragma unroll
-                            for (int r = 0; r < KEEP; ++r) Io<IO>::st(yp + (q - (G - 1) + base + r) * D, yv[r]);
-                        }
-                    }
-                }
-                j = T;
-            } else if (nsteps == T) {
+            if (nsteps == T) {
 #pragma unroll
                 for (int j0 = 0; j0 < T; j0 += G) group(j0);
                 j = T;

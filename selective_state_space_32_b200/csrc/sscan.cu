@@ -60,11 +60,15 @@ constexpr KCfg kChainedCfgs[] = {
     {32, 8, 32, 4, 4},   // 5: 8 channels per warp
     {64, 16, 16, 3, 8},  // 6: 8 channels per warp, 2 warps per sub-partition
 };
-// Order in which the shapes are tried (measured on B200: for N = 16, fp32 I/O
-// runs fastest at 8 states per lane and one consumer warp per sub-partition,
-// bf16 I/O at 4 states per lane and two).
+// Order in which the shapes are tried (measured on B200: for N = 16 both I/O
+// types run fastest at 8 states per lane and one consumer warp per SM
+// sub-partition, then at 4 states per lane and two).
 constexpr int kPrefF32[] = {3, 2, 1, 4, 5, 6, 0};
-constexpr int kPrefBF16[] = {0, 2, 3, 1, 4, 5, 6};
+constexpr int kPrefBF16[] = {3, 0, 2, 1, 4, 5, 6};
+// The split mode can use any number of warps (pieces are independent until the
+// fix-up), so it prefers two consumer warps per sub-partition.
+constexpr int kPrefSplitF32[] = {2, 3, 1, 4, 5, 6, 0};
+constexpr int kPrefSplitBF16[] = {0, 2, 3, 1, 4, 5, 6};
 constexpr int kNumCfgs = sizeof(kChainedCfgs) / sizeof(kChainedCfgs[0]);
 
 std::atomic<uint32_t> g_epoch{1};  // launch tags of the chained kernel (unique per process)
@@ -170,7 +174,8 @@ void choose_schedule(sscan_plan *p) {
     // 2) split: fewer chains than warps; cut them into pieces scanned concurrently
     for (int pass = force_split ? 1 : 0; pass < 2; ++pass) {
         for (int oi = 0; oi < kNumCfgs; ++oi) {
-            const int i = es == 4 ? kPrefF32[oi] : kPrefBF16[oi];
+            const int i = pass == 0 ? (es == 4 ? kPrefF32[oi] : kPrefBF16[oi])
+                                    : (es == 4 ? kPrefSplitF32[oi] : kPrefSplitBF16[oi]);
             const KCfg &k = kChainedCfgs[i];
             if (k.N != p->N) continue;
             if (want >= 0 && want != i) continue;

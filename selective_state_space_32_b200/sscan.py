@@ -184,7 +184,7 @@ def forward(u, delta, A, B, C, h0=None, zoh: bool = False, want_final: bool = Tr
 
 
 def forward_host(u, delta, A, B, C, h0=None, zoh: bool = False, device="cuda", out=None,
-                 chunks: int = 4):
+                 chunks: int = 2):
     """Forward on host (CPU) tensors: copies the inputs to the device, runs the scan
     and copies y and h_final back, then waits for the copies.
 
