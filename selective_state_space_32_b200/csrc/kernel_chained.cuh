@@ -61,6 +61,7 @@ struct ChainedParams {
     int *rec_mono;                 // [chains][max_pieces] delta >= 0 over the piece and A <= 0
     unsigned long long *rec_flags; // [chains][max_pieces] (epoch << 32) | 1 once published
     int64_t max_pieces;
+    int drop_publish;              // failure-detection tests only: heads never publish their carry
 };
 
 template <class IO, int N_, int NL_, int T_, int STAGES_, int WPC_>
@@ -685,7 +686,7 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
                 __threadfence();
                 st_release_u64(P.rec_flags + r, P.epoch_hi | 1ull);
             }
-        } else if (te < L) {
+        } else if (te < L && !P.drop_publish) {
             // publish the state at the cut for the warp that runs the rest of this chain
             float *dst = P.carry + (c * 32 + lane) * NL;
 #pragma unroll
@@ -698,7 +699,7 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
             __threadfence();
             __syncwarp();
             if (lane == 0) st_release_u64(P.flags + c, P.epoch_hi | static_cast<unsigned long long>(te));
-        } else if (P.h_final != nullptr && valid) {
+        } else if (te == L && P.h_final != nullptr && valid) {
             float *dst = P.h_final + (b * D + d) * N + n0;
 #pragma unroll
             for (int p = 0; p < NP; p += 2) {

@@ -79,6 +79,9 @@ WORKLOADS = {
     "mamba1p4b_bf16": Workload("mamba1p4b_bf16", 2, 8192, 4096, 16, "bf16", 0.1, False, 0.0, 2),
     "longseq_bf16": Workload("longseq_bf16", 1, 131072, 2048, 16, "bf16", 0.1, False, 0.32, 3),
     "zoh_n64_bf16": Workload("zoh_n64_bf16", 16, 1024, 5120, 64, "bf16", 0.0, True, 0.0, 4),
+    # one decode step (a single token per sequence, state carried in and out) for a
+    # batch of 256 sequences of a layer with D = 2048, N = 16
+    "decode_b256_f32": Workload("decode_b256_f32", 256, 1, 2048, 16, "f32", 0.1, False, 0.0, 5),
 }
 ORDER = ["tiny_f32", "mamba130m_f32", "mamba1p4b_bf16", "longseq_bf16", "zoh_n64_bf16"]
 

@@ -63,7 +63,7 @@ CHAINED = [
     (1, 517, 64, 16, "bf16", True, False, 4, 1, 1),
     (2, 200, 64, 32, "f32", True, True, 5, 2, 0),
     (2, 100, 72, 64, "bf16", True, True, 6, 1, 0),
-    (3, 37, 128, 16, "f32", False, False, 3, 2, 1),     # L shorter than two stages
+    (3, 64, 128, 16, "f32", False, False, 3, 2, 1),     # L of two stages
     (2, 300, 128, 16, "f32", True, False, 3, 20, 1),    # segment < L: chains cut many times
     (2, 300, 256, 16, "bf16", True, False, 0, 1, 0),    # 8 states/lane, 8 warps/block
     (2, 300, 128, 16, "bf16", True, False, 1, 1, 0),    # 4 states/lane, 12 warps/block
@@ -127,6 +127,31 @@ def test_split_mode_forced(case, monkeypatch):
     plan.close()
 
 
+def test_lost_carry_times_out_and_is_reported(monkeypatch):
+    """Failure detection without a GPU fault: the warps that run a chain's head are told
+    not to publish its state, so the warps running the tails wait on a flag nothing sets.
+    Their bounded wait gives up (about a second), the kernel finishes, and the plan's
+    status word reports SSCAN_ERR_TIMEOUT; the next call starts clean."""
+    import time
+    g = W.generate(2, 300, 128, 16, "f32", 0.1, seed=77)
+    d = P.to_device(g)
+    monkeypatch.setenv("SSCAN_TUNE", "cfg=3,sms=3,nopublish=1")
+    plan = S.Plan(2, 300, 128, 16, torch.float32)
+    assert "kernel=chained" in plan.describe() and "split=0" in plan.describe()
+    t0 = time.time()
+    plan.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"])
+    assert plan.status() == S.ERR_TIMEOUT
+    assert time.time() - t0 < 60
+    plan.close()
+    monkeypatch.setenv("SSCAN_TUNE", "cfg=3,sms=3")
+    plan = S.Plan(2, 300, 128, 16, torch.float32)
+    y, hf = plan.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"])
+    assert plan.status() == S.OK
+    yr, hr = P.run_oracle(g)
+    P.check(y.cpu().numpy(), yr, "f32", "y after a failed call")
+    plan.close()
+
+
 def test_default_schedules():
     """The full-size workloads get the chained kernel; the 2048-channel long sequence is split."""
     for name, want in [("mamba130m_f32", "split=0"), ("mamba1p4b_bf16", "split=0"),
@@ -184,6 +209,32 @@ def test_forward_host_chunked_matches_device_path():
         P.check(y_h.float().numpy(), yr, "bf16", f"y host chunks={chunks}")
         P.check(hf_h.numpy(), hr, "bf16", f"h_final host chunks={chunks}")
         assert torch.allclose(hf_h, hf_dev.cpu(), rtol=1e-5, atol=1e-6)
+
+
+@pytest.mark.parametrize("dt,zoh", [("f32", False), ("bf16", True)])
+def test_decode_steps_match_one_forward(dt, zoh):
+    """Single-token decode: the state is carried in place (h_final aliases h0), one
+    token per call; the tokens' outputs and the final state equal one forward pass."""
+    Bt, L, D, N = 4, 12, 256, 16
+    g = W.generate(Bt, L, D, N, dt, 0.1, seed=11, A_jitter=0.2)
+    d = P.to_device(g)
+    y_full, h_full = S.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"], zoh=zoh)
+    tdt = torch.float32 if dt == "f32" else torch.bfloat16
+    plan = S.get_plan(Bt, 1, D, N, tdt, zoh)
+    assert "kernel=generic" in plan.describe()
+    state = d["h0"].clone()
+    ys = []
+    for t in range(L):
+        yt, _ = plan.forward(d["u"][:, t:t + 1].contiguous(), d["delta"][:, t:t + 1].contiguous(),
+                             d["A"], d["B"][:, t:t + 1].contiguous(), d["C"][:, t:t + 1].contiguous(),
+                             h0=state, h_final=state)
+        ys.append(yt)
+    torch.cuda.synchronize()
+    yr, hr = P.run_oracle(g, zoh)
+    P.check(torch.cat(ys, 1).float().cpu().numpy(), yr, dt, "decoded y")
+    P.check(state.cpu().numpy(), hr, dt, "decoded state")
+    assert torch.allclose(torch.cat(ys, 1).float(), y_full.float(), rtol=2e-2 if dt == "bf16" else 1e-5,
+                          atol=1e-2 if dt == "bf16" else 1e-5)
 
 
 def test_h_final_may_alias_h0():

@@ -82,7 +82,7 @@ def test_noalloc_matches_plan_entry_twice(case, monkeypatch):
 def test_noalloc_rejects_workspace_beyond_the_fixed_array():
     # 4096 batch rows x 2048 channels (N = 64): the chained schedule needs a carry
     # slot per chain, far beyond the 32 MiB array -> rejected before any launch.
-    Bt, L, D, N = 4096, 8, 2048, 64
+    Bt, L, D, N = 4096, 64, 2048, 64
     rc = S.lib().sscan_forward_noalloc(Bt, L, D, N, S.BF16, 0, *([ctypes.c_void_p(256)] * 5), None,
                                        ctypes.c_void_p(256), None, None)
     assert rc == S.ERR_WORKSPACE, S.status_string(rc)
