@@ -106,6 +106,7 @@ template <> struct Io<float> {
     // NP consecutive pairs (2*NP values) starting at a 16-byte aligned p
     template <int NP>
     static __device__ __forceinline__ void ld_pairs(const float *p, f2 (&out)[NP]) {
+        static_assert(NP % 2 == 0, "pairs are loaded 4 values at a time");
 #pragma unroll
         for (int i = 0; i < NP / 2; ++i) {
             const float4 v = __ldg(reinterpret_cast<const float4 *>(p) + i);
@@ -125,15 +126,24 @@ template <> struct Io<uint16_t> {  // bf16 bit patterns
         asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(v));
         *p = r;
     }
+    // NP consecutive pairs (2*NP bf16 values) starting at p (8-byte aligned for NP = 2,
+    // 16-byte aligned otherwise); each 32-bit word holds one pair
     template <int NP>
     static __device__ __forceinline__ void ld_pairs(const uint16_t *p, f2 (&out)[NP]) {
+        static_assert(NP == 2 || NP % 4 == 0, "pairs are loaded 2 or 4 words at a time");
+        if constexpr (NP == 2) {
+            const uint2 v = __ldg(reinterpret_cast<const uint2 *>(p));
+            out[0] = pack2(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u));
+            out[1] = pack2(__uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+        } else {
 #pragma unroll
-        for (int i = 0; i < NP / 4; ++i) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p) + i);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            for (int i = 0; i < NP / 4; ++i) {
+                const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p) + i);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j)  // low half = even state, high half = odd state
-                out[4 * i + j] = pack2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xffff0000u));
+                for (int j = 0; j < 4; ++j)  // low half = even state, high half = odd state
+                    out[4 * i + j] = pack2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xffff0000u));
+            }
         }
     }
 };

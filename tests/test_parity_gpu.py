@@ -95,6 +95,8 @@ SPLIT = [
     # (B, L, D, N, dtype, h0, zoh, reset_frac, blocks, negate): split mode forced on a small
     # grid: pieces scanned from zero, exact carry-in by look-back, bounded fix-up of y
     (1, 4096, 64, 16, "bf16", True, False, 0.32, 8, False),   # resets: short fix-up windows
+    (1, 4096, 64, 16, "bf16", True, False, 0.32, -8, False),  # same, 4 states per lane (cfg 2)
+    (2, 3000, 64, 16, "bf16", True, True, 0.0, -8, False),    # 4 states per lane, ZOH, long windows
     (1, 4096, 64, 16, "f32", True, False, 0.32, 8, False),
     (2, 3000, 64, 16, "f32", True, False, 0.0, 8, False),     # slow decay: long windows
     (1, 2050, 128, 16, "f32", True, True, 0.0, 6, False),     # exact ZOH, ragged pieces
@@ -114,7 +116,8 @@ def test_split_mode_forced(case, monkeypatch):
         v = W.as_f32(g["delta"], dt).copy()
         v[:, 100:103, :] *= -0.5
         g["delta"] = v if dt == "f32" else W.f32_to_bf16_bits(v)
-    monkeypatch.setenv("SSCAN_TUNE", f"split=1,sms={blocks}")
+    # negative blocks: force the 4-states-per-lane shape (cfg 2) on |blocks| blocks
+    monkeypatch.setenv("SSCAN_TUNE", f"split=1,sms={abs(blocks)}" + (",cfg=2" if blocks < 0 else ""))
     plan = S.Plan(Bt, L, D, N, torch.float32 if dt == "f32" else torch.bfloat16, zoh)
     desc = plan.describe()
     assert "kernel=chained" in desc and "split=1" in desc, desc
