@@ -93,7 +93,7 @@ class ClockSampler:
         "display_clock_setting": 0x100,
     }
 
-    def __init__(self, index: int, period_s: float = 0.005):
+    def __init__(self, index: int, period_s: float = 0.001):
         self.index, self.period = index, period_s
         self.samples, self.reasons = [], set()
         self.max_mhz = None
@@ -280,6 +280,9 @@ def run_ours(args, rank, world, local_rank):
     hbm_achieved = alg_bytes / (kmean / 1e3) / 1e9
     upd_rate = w.updates / (kmean / 1e3) / 1e9
     alu_peak = ALU_UPDATES_PER_SM_CLK * SM_COUNT * sm_max * 1e6 / 1e9
+    mufu_peak = 16.0 * SM_COUNT * sm_max * 1e6 / 1e9     # one exp2 per update, MUFU only
+    kernel_name = ("sscan_chained_kernel" if plan.describe().startswith("kernel=chained")
+                   else "sscan_generic_kernel")
     traffic = measured_traffic(args.workload)
     cpu_value, cores, sample = cpu_oracle_rate(g, w, args.cpu_seconds, 3 * args.cpu_seconds)
     out = {
@@ -294,9 +297,10 @@ def run_ours(args, rank, world, local_rank):
                          f"{L2_BYTES / 2**20:.0f} MiB L2); no flush"},
         "roofline": {"bound": "alu", "achieved": upd_rate, "peak": alu_peak,
                      "unit": "Gupdates/s", "frac": upd_rate / alu_peak, "traffic": traffic,
-                     "kernel": "sscan_fwd_kernel",
+                     "kernel": kernel_name, "schedule": plan.describe(),
                      "peak_basis": f"{ALU_UPDATES_PER_SM_CLK:.1f} state updates/SM/clk "
-                                   f"(16 MUFU + 128 FMA lanes) x {SM_COUNT} SMs x {sm_max:.0f} MHz"},
+                                   f"(16 MUFU + 128 FMA lanes) x {SM_COUNT} SMs x {sm_max:.0f} MHz",
+                     "mufu_only_peak": mufu_peak, "mufu_only_frac": upd_rate / mufu_peak},
         "hbm": {"achieved": hbm_achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": hbm_achieved / hbm_peak, "peak_source": peak_src,
                 "algorithmic_bytes_per_step": alg_bytes},

@@ -61,6 +61,7 @@ struct ChainedParams {
     int *rec_mono;                 // [chains][max_pieces] delta >= 0 over the piece and A <= 0
     unsigned long long *rec_flags; // [chains][max_pieces] (epoch << 32) | 1 once published
     int64_t max_pieces;
+    void *ysink;                   // [warps][32] 4-byte slots: y stores of lanes past the last channel
     int drop_publish;              // failure-detection tests only: heads never publish their carry
 };
 
@@ -596,7 +597,12 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
 
         double dsum = 0.0;      // split mode: sum of delta over the part (for prod Abar)
         float dmin = 3.0e38f;   // split mode: smallest delta of the part
-        IO *ybase = static_cast<IO *>(P.y) + b * L * D + d;
+        // Lanes past the last channel (d >= D) store into their own sink slot
+        // (stride 0) instead of skipping the store: the stores of a stage are then
+        // unconditional, which measured faster than a per-lane guard.
+        IO *ybase = valid ? static_cast<IO *>(P.y) + b * L * D + d
+                          : reinterpret_cast<IO *>(static_cast<float *>(P.ysink) + wk * 32 + lane);
+        const int64_t ystr = valid ? D : 0;
         for (int64_t t0 = ts; t0 < te; t0 += T) {
             const int s = static_cast<int>(consumed % STAGES);
             const uint32_t par = static_cast<uint32_t>((consumed / STAGES) & 1);
@@ -639,7 +645,7 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
                 Cs = convC;
             }
             const int nsteps = static_cast<int>(te - t0 < T ? te - t0 : T);
-            IO *yp = ybase + t0 * D;
+            IO *yp = ybase + t0 * ystr;
             int j = 0;
             float ssum = 0.0f;  // split mode: this stage's share of dsum
             // Groups of G tokens: discretize the whole group first (independent of h),
@@ -648,7 +654,7 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
             constexpr int G = Cfg::G;
             constexpr int GZ = Cfg::GZ;
             constexpr int KEEP = G / LPC > 0 ? G / LPC : 1;
-            const bool g_store = valid && (LPC <= G || (g & (LPC / G - 1)) == 0);
+            const bool g_store = LPC <= G || (g & (LPC / G - 1)) == 0;
             auto group_euler = [&](int j0) {
                 f2 ab[G][NP];
                 float duv[G];
@@ -673,13 +679,13 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
                 const int base = reduce_scatter<LPC, G>(yv, g);
                 if (g_store) {
 #pragma unroll
-                    for (int q = 0; q < KEEP; ++q) Io<IO>::st(yp + (j0 + base + q) * D, yv[q]);
+                    for (int q = 0; q < KEEP; ++q) Io<IO>::st(yp + (j0 + base + q) * ystr, yv[q]);
                 }
             };
             auto group = [&](int j0) {  // ZOH: Abar and the ZOH coefficient per token
                 constexpr int G = GZ;
                 constexpr int KEEP = G / LPC > 0 ? G / LPC : 1;
-                const bool g_store = valid && (LPC <= G || (g & (LPC / G - 1)) == 0);
+                const bool g_store = LPC <= G || (g & (LPC / G - 1)) == 0;
                 f2 ab[G][NP], bu[G][NP];
 #pragma unroll
                 for (int q = 0; q < G; ++q) {
@@ -700,7 +706,7 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
                 const int base = reduce_scatter<LPC, G>(yv, g);
                 if (g_store) {
 #pragma unroll
-                    for (int q = 0; q < KEEP; ++q) Io<IO>::st(yp + (j0 + base + q) * D, yv[q]);
+                    for (int q = 0; q < KEEP; ++q) Io<IO>::st(yp + (j0 + base + q) * ystr, yv[q]);
                 }
             };
             if (!ZOH) {
@@ -732,7 +738,7 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
                 float yv = advance<NP>(h, ab, bu, Cs + j * N + n0);
 #pragma unroll
                 for (int o = 1; o < LPC; o <<= 1) yv += __shfl_xor_sync(0xffffffffu, yv, o);
-                if (valid && g == 0) Io<IO>::st(yp + j * D, yv);
+                if (g == 0) Io<IO>::st(yp + j * ystr, yv);
             }
             if (SPLIT) dsum += static_cast<double>(ssum);
             // every lane is done reading the slot: release it to the producer

@@ -104,6 +104,7 @@ struct sscan_plan {
     int64_t chains_per_row, chains, workers, seg, max_pieces;
     size_t flag_off, flag_bytes;                // flags cleared on a workspace's first use
     size_t rec_s_off, rec_mono_off, ws_bytes;   // split-mode record arrays (rec_h at 0)
+    size_t sink_off;                            // y sink of lanes past the last channel
     const void *last_ws;  // workspace whose flags were last cleared
     // tensor-map cache
     const void *tm_ptr[4];
@@ -222,7 +223,8 @@ void choose_schedule(sscan_plan *p) {
                 p->flag_off = align_up(size_t(chains) * 32 * k.NL * sizeof(float), 256);
                 p->flag_bytes = size_t(chains) * sizeof(unsigned long long);
             }
-            p->ws_bytes = p->flag_off + align_up(p->flag_bytes, 256);
+            p->sink_off = p->flag_off + align_up(p->flag_bytes, 256);
+            p->ws_bytes = p->sink_off + align_up(size_t(workers) * 32 * sizeof(float), 256);
             return;
         }
     }
@@ -323,6 +325,7 @@ int launch_chained_t(sscan_plan *p, const void *u, const void *dl, const float *
     prm.rec_mono = reinterpret_cast<int *>(w + p->rec_mono_off);
     prm.rec_flags = flags;
     prm.max_pieces = p->max_pieces;
+    prm.ysink = w + p->sink_off;
     prm.drop_publish = p->drop_publish ? 1 : 0;
     prm.status = p->d_status;
     prm.epoch_hi = static_cast<unsigned long long>(ep) << 32;

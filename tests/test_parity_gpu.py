@@ -59,7 +59,10 @@ CHAINED = [
     # cfg indexes the library's shape table (see csrc/sscan.cu).
     (2, 300, 128, 16, "f32", True, False, 3, 3, 1),     # 8 states/lane, FMA-pipe exp on
     (2, 300, 128, 16, "f32", True, False, 3, 3, 0),
-    (2, 300, 136, 16, "f32", True, False, 2, 2, 0),     # 4 states/lane; ragged last chain
+    (2, 300, 136, 16, "f32", True, False, 2, 2, 0),     # 4 states/lane
+    (2, 300, 136, 16, "f32", True, False, 3, 2, 0),     # D % 16 != 0: last chain's upper lanes idle
+    (2, 300, 200, 16, "bf16", True, False, 0, 1, 0),    # the same with bf16 I/O, 8 warps/block
+    (2, 200, 68, 32, "f32", True, True, 5, 2, 0),       # ZOH, N = 32, D % 8 != 0
     (1, 517, 64, 16, "bf16", True, False, 4, 1, 1),
     (2, 200, 64, 32, "f32", True, True, 5, 2, 0),
     (2, 100, 72, 64, "bf16", True, True, 6, 1, 0),
@@ -102,6 +105,7 @@ SPLIT = [
     (1, 2050, 128, 16, "f32", True, True, 0.0, 6, False),     # exact ZOH, ragged pieces
     (1, 1500, 64, 16, "f32", True, False, 0.32, 4, True),     # some delta < 0: no early exit
     (2, 700, 72, 64, "bf16", True, True, 0.32, 4, False),     # N = 64 (32 warps > 18 chains)
+    (1, 3000, 68, 16, "f32", True, False, 0.32, 8, False),    # D % 8 != 0: idle upper lanes
 ]
 
 
