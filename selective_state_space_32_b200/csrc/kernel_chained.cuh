@@ -9,9 +9,11 @@
 // section 2), so a chain's steps must run in order; chains are independent.
 //
 // Schedule.  The B*ceil(D/CPW) chains are laid end to end (chain-major, then
-// time) and cut into W equal segments of S = ceil(chains*L / W) chain-steps,
-// one per warp of a persistent grid, so every warp does the same number of
-// state updates.  With S >= L a chain is cut at most once, between two
+// time) and cut into W segments of S = ceil(chains*L / W) chain-steps on
+// average, one per warp of a persistent grid, so every warp does the same
+// number of state updates (up to a small shift that evens out finishing times:
+// the warps sharing an SM sub-partition with the producer run S - 3x steps, the
+// others S + x).  With segments >= L a chain is cut at most once, between two
 // consecutive warps: the earlier warp runs the chain's head (from t = 0) FIRST
 // and publishes the state at the cut; the later warp runs its own head and
 // whole chains first and the chain's tail LAST, after reading that state.
@@ -52,7 +54,9 @@ struct ChainedParams {
     int64_t L, D;
     int64_t chains_per_row;        // ceil(D / CPW)
     int64_t chains;                // B * chains_per_row
-    int64_t seg;                   // chain-steps per warp (S)
+    int64_t seg;                   // chain-steps per warp (S), on average
+    int64_t seg_shift;             // x: warps j = 0 mod 4 of a block run S - 3x steps, the others S + x
+    int wpc;                       // consumer warps per block
     // split mode (chains cut into several pieces that are scanned concurrently)
     const void *delta;             // [B][L][D], read again by the fix-up
     const void *Cm;                // [B][L][N], read again by the fix-up
@@ -217,9 +221,15 @@ struct Segment {
     int64_t c_first, t_first, c_last, t_last, f_lo, n_full, n_parts;
     int n_head;
     bool single;
+    // First chain-step of warp w: w*S shifted by x per heavier warp before it in its
+    // block minus 3x per lighter one (a block's total stays WPC*S).
+    static __device__ __forceinline__ int64_t start(int64_t w, const ChainedParams &P) {
+        const int j = static_cast<int>(w % P.wpc);
+        return w * P.seg + P.seg_shift * (j - 4 * ((j + 3) / 4));
+    }
     __device__ __forceinline__ Segment(int64_t wk, const ChainedParams &P) {
         const int64_t L = P.L, Q = P.chains * L;
-        const int64_t q0 = wk * P.seg;
+        const int64_t q0 = start(wk, P);
         if (q0 >= Q) {
             n_parts = 0;
             c_first = t_first = c_last = t_last = f_lo = n_full = 0;
@@ -227,7 +237,8 @@ struct Segment {
             single = true;
             return;
         }
-        const int64_t q1 = q0 + P.seg < Q ? q0 + P.seg : Q;
+        const int64_t q1e = start(wk + 1, P);
+        const int64_t q1 = q1e < Q ? q1e : Q;
         c_first = q0 / L;
         t_first = q0 - c_first * L;
         c_last = (q1 - 1) / L;

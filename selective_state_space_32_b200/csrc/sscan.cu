@@ -74,6 +74,11 @@ constexpr int kNumCfgs = sizeof(kChainedCfgs) / sizeof(kChainedCfgs[0]);
 std::atomic<uint32_t> g_epoch{1};  // launch tags of the chained kernel (unique per process)
 
 constexpr int kMaxSmem = 227 * 1024;  // dynamic shared memory per block on B200
+// The consumer warps that share an SM sub-partition with the producer warp (warp
+// index a multiple of 4) ran ~4% slower than the other three on B200, and the
+// launch ends with its slowest warp; they get 3x fewer chain-steps and the others
+// x more, x = S * kLightPermille / 1000, which evens out the finishing times.
+constexpr int kLightPermille = 10;
 constexpr int64_t kMinChainedL = 64;  // shorter sequences use the generic kernel
 
 // Shared memory of a chained-kernel shape (mirrors ChainedCfg::kSmem).
@@ -102,6 +107,7 @@ struct sscan_plan {
     bool split;        // chains cut into concurrently scanned pieces + look-back fix-up
     bool drop_publish; // failure-detection tests: heads skip publishing (see read_tune)
     int64_t chains_per_row, chains, workers, seg, max_pieces;
+    int64_t seg_shift;  // segment re-balancing unit x (see ChainedParams::seg_shift)
     size_t flag_off, flag_bytes;                // flags cleared on a workspace's first use
     size_t rec_s_off, rec_mono_off, ws_bytes;   // split-mode record arrays (rec_h at 0)
     size_t sink_off;                            // y sink of lanes past the last channel
@@ -146,13 +152,16 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // many blocks, split=1 forces the split mode (tests use the last two to cut
 // chains on small problems), nopublish=1 makes the warps running a chain's
 // head skip publishing the carried state (failure-detection tests: the
-// bounded waits of the warps running the tails must give up and report it).
-void read_tune(int &cfg, int &poly, int &sms, int &split, int &nopublish) {
+// bounded waits of the warps running the tails must give up and report it),
+// light=<per mille> sets how much shorter the segments of the warps that share
+// an SM sub-partition with the producer warp are (see kLightPermille).
+void read_tune(int &cfg, int &poly, int &sms, int &split, int &nopublish, int &light) {
     cfg = -2;
     poly = -1;
     sms = 0;
     split = 0;
     nopublish = 0;
+    light = -1;
     const char *s = getenv("SSCAN_TUNE");
     if (!s) return;
     if (const char *c = strstr(s, "cfg=")) cfg = atoi(c + 4);
@@ -160,6 +169,7 @@ void read_tune(int &cfg, int &poly, int &sms, int &split, int &nopublish) {
     if (const char *c = strstr(s, "sms=")) sms = atoi(c + 4);
     if (const char *c = strstr(s, "split=")) split = atoi(c + 6);
     if (const char *c = strstr(s, "nopublish=")) nopublish = atoi(c + 10);
+    if (const char *c = strstr(s, "light=")) light = atoi(c + 6);
 }
 
 void choose_schedule(sscan_plan *p) {
@@ -167,8 +177,8 @@ void choose_schedule(sscan_plan *p) {
     p->mode = kGeneric;
     p->g_nl = p->N == 16 ? 8 : 16;
     p->g_lpc = static_cast<int>(p->N) / p->g_nl;
-    int want = -2, poly = -1, sms = 0, force_split = 0, nopublish = 0;
-    read_tune(want, poly, sms, force_split, nopublish);
+    int want = -2, poly = -1, sms = 0, force_split = 0, nopublish = 0, light = -1;
+    read_tune(want, poly, sms, force_split, nopublish, light);
     p->drop_publish = nopublish != 0;
     const int blocks = (sms > 0 && sms < p->sm_count) ? sms : p->sm_count;
     // the FMA-pipe exponent measured slower than MUFU alone at every occupancy: off unless asked
@@ -210,6 +220,8 @@ void choose_schedule(sscan_plan *p) {
             p->chains = chains;
             p->workers = workers;
             p->seg = ceil_div(chains * p->L, workers);
+            // split mode indexes pieces by equal segments; the chained mode balances time
+            p->seg_shift = p->split ? 0 : p->seg * (light >= 0 ? light : kLightPermille) / 1000;
             if (p->split) {
                 p->max_pieces = p->L / p->seg + 2;
                 const size_t recs = size_t(chains) * size_t(p->max_pieces);
@@ -334,6 +346,8 @@ int launch_chained_t(sscan_plan *p, const void *u, const void *dl, const float *
     prm.chains_per_row = p->chains_per_row;
     prm.chains = p->chains;
     prm.seg = p->seg;
+    prm.seg_shift = p->seg_shift;
+    prm.wpc = k.WPC;
     void *args[] = {&p->tm[0], &p->tm[1], &p->tm[2], &p->tm[3], &prm};
     const dim3 grid(static_cast<unsigned>(p->workers / k.WPC)), block(Cfg::kThreads);
     const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kern), grid, block, args,
@@ -480,13 +494,13 @@ int sscan_plan_describe(sscan_plan_t plan, char *buf, size_t len) {
         n = snprintf(tmp, sizeof tmp,
                      "kernel=chained B=%lld L=%lld D=%lld N=%lld dtype=%s zoh=%d states_per_thread=%d "
                      "threads_per_channel=%d channels_per_warp=%d warps_per_block=%d tokens_per_stage=%d "
-                     "stages=%d fma_pipe_exp=%d split=%d chains=%lld warps=%lld segment=%lld workspace=%zu "
+                     "stages=%d fma_pipe_exp=%d split=%d chains=%lld warps=%lld segment=%lld shift=%lld workspace=%zu "
                      "sms=%d",
                      (long long)plan->B, (long long)plan->L, (long long)plan->D, (long long)plan->N,
                      plan->dtype == SSCAN_F32 ? "f32" : "bf16", (plan->flags & SSCAN_ZOH) ? 1 : 0, k.NL,
                      k.N / k.NL, 32 / (k.N / k.NL), k.WPC, k.T, k.STAGES, plan->poly ? 1 : 0,
                      plan->split ? 1 : 0,
-                     (long long)plan->chains, (long long)plan->workers, (long long)plan->seg, plan->ws_bytes,
+                     (long long)plan->chains, (long long)plan->workers, (long long)plan->seg, (long long)plan->seg_shift, plan->ws_bytes,
                      plan->sm_count);
     } else {
         n = snprintf(tmp, sizeof tmp,
