@@ -14,7 +14,10 @@ The C code computes the plain definition (one sequential loop over tokens per
     y      = sum_n C[n] * h[n]                              state after the update
     h_final = h after the last token
 
-following "tm_ssm_selective" (Transformer Math), section "Discretization becomes
+and, optionally, the fused prologue delta <- softplus(delta + delta_bias[d]) and
+epilogue y <- y * silu(z) ("tm_ssm_selective", section "The mechanism:
+parameters as functions of the input"; "Selective State-Space Models (Mamba)
+and Hardware-Aware Scans", section 4), following "tm_ssm_selective" (Transformer Math), section "Discretization becomes
 a per-token operation", and the selective_scan reference loop of "12. Selective
 State Space".  The header comment of ``sscan_oracle.c`` lists the readings taken
 where the pages are silent.
@@ -71,6 +74,12 @@ def _bind(path):
     lib.sscan_oracle_rows.argtypes = [i64, i64, i64, i64, dp, dp, dp, dp, dp, dp, dp,
                                       ip, dp, dp, ip]
     lib.sscan_oracle_rows.restype = ip
+    lib.sscan_oracle_forward_ex.argtypes = [i64, i64, i64, i64, dp, dp, dp, dp, dp, dp,
+                                            ip, dp, ip, dp, dp, dp, ip]
+    lib.sscan_oracle_forward_ex.restype = ip
+    lib.sscan_oracle_rows_ex.argtypes = [i64, i64, i64, i64, dp, dp, dp, dp, dp, dp, dp,
+                                         ip, dp, ip, dp, dp, dp, ip]
+    lib.sscan_oracle_rows_ex.restype = ip
     return lib
 
 
@@ -98,36 +107,44 @@ def _ptr(a):
     return None if a is None else a.ctypes.data
 
 
-def forward(u, delta, A, B, C, h0=None, zoh=False, nthreads=None, lib=None):
+def forward(u, delta, A, B, C, h0=None, zoh=False, nthreads=None, lib=None,
+            delta_bias=None, softplus=False, z=None):
     """Selective-scan forward in fp64 over full tensors.
 
     u, delta: [Bt, L, D]; A: [D, N]; B, C: [Bt, L, N]; h0: [Bt, D, N] or None.
+    delta_bias: [D] or None; softplus: apply softplus to delta (+ bias);
+    z: [Bt, L, D] gate or None (y is multiplied by silu(z)).
     Inputs are widened to fp64 exactly (fp32 and bf16 values are exact in fp64).
     Returns (y [Bt, L, D], h_final [Bt, D, N]) as float64 arrays.
     ``lib`` selects another build of the same C source (default: the oracle's own).
     """
-    u, delta, A, B, C, h0 = map(_f64, (u, delta, A, B, C, h0))
+    u, delta, A, B, C, h0, delta_bias, z = map(_f64, (u, delta, A, B, C, h0, delta_bias, z))
     Bt, L, D = u.shape
     N = A.shape[1]
     assert delta.shape == (Bt, L, D) and A.shape == (D, N)
     assert B.shape == (Bt, L, N) and C.shape == (Bt, L, N)
     assert h0 is None or h0.shape == (Bt, D, N)
+    assert delta_bias is None or delta_bias.shape == (D,)
+    assert z is None or z.shape == (Bt, L, D)
     y = np.empty((Bt, L, D), dtype=np.float64)
     hf = np.empty((Bt, D, N), dtype=np.float64)
-    rc = (lib or _load()).sscan_oracle_forward(Bt, L, D, N, _ptr(u), _ptr(delta), _ptr(A), _ptr(B),
-                                      _ptr(C), _ptr(h0), int(bool(zoh)), _ptr(y), _ptr(hf),
-                                      int(nthreads or host_threads()))
+    rc = (lib or _load()).sscan_oracle_forward_ex(
+        Bt, L, D, N, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(h0), int(bool(zoh)),
+        _ptr(delta_bias), int(bool(softplus)), _ptr(z), _ptr(y), _ptr(hf),
+        int(nthreads or host_threads()))
     if rc != 0:
         raise RuntimeError(f"oracle failed with code {rc}")
     return y, hf
 
 
-def forward_rows(rows, u, delta, A, B, C, h0=None, zoh=False, nthreads=None, lib=None):
+def forward_rows(rows, u, delta, A, B, C, h0=None, zoh=False, nthreads=None, lib=None,
+                 delta_bias=None, softplus=False, z=None):
     """The recurrence on selected (b, d) rows only (rows are independent, so exact).
 
     rows: sequence of (b, d) pairs.  u, delta: [Bt, L, D] arrays of any float
     dtype (only the selected channels are gathered and widened); A: [D, N];
-    B, C: [Bt, L, N]; h0: [Bt, D, N] or None.
+    B, C: [Bt, L, N]; h0: [Bt, D, N] or None; delta_bias [D], softplus and the
+    gate z [Bt, L, D] as in ``forward``.
     Returns (y_rows [R, L], h_final_rows [R, N]) as float64.
     """
     rows = np.asarray(rows, dtype=np.int64).reshape(-1, 2)
@@ -140,12 +157,16 @@ def forward_rows(rows, u, delta, A, B, C, h0=None, zoh=False, nthreads=None, lib
     d_r = np.ascontiguousarray(np.asarray(delta)[rb, :, rd].astype(np.float64))
     A_r = np.ascontiguousarray(np.asarray(A, dtype=np.float64)[rd])
     h0_r = None if h0 is None else np.ascontiguousarray(np.asarray(h0, dtype=np.float64)[rb, rd])
+    bias_r = None if delta_bias is None else np.ascontiguousarray(
+        np.asarray(delta_bias, dtype=np.float64)[rd])
+    z_r = None if z is None else np.ascontiguousarray(np.asarray(z)[rb, :, rd].astype(np.float64))
     B64, C64 = _f64(B), _f64(C)
     y = np.empty((R, L), dtype=np.float64)
     hf = np.empty((R, N), dtype=np.float64)
-    rc = (lib or _load()).sscan_oracle_rows(R, L, N, Bt, _ptr(rb), _ptr(u_r), _ptr(d_r), _ptr(A_r),
-                                   _ptr(B64), _ptr(C64), _ptr(h0_r), int(bool(zoh)),
-                                   _ptr(y), _ptr(hf), int(nthreads or host_threads()))
+    rc = (lib or _load()).sscan_oracle_rows_ex(
+        R, L, N, Bt, _ptr(rb), _ptr(u_r), _ptr(d_r), _ptr(A_r), _ptr(B64), _ptr(C64), _ptr(h0_r),
+        int(bool(zoh)), _ptr(bias_r), int(bool(softplus)), _ptr(z_r), _ptr(y), _ptr(hf),
+        int(nthreads or host_threads()))
     if rc != 0:
         raise RuntimeError(f"oracle failed with code {rc}")
     return y, hf

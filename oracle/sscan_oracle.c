@@ -17,6 +17,13 @@
  *   y[b,t,d] = sum_n C[b,t,n] * h[n]              (state AFTER token t)
  *   h_final[b,d,n] = h[n] after the last token
  *
+ * Optional fused prologue / epilogue (the _ex entry points):
+ *
+ *   delta  <- delta + delta_bias[d]                 (when a bias is given)
+ *   delta  <- softplus(delta) = log(1 + exp(delta)) (when softplus is set)
+ *   y[b,t,d] <- y[b,t,d] * silu(z[b,t,d]),  silu(z) = z / (1 + exp(-z))
+ *                                                   (when a gate z is given)
+ *
  * Sources (page title, section):
  *  - "tm_ssm_selective" (Transformer Math page on selective SSMs), section
  *    "Discretization becomes a per-token operation": per-token ZOH
@@ -32,13 +39,23 @@
  *  - "Mamba & Mamba-2 Architecture", section 1 (shapes B,C:[B,L,N],
  *    Delta:[B,L,D], A:[D,N]) and the numpy listing in section "Code"
  *    (update, then y_t = c_t . h).
+ *  - Prologue: "tm_ssm_selective", section "The mechanism: parameters as
+ *    functions of the input": Delta_t = softplus(d_bias + Linear_D(u_t)); the
+ *    scan is given Linear_D(u_t) as delta and d_bias per channel.
+ *  - Epilogue: "Selective State-Space Models (Mamba) and Hardware-Aware
+ *    Scans", section 4: the block's second branch gates the SSM output
+ *    multiplicatively, as in gated feed-forward layers.
  *
  * Readings where the pages leave a step open:
  *  - y at step t reads the state after token t's update (all listings agree).
  *  - h0 is an optional input (the pages start from zero); NULL means zero.
  *  - ZOH with A[d,n] == 0 takes the limit (exp(Delta*A)-1)/A -> Delta.
- *  - Delta arrives already positive: softplus belongs to the projection
- *    layer that produces it, not to the scan.
+ *  - Without the prologue, delta arrives already positive (softplus done by
+ *    the projection layer that produces it).
+ *  - The gate branch goes through SiLU (the gated feed-forward form the page
+ *    compares it to); the pages give no skip term D*u, so none is added.
+ *  - softplus is evaluated as max(s, 0) + log1p(exp(-|s|)), the same value
+ *    as log(1 + exp(s)) without overflow.
  *
  * Rows are independent (each (b,d) row has its own state), so rows are
  * spread over POSIX threads; the per-row arithmetic is the same sequential
@@ -52,8 +69,22 @@
 #include <stdint.h>
 #include <stdlib.h>
 
+/* softplus(s) = log(1 + exp(s)), written so that exp never overflows. */
+static double softplus(double s)
+{
+    return (s > 0.0 ? s : 0.0) + log1p(exp(-fabs(s)));
+}
+
+/* silu(z) = z * sigmoid(z) = z / (1 + exp(-z)). */
+static double silu(double z)
+{
+    return z / (1.0 + exp(-z));
+}
+
 /* One (b,d) row: the sequential recurrence over L tokens.
  *   u[t*su], dl[t*sd]   input and step size of this channel at token t
+ *   bias, sp            delta <- delta + bias, then softplus when sp != 0
+ *   z[t*sz]             gate of this channel at token t, or NULL
  *   a[n]                the channel's diagonal A row
  *   Bm[t*N+n], Cm[t*N+n] the batch's input / output projections
  *   h0[n]               initial state, or NULL for zero
@@ -66,12 +97,15 @@ static void scan_row(int64_t L, int64_t N,
                      const double *a,
                      const double *Bm, const double *Cm,
                      const double *h0, int zoh,
+                     double bias, int sp, const double *z, int64_t sz,
                      double *y, int64_t sy, double *hfin, double *h)
 {
     for (int64_t n = 0; n < N; ++n)
         h[n] = h0 ? h0[n] : 0.0;
     for (int64_t t = 0; t < L; ++t) {
-        const double delta = dl[t * sd];
+        double delta = dl[t * sd] + bias;
+        if (sp)
+            delta = softplus(delta);
         const double x = u[t * su];
         const double *Bt = Bm + t * N;
         const double *Ct = Cm + t * N;
@@ -86,7 +120,7 @@ static void scan_row(int64_t L, int64_t N,
             h[n] = abar * h[n] + bbar * x;
             acc += Ct[n] * h[n];
         }
-        y[t * sy] = acc;
+        y[t * sy] = z ? acc * silu(z[t * sz]) : acc;
     }
     if (hfin)
         for (int64_t n = 0; n < N; ++n)
@@ -102,6 +136,9 @@ typedef struct {
     const int64_t *row_b;     /* rows_mode 1: batch index of each row */
     int64_t nrows;
     int zoh;
+    const double *bias;       /* [D] (rows_mode 1: [R]) or NULL */
+    int softplus;
+    const double *z;          /* like u, or NULL */
 } job_t;
 
 typedef struct {
@@ -122,6 +159,8 @@ static void run_row(const job_t *j, int64_t r, double *h)
                  j->A + d * N,
                  j->Bm + b * L * N, j->Cm + b * L * N,
                  j->h0 ? j->h0 + (b * D + d) * N : NULL, j->zoh,
+                 j->bias ? j->bias[d] : 0.0, j->softplus,
+                 j->z ? j->z + b * L * D + d : NULL, D,
                  j->y + b * L * D + d, D,
                  j->hfin ? j->hfin + (b * D + d) * N : NULL, h);
     } else {
@@ -133,6 +172,8 @@ static void run_row(const job_t *j, int64_t r, double *h)
                  j->A + r * N,
                  j->Bm + b * L * N, j->Cm + b * L * N,
                  j->h0 ? j->h0 + r * N : NULL, j->zoh,
+                 j->bias ? j->bias[r] : 0.0, j->softplus,
+                 j->z ? j->z + r * L : NULL, 1,
                  j->y + r * L, 1,
                  j->hfin ? j->hfin + r * N : NULL, h);
     }
@@ -177,22 +218,36 @@ static int run_job(const job_t *j, int64_t nrows, int nthreads)
     return rc;
 }
 
-/* Full forward over contiguous row-major tensors.
+/* Full forward over contiguous row-major tensors, with the optional
+ * prologue / epilogue.
  *   u, delta, y : [B][L][D]     A : [D][N]     Bm, Cm : [B][L][N]
  *   h0, h_final : [B][D][N]     (either may be NULL)
+ *   delta_bias  : [D] or NULL   softplus: 0 or 1     z : [B][L][D] or NULL
  * Returns 0 on success, 1 for bad sizes or pointers, 2/3 on allocation or
  * thread-creation failure. */
-int sscan_oracle_forward(int64_t B, int64_t L, int64_t D, int64_t N,
-                         const double *u, const double *delta, const double *A,
-                         const double *Bm, const double *Cm, const double *h0,
-                         int zoh, double *y, double *h_final, int nthreads)
+int sscan_oracle_forward_ex(int64_t B, int64_t L, int64_t D, int64_t N,
+                            const double *u, const double *delta, const double *A,
+                            const double *Bm, const double *Cm, const double *h0,
+                            int zoh, const double *delta_bias, int softplus, const double *z,
+                            double *y, double *h_final, int nthreads)
 {
     if (B < 0 || L < 0 || D < 0 || N < 0) return 1;
     if (B == 0 || D == 0) return 0;
     if (N > 0 && (!A || ((L > 0) && (!Bm || !Cm)))) return 1;
     if (L > 0 && (!u || !delta || !y)) return 1;
-    job_t j = {B, L, D, N, 0, u, delta, A, Bm, Cm, h0, y, h_final, NULL, B * D, zoh};
+    job_t j = {B, L, D, N, 0, u, delta, A, Bm, Cm, h0, y, h_final, NULL, B * D, zoh,
+               delta_bias, softplus != 0, z};
     return run_job(&j, B * D, nthreads);
+}
+
+/* The plain forward: no bias, no softplus, no gate. */
+int sscan_oracle_forward(int64_t B, int64_t L, int64_t D, int64_t N,
+                         const double *u, const double *delta, const double *A,
+                         const double *Bm, const double *Cm, const double *h0,
+                         int zoh, double *y, double *h_final, int nthreads)
+{
+    return sscan_oracle_forward_ex(B, L, D, N, u, delta, A, Bm, Cm, h0, zoh, NULL, 0, NULL,
+                                   y, h_final, nthreads);
 }
 
 /* The same recurrence on an explicit list of R rows (for sampling large
@@ -200,12 +255,15 @@ int sscan_oracle_forward(int64_t B, int64_t L, int64_t D, int64_t N,
  *   row_b      : [R]     batch index of each row (indexes Bm/Cm)
  *   u_rows, delta_rows, y_rows : [R][L]   the row's channel, gathered
  *   A_rows, h0_rows, hfin_rows : [R][N]   (h0_rows / hfin_rows may be NULL)
- *   Bm, Cm     : [Bn][L][N] */
-int sscan_oracle_rows(int64_t R, int64_t L, int64_t N, int64_t Bn,
-                      const int64_t *row_b,
-                      const double *u_rows, const double *delta_rows, const double *A_rows,
-                      const double *Bm, const double *Cm, const double *h0_rows,
-                      int zoh, double *y_rows, double *hfin_rows, int nthreads)
+ *   Bm, Cm     : [Bn][L][N]
+ *   bias_rows  : [R] delta bias of each row's channel, or NULL
+ *   z_rows     : [R][L] gate of each row, or NULL */
+int sscan_oracle_rows_ex(int64_t R, int64_t L, int64_t N, int64_t Bn,
+                         const int64_t *row_b,
+                         const double *u_rows, const double *delta_rows, const double *A_rows,
+                         const double *Bm, const double *Cm, const double *h0_rows,
+                         int zoh, const double *bias_rows, int softplus, const double *z_rows,
+                         double *y_rows, double *hfin_rows, int nthreads)
 {
     if (R < 0 || L < 0 || N < 0 || Bn < 0) return 1;
     if (R == 0) return 0;
@@ -213,6 +271,17 @@ int sscan_oracle_rows(int64_t R, int64_t L, int64_t N, int64_t Bn,
     for (int64_t r = 0; r < R; ++r)
         if (row_b[r] < 0 || row_b[r] >= Bn) return 1;
     job_t j = {Bn, L, 0, N, 1, u_rows, delta_rows, A_rows, Bm, Cm, h0_rows,
-               y_rows, hfin_rows, row_b, R, zoh};
+               y_rows, hfin_rows, row_b, R, zoh, bias_rows, softplus != 0, z_rows};
     return run_job(&j, R, nthreads);
+}
+
+/* Row list without prologue / epilogue. */
+int sscan_oracle_rows(int64_t R, int64_t L, int64_t N, int64_t Bn,
+                      const int64_t *row_b,
+                      const double *u_rows, const double *delta_rows, const double *A_rows,
+                      const double *Bm, const double *Cm, const double *h0_rows,
+                      int zoh, double *y_rows, double *hfin_rows, int nthreads)
+{
+    return sscan_oracle_rows_ex(R, L, N, Bn, row_b, u_rows, delta_rows, A_rows, Bm, Cm, h0_rows,
+                                zoh, NULL, 0, NULL, y_rows, hfin_rows, nthreads);
 }

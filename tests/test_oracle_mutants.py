@@ -35,6 +35,17 @@ MUTANTS = {
     "u_stride": ("j->u + b * L * D + d, D,", "j->u + b * L * D + d, 1,"),
     "B_time_index": ("const double *Bt = Bm + t * N;", "const double *Bt = Bm + (t > 0 ? t - 1 : 0) * N;"),
     "hfinal_stale": ("hfin[n] = h[n];", "hfin[n] = h0 ? h0[n] : 0.0;"),
+    # fused prologue / epilogue
+    "softplus_as_exp": ("return (s > 0.0 ? s : 0.0) + log1p(exp(-fabs(s)));", "return exp(s);"),
+    "softplus_sign": ("log1p(exp(-fabs(s)))", "log1p(exp(fabs(s)))"),
+    "bias_dropped": ("double delta = dl[t * sd] + bias;", "double delta = dl[t * sd];"),
+    "bias_after_softplus": ("double delta = dl[t * sd] + bias;\n        if (sp)\n            delta = softplus(delta);",
+                            "double delta = dl[t * sd];\n        if (sp)\n            delta = softplus(delta);\n"
+                            "        delta += bias;"),
+    "bias_batch_index": ("j->bias ? j->bias[d] : 0.0", "j->bias ? j->bias[b] : 0.0"),
+    "gate_sigmoid_only": ("return z / (1.0 + exp(-z));", "return 1.0 / (1.0 + exp(-z));"),
+    "gate_additive": ("acc * silu(z[t * sz])", "acc + silu(z[t * sz])"),
+    "gate_stride": ("j->z ? j->z + b * L * D + d : NULL, D,", "j->z ? j->z + b * L * D + d : NULL, 1,"),
 }
 
 
@@ -53,8 +64,8 @@ def test_mutant_is_caught(name, source, tmp_path):
     src.write_text(mutated)
     lib = O.load_library(O.compile_source(str(src), str(tmp_path / f"lib{name}.so")))
 
-    def fwd(u, delta, A, B, C, h0, zoh):
-        return O.forward(u, delta, A, B, C, h0, zoh, lib=lib)
+    def fwd(u, delta, A, B, C, h0, zoh, **kw):
+        return O.forward(u, delta, A, B, C, h0, zoh, lib=lib, **kw)
 
     caught = []
     for pin in P.PINS:

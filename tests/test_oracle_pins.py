@@ -265,13 +265,100 @@ def pin_split_resume(fwd):
         assert np.array_equal(h2, hf)
 
 
+# ---- fused prologue (delta <- softplus(delta + bias)) and epilogue (y * silu(z)) ----
+
+def _expit(x):
+    from scipy.special import expit  # library logistic function
+    return expit(x)
+
+
+def pin_fused_softplus_gru(fwd):
+    # "tm_ssm_selective", "Delta is a gate, exactly": N = 1, A = -1, B = 1 and
+    # Delta = softplus(s) make the ZOH step the GRU update with g = sigmoid(s).
+    # Here s reaches the scan as a raw delta s - b plus the channel bias b.
+    rng = np.random.default_rng(31)
+    L, bias = 40, 0.75
+    s = rng.normal(0.0, 2.5, L)
+    u = rng.standard_normal(L)
+    g = _expit(s)
+    h, want = -0.4, []
+    for t in range(L):
+        h = (1.0 - g[t]) * h + g[t] * u[t]
+        want.append(h)
+    ones = np.ones((1, L, 1))
+    y, hf = fwd(u.reshape(1, L, 1), (s - bias).reshape(1, L, 1), np.array([[-1.0]]), ones, ones,
+                np.array([[[-0.4]]]), True, delta_bias=np.array([bias]), softplus=True)
+    assert np.abs(y[0, :, 0] - np.array(want)).max() <= 1e-13
+    assert abs(hf[0, 0, 0] - want[-1]) <= 1e-13
+
+
+def pin_fused_softplus_at_zero(fwd):
+    # softplus(0) = log 2: with A = -1 the retention is exactly 1/2 and the Euler
+    # input weight log 2.
+    u = np.array([0.3, -1.2, 2.0])
+    h, want = 0.8, []
+    for t in range(3):
+        h = 0.5 * h + math.log(2.0) * u[t]
+        want.append(h)
+    ones = np.ones((1, 3, 1))
+    y, _ = fwd(u.reshape(1, 3, 1), np.zeros((1, 3, 1)), np.array([[-1.0]]), ones, ones,
+               np.array([[[0.8]]]), False, softplus=True)
+    assert np.abs(y[0, :, 0] - np.array(want)).max() <= 1e-15
+
+
+def pin_fused_softplus_limits(fwd):
+    # softplus(s) -> s for large s (gap e^-40 ~ 4e-18) and -> 0 for very negative s
+    # (the "Delta -> 0 keeps the state" gate of "tm_ssm_selective").
+    rng = np.random.default_rng(32)
+    u, delta, A, B, C, h0 = _rand_problem(rng, 2, 9, 3, 4)
+    big = np.full_like(delta, 40.0)
+    y1, h1 = fwd(u, big, A, B, C, h0, False, softplus=True)
+    y2, h2 = fwd(u, big, A, B, C, h0, False)
+    assert np.abs(y1 - y2).max() <= 1e-12 * (1 + np.abs(y2).max())
+    y3, h3 = fwd(u, np.full_like(delta, -60.0), A, B, C, h0, False, softplus=True)
+    assert np.abs(h3 - h0).max() <= 1e-20 * (1 + np.abs(h0).max()) + 1e-24
+    assert np.abs(y3 - np.einsum("btn,bdn->btd", C, h0)).max() <= 1e-15
+
+
+def pin_fused_bias_per_channel(fwd):
+    # the bias is one value per channel d, added to delta before softplus
+    rng = np.random.default_rng(33)
+    u, delta, A, B, C, h0 = _rand_problem(rng, 3, 11, 4, 5)
+    bias = rng.normal(0.0, 1.0, 4)
+    for sp, zoh in ((False, False), (True, False), (True, True)):
+        y1, h1 = fwd(u, delta, A, B, C, h0, zoh, delta_bias=bias, softplus=sp)
+        d2 = delta + bias[None, None, :]
+        if sp:
+            d2 = np.maximum(d2, 0.0) + np.log1p(np.exp(-np.abs(d2)))
+        y2, h2 = fwd(u, d2, A, B, C, h0, zoh)
+        assert np.abs(y1 - y2).max() <= 1e-13 * (1 + np.abs(y2).max())
+        assert np.abs(h1 - h2).max() <= 1e-13 * (1 + np.abs(h2).max())
+
+
+def pin_fused_gate(fwd):
+    # "Selective State-Space Models (Mamba) and Hardware-Aware Scans", section 4:
+    # the second branch gates the SSM output; y * silu(z), silu(z) = z * sigmoid(z).
+    rng = np.random.default_rng(34)
+    u, delta, A, B, C, h0 = _rand_problem(rng, 2, 13, 3, 4)
+    z = rng.normal(0.0, 2.0, u.shape)
+    for zoh in (False, True):
+        y0, h0f = fwd(u, delta, A, B, C, h0, zoh)
+        yg, hgf = fwd(u, delta, A, B, C, h0, zoh, z=z)
+        assert np.abs(yg - y0 * z * _expit(z)).max() <= 1e-14 * (1 + np.abs(y0).max())
+        assert np.array_equal(hgf, h0f)            # the gate acts on y only
+        yz, _ = fwd(u, delta, A, B, C, h0, zoh, z=np.zeros_like(z))
+        assert np.array_equal(yz, np.zeros_like(yz))
+
+
 PINS = [pin_p2_listing, pin_p2_worked_example, pin_p5_horizon_table, pin_brute_force,
         pin_lti_convolution, pin_gru_identity, pin_delta_zero, pin_reset,
-        pin_zoh_fixed_point, pin_state_bound, pin_split_resume]
+        pin_zoh_fixed_point, pin_state_bound, pin_split_resume,
+        pin_fused_softplus_gru, pin_fused_softplus_at_zero, pin_fused_softplus_limits,
+        pin_fused_bias_per_channel, pin_fused_gate]
 
 
-def oracle_fwd(u, delta, A, B, C, h0, zoh, lib=None):
-    return O.forward(u, delta, A, B, C, h0, zoh, lib=lib)
+def oracle_fwd(u, delta, A, B, C, h0, zoh, lib=None, **kw):
+    return O.forward(u, delta, A, B, C, h0, zoh, lib=lib, **kw)
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
