@@ -146,14 +146,16 @@ def cpu_oracle_rate(g, w, min_seconds=10.0, max_seconds=30.0):
     """Time the fp64 oracle as it stands on this host's cores: full passes over the
     workload until at least ``min_seconds`` elapsed.  Returns (elements/s, cores, sample)."""
     from oracle import oracle as O
-    v = {k: (None if g[k] is None else W.as_f32(g[k], g["dtype"]).astype(np.float64))
-         for k in ("u", "delta", "B", "C")}
+    v = {k: (None if g.get(k) is None else W.as_f32(g[k], g["dtype"]).astype(np.float64))
+         for k in ("u", "delta", "B", "C", "z")}
     A = g["A"].astype(np.float64)
     h0 = None if g["h0"] is None else g["h0"].astype(np.float64)
+    bias = None if g.get("delta_bias") is None else g["delta_bias"].astype(np.float64)
     cores = O.host_threads()
     n, t0 = 0, time.perf_counter()
     while True:
-        O.forward(v["u"], v["delta"], A, v["B"], v["C"], h0, w.zoh, nthreads=cores)
+        O.forward(v["u"], v["delta"], A, v["B"], v["C"], h0, w.zoh, nthreads=cores,
+                  delta_bias=bias, softplus=w.fused, z=v["z"])
         n += 1
         el = time.perf_counter() - t0
         if el >= min_seconds or el + el / n > max_seconds:
@@ -190,7 +192,7 @@ def run_ours(args, rank, world, local_rank):
     w = W.WORKLOADS[args.workload]
     # shard: rank r owns batch rows [r*B, (r+1)*B) of an N*B-row job (own seed)
     g = W.generate(w.B, w.L, w.D, w.N, w.dtype, w.h0_std, w.reset_frac,
-                   seed=shard_seed(w, rank))
+                   seed=shard_seed(w, rank), fused=w.fused)
     tdt = torch.float32 if w.dtype == "f32" else torch.bfloat16
 
     def host(x, dt):
@@ -204,9 +206,10 @@ def run_ours(args, rank, world, local_rank):
 
     hin = {"u": host(g["u"], w.dtype), "delta": host(g["delta"], w.dtype),
            "A": host(g["A"], "f32"), "B": host(g["B"], w.dtype), "C": host(g["C"], w.dtype),
-           "h0": host(g["h0"], "f32")}
+           "h0": host(g["h0"], "f32"), "delta_bias": host(g["delta_bias"], "f32"),
+           "z": host(g["z"], w.dtype)}
     din = {k: (None if v is None else v.to(dev)) for k, v in hin.items()}
-    plan = S.Plan(w.B, w.L, w.D, w.N, tdt, w.zoh)
+    plan = S.Plan(w.B, w.L, w.D, w.N, tdt, w.zoh, delta_softplus=w.fused)
     ws = plan.new_workspace(dev)
     y = torch.empty((w.B, w.L, w.D), dtype=tdt, device=dev)
     hf = torch.empty((w.B, w.D, w.N), dtype=torch.float32, device=dev)
@@ -214,7 +217,8 @@ def run_ours(args, rank, world, local_rank):
 
     def step():
         plan.forward(din["u"], din["delta"], din["A"], din["B"], din["C"], din["h0"],
-                     y=y, h_final=hf, workspace=ws, stream=stream)
+                     y=y, h_final=hf, workspace=ws, stream=stream,
+                     delta_bias=din["delta_bias"], z=din["z"])
 
     for _ in range(args.warmup):
         step()
@@ -251,7 +255,8 @@ def run_ours(args, rank, world, local_rank):
 
     def e2e_step():
         S.forward_host(hin["u"], hin["delta"], hin["A"], hin["B"], hin["C"], hin["h0"],
-                       zoh=w.zoh, device=dev, out=out_h)
+                       zoh=w.zoh, device=dev, out=out_h, delta_bias=hin["delta_bias"],
+                       delta_softplus=w.fused, z=hin["z"])
 
     for _ in range(min(args.warmup, 3)):
         e2e_step()
@@ -290,7 +295,8 @@ def run_ours(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": f"{w.name}: B={w.B} L={w.L} D={w.D} N={w.N} io={w.dtype} "
-                               f"{'ZOH' if w.zoh else 'Euler'} h0={'yes' if w.h0_std else 'no'}",
+                               f"{'ZOH' if w.zoh else 'Euler'} h0={'yes' if w.h0_std else 'no'}"
+                               f"{' fused softplus(delta+bias), y*silu(z)' if w.fused else ''}",
                    "B": w.B, "L": w.L, "D": w.D, "N": w.N, "io_dtype": w.dtype,
                    "parallelism": f"dp{world} (independent batch-row shards, no collective)",
                    "l2": f"inputs larger than L2 ({alg_bytes / 1e6:.0f} MB per step vs "
@@ -322,27 +328,30 @@ def run_reference(args):
     w = W.WORKLOADS[args.workload]
     g = W.make_inputs(w)
     from oracle import oracle as O
-    v = {k: W.as_f32(g[k], g["dtype"]).astype(np.float64) for k in ("u", "delta", "B", "C")}
+    v = {k: (None if g.get(k) is None else W.as_f32(g[k], g["dtype"]).astype(np.float64))
+         for k in ("u", "delta", "B", "C", "z")}
     A = g["A"].astype(np.float64)
     h0 = None if g["h0"] is None else g["h0"].astype(np.float64)
+    fk = {"delta_bias": None if g.get("delta_bias") is None else g["delta_bias"].astype(np.float64),
+          "softplus": w.fused, "z": v["z"]}
     cores = O.host_threads()
     # each step: a bounded sample of the workload's rows (rows are independent)
     target = max(1.0, args.ref_step_seconds)
     rows_all = [(b, d) for b in range(w.B) for d in range(w.D)]
     probe = rows_all[: max(1, len(rows_all) // 64)]
     t0 = time.perf_counter()
-    O.forward_rows(probe, v["u"], v["delta"], A, v["B"], v["C"], h0, w.zoh, nthreads=cores)
+    O.forward_rows(probe, v["u"], v["delta"], A, v["B"], v["C"], h0, w.zoh, nthreads=cores, **fk)
     per_row = (time.perf_counter() - t0) / len(probe)
     nrows = int(min(len(rows_all), max(1, target / max(per_row, 1e-9))))
     rng = np.random.default_rng(0)
     sel = [rows_all[i] for i in sorted(rng.choice(len(rows_all), nrows, replace=False))]
     for _ in range(args.warmup):
         O.forward_rows(sel[: max(1, nrows // 8)], v["u"], v["delta"], A, v["B"], v["C"], h0,
-                       w.zoh, nthreads=cores)
+                       w.zoh, nthreads=cores, **fk)
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        O.forward_rows(sel, v["u"], v["delta"], A, v["B"], v["C"], h0, w.zoh, nthreads=cores)
+        O.forward_rows(sel, v["u"], v["delta"], A, v["B"], v["C"], h0, w.zoh, nthreads=cores, **fk)
         times.append(time.perf_counter() - t0)
     tot = sum(times)
     value = nrows * w.L * args.steps / tot
@@ -353,7 +362,8 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": f"{w.name}: B={w.B} L={w.L} D={w.D} N={w.N} io={w.dtype} "
-                               f"{'ZOH' if w.zoh else 'Euler'} h0={'yes' if w.h0_std else 'no'}",
+                               f"{'ZOH' if w.zoh else 'Euler'} h0={'yes' if w.h0_std else 'no'}"
+                               f"{' fused softplus(delta+bias), y*silu(z)' if w.fused else ''}",
                    "B": w.B, "L": w.L, "D": w.D, "N": w.N, "io_dtype": w.dtype},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},

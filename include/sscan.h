@@ -70,7 +70,13 @@ enum {
     /* exact zero-order-hold input term (exp(delta*A)-1)/A * B * u instead of
      * the Euler term delta * B * u ("tm_ssm_selective", section
      * "Discretization becomes a per-token operation") */
-    SSCAN_ZOH = 1u << 0
+    SSCAN_ZOH = 1u << 0,
+    /* fused prologue: the scan uses delta' = softplus(delta + delta_bias[d])
+     * = log(1 + exp(delta + delta_bias[d])) instead of delta, i.e. delta is
+     * the raw projection Linear_D(u_t) and the bias d_bias of
+     * "tm_ssm_selective", section "The mechanism: parameters as functions of
+     * the input" (Delta_t = softplus(d_bias + Linear_D(u_t))) */
+    SSCAN_DELTA_SOFTPLUS = 1u << 1
 };
 
 /* status codes */
@@ -89,7 +95,7 @@ enum {
  *   N        state size per channel, one of 16, 32, 64 (the pages use 16;
  *            "12. Selective State Space" discusses 64 and 128)
  *   dtype    SSCAN_F32 or SSCAN_BF16
- *   flags    0 or SSCAN_ZOH
+ *   flags    0 or any of SSCAN_ZOH, SSCAN_DELTA_SOFTPLUS
  * On success *plan receives the plan and SSCAN_OK is returned; otherwise
  * *plan is set to NULL.  Sizes are validated before any CUDA call, so
  * SSCAN_ERR_INVALID / SSCAN_ERR_UNSUPPORTED come back without a device. */
@@ -116,6 +122,23 @@ SSCAN_API size_t sscan_workspace_bytes(sscan_plan_t plan);
 SSCAN_API int sscan_forward(sscan_plan_t plan, const void *u, const void *delta, const float *A,
                   const void *B, const void *C, const float *h0, void *y, float *h_final,
                   void *workspace, void *stream);
+
+/* sscan_forward with the fused prologue and epilogue of the Mamba block:
+ *   delta_bias      [D] fp32 added to delta before use (and before softplus
+ *                   when the plan has SSCAN_DELTA_SOFTPLUS), or NULL
+ *   z               [B][L][D], plan dtype: the output is y * silu(z),
+ *                   silu(z) = z / (1 + exp(-z)), or NULL for no gate
+ *                   ("Selective State-Space Models (Mamba) and Hardware-Aware
+ *                   Scans", section 4: the block's second branch gates the
+ *                   SSM output multiplicatively)
+ * h_final is the state of the scan (the gate acts on y only).  All other
+ * arguments, the ownership (caller-owned device buffers, nothing retained)
+ * and the errors are those of sscan_forward; delta_bias and z must be
+ * 16-byte aligned and must not overlap y or h_final.  sscan_forward is this
+ * call with delta_bias = z = NULL. */
+SSCAN_API int sscan_forward_gated(sscan_plan_t plan, const void *u, const void *delta, const float *A,
+                        const void *B, const void *C, const float *h0, const float *delta_bias,
+                        const void *z, void *y, float *h_final, void *workspace, void *stream);
 
 /* Wait for `stream`, then read and clear the plan's device status word.
  * Returns SSCAN_OK, SSCAN_ERR_TIMEOUT, or SSCAN_ERR_CUDA. */

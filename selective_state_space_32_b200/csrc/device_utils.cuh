@@ -95,6 +95,37 @@ __device__ __forceinline__ f2 zoh_coef_pair(f2 dd, f2 a1, f2 ia, f2 abar) {
     return pack2(fabsf(z0) <= 0.25f ? s0 : g0, fabsf(z1) <= 0.25f ? s1 : g1);
 }
 
+// softplus(s) = log(1 + e^s) for the fused prologue.  s itself above 20 (the
+// remainder log1p(e^-s) < 2.1e-9 is below half an ulp of s); otherwise with
+// w = e^s (MUFU ex2, relative error ~2^-22): for w < 1/8 the Taylor series of
+// log1p(w) to w^8 (truncation below w^9/9, i.e. < 7e-9 relative), else
+// ln 2 * log2(1 + w) on the MUFU (result >= 0.117 there, so the lg2
+// approximation's ~2^-22 absolute error stays below ~2e-6 relative).  Both
+// branches are evaluated and one is selected (no divergence).
+__device__ __forceinline__ float softplus_f(float s) {
+    const float w = ex2(fminf(s, 20.0f) * 1.4426950408889634f);
+    float q = fmaf(w, -0.125f, 0.14285714285714285f);
+    q = fmaf(q, w, -0.16666666666666666f);
+    q = fmaf(q, w, 0.2f);
+    q = fmaf(q, w, -0.25f);
+    q = fmaf(q, w, 0.3333333333333333f);
+    q = fmaf(q, w, -0.5f);
+    q = fmaf(q, w, 1.0f);
+    const float series = w * q;
+    float l;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(1.0f + w));
+    const float big = l * 0.6931471805599453f;
+    return s > 20.0f ? s : (w < 0.125f ? series : big);
+}
+
+// silu(z) = z * sigmoid(z) = z / (1 + e^-z) with the MUFU reciprocal (relative
+// error ~2^-23); 1 + e^-z = inf (z < -88) gives rcp = 0 and silu = -0.
+__device__ __forceinline__ float silu_f(float z) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + ex2(-z * 1.4426950408889634f)));
+    return z * r;
+}
+
 // ------------------------------------------------------------- storage types
 
 template <class IO> struct Io;

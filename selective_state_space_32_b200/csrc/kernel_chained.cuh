@@ -66,6 +66,10 @@ struct ChainedParams {
     unsigned long long *rec_flags; // [chains][max_pieces] (epoch << 32) | 1 once published
     int64_t max_pieces;
     void *ysink;                   // [warps][32] 4-byte slots: y stores of lanes past the last channel
+    // fused prologue / epilogue (FUSED kernels only)
+    const float *delta_bias;       // [D] added to delta, or null
+    const void *z;                 // [B][L][D] gate: y *= silu(z), or null
+    int softplus;                  // delta <- softplus(delta + bias)
     int drop_publish;              // failure-detection tests only: heads never publish their carry
 };
 
@@ -87,6 +91,12 @@ struct ChainedCfg {
     static constexpr int kWarp = ((STAGES * kStage + kConv) + 127) / 128 * 128;
     static constexpr int kBars = (2 * WPC * STAGES * 8 + 127) / 128 * 128;  // full + empty per slot
     static constexpr int kSmem = WPC * kWarp + kBars;
+    // fused kernels: each stage also holds the gate tile z [T][CPW]; two fp32 [T][CPW]
+    // tiles hold the stage's delta after bias / softplus and silu(z)
+    static constexpr int kStageF = kStage + kU;
+    static constexpr int kDsf = T * CPW * 4;
+    static constexpr int kWarpF = ((STAGES * kStageF + kConv + 2 * kDsf) + 127) / 128 * 128;
+    static constexpr int kSmemF = WPC * kWarpF + kBars;
     static constexpr int kThreads = (WPC + 1) * 32;  // WPC consumer warps + 1 producer warp
     static_assert(LPC >= 1 && LPC <= 8 && N % NL == 0 && NL % 4 == 0, "bad split");
     static_assert(CPW * ES % 16 == 0 && N * ES % 16 == 0, "TMA rows must be 16-byte multiples");
@@ -275,7 +285,7 @@ struct Segment {
 // 2^-40 max(1, |h_in|) and delta >= 0, A <= 0 over the piece guarantee that
 // it can only shrink further ("Delta is a gate": large steps reset the state,
 // "tm_ssm_selective").  The piece's final state is hloc + P_piece h_in.
-template <class IO, class Cfg>
+template <class IO, class Cfg, bool FUSED>
 __device__ __noinline__ void split_fixup(const ChainedParams &P, int64_t c, int64_t ts, int64_t te,
                                          int64_t wk, int lane) {
     constexpr int N = Cfg::N, NL = Cfg::NL, LPC = Cfg::LPC, CPW = Cfg::CPW, NP = Cfg::NP;
@@ -354,16 +364,25 @@ __device__ __noinline__ void split_fixup(const ChainedParams &P, int64_t c, int6
     const IO *cptr = static_cast<const IO *>(P.Cm) + b * L * N + n0;
     IO *yptr = static_cast<IO *>(P.y) + b * L * D + dcl;
     const bool writer = valid && g == 0;
+    // fused: the same delta transform as the scan; the correction is gated like y
+    const float biasv = (FUSED && P.delta_bias != nullptr) ? __ldg(P.delta_bias + dcl) : 0.0f;
+    const bool gate = FUSED && P.z != nullptr;
+    const IO *zptr = gate ? static_cast<const IO *>(P.z) + b * L * D + dcl : nullptr;
     for (int64_t tb = ts; tb < te; tb += FB) {
         const int nb = static_cast<int>(te - tb < FB ? te - tb : FB);
-        float dl[FB], yo[FB];
+        float dl[FB], yo[FB], gq[FB];
         f2 cv[FB][NP];
 #pragma unroll
         for (int q = 0; q < FB; ++q) {
             const int64_t t = tb + (q < nb ? q : 0);
             dl[q] = Io<IO>::widen(Io<IO>::ld(dptr + t * D));
+            if (FUSED) {
+                dl[q] += biasv;
+                if (P.softplus) dl[q] = softplus_f(dl[q]);
+            }
             Io<IO>::template ld_pairs<NP>(cptr + t * N, cv[q]);
             yo[q] = writer ? Io<IO>::widen(__ldcg(yptr + t * D)) : 0.0f;
+            gq[q] = (gate && writer) ? silu_f(Io<IO>::widen(Io<IO>::ld(zptr + t * D))) : 1.0f;
         }
 #pragma unroll
         for (int q = 0; q < FB; ++q) {
@@ -381,7 +400,7 @@ __device__ __noinline__ void split_fixup(const ChainedParams &P, int64_t c, int6
                 float corr = y0 + y1;
 #pragma unroll
                 for (int o = 1; o < LPC; o <<= 1) corr += __shfl_xor_sync(0xffffffffu, corr, o);
-                if (writer) Io<IO>::st(yptr + (tb + q) * D, yo[q] + corr);
+                if (writer) Io<IO>::st(yptr + (tb + q) * D, yo[q] + corr * gq[q]);
             }
         }
         if (mono) {
@@ -426,9 +445,10 @@ __device__ __noinline__ void split_fixup(const ChainedParams &P, int64_t c, int6
 // stage that used the slot before.  No lane ever blocks on one consumer (a
 // consumer may be waiting for another warp's carry): each lane tests its
 // consumer's barrier, and the warp backs off briefly when no lane could issue.
-template <class IO, class Cfg>
+template <class IO, class Cfg, bool FUSED>
 __device__ __forceinline__ void produce(const CUtensorMap *tm_u, const CUtensorMap *tm_d, const CUtensorMap *tm_b,
-                                        const CUtensorMap *tm_c, const ChainedParams &P, unsigned char *smem,
+                                        const CUtensorMap *tm_c, const CUtensorMap *tm_z, const ChainedParams &P,
+                                        unsigned char *smem,
                                         uint64_t *full, uint64_t *empty, int lane) {
     constexpr int WPC = Cfg::WPC, T = Cfg::T, STAGES = Cfg::STAGES, CPW = Cfg::CPW;
     if (lane == 0) {
@@ -436,7 +456,10 @@ __device__ __forceinline__ void produce(const CUtensorMap *tm_u, const CUtensorM
         tma_prefetch_desc(tm_d);
         tma_prefetch_desc(tm_b);
         tma_prefetch_desc(tm_c);
+        if (FUSED && P.z != nullptr) tma_prefetch_desc(tm_z);
     }
+    constexpr int kStageB = FUSED ? Cfg::kStageF : Cfg::kStage;
+    const bool zt = FUSED && P.z != nullptr;  // the gate tile is loaded with each stage
     const int64_t L = P.L;
     const int i = lane;  // the consumer this lane serves
     const Segment sg(static_cast<int64_t>(blockIdx.x) * WPC + (i < WPC ? i : 0), P);
@@ -452,21 +475,22 @@ __device__ __forceinline__ void produce(const CUtensorMap *tm_u, const CUtensorM
         row = static_cast<int>(b * L);
     };
     if (k >= 0) begin_part();
-    unsigned char *ring = smem + (i < WPC ? i : 0) * Cfg::kWarp;
+    unsigned char *ring = smem + (i < WPC ? i : 0) * (FUSED ? Cfg::kWarpF : Cfg::kWarp);
     uint32_t idle = 0;
     while (__any_sync(0xffffffffu, k >= 0)) {
         const int s = static_cast<int>(r % STAGES);
         const bool ready = k >= 0 && (r < STAGES || mbar_test_wait(&empty[i * STAGES + s],
                                                                    static_cast<uint32_t>((r / STAGES - 1) & 1)));
         if (ready) {
-            unsigned char *slot = ring + s * Cfg::kStage;
+            unsigned char *slot = ring + s * kStageB;
             uint64_t *bar = &full[i * STAGES + s];
             const int yrow = row + static_cast<int>(t);
-            mbar_expect_tx(bar, Cfg::kStage);
+            mbar_expect_tx(bar, zt ? Cfg::kStageF : Cfg::kStage);
             tma_load_2d(slot, tm_u, x, yrow, bar);
             tma_load_2d(slot + Cfg::kU, tm_d, x, yrow, bar);
             tma_load_2d(slot + 2 * Cfg::kU, tm_b, 0, yrow, bar);
             tma_load_2d(slot + 2 * Cfg::kU + Cfg::kB, tm_c, 0, yrow, bar);
+            if (zt) tma_load_2d(slot + Cfg::kStage, tm_z, x, yrow, bar);
             ++r;
             t += T;
             if (t >= te) {
@@ -488,28 +512,32 @@ __device__ __forceinline__ void produce(const CUtensorMap *tm_u, const CUtensorM
     }
 }
 
-template <class IO, class Cfg, bool ZOH, bool POLY, bool SPLIT>
+template <class IO, class Cfg, bool ZOH, bool POLY, bool SPLIT, bool FUSED>
 __global__ void __launch_bounds__(Cfg::kThreads, 1)
 sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_d,
                      const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
-                     const ChainedParams P) {
+                     const __grid_constant__ CUtensorMap tm_z, const ChainedParams P) {
     constexpr int N = Cfg::N, NL = Cfg::NL, T = Cfg::T, STAGES = Cfg::STAGES;
     constexpr int LPC = Cfg::LPC, CPW = Cfg::CPW, NP = Cfg::NP;
     extern __shared__ __align__(128) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::WPC * Cfg::kWarp);
+    constexpr int kWarpB = FUSED ? Cfg::kWarpF : Cfg::kWarp;  // bytes of one consumer's region
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::WPC * kWarpB);
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2 * Cfg::WPC * STAGES; ++i) mbar_init(&bars[i], 1);
         mbar_fence_init();
     }
     __syncthreads();  // the only block-wide barrier
     if (warp == Cfg::WPC) {
-        produce<IO, Cfg>(&tm_u, &tm_d, &tm_b, &tm_c, P, smem, bars, bars + Cfg::WPC * STAGES, lane);
+        produce<IO, Cfg, FUSED>(&tm_u, &tm_d, &tm_b, &tm_c, &tm_z, P, smem, bars, bars + Cfg::WPC * STAGES, lane);
         return;
     }
-    unsigned char *wbase = smem + warp * Cfg::kWarp;
-    float *convB = reinterpret_cast<float *>(wbase + STAGES * Cfg::kStage);
+    constexpr int kStageB = FUSED ? Cfg::kStageF : Cfg::kStage;  // bytes of one stage
+    unsigned char *wbase = smem + warp * kWarpB;
+    float *convB = reinterpret_cast<float *>(wbase + STAGES * kStageB);
     float *convC = convB + T * N;
+    float *dsf = reinterpret_cast<float *>(wbase + STAGES * kStageB + Cfg::kConv);  // FUSED: delta'
+    float *gsf = dsf + T * CPW;                                                      // FUSED: silu(z)
     uint64_t *full = bars + warp * STAGES;
     uint64_t *empty = bars + (Cfg::WPC + warp) * STAGES;
 
@@ -520,12 +548,13 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
     const int64_t n_parts = seg.n_parts;
     auto part = [&](int64_t k, int64_t &c, int64_t &ts, int64_t &te) { seg.part(k, L, c, ts, te); };
 
-    auto tile_u = [&](int s) { return reinterpret_cast<IO *>(wbase + s * Cfg::kStage); };
-    auto tile_d = [&](int s) { return reinterpret_cast<IO *>(wbase + s * Cfg::kStage + Cfg::kU); };
-    auto tile_b = [&](int s) { return reinterpret_cast<IO *>(wbase + s * Cfg::kStage + 2 * Cfg::kU); };
+    auto tile_u = [&](int s) { return reinterpret_cast<IO *>(wbase + s * kStageB); };
+    auto tile_d = [&](int s) { return reinterpret_cast<IO *>(wbase + s * kStageB + Cfg::kU); };
+    auto tile_b = [&](int s) { return reinterpret_cast<IO *>(wbase + s * kStageB + 2 * Cfg::kU); };
     auto tile_c = [&](int s) {
-        return reinterpret_cast<IO *>(wbase + s * Cfg::kStage + 2 * Cfg::kU + Cfg::kB);
+        return reinterpret_cast<IO *>(wbase + s * kStageB + 2 * Cfg::kU + Cfg::kB);
     };
+    auto tile_z = [&](int s) { return reinterpret_cast<IO *>(wbase + s * kStageB + Cfg::kStage); };
 
     const int cl = lane / LPC;   // channel within the chain
     const int g = lane % LPC;    // state group
@@ -614,6 +643,14 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
         IO *ybase = valid ? static_cast<IO *>(P.y) + b * L * D + d
                           : reinterpret_cast<IO *>(static_cast<float *>(P.ysink) + wk * 32 + lane);
         const int64_t ystr = valid ? D : 0;
+        // fused prologue: this lane transforms tile entries lane, lane + 32, ...,
+        // all of channel lane % CPW of the chain (32 is a multiple of CPW)
+        float biasv = 0.0f;
+        if (FUSED && P.delta_bias != nullptr) {
+            const int64_t dp = cw * CPW + lane % CPW;
+            biasv = dp < D ? __ldg(P.delta_bias + dp) : 0.0f;
+        }
+        const bool gate = FUSED && P.z != nullptr;
         for (int64_t t0 = ts; t0 < te; t0 += T) {
             const int s = static_cast<int>(consumed % STAGES);
             const uint32_t par = static_cast<uint32_t>((consumed / STAGES) & 1);
@@ -655,6 +692,17 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
                 Bs = convB;
                 Cs = convC;
             }
+            if (FUSED) {  // once per tile entry: delta' = softplus(delta + bias), silu(z), fp32
+                const IO *zs = tile_z(s);
+#pragma unroll
+                for (int i = lane; i < T * CPW; i += 32) {
+                    const float v = Io<IO>::widen(dsm[i]) + biasv;
+                    dsf[i] = P.softplus ? softplus_f(v) : v;
+                    gsf[i] = gate ? silu_f(Io<IO>::widen(zs[i])) : 1.0f;
+                }
+                __syncwarp();
+            }
+            auto delta_at = [&](int idx) { return FUSED ? dsf[idx] : Io<IO>::widen(dsm[idx]); };
             const int nsteps = static_cast<int>(te - t0 < T ? te - t0 : T);
             IO *yp = ybase + t0 * ystr;
             int j = 0;
@@ -672,7 +720,7 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
 #pragma unroll
                 for (int q = 0; q < G; ++q) {
                     const float x = Io<IO>::widen(us[(j0 + q) * CPW + cl]);
-                    const float dl = Io<IO>::widen(dsm[(j0 + q) * CPW + cl]);
+                    const float dl = delta_at((j0 + q) * CPW + cl);
                     if (SPLIT) {
                         ssum += dl;
                         dmin = fminf(dmin, dl);
@@ -688,6 +736,10 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
                 for (int q = 0; q < G; ++q)
                     yv[q] = advance_euler<NP>(h, ab[q], duv[q], Bs + (j0 + q) * N + n0, Cs + (j0 + q) * N + n0);
                 const int base = reduce_scatter<LPC, G>(yv, g);
+                if (FUSED) {
+#pragma unroll
+                    for (int q = 0; q < KEEP; ++q) yv[q] *= gsf[(j0 + base + q) * CPW + cl];
+                }
                 if (g_store) {
 #pragma unroll
                     for (int q = 0; q < KEEP; ++q) Io<IO>::st(yp + (j0 + base + q) * ystr, yv[q]);
@@ -701,7 +753,7 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
 #pragma unroll
                 for (int q = 0; q < G; ++q) {
                     const float x = Io<IO>::widen(us[(j0 + q) * CPW + cl]);
-                    const float dl = Io<IO>::widen(dsm[(j0 + q) * CPW + cl]);
+                    const float dl = delta_at((j0 + q) * CPW + cl);
                     if (SPLIT) {
                         ssum += dl;
                         dmin = fminf(dmin, dl);
@@ -715,6 +767,10 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
 #pragma unroll
                 for (int q = 0; q < G; ++q) yv[q] = advance<NP>(h, ab[q], bu[q], Cs + (j0 + q) * N + n0);
                 const int base = reduce_scatter<LPC, G>(yv, g);
+                if (FUSED) {
+#pragma unroll
+                    for (int q = 0; q < KEEP; ++q) yv[q] *= gsf[(j0 + base + q) * CPW + cl];
+                }
                 if (g_store) {
 #pragma unroll
                     for (int q = 0; q < KEEP; ++q) Io<IO>::st(yp + (j0 + base + q) * ystr, yv[q]);
@@ -740,7 +796,7 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
             for (; j < nsteps; ++j) {  // ragged end of a part
                 f2 ab[NP], bu[NP];
                 const float x = Io<IO>::widen(us[j * CPW + cl]);
-                const float dl = Io<IO>::widen(dsm[j * CPW + cl]);
+                const float dl = delta_at(j * CPW + cl);
                 if (SPLIT) {
                     ssum += dl;
                     dmin = fminf(dmin, dl);
@@ -749,6 +805,7 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
                 float yv = advance<NP>(h, ab, bu, Cs + j * N + n0);
 #pragma unroll
                 for (int o = 1; o < LPC; o <<= 1) yv += __shfl_xor_sync(0xffffffffu, yv, o);
+                if (FUSED) yv *= gsf[j * CPW + cl];
                 if (g == 0) Io<IO>::st(yp + j * ystr, yv);
             }
             if (SPLIT) dsum += static_cast<double>(ssum);
@@ -817,7 +874,7 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
             int64_t c, ts, te;
             part(k, c, ts, te);
             if (ts == 0) continue;
-            split_fixup<IO, Cfg>(P, c, ts, te, wk, lane);
+            split_fixup<IO, Cfg, FUSED>(P, c, ts, te, wk, lane);
         }
     }
     if (failed) {

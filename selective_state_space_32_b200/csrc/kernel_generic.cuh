@@ -26,7 +26,8 @@ __global__ void __launch_bounds__(kGenericThreads)
 sscan_generic_kernel(const IO *__restrict__ u, const IO *__restrict__ delta,
                  const float *__restrict__ A, const IO *__restrict__ Bm,
                  const IO *__restrict__ Cm, const float *h0, IO *__restrict__ y,
-                 float *h_final, int64_t L, int64_t D) {
+                 float *h_final, int64_t L, int64_t D, const float *__restrict__ delta_bias,
+                 const IO *__restrict__ z, int softplus) {
     constexpr int N = NL * LPC;
     constexpr int NP = NL / 2;  // packed pairs per thread
     constexpr int CPB = kGenericThreads / LPC;
@@ -69,6 +70,9 @@ sscan_generic_kernel(const IO *__restrict__ u, const IO *__restrict__ delta,
     const IO *cp = Cm + b * L * N + n0;
     IO *yp = y + b * L * D + dc;
     const bool writer = valid && g == 0;
+    // fused prologue / epilogue: delta <- softplus(delta + bias[d]), y <- y * silu(z)
+    const float biasv = delta_bias != nullptr ? __ldg(delta_bias + dc) : 0.0f;
+    const IO *zp = z != nullptr ? z + b * L * D + dc : nullptr;
 
     IO ubuf[kPrefetch], dbuf[kPrefetch];
 #pragma unroll
@@ -84,7 +88,8 @@ sscan_generic_kernel(const IO *__restrict__ u, const IO *__restrict__ delta,
             const int64_t t = t0 + k;
             if (t < L) {
                 const float x = Io<IO>::widen(ubuf[k]);
-                const float dl = Io<IO>::widen(dbuf[k]);
+                float dl = Io<IO>::widen(dbuf[k]) + biasv;
+                if (softplus) dl = softplus_f(dl);
                 if (t + kPrefetch < L) {
                     ubuf[k] = Io<IO>::ld(up + (t + kPrefetch) * D);
                     dbuf[k] = Io<IO>::ld(dp + (t + kPrefetch) * D);
@@ -120,7 +125,10 @@ sscan_generic_kernel(const IO *__restrict__ u, const IO *__restrict__ delta,
                 float yv = y0 + y1;
 #pragma unroll
                 for (int o = 1; o < LPC; o <<= 1) yv += __shfl_xor_sync(0xffffffffu, yv, o);
-                if (writer) Io<IO>::st(yp + t * D, yv);
+                if (writer) {
+                    if (zp != nullptr) yv *= silu_f(Io<IO>::widen(Io<IO>::ld(zp + t * D)));
+                    Io<IO>::st(yp + t * D, yv);
+                }
             }
         }
     }

@@ -81,7 +81,8 @@ constexpr int kMaxSmem = 227 * 1024;  // dynamic shared memory per block on B200
 constexpr int kLightPermille = 10;
 constexpr int64_t kMinChainedL = 64;  // shorter sequences use the generic kernel
 
-// Shared memory of a chained-kernel shape (mirrors ChainedCfg::kSmem).
+// Shared memory of a chained-kernel shape (mirrors ChainedCfg::kSmem; a fused call on a
+// shape whose larger ChainedCfg::kSmemF does not fit runs the generic kernel).
 int chained_smem_bytes(const KCfg &k, int es) {
     const int lpc = k.N / k.NL, cpw = 32 / lpc;
     const int kU = k.T * cpw * es, kB = k.T * k.N * es;
@@ -113,8 +114,8 @@ struct sscan_plan {
     size_t sink_off;                            // y sink of lanes past the last channel
     const void *last_ws;  // workspace whose flags were last cleared
     // tensor-map cache
-    const void *tm_ptr[4];
-    CUtensorMap tm[4];
+    const void *tm_ptr[5];
+    CUtensorMap tm[5];  // u, delta, B, C, gate z (z: fused calls with a gate; else a copy of u's)
     bool tm_valid;
     // generic kernel
     int g_nl, g_lpc;
@@ -242,32 +243,38 @@ void choose_schedule(sscan_plan *p) {
     }
 }
 
+// Arguments of the fused prologue / epilogue of one call.
+struct Fused {
+    const float *bias;  // [D] or null
+    const void *z;      // [B][L][D] gate or null
+    bool softplus;      // plan flag SSCAN_DELTA_SOFTPLUS
+    bool on() const { return bias != nullptr || z != nullptr || softplus; }
+};
+
 // ------------------------------------------------------------ generic launch
 
 template <class IO, int NL, int LPC>
 cudaError_t launch_generic_t(const sscan_plan *p, const void *u, const void *dl, const float *A,
                              const void *Bm, const void *Cm, const float *h0, void *y, float *hf,
-                             cudaStream_t s) {
+                             const Fused &fu, cudaStream_t s) {
     const dim3 grid(static_cast<unsigned>(ceil_div(p->D, kGenericThreads / LPC)), static_cast<unsigned>(p->B));
-    if (p->flags & SSCAN_ZOH)
-        sscan_generic_kernel<IO, NL, LPC, true><<<grid, kGenericThreads, 0, s>>>(
-            static_cast<const IO *>(u), static_cast<const IO *>(dl), A, static_cast<const IO *>(Bm),
-            static_cast<const IO *>(Cm), h0, static_cast<IO *>(y), hf, p->L, p->D);
-    else
-        sscan_generic_kernel<IO, NL, LPC, false><<<grid, kGenericThreads, 0, s>>>(
-            static_cast<const IO *>(u), static_cast<const IO *>(dl), A, static_cast<const IO *>(Bm),
-            static_cast<const IO *>(Cm), h0, static_cast<IO *>(y), hf, p->L, p->D);
+    auto kern = (p->flags & SSCAN_ZOH) ? sscan_generic_kernel<IO, NL, LPC, true>
+                                       : sscan_generic_kernel<IO, NL, LPC, false>;
+    kern<<<grid, kGenericThreads, 0, s>>>(
+        static_cast<const IO *>(u), static_cast<const IO *>(dl), A, static_cast<const IO *>(Bm),
+        static_cast<const IO *>(Cm), h0, static_cast<IO *>(y), hf, p->L, p->D, fu.bias,
+        static_cast<const IO *>(fu.z), fu.softplus ? 1 : 0);
     return cudaGetLastError();
 }
 
 template <class IO>
 cudaError_t launch_generic(const sscan_plan *p, const void *u, const void *dl, const float *A,
                            const void *Bm, const void *Cm, const float *h0, void *y, float *hf,
-                           cudaStream_t s) {
+                           const Fused &fu, cudaStream_t s) {
     switch (p->N) {
-        case 16: return launch_generic_t<IO, 8, 2>(p, u, dl, A, Bm, Cm, h0, y, hf, s);
-        case 32: return launch_generic_t<IO, 16, 2>(p, u, dl, A, Bm, Cm, h0, y, hf, s);
-        default: return launch_generic_t<IO, 16, 4>(p, u, dl, A, Bm, Cm, h0, y, hf, s);
+        case 16: return launch_generic_t<IO, 8, 2>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s);
+        case 32: return launch_generic_t<IO, 16, 2>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s);
+        default: return launch_generic_t<IO, 16, 4>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s);
     }
 }
 
@@ -292,30 +299,40 @@ bool encode_map(CUtensorMap *m, const void *ptr, int es, uint64_t inner, uint64_
     return r == CUDA_SUCCESS;
 }
 
-template <class IO, int CFG, bool ZOH, bool POLY, bool SPLIT>
+template <class IO, int CFG, bool ZOH, bool POLY, bool SPLIT, bool FUSED>
 int launch_chained_t(sscan_plan *p, const void *u, const void *dl, const float *A, const void *Bm,
-                     const void *Cm, const float *h0, void *y, float *hf, void *ws, cudaStream_t s) {
+                     const void *Cm, const float *h0, void *y, float *hf, void *ws, const Fused &fu,
+                     cudaStream_t s) {
     constexpr KCfg k = kChainedCfgs[CFG];
     using Cfg = ChainedCfg<IO, k.N, k.NL, k.T, k.STAGES, k.WPC>;
-    auto kern = sscan_chained_kernel<IO, Cfg, ZOH, POLY, SPLIT>;
+    if constexpr (FUSED && Cfg::kSmemF > kMaxSmem) {
+        // the fused stage ring of this shape does not fit: the generic kernel serves the call
+        (void)ws;
+        return launch_generic<IO>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s) == cudaSuccess ? SSCAN_OK
+                                                                                       : SSCAN_ERR_CUDA;
+    } else {
+    constexpr int smem_bytes = FUSED ? Cfg::kSmemF : Cfg::kSmem;
+    auto kern = sscan_chained_kernel<IO, Cfg, ZOH, POLY, SPLIT, FUSED>;
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [&] {
-        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
     });
     if (attr_err != cudaSuccess) return SSCAN_ERR_CUDA;
 
     const int es = sizeof(IO);
-    const void *ptrs[4] = {u, dl, Bm, Cm};
+    const void *ptrs[5] = {u, dl, Bm, Cm, fu.z};
     if (!p->tm_valid || memcmp(ptrs, p->tm_ptr, sizeof ptrs) != 0) {
         const uint64_t rows = static_cast<uint64_t>(p->B * p->L);
         if (!encode_map(&p->tm[0], u, es, p->D, rows, Cfg::CPW, Cfg::T) ||
             !encode_map(&p->tm[1], dl, es, p->D, rows, Cfg::CPW, Cfg::T) ||
             !encode_map(&p->tm[2], Bm, es, p->N, rows, p->N, Cfg::T) ||
-            !encode_map(&p->tm[3], Cm, es, p->N, rows, p->N, Cfg::T)) {
+            !encode_map(&p->tm[3], Cm, es, p->N, rows, p->N, Cfg::T) ||
+            (fu.z != nullptr && !encode_map(&p->tm[4], fu.z, es, p->D, rows, Cfg::CPW, Cfg::T))) {
             p->tm_valid = false;
             return SSCAN_ERR_CUDA;
         }
+        if (fu.z == nullptr) p->tm[4] = p->tm[0];  // never loaded (the kernel sees no gate)
         memcpy(p->tm_ptr, ptrs, sizeof ptrs);
         p->tm_valid = true;
     }
@@ -352,40 +369,54 @@ int launch_chained_t(sscan_plan *p, const void *u, const void *dl, const float *
     prm.seg = p->seg;
     prm.seg_shift = p->seg_shift;
     prm.wpc = k.WPC;
-    void *args[] = {&p->tm[0], &p->tm[1], &p->tm[2], &p->tm[3], &prm};
+    prm.delta_bias = fu.bias;
+    prm.z = fu.z;
+    prm.softplus = fu.softplus ? 1 : 0;
+    void *args[] = {&p->tm[0], &p->tm[1], &p->tm[2], &p->tm[3], &p->tm[4], &prm};
     const dim3 grid(static_cast<unsigned>(p->workers / k.WPC)), block(Cfg::kThreads);
     const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kern), grid, block, args,
-                                                      Cfg::kSmem, s);
+                                                      smem_bytes, s);
     return e == cudaSuccess ? SSCAN_OK : SSCAN_ERR_CUDA;
+    }
 }
 
+// Fused calls (bias, softplus or gate) take the FUSED kernels, which keep every
+// exponent on the MUFU pipe.
 template <class IO, int CFG, bool SPLIT>
 int launch_chained_mode(sscan_plan *p, const void *u, const void *dl, const float *A, const void *Bm,
-                        const void *Cm, const float *h0, void *y, float *hf, void *ws, cudaStream_t s) {
-    if (p->flags & SSCAN_ZOH)
-        return launch_chained_t<IO, CFG, true, false, SPLIT>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
-    if (p->poly) return launch_chained_t<IO, CFG, false, true, SPLIT>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
-    return launch_chained_t<IO, CFG, false, false, SPLIT>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
+                        const void *Cm, const float *h0, void *y, float *hf, void *ws, const Fused &fu,
+                        cudaStream_t s) {
+    const bool zoh = (p->flags & SSCAN_ZOH) != 0;
+    if (fu.on())
+        return zoh ? launch_chained_t<IO, CFG, true, false, SPLIT, true>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s)
+                   : launch_chained_t<IO, CFG, false, false, SPLIT, true>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s);
+    if (zoh)
+        return launch_chained_t<IO, CFG, true, false, SPLIT, false>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s);
+    if (p->poly)
+        return launch_chained_t<IO, CFG, false, true, SPLIT, false>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s);
+    return launch_chained_t<IO, CFG, false, false, SPLIT, false>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s);
 }
 
 template <class IO, int CFG>
 int launch_chained_cfg(sscan_plan *p, const void *u, const void *dl, const float *A, const void *Bm,
-                       const void *Cm, const float *h0, void *y, float *hf, void *ws, cudaStream_t s) {
-    return p->split ? launch_chained_mode<IO, CFG, true>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s)
-                    : launch_chained_mode<IO, CFG, false>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
+                       const void *Cm, const float *h0, void *y, float *hf, void *ws, const Fused &fu,
+                       cudaStream_t s) {
+    return p->split ? launch_chained_mode<IO, CFG, true>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s)
+                    : launch_chained_mode<IO, CFG, false>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s);
 }
 
 template <class IO>
 int launch_chained(sscan_plan *p, const void *u, const void *dl, const float *A, const void *Bm,
-                   const void *Cm, const float *h0, void *y, float *hf, void *ws, cudaStream_t s) {
+                   const void *Cm, const float *h0, void *y, float *hf, void *ws, const Fused &fu,
+                   cudaStream_t s) {
     switch (p->cfg) {
-        case 0: return launch_chained_cfg<IO, 0>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
-        case 1: return launch_chained_cfg<IO, 1>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
-        case 2: return launch_chained_cfg<IO, 2>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
-        case 3: return launch_chained_cfg<IO, 3>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
-        case 4: return launch_chained_cfg<IO, 4>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
-        case 5: return launch_chained_cfg<IO, 5>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
-        case 6: return launch_chained_cfg<IO, 6>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, s);
+        case 0: return launch_chained_cfg<IO, 0>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s);
+        case 1: return launch_chained_cfg<IO, 1>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s);
+        case 2: return launch_chained_cfg<IO, 2>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s);
+        case 3: return launch_chained_cfg<IO, 3>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s);
+        case 4: return launch_chained_cfg<IO, 4>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s);
+        case 5: return launch_chained_cfg<IO, 5>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s);
+        case 6: return launch_chained_cfg<IO, 6>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s);
         default: return SSCAN_ERR_UNSUPPORTED;
     }
 }
@@ -449,7 +480,7 @@ int sscan_plan_create(sscan_plan_t *plan, int64_t B, int64_t L, int64_t D, int64
     if (B < 1 || D < 1 || L < 0) return SSCAN_ERR_INVALID;
     if (B > 65535 || D > (int64_t(1) << 31) || L > (int64_t(1) << 40)) return SSCAN_ERR_UNSUPPORTED;
     if (dtype != SSCAN_F32 && dtype != SSCAN_BF16) return SSCAN_ERR_INVALID;
-    if (flags & ~static_cast<uint32_t>(SSCAN_ZOH)) return SSCAN_ERR_INVALID;
+    if (flags & ~static_cast<uint32_t>(SSCAN_ZOH | SSCAN_DELTA_SOFTPLUS)) return SSCAN_ERR_INVALID;
     if (N != 16 && N != 32 && N != 64) return SSCAN_ERR_UNSUPPORTED;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return SSCAN_ERR_UNSUPPORTED;
@@ -524,6 +555,12 @@ int sscan_plan_describe(sscan_plan_t plan, char *buf, size_t len) {
 int sscan_forward(sscan_plan_t plan, const void *u, const void *delta, const float *A,
                   const void *B, const void *C, const float *h0, void *y, float *h_final,
                   void *workspace, void *stream) {
+    return sscan_forward_gated(plan, u, delta, A, B, C, h0, nullptr, nullptr, y, h_final, workspace, stream);
+}
+
+int sscan_forward_gated(sscan_plan_t plan, const void *u, const void *delta, const float *A,
+                        const void *B, const void *C, const float *h0, const float *delta_bias,
+                        const void *z, void *y, float *h_final, void *workspace, void *stream) {
     if (!plan) return SSCAN_ERR_INVALID;
     sscan_plan *p = plan;
     const size_t es = p->dtype == SSCAN_F32 ? 4 : 2;
@@ -534,16 +571,18 @@ int sscan_forward(sscan_plan_t plan, const void *u, const void *delta, const flo
     if (!A) return SSCAN_ERR_INVALID;
     if (n_bld && (!u || !delta || !y)) return SSCAN_ERR_INVALID;
     if (n_bln && (!B || !C)) return SSCAN_ERR_INVALID;
-    const void *ptrs[] = {u, delta, A, B, C, h0, y, h_final};
+    const void *ptrs[] = {u, delta, A, B, C, h0, y, h_final, delta_bias, z};
     for (const void *q : ptrs)
         if (q && !aligned16(q)) return SSCAN_ERR_ALIGN;
     // y must not overlap any input; h_final may equal h0 but not overlap anything else
-    const void *ins[] = {u, delta, A, B, C, h0};
-    const size_t insz[] = {n_bld * es, n_bld * es, n_dn * 4, n_bln * es, n_bln * es, n_bdn * 4};
-    for (int i = 0; i < 6; ++i) {
+    const void *ins[] = {u, delta, A, B, C, delta_bias, z, h0};
+    const size_t insz[] = {n_bld * es, n_bld * es, n_dn * 4, n_bln * es, n_bln * es,
+                           static_cast<size_t>(p->D) * 4, n_bld * es, n_bdn * 4};
+    for (int i = 0; i < 8; ++i) {
         if (overlaps(y, n_bld * es, ins[i], insz[i])) return SSCAN_ERR_INVALID;
-        if (i < 5 && overlaps(h_final, n_bdn * 4, ins[i], insz[i])) return SSCAN_ERR_INVALID;
+        if (i < 7 && overlaps(h_final, n_bdn * 4, ins[i], insz[i])) return SSCAN_ERR_INVALID;
     }
+    const Fused fu{delta_bias, z, (p->flags & SSCAN_DELTA_SOFTPLUS) != 0};
     if (h0 && h_final && h0 != h_final && overlaps(h_final, n_bdn * 4, h0, n_bdn * 4))
         return SSCAN_ERR_INVALID;
     if (overlaps(h_final, n_bdn * 4, y, n_bld * es)) return SSCAN_ERR_INVALID;
@@ -551,17 +590,17 @@ int sscan_forward(sscan_plan_t plan, const void *u, const void *delta, const flo
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (p->mode == kChained) {
         if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SSCAN_ERR_WORKSPACE;
-        const size_t sz[8] = {n_bld * es, n_bld * es, n_dn * 4, n_bln * es,
-                              n_bln * es, n_bdn * 4, n_bld * es, n_bdn * 4};
-        for (int i = 0; i < 8; ++i)
+        const size_t sz[10] = {n_bld * es, n_bld * es, n_dn * 4, n_bln * es, n_bln * es,
+                               n_bdn * 4, n_bld * es, n_bdn * 4, static_cast<size_t>(p->D) * 4, n_bld * es};
+        for (int i = 0; i < 10; ++i)
             if (overlaps(workspace, p->ws_bytes, ptrs[i], sz[i])) return SSCAN_ERR_WORKSPACE;
         return p->dtype == SSCAN_F32
-                   ? launch_chained<float>(p, u, delta, A, B, C, h0, y, h_final, workspace, s)
-                   : launch_chained<uint16_t>(p, u, delta, A, B, C, h0, y, h_final, workspace, s);
+                   ? launch_chained<float>(p, u, delta, A, B, C, h0, y, h_final, workspace, fu, s)
+                   : launch_chained<uint16_t>(p, u, delta, A, B, C, h0, y, h_final, workspace, fu, s);
     }
     const cudaError_t e =
-        p->dtype == SSCAN_F32 ? launch_generic<float>(p, u, delta, A, B, C, h0, y, h_final, s)
-                              : launch_generic<uint16_t>(p, u, delta, A, B, C, h0, y, h_final, s);
+        p->dtype == SSCAN_F32 ? launch_generic<float>(p, u, delta, A, B, C, h0, y, h_final, fu, s)
+                              : launch_generic<uint16_t>(p, u, delta, A, B, C, h0, y, h_final, fu, s);
     return e == cudaSuccess ? SSCAN_OK : SSCAN_ERR_CUDA;
 }
 
@@ -583,7 +622,7 @@ int sscan_forward_noalloc(int64_t B, int64_t L, int64_t D, int64_t N, int dtype,
     if (B < 1 || D < 1 || L < 0) return SSCAN_ERR_INVALID;
     if (B > 65535 || D > (int64_t(1) << 31) || L > (int64_t(1) << 40)) return SSCAN_ERR_UNSUPPORTED;
     if (dtype != SSCAN_F32 && dtype != SSCAN_BF16) return SSCAN_ERR_INVALID;
-    if (flags & ~static_cast<uint32_t>(SSCAN_ZOH)) return SSCAN_ERR_INVALID;
+    if (flags & ~static_cast<uint32_t>(SSCAN_ZOH | SSCAN_DELTA_SOFTPLUS)) return SSCAN_ERR_INVALID;
     if (N != 16 && N != 32 && N != 64) return SSCAN_ERR_UNSUPPORTED;
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return SSCAN_ERR_UNSUPPORTED;

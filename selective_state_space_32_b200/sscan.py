@@ -18,11 +18,12 @@ LIB_PATH = os.path.join(_HERE, "libsscan.so")
 
 F32, BF16 = 0, 1
 ZOH = 1
+DELTA_SOFTPLUS = 2
 OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(7)
 
 SYMBOLS = ("sscan_plan_create", "sscan_plan_destroy", "sscan_workspace_bytes", "sscan_forward",
            "sscan_get_status", "sscan_status_string", "sscan_plan_describe", "sscan_version",
-           "sscan_forward_noalloc")
+           "sscan_forward_noalloc", "sscan_forward_gated")
 
 
 class SscanError(RuntimeError):
@@ -64,6 +65,8 @@ def lib() -> ctypes.CDLL:
             L.sscan_version.restype = ip
             L.sscan_forward_noalloc.argtypes = [i64, i64, i64, i64, ip, u32] + [vp] * 9
             L.sscan_forward_noalloc.restype = ip
+            L.sscan_forward_gated.argtypes = [vp] * 13
+            L.sscan_forward_gated.restype = ip
             _lib = L
     return _lib
 
@@ -85,16 +88,17 @@ def _ptr(t: Optional[torch.Tensor]):
 
 
 class Plan:
-    """A sscan_plan for one (B, L, D, N, dtype, zoh) shape on the current device."""
+    """A sscan_plan for one (B, L, D, N, dtype, zoh, delta_softplus) shape on the current device."""
 
     def __init__(self, B: int, L: int, D: int, N: int, dtype: torch.dtype = torch.float32,
-                 zoh: bool = False):
+                 zoh: bool = False, delta_softplus: bool = False):
         self.shape = (int(B), int(L), int(D), int(N))
         self.dtype = dtype
         self.zoh = bool(zoh)
+        self.delta_softplus = bool(delta_softplus)
         h = ctypes.c_void_p()
         rc = lib().sscan_plan_create(ctypes.byref(h), *self.shape, _dtype_code(dtype),
-                                     ZOH if zoh else 0)
+                                     (ZOH if zoh else 0) | (DELTA_SOFTPLUS if delta_softplus else 0))
         if rc != OK:
             raise SscanError(rc, "sscan_plan_create")
         self._h = h
@@ -122,8 +126,12 @@ class Plan:
         return torch.empty(self.workspace_bytes, dtype=torch.uint8, device=device or "cuda")
 
     def forward(self, u, delta, A, B, C, h0=None, y=None, h_final=None, workspace=None,
-                want_final: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-        """Enqueue the forward on ``stream`` (default: torch's current stream)."""
+                want_final: bool = True, stream=None, delta_bias=None,
+                z=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+        """Enqueue the forward on ``stream`` (default: torch's current stream).
+
+        delta_bias ([D] float32) and z ([B, L, D], plan dtype) select the fused
+        prologue / epilogue (``sscan_forward_gated``)."""
         Bt, L, D, N = self.shape
         if y is None:
             y = torch.empty((Bt, L, D), dtype=self.dtype, device=u.device)
@@ -136,7 +144,9 @@ class Plan:
                                    ("C", C, (Bt, L, N), self.dtype),
                                    ("h0", h0, (Bt, D, N), torch.float32),
                                    ("y", y, (Bt, L, D), self.dtype),
-                                   ("h_final", h_final, (Bt, D, N), torch.float32)):
+                                   ("h_final", h_final, (Bt, D, N), torch.float32),
+                                   ("delta_bias", delta_bias, (D,), torch.float32),
+                                   ("z", z, (Bt, L, D), self.dtype)):
             if t is None:
                 continue
             if tuple(t.shape) != shape or t.dtype != dt or not t.is_cuda or not t.is_contiguous():
@@ -146,11 +156,18 @@ class Plan:
             workspace = self.new_workspace(u.device)
         if stream is None:
             stream = torch.cuda.current_stream(u.device)
-        rc = lib().sscan_forward(self._h, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
-                                 _ptr(h0), _ptr(y), _ptr(h_final), _ptr(workspace),
-                                 ctypes.c_void_p(stream.cuda_stream))
+        if delta_bias is None and z is None:
+            rc = lib().sscan_forward(self._h, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+                                     _ptr(h0), _ptr(y), _ptr(h_final), _ptr(workspace),
+                                     ctypes.c_void_p(stream.cuda_stream))
+            what = "sscan_forward"
+        else:
+            rc = lib().sscan_forward_gated(self._h, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+                                           _ptr(h0), _ptr(delta_bias), _ptr(z), _ptr(y), _ptr(h_final),
+                                           _ptr(workspace), ctypes.c_void_p(stream.cuda_stream))
+            what = "sscan_forward_gated"
         if rc != OK:
-            raise SscanError(rc, "sscan_forward")
+            raise SscanError(rc, what)
         return y, h_final
 
     def status(self, stream=None) -> int:
@@ -163,28 +180,32 @@ class Plan:
 _plans: dict = {}
 
 
-def get_plan(B, L, D, N, dtype=torch.float32, zoh=False) -> Plan:
-    key = (int(B), int(L), int(D), int(N), dtype, bool(zoh), torch.cuda.current_device())
+def get_plan(B, L, D, N, dtype=torch.float32, zoh=False, delta_softplus=False) -> Plan:
+    key = (int(B), int(L), int(D), int(N), dtype, bool(zoh), bool(delta_softplus),
+           torch.cuda.current_device())
     p = _plans.get(key)
     if p is None:
-        p = _plans[key] = Plan(B, L, D, N, dtype, zoh)
+        p = _plans[key] = Plan(B, L, D, N, dtype, zoh, delta_softplus)
     return p
 
 
-def forward(u, delta, A, B, C, h0=None, zoh: bool = False, want_final: bool = True):
+def forward(u, delta, A, B, C, h0=None, zoh: bool = False, want_final: bool = True,
+            delta_bias=None, delta_softplus: bool = False, z=None):
     """Selective-scan forward on CUDA tensors: returns (y [B,L,D], h_final [B,D,N] or None).
 
     u, delta: [B, L, D] float32 or bfloat16; A: [D, N] float32; B, C: [B, L, N]
-    (dtype of u); h0: [B, D, N] float32 or None.
+    (dtype of u); h0: [B, D, N] float32 or None.  Fused prologue / epilogue:
+    delta_bias [D] float32 and delta_softplus (delta <- softplus(delta + bias)),
+    z [B, L, D] (dtype of u; y <- y * silu(z)).
     """
     Bt, L, D = u.shape
     N = A.shape[1]
-    return get_plan(Bt, L, D, N, u.dtype, zoh).forward(u, delta, A, B, C, h0,
-                                                        want_final=want_final)
+    return get_plan(Bt, L, D, N, u.dtype, zoh, delta_softplus).forward(
+        u, delta, A, B, C, h0, want_final=want_final, delta_bias=delta_bias, z=z)
 
 
 def forward_host(u, delta, A, B, C, h0=None, zoh: bool = False, device="cuda", out=None,
-                 chunks: int = 2):
+                 chunks: int = 2, delta_bias=None, delta_softplus: bool = False, z=None):
     """Forward on host (CPU) tensors: copies the inputs to the device, runs the scan
     and copies y and h_final back, then waits for the copies.
 
@@ -192,7 +213,8 @@ def forward_host(u, delta, A, B, C, h0=None, zoh: bool = False, device="cuda", o
     flow through two streams: a piece's host-to-device copy overlaps the previous
     piece's scan and device-to-host copy (the transfer, not the scan, bounds this
     path).  Pinned host tensors are needed for the copies to be asynchronous;
-    ``out`` = (y_host, h_final_host) reuses output buffers.
+    ``out`` = (y_host, h_final_host) reuses output buffers; delta_bias, delta_softplus
+    and z select the fused prologue / epilogue (z is cut like u).
     Returns (y_host, h_final_host)."""
     dev = torch.device(device)
     Bt, L, D = u.shape
@@ -206,6 +228,7 @@ def forward_host(u, delta, A, B, C, h0=None, zoh: bool = False, device="cuda", o
     main = torch.cuda.current_stream(dev)
     streams = [torch.cuda.Stream(dev) for _ in range(min(2, n))]
     A_d = A.to(dev, non_blocking=True)
+    bias_d = None if delta_bias is None else delta_bias.to(dev, non_blocking=True)
     for st in streams:
         st.wait_stream(main)
     for i in range(n):
@@ -213,12 +236,13 @@ def forward_host(u, delta, A, B, C, h0=None, zoh: bool = False, device="cuda", o
         st = streams[i % len(streams)]
         with torch.cuda.stream(st):
             dv = [None if t is None else t[b0:b1].to(dev, non_blocking=True)
-                  for t in (u, delta, B, C, h0)]
-            plan = get_plan(b1 - b0, L, D, N, u.dtype, zoh)
-            y, hf = plan.forward(dv[0], dv[1], A_d, dv[2], dv[3], dv[4], stream=st)
+                  for t in (u, delta, B, C, h0, z)]
+            plan = get_plan(b1 - b0, L, D, N, u.dtype, zoh, delta_softplus)
+            y, hf = plan.forward(dv[0], dv[1], A_d, dv[2], dv[3], dv[4], stream=st,
+                                 delta_bias=bias_d, z=dv[5])
             out[0][b0:b1].copy_(y, non_blocking=True)
             out[1][b0:b1].copy_(hf, non_blocking=True)
-            for t in (*dv, y, hf):  # keep the caching allocator from reusing them early
+            for t in (*dv, y, hf, bias_d):  # keep the caching allocator from reusing them early
                 if t is not None:
                     t.record_stream(st)
     for st in streams:

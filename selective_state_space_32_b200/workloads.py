@@ -17,7 +17,12 @@ Distributions (the same for every workload unless noted):
   * A = -exp(A_log) with A_log[d, n] = log(n + 1) (S4D-real), so A[d, n] = -(n + 1),
   * h0 ~ N(0, 0.1^2) where a workload has a nonzero initial state,
   * the long-sequence workload marks round(0.32 L) time positions per batch row
-    as reset tokens (delta + 3) and scales delta by 0.01 elsewhere.
+    as reset tokens (delta + 3) and scales delta by 0.01 elsewhere,
+  * fused workloads (the kernel applies delta <- softplus(delta + bias) and
+    y <- y * silu(z) itself) store the raw delta 0.5 z and the per-channel
+    bias softplus^-1(dt[d]) (fp32), so the effective delta has the same
+    distribution as above; their gate z ~ N(0, 1) is drawn after everything
+    else.
 
 Draw order from numpy PCG64(seed): dt, reset mask, z, u, B, C, h0, all fp64 in
 C order.  Values are then rounded to fp32 (numpy, round-to-nearest-even) and,
@@ -46,6 +51,7 @@ class Workload:
     zoh: bool             # exact zero-order-hold input term instead of Euler
     reset_frac: float     # fraction of time positions that are reset tokens (0: none)
     index: int            # seed offset
+    fused: bool = False   # raw delta + bias + gate z (the kernel's fused prologue / epilogue)
 
     @property
     def elements(self) -> int:
@@ -66,11 +72,12 @@ class Workload:
         A ([D,N] fp32), h_final and, when given, h0 ([B,D,N] fp32)."""
         s = self.itemsize
         return (3 * s * self.B * self.L * self.D + 2 * s * self.B * self.L * self.N
-                + 4 * self.D * self.N + 4 * self.B * self.D * self.N * (1 + (self.h0_std > 0)))
+                + 4 * self.D * self.N + 4 * self.B * self.D * self.N * (1 + (self.h0_std > 0))
+                + (s * self.B * self.L * self.D + 4 * self.D if self.fused else 0))
 
     def shape_dict(self) -> dict:
         return {"B": self.B, "L": self.L, "D": self.D, "N": self.N, "dtype": self.dtype,
-                "h0": self.h0_std > 0, "zoh": self.zoh}
+                "h0": self.h0_std > 0, "zoh": self.zoh, "fused": self.fused}
 
 
 WORKLOADS = {
@@ -82,6 +89,11 @@ WORKLOADS = {
     # one decode step (a single token per sequence, state carried in and out) for a
     # batch of 256 sequences of a layer with D = 2048, N = 16
     "decode_b256_f32": Workload("decode_b256_f32", 256, 1, 2048, 16, "f32", 0.1, False, 0.0, 5),
+    # the bench shape with the Mamba block's softplus(delta + bias) and silu(z) gate fused
+    "mamba130m_fused_f32": Workload("mamba130m_fused_f32", 8, 2048, 1536, 16, "f32", 0.0, False, 0.0, 6,
+                                    fused=True),
+    "mamba1p4b_fused_bf16": Workload("mamba1p4b_fused_bf16", 2, 8192, 4096, 16, "bf16", 0.1, False, 0.0, 7,
+                                     fused=True),
 }
 ORDER = ["tiny_f32", "mamba130m_f32", "mamba1p4b_bf16", "longseq_bf16", "zoh_n64_bf16"]
 
@@ -119,16 +131,18 @@ def _inv_softplus(y):
 
 def generate(B: int, L: int, D: int, N: int, dtype: str = "f32", h0_std: float = 0.0,
              reset_frac: float = 0.0, seed: int = SEED_BASE, A_jitter: float = 0.0,
-             block: int = 1 << 22) -> dict:
+             block: int = 1 << 22, fused: bool = False) -> dict:
     """Seeded inputs of the given shape (see the module docstring for the recipe).
 
     A_jitter > 0 adds N(0, A_jitter^2) to A_log (drawn last), so tests can use
     a non-integer A.  Large arrays are drawn in blocks of ``block`` values; the
     stream is the same as a single draw.
     Returns a dict with u, delta ([B,L,D]), A ([D,N] fp32), B, C ([B,L,N]),
-    h0 ([B,D,N] fp32 or None) and dtype.
+    h0 ([B,D,N] fp32 or None) and dtype; with ``fused`` also delta_bias ([D]
+    fp32) and z ([B,L,D]), and delta is the raw (pre-softplus) value.
     """
     assert dtype in ("f32", "bf16")
+    assert not (fused and reset_frac > 0)
     rng = np.random.Generator(np.random.PCG64(seed))
     dt = np.exp(rng.uniform(math.log(1e-3), math.log(1e-1), size=D))
     reset = None
@@ -138,6 +152,7 @@ def generate(B: int, L: int, D: int, N: int, dtype: str = "f32", h0_std: float =
         for b in range(B):
             reset[b, rng.permutation(L)[:k]] = True
     bias = _inv_softplus(dt)
+    bias32 = bias.astype(np.float32)
 
     total = B * L * D
     sdt = np.uint16 if dtype == "bf16" else np.float32
@@ -147,7 +162,7 @@ def generate(B: int, L: int, D: int, N: int, dtype: str = "f32", h0_std: float =
         z = rng.standard_normal(e - s)
         idx = np.arange(s, e)
         d = idx % D
-        v = _softplus(0.5 * z + bias[d])
+        v = 0.5 * z if fused else _softplus(0.5 * z + bias[d])
         if reset is not None:
             bt = idx // D
             r = reset.reshape(-1)[bt]
@@ -166,10 +181,19 @@ def generate(B: int, L: int, D: int, N: int, dtype: str = "f32", h0_std: float =
     if A_jitter > 0:
         A_log = A_log + A_jitter * rng.standard_normal((D, N))
     A = (-np.exp(A_log)).astype(np.float32)
-    return {"u": u.reshape(B, L, D), "delta": delta.reshape(B, L, D), "A": A,
-            "B": Bm, "C": Cm, "h0": h0, "dtype": dtype}
+    out = {"u": u.reshape(B, L, D), "delta": delta.reshape(B, L, D), "A": A,
+           "B": Bm, "C": Cm, "h0": h0, "dtype": dtype, "delta_bias": None, "z": None}
+    if fused:
+        out["delta_bias"] = bias32
+        zg = np.empty(B * L * D, dtype=sdt)
+        for s in range(0, B * L * D, block):
+            e = min(B * L * D, s + block)
+            zg[s:e] = _store(rng.standard_normal(e - s), dtype)
+        out["z"] = zg.reshape(B, L, D)
+    return out
 
 
 def make_inputs(w: Workload) -> dict:
     """Inputs of a named workload, seeded with SEED_BASE + its index."""
-    return generate(w.B, w.L, w.D, w.N, w.dtype, w.h0_std, w.reset_frac, SEED_BASE + w.index)
+    return generate(w.B, w.L, w.D, w.N, w.dtype, w.h0_std, w.reset_frac, SEED_BASE + w.index,
+                    fused=w.fused)

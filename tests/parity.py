@@ -29,26 +29,31 @@ def to_device(g, device="cuda"):
         return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(device)
     dt = g["dtype"]
     return {"u": t(g["u"], dt), "delta": t(g["delta"], dt), "A": t(g["A"], "f32"),
-            "B": t(g["B"], dt), "C": t(g["C"], dt), "h0": t(g["h0"], "f32")}
+            "B": t(g["B"], dt), "C": t(g["C"], dt), "h0": t(g["h0"], "f32"),
+            "delta_bias": t(g.get("delta_bias"), "f32"), "z": t(g.get("z"), dt)}
 
 
 def host_values(g):
     """The exact fp32 values of every generated input (bf16 widened)."""
     dt = g["dtype"]
+    z = g.get("z")
     return {"u": W.as_f32(g["u"], dt), "delta": W.as_f32(g["delta"], dt), "A": g["A"],
-            "B": W.as_f32(g["B"], dt), "C": W.as_f32(g["C"], dt), "h0": g["h0"]}
+            "B": W.as_f32(g["B"], dt), "C": W.as_f32(g["C"], dt), "h0": g["h0"],
+            "delta_bias": g.get("delta_bias"), "z": None if z is None else W.as_f32(z, dt)}
 
 
-def run_gpu(g, zoh=False, device="cuda"):
+def run_gpu(g, zoh=False, device="cuda", softplus=False):
     d = to_device(g, device)
-    y, hf = S.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"], zoh=zoh)
+    y, hf = S.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"], zoh=zoh,
+                      delta_bias=d["delta_bias"], delta_softplus=softplus, z=d["z"])
     torch.cuda.synchronize()
     return y.float().cpu().numpy(), hf.cpu().numpy()
 
 
-def run_oracle(g, zoh=False):
+def run_oracle(g, zoh=False, softplus=False):
     v = host_values(g)
-    return O.forward(v["u"], v["delta"], v["A"], v["B"], v["C"], v["h0"], zoh)
+    return O.forward(v["u"], v["delta"], v["A"], v["B"], v["C"], v["h0"], zoh,
+                     delta_bias=v["delta_bias"], softplus=softplus, z=v["z"])
 
 
 def rel_l2(got, ref):

@@ -57,3 +57,19 @@ def test_workload_table():
     assert W.WORKLOADS["mamba1p4b_bf16"].algorithmic_bytes() == 405012480
     assert W.WORKLOADS["longseq_bf16"].algorithmic_bytes() == 1619394560
     assert W.WORKLOADS["zoh_n64_bf16"].algorithmic_bytes() == 529793024
+
+
+def test_fused_generator_matches_the_unfused_recipe():
+    # same seed: u, B, C, h0 identical; softplus(raw delta + bias) is the unfused delta
+    # up to the fp32 rounding of the raw value and of the bias
+    a = W.generate(2, 40, 24, 16, "f32", 0.1, seed=77)
+    b = W.generate(2, 40, 24, 16, "f32", 0.1, seed=77, fused=True)
+    for k in ("u", "B", "C", "h0", "A"):
+        assert np.array_equal(a[k], b[k]), k
+    s = b["delta"].astype(np.float64) + b["delta_bias"].astype(np.float64)[None, None, :]
+    eff = np.maximum(s, 0.0) + np.log1p(np.exp(-np.abs(s)))
+    assert np.allclose(eff, a["delta"], rtol=2e-6, atol=0)
+    assert b["z"].shape == (2, 40, 24) and b["delta_bias"].dtype == np.float32
+    assert a["z"] is None and a["delta_bias"] is None
+    w = W.WORKLOADS["mamba130m_fused_f32"]
+    assert w.algorithmic_bytes() == W.WORKLOADS["mamba130m_f32"].algorithmic_bytes() + 4 * 8 * 2048 * 1536 + 4 * 1536
