@@ -97,6 +97,15 @@ struct ChainedCfg {
     static constexpr int kDsf = T * CPW * 4;
     static constexpr int kWarpF = ((STAGES * kStageF + kConv + 2 * kDsf) + 127) / 128 * 128;
     static constexpr int kSmemF = WPC * kWarpF + kBars;
+    // fused kernels of 4-consumer shapes: one helper warp per consumer, on the same SM
+    // sub-partition, computes those two tiles for every stage into a ring of STAGES
+    // (the consumer's MUFU pipe is idle during its state updates; a ninth warp fits the
+    // register file at the consumer's register count)
+    static constexpr int kWarpH = ((STAGES * kStageF + kConv + 2 * STAGES * kDsf) + 127) / 128 * 128;
+    static constexpr int kBarsH = (3 * WPC * STAGES * 8 + 127) / 128 * 128;  // full, empty, ready
+    static constexpr int kSmemH = WPC * kWarpH + kBarsH;
+    static constexpr int kThreadsH = (2 * WPC + 1) * 32;
+    static constexpr bool kHelp = WPC == 4 && kSmemH <= 227 * 1024;
     static constexpr int kThreads = (WPC + 1) * 32;  // WPC consumer warps + 1 producer warp
     static_assert(LPC >= 1 && LPC <= 8 && N % NL == 0 && NL % 4 == 0, "bad split");
     static_assert(CPW * ES % 16 == 0 && N * ES % 16 == 0, "TMA rows must be 16-byte multiples");
@@ -436,6 +445,73 @@ __device__ __noinline__ void split_fixup(const ChainedParams &P, int64_t c, int6
     }
 }
 
+// The fused per-stage transform of one [T][CPW] tile: delta' = softplus(delta + bias)
+// (or delta + bias) and silu(z) (or 1) in fp32, lane-strided entries (entry i is
+// channel i % CPW, the same for every entry of a lane since 32 is a multiple of CPW).
+// A fixed trip count keeps the independent exponentials in flight together.
+template <class IO, class Cfg>
+__device__ __forceinline__ void fused_tile(const IO *dsm, const IO *zs, float *dsf, float *gsf, float biasv,
+                                           bool softplus, bool gate, int lane) {
+    constexpr int kPer = Cfg::T * Cfg::CPW / 32;
+    static_assert(Cfg::T * Cfg::CPW % 32 == 0, "tile entries per lane");
+    if (softplus) {
+#pragma unroll
+        for (int k = 0; k < kPer; ++k)
+            dsf[lane + 32 * k] = softplus_f(Io<IO>::widen(dsm[lane + 32 * k]) + biasv);
+    } else {
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) dsf[lane + 32 * k] = Io<IO>::widen(dsm[lane + 32 * k]) + biasv;
+    }
+    if (gate) {
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) gsf[lane + 32 * k] = silu_f(Io<IO>::widen(zs[lane + 32 * k]));
+    } else {
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) gsf[lane + 32 * k] = 1.0f;
+    }
+}
+
+// Helper warp j (fused 4-consumer shapes): walks consumer j's stages in its order,
+// waits for each stage to land, writes its transformed tiles into ring slot s and
+// arrives on ready[s].  It never runs more than a ring ahead: a slot is refilled
+// only after the consumer has released it.  Every wait is bounded.
+template <class IO, class Cfg>
+__device__ __forceinline__ void help(const ChainedParams &P, unsigned char *smem, uint64_t *full,
+                                     uint64_t *ready, int j, int lane) {
+    constexpr int T = Cfg::T, STAGES = Cfg::STAGES, CPW = Cfg::CPW;
+    const int64_t L = P.L, D = P.D;
+    const Segment sg(static_cast<int64_t>(blockIdx.x) * Cfg::WPC + j, P);
+    unsigned char *wbase = smem + j * Cfg::kWarpH;
+    float *dring = reinterpret_cast<float *>(wbase + STAGES * Cfg::kStageF + Cfg::kConv);
+    float *gring = dring + STAGES * T * CPW;
+    const bool gate = P.z != nullptr;
+    int64_t r = 0;
+    for (int64_t k = 0; k < sg.n_parts; ++k) {
+        int64_t c, ts, te;
+        sg.part(k, L, c, ts, te);
+        const int64_t cw = c % P.chains_per_row;
+        float biasv = 0.0f;
+        if (P.delta_bias != nullptr) {
+            const int64_t dp = cw * CPW + lane % CPW;
+            biasv = dp < D ? __ldg(P.delta_bias + dp) : 0.0f;
+        }
+        for (int64_t t0 = ts; t0 < te; t0 += T, ++r) {
+            const int s = static_cast<int>(r % STAGES);
+            const bool landed = mbar_wait(&full[s], static_cast<uint32_t>((r / STAGES) & 1));
+            if (!__all_sync(0xffffffffu, landed)) {
+                if (lane == 0) atomicOr(P.status, 8);
+                return;  // the consumer's bounded wait on ready[s] then gives up too
+            }
+            const IO *dsm = reinterpret_cast<const IO *>(wbase + s * Cfg::kStageF + Cfg::kU);
+            const IO *zs = reinterpret_cast<const IO *>(wbase + s * Cfg::kStageF + Cfg::kStage);
+            fused_tile<IO, Cfg>(dsm, zs, dring + s * T * CPW, gring + s * T * CPW, biasv, P.softplus != 0,
+                                gate, lane);
+            __syncwarp();  // every lane's tile entries before the arrive (release)
+            if (lane == 0) mbar_arrive(&ready[s]);
+        }
+    }
+}
+
 // The producer: the block's last warp keeps every consumer warp's ring filled,
 // lane i serving consumer warp i, all lanes in lockstep so that one TMA
 // instruction issues the loads of every consumer that has a free slot (issuing
@@ -445,7 +521,7 @@ __device__ __noinline__ void split_fixup(const ChainedParams &P, int64_t c, int6
 // stage that used the slot before.  No lane ever blocks on one consumer (a
 // consumer may be waiting for another warp's carry): each lane tests its
 // consumer's barrier, and the warp backs off briefly when no lane could issue.
-template <class IO, class Cfg, bool FUSED>
+template <class IO, class Cfg, bool FUSED, int kRegion>
 __device__ __forceinline__ void produce(const CUtensorMap *tm_u, const CUtensorMap *tm_d, const CUtensorMap *tm_b,
                                         const CUtensorMap *tm_c, const CUtensorMap *tm_z, const ChainedParams &P,
                                         unsigned char *smem,
@@ -475,7 +551,7 @@ __device__ __forceinline__ void produce(const CUtensorMap *tm_u, const CUtensorM
         row = static_cast<int>(b * L);
     };
     if (k >= 0) begin_part();
-    unsigned char *ring = smem + (i < WPC ? i : 0) * (FUSED ? Cfg::kWarpF : Cfg::kWarp);
+    unsigned char *ring = smem + (i < WPC ? i : 0) * kRegion;
     uint32_t idle = 0;
     while (__any_sync(0xffffffffu, k >= 0)) {
         const int s = static_cast<int>(r % STAGES);
@@ -513,7 +589,7 @@ __device__ __forceinline__ void produce(const CUtensorMap *tm_u, const CUtensorM
 }
 
 template <class IO, class Cfg, bool ZOH, bool POLY, bool SPLIT, bool FUSED>
-__global__ void __launch_bounds__(Cfg::kThreads, 1)
+__global__ void __launch_bounds__((FUSED && Cfg::kHelp) ? Cfg::kThreadsH : Cfg::kThreads, 1)
 sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_d,
                      const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
                      const __grid_constant__ CUtensorMap tm_z, const ChainedParams P) {
@@ -521,25 +597,33 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
     constexpr int LPC = Cfg::LPC, CPW = Cfg::CPW, NP = Cfg::NP;
     extern __shared__ __align__(128) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int kWarpB = FUSED ? Cfg::kWarpF : Cfg::kWarp;  // bytes of one consumer's region
+    constexpr bool HELP = FUSED && Cfg::kHelp;  // helper warps compute the fused tiles
+    constexpr int kWarpB = HELP ? Cfg::kWarpH : (FUSED ? Cfg::kWarpF : Cfg::kWarp);  // one consumer's region
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::WPC * kWarpB);
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2 * Cfg::WPC * STAGES; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < (HELP ? 3 : 2) * Cfg::WPC * STAGES; ++i) mbar_init(&bars[i], 1);
         mbar_fence_init();
     }
     __syncthreads();  // the only block-wide barrier
-    if (warp == Cfg::WPC) {
-        produce<IO, Cfg, FUSED>(&tm_u, &tm_d, &tm_b, &tm_c, &tm_z, P, smem, bars, bars + Cfg::WPC * STAGES, lane);
+    if (warp == (HELP ? 2 * Cfg::WPC : Cfg::WPC)) {
+        produce<IO, Cfg, FUSED, kWarpB>(&tm_u, &tm_d, &tm_b, &tm_c, &tm_z, P, smem, bars,
+                                        bars + Cfg::WPC * STAGES, lane);
+        return;
+    }
+    if (HELP && warp >= Cfg::WPC) {
+        const int j = warp - Cfg::WPC;
+        help<IO, Cfg>(P, smem, bars + j * STAGES, bars + (2 * Cfg::WPC + j) * STAGES, j, lane);
         return;
     }
     constexpr int kStageB = FUSED ? Cfg::kStageF : Cfg::kStage;  // bytes of one stage
     unsigned char *wbase = smem + warp * kWarpB;
     float *convB = reinterpret_cast<float *>(wbase + STAGES * kStageB);
     float *convC = convB + T * N;
-    float *dsf = reinterpret_cast<float *>(wbase + STAGES * kStageB + Cfg::kConv);  // FUSED: delta'
-    float *gsf = dsf + T * CPW;                                                      // FUSED: silu(z)
+    float *dsf0 = reinterpret_cast<float *>(wbase + STAGES * kStageB + Cfg::kConv);  // FUSED: delta'
+    float *gsf0 = dsf0 + (HELP ? STAGES : 1) * T * CPW;                               // FUSED: silu(z)
     uint64_t *full = bars + warp * STAGES;
     uint64_t *empty = bars + (Cfg::WPC + warp) * STAGES;
+    uint64_t *ready = bars + (2 * Cfg::WPC + warp) * STAGES;  // HELP only
 
     const int64_t L = P.L, D = P.D;
     const int64_t wk = static_cast<int64_t>(blockIdx.x) * Cfg::WPC + warp;  // this warp's segment
@@ -654,7 +738,8 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
         for (int64_t t0 = ts; t0 < te; t0 += T) {
             const int s = static_cast<int>(consumed % STAGES);
             const uint32_t par = static_cast<uint32_t>((consumed / STAGES) & 1);
-            const bool landed = mbar_wait(&full[s], par);
+            bool landed = mbar_wait(&full[s], par);
+            if (HELP) landed = landed && mbar_wait(&ready[s], par);  // the helper's tiles of this stage
             if (!__all_sync(0xffffffffu, landed)) {
                 if (lane == 0) atomicOr(P.status, 2);
                 failed = true;
@@ -692,14 +777,11 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
                 Bs = convB;
                 Cs = convC;
             }
-            if (FUSED) {  // once per tile entry: delta' = softplus(delta + bias), silu(z), fp32
-                const IO *zs = tile_z(s);
-#pragma unroll
-                for (int i = lane; i < T * CPW; i += 32) {
-                    const float v = Io<IO>::widen(dsm[i]) + biasv;
-                    dsf[i] = P.softplus ? softplus_f(v) : v;
-                    gsf[i] = gate ? silu_f(Io<IO>::widen(zs[i])) : 1.0f;
-                }
+            // fused tiles of this stage: the helper's ring slot, or computed here
+            const float *dsf = HELP ? dsf0 + s * T * CPW : dsf0;
+            const float *gsf = HELP ? gsf0 + s * T * CPW : gsf0;
+            if (FUSED && !HELP) {
+                fused_tile<IO, Cfg>(dsm, tile_z(s), dsf0, gsf0, biasv, P.softplus != 0, gate, lane);
                 __syncwarp();
             }
             auto delta_at = [&](int idx) { return FUSED ? dsf[idx] : Io<IO>::widen(dsm[idx]); };

@@ -305,13 +305,15 @@ int launch_chained_t(sscan_plan *p, const void *u, const void *dl, const float *
                      cudaStream_t s) {
     constexpr KCfg k = kChainedCfgs[CFG];
     using Cfg = ChainedCfg<IO, k.N, k.NL, k.T, k.STAGES, k.WPC>;
-    if constexpr (FUSED && Cfg::kSmemF > kMaxSmem) {
+    if constexpr (FUSED && !Cfg::kHelp && Cfg::kSmemF > kMaxSmem) {
         // the fused stage ring of this shape does not fit: the generic kernel serves the call
         (void)ws;
         return launch_generic<IO>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s) == cudaSuccess ? SSCAN_OK
                                                                                        : SSCAN_ERR_CUDA;
     } else {
-    constexpr int smem_bytes = FUSED ? Cfg::kSmemF : Cfg::kSmem;
+    constexpr bool help = FUSED && Cfg::kHelp;  // helper warps (see ChainedCfg::kHelp)
+    constexpr int smem_bytes = help ? Cfg::kSmemH : (FUSED ? Cfg::kSmemF : Cfg::kSmem);
+    constexpr int threads = help ? Cfg::kThreadsH : Cfg::kThreads;
     auto kern = sscan_chained_kernel<IO, Cfg, ZOH, POLY, SPLIT, FUSED>;
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
@@ -373,7 +375,7 @@ int launch_chained_t(sscan_plan *p, const void *u, const void *dl, const float *
     prm.z = fu.z;
     prm.softplus = fu.softplus ? 1 : 0;
     void *args[] = {&p->tm[0], &p->tm[1], &p->tm[2], &p->tm[3], &p->tm[4], &prm};
-    const dim3 grid(static_cast<unsigned>(p->workers / k.WPC)), block(Cfg::kThreads);
+    const dim3 grid(static_cast<unsigned>(p->workers / k.WPC)), block(threads);
     const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kern), grid, block, args,
                                                       smem_bytes, s);
     return e == cudaSuccess ? SSCAN_OK : SSCAN_ERR_CUDA;
