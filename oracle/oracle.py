@@ -80,6 +80,8 @@ def _bind(path):
     lib.sscan_oracle_rows_ex.argtypes = [i64, i64, i64, i64, dp, dp, dp, dp, dp, dp, dp,
                                          ip, dp, ip, dp, dp, dp, ip]
     lib.sscan_oracle_rows_ex.restype = ip
+    lib.sscan_oracle_backward.argtypes = [i64, i64, i64, i64] + [dp] * 6 + [ip] + [dp] * 8 + [ip]
+    lib.sscan_oracle_backward.restype = ip
     return lib
 
 
@@ -170,3 +172,22 @@ def forward_rows(rows, u, delta, A, B, C, h0=None, zoh=False, nthreads=None, lib
     if rc != 0:
         raise RuntimeError(f"oracle failed with code {rc}")
     return y, hf
+
+
+def backward(u, delta, A, B, C, h0=None, zoh=False, dy=None, dh_final=None, nthreads=None, lib=None):
+    """Gradients of the plain forward in fp64: given dy [Bt, L, D] (and optionally
+    dh_final [Bt, D, N]) returns a dict with du, ddelta ([Bt, L, D]), dA ([D, N]),
+    dB, dC ([Bt, L, N]) and dh0 ([Bt, D, N]).  See ``sscan_oracle.c`` ("backward")."""
+    u, delta, A, B, C, h0, dy, dh_final = map(_f64, (u, delta, A, B, C, h0, dy, dh_final))
+    Bt, L, D = u.shape
+    N = A.shape[1]
+    assert dy is not None and dy.shape == (Bt, L, D)
+    out = {"du": np.empty((Bt, L, D)), "ddelta": np.empty((Bt, L, D)), "dA": np.empty((D, N)),
+           "dB": np.empty((Bt, L, N)), "dC": np.empty((Bt, L, N)), "dh0": np.empty((Bt, D, N))}
+    rc = (lib or _load()).sscan_oracle_backward(
+        Bt, L, D, N, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(h0), int(bool(zoh)),
+        _ptr(dy), _ptr(dh_final), _ptr(out["du"]), _ptr(out["ddelta"]), _ptr(out["dA"]), _ptr(out["dB"]),
+        _ptr(out["dC"]), _ptr(out["dh0"]), int(nthreads or host_threads()))
+    if rc != 0:
+        raise RuntimeError(f"oracle backward failed with code {rc}")
+    return out

@@ -285,3 +285,159 @@ int sscan_oracle_rows(int64_t R, int64_t L, int64_t N, int64_t Bn,
     return sscan_oracle_rows_ex(R, L, N, Bn, row_b, u_rows, delta_rows, A_rows, Bm, Cm, h0_rows,
                                 zoh, NULL, 0, NULL, y_rows, hfin_rows, nthreads);
 }
+
+/* ------------------------------------------------------------------ backward
+ *
+ * Gradients of a scalar loss through the forward above (plain forward, no
+ * prologue / epilogue), given dy = dLoss/dy [B][L][D] and optionally
+ * dh_final = dLoss/dh_final [B][D][N].  Written out from the recurrence by the
+ * chain rule, in the order the forward computes it ("Selective State-Space
+ * Models (Mamba) and Hardware-Aware Scans", section 3: the backward pass
+ * recomputes the states instead of storing them; here every state of a row is
+ * kept, the plain way):
+ *
+ *   a_t = exp(delta_t A_n),  beta_t = delta_t B_t[n]        (Euler)
+ *                            beta_t = (a_t - 1)/A_n B_t[n]   (ZOH; delta_t B_t[n] at A_n = 0)
+ *   h_t = a_t h_{t-1} + beta_t u_t,   y_t = sum_n C_t[n] h_t
+ *
+ *   g_t = dLoss/dh_t = C_t[n] dy_t + a_{t+1} g_{t+1},  g_{L-1} = C dy + dh_final
+ *   du_t      = sum_n g_t beta_t
+ *   ddelta_t  = sum_n g_t (h_{t-1} A_n a_t + u_t dbeta/ddelta)
+ *               dbeta/ddelta = B_t[n] (Euler), a_t B_t[n] (ZOH)
+ *   dA[d,n]   = sum_{b,t} g_t (h_{t-1} delta_t a_t + u_t dbeta/dA)
+ *               dbeta/dA = 0 (Euler), B_t[n] (delta_t a_t A_n - (a_t - 1)) / A_n^2
+ *               (ZOH; delta_t^2 B_t[n] / 2 at A_n = 0)
+ *   dB_t[n]   = sum_d g_t u_t dbeta/dB,  dbeta/dB = delta_t (Euler), (a_t - 1)/A_n (ZOH)
+ *   dC_t[n]   = sum_d dy_t h_t
+ *   dh0       = a_0 g_0
+ *
+ * Outputs are overwritten (not accumulated into).  One thread per batch row b
+ * (dB, dC of row b are its own); each thread sums its dA into a private
+ * buffer that is added up in b order at the end, so the result does not
+ * depend on the thread count. */
+
+typedef struct {
+    int64_t B, L, D, N;
+    const double *u, *dl, *A, *Bm, *Cm, *h0, *dy, *dhf;
+    int zoh;
+    double *du, *ddl, *dA_part, *dB, *dC, *dh0;
+    int64_t b0, b1;
+    int status;
+} bwd_t;
+
+static void bwd_row(const bwd_t *j, int64_t b, int64_t d, double *hs, double *g, double *dA)
+{
+    const int64_t L = j->L, D = j->D, N = j->N;
+    const double *u = j->u + b * L * D + d, *dl = j->dl + b * L * D + d, *dy = j->dy + b * L * D + d;
+    const double *a_row = j->A + d * N;
+    const double *Bm = j->Bm + b * L * N, *Cm = j->Cm + b * L * N;
+    /* forward: hs[(t+1)*N + n] = h_t, hs[n] = h_{-1} = h0 */
+    for (int64_t n = 0; n < N; ++n)
+        hs[n] = j->h0 ? j->h0[(b * D + d) * N + n] : 0.0;
+    for (int64_t t = 0; t < L; ++t)
+        for (int64_t n = 0; n < N; ++n) {
+            const double delta = dl[t * D], an = a_row[n];
+            const double abar = exp(delta * an);
+            const double beta = j->zoh ? (an != 0.0 ? expm1(delta * an) / an * Bm[t * N + n] : delta * Bm[t * N + n])
+                                       : delta * Bm[t * N + n];
+            hs[(t + 1) * N + n] = abar * hs[t * N + n] + beta * u[t * D];
+        }
+    /* backward */
+    for (int64_t n = 0; n < N; ++n)
+        g[n] = j->dhf ? j->dhf[(b * D + d) * N + n] : 0.0;
+    for (int64_t t = L - 1; t >= 0; --t) {
+        const double delta = dl[t * D], x = u[t * D], dyt = dy[t * D];
+        double du = 0.0, ddl = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+            const double an = a_row[n], Bn = Bm[t * N + n], Cn = Cm[t * N + n];
+            const double abar = exp(delta * an);
+            const double hprev = hs[t * N + n], ht = hs[(t + 1) * N + n];
+            g[n] += Cn * dyt;                                   /* g_t = C dy + (carried a_{t+1} g_{t+1}) */
+            j->dC[(b * L + t) * N + n] += dyt * ht;
+            double beta, dbeta_ddl, dbeta_dA, dbeta_dB;
+            if (!j->zoh) {
+                beta = delta * Bn; dbeta_ddl = Bn; dbeta_dA = 0.0; dbeta_dB = delta;
+            } else if (an != 0.0) {
+                const double em1 = expm1(delta * an);
+                beta = em1 / an * Bn; dbeta_ddl = abar * Bn;
+                dbeta_dA = Bn * (delta * abar * an - em1) / (an * an); dbeta_dB = em1 / an;
+            } else {
+                beta = delta * Bn; dbeta_ddl = Bn; dbeta_dA = 0.5 * delta * delta * Bn; dbeta_dB = delta;
+            }
+            du += g[n] * beta;
+            ddl += g[n] * (hprev * an * abar + x * dbeta_ddl);
+            dA[d * N + n] += g[n] * (hprev * delta * abar + x * dbeta_dA);
+            j->dB[(b * L + t) * N + n] += g[n] * x * dbeta_dB;
+            g[n] *= abar;                                       /* now a_t g_t: carried to t-1 */
+        }
+        j->du[(b * L + t) * D + d] = du;
+        j->ddl[(b * L + t) * D + d] = ddl;
+    }
+    if (j->dh0)
+        for (int64_t n = 0; n < N; ++n)
+            j->dh0[(b * D + d) * N + n] = g[n];               /* a_0 g_0 */
+}
+
+static void *bwd_slice(void *arg)
+{
+    bwd_t *j = (bwd_t *)arg;
+    const int64_t L = j->L, N = j->N;
+    double *hs = (double *)malloc(sizeof(double) * (size_t)((L + 1) * N + 1));
+    double *g = (double *)malloc(sizeof(double) * (size_t)(N + 1));
+    if (!hs || !g) { free(hs); free(g); j->status = 2; return NULL; }
+    for (int64_t b = j->b0; b < j->b1; ++b) {
+        for (int64_t i = 0; i < L * N; ++i) { j->dB[b * L * N + i] = 0.0; j->dC[b * L * N + i] = 0.0; }
+        for (int64_t d = 0; d < j->D; ++d)
+            bwd_row(j, b, d, hs, g, j->dA_part + b * j->D * N);
+    }
+    free(hs);
+    free(g);
+    j->status = 0;
+    return NULL;
+}
+
+/* Backward over full tensors.  Inputs as for sscan_oracle_forward plus
+ *   dy       : [B][L][D]      dh_final : [B][D][N] or NULL (zero)
+ * Outputs (all overwritten):
+ *   du, ddelta : [B][L][D]    dA : [D][N]    dB, dC : [B][L][N]    dh0 : [B][D][N] or NULL
+ * Returns 0 on success, 1 for bad arguments, 2/3 on allocation or thread failure. */
+int sscan_oracle_backward(int64_t B, int64_t L, int64_t D, int64_t N,
+                          const double *u, const double *delta, const double *A,
+                          const double *Bm, const double *Cm, const double *h0, int zoh,
+                          const double *dy, const double *dh_final,
+                          double *du, double *ddelta, double *dA, double *dB, double *dC,
+                          double *dh0, int nthreads)
+{
+    if (B < 1 || L < 0 || D < 1 || N < 1) return 1;
+    if (!A || !dA || (L > 0 && (!u || !delta || !Bm || !Cm || !dy || !du || !ddelta || !dB || !dC))) return 1;
+    double *part = (double *)calloc((size_t)(B * D * N), sizeof(double));
+    if (!part) return 2;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > B) nthreads = (int)B;
+    bwd_t *jobs = (bwd_t *)calloc((size_t)nthreads, sizeof(bwd_t));
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !th) { free(part); free(jobs); free(th); return 2; }
+    int rc = 0, started = 0;
+    for (int i = 0; i < nthreads; ++i) {
+        bwd_t j = {B, L, D, N, u, delta, A, Bm, Cm, h0, dy, dh_final, zoh,
+                   du, ddelta, part, dB, dC, dh0, B * i / nthreads, B * (i + 1) / nthreads, 1};
+        jobs[i] = j;
+        if (i == nthreads - 1) break;
+        if (pthread_create(&th[i], NULL, bwd_slice, &jobs[i]) != 0) { rc = 3; break; }
+        ++started;
+    }
+    if (rc == 0) bwd_slice(&jobs[nthreads - 1]);
+    for (int i = 0; i < started; ++i) pthread_join(th[i], NULL);
+    for (int i = 0; rc == 0 && i < nthreads; ++i)
+        if (jobs[i].status != 0) rc = jobs[i].status;
+    if (rc == 0)
+        for (int64_t k = 0; k < D * N; ++k) {
+            double s = 0.0;
+            for (int64_t b = 0; b < B; ++b) s += part[b * D * N + k];
+            dA[k] = s;
+        }
+    free(part);
+    free(jobs);
+    free(th);
+    return rc;
+}
