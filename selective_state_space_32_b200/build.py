@@ -15,7 +15,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SOURCES = [os.path.join(HERE, "csrc", "sscan.cu")]
 HEADERS = [os.path.join(ROOT, "include", "sscan.h")] + [
-    os.path.join(HERE, "csrc", f) for f in ("device_utils.cuh", "kernel_chained.cuh", "kernel_generic.cuh")]
+    os.path.join(HERE, "csrc", f) for f in ("device_utils.cuh", "kernel_chained.cuh", "kernel_generic.cuh",
+                                            "kernel_backward.cuh")]
 LIB = os.path.join(HERE, "libsscan.so")
 
 NVCC_FLAGS = [

@@ -23,7 +23,7 @@ OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPAC
 
 SYMBOLS = ("sscan_plan_create", "sscan_plan_destroy", "sscan_workspace_bytes", "sscan_forward",
            "sscan_get_status", "sscan_status_string", "sscan_plan_describe", "sscan_version",
-           "sscan_forward_noalloc", "sscan_forward_gated")
+           "sscan_forward_noalloc", "sscan_forward_gated", "sscan_backward", "sscan_backward_workspace_bytes")
 
 
 class SscanError(RuntimeError):
@@ -67,6 +67,10 @@ def lib() -> ctypes.CDLL:
             L.sscan_forward_noalloc.restype = ip
             L.sscan_forward_gated.argtypes = [vp] * 13
             L.sscan_forward_gated.restype = ip
+            L.sscan_backward.argtypes = [vp] * 17
+            L.sscan_backward.restype = ip
+            L.sscan_backward_workspace_bytes.argtypes = [vp]
+            L.sscan_backward_workspace_bytes.restype = sz
             _lib = L
     return _lib
 
@@ -169,6 +173,29 @@ class Plan:
         if rc != OK:
             raise SscanError(rc, what)
         return y, h_final
+
+    def backward(self, u, delta, A, B, C, h0, dy, dh_final=None, want_dh0: bool = True, stream=None) -> dict:
+        """Gradients of the plain forward (N = 16): returns a dict with du, ddelta (plan dtype),
+        dA, dB, dC and dh0 (fp32) given dy (and optionally dh_final)."""
+        Bt, L, D, N = self.shape
+        dev = u.device
+        out = {"du": torch.empty((Bt, L, D), dtype=self.dtype, device=dev),
+               "ddelta": torch.empty((Bt, L, D), dtype=self.dtype, device=dev),
+               "dA": torch.empty((D, N), dtype=torch.float32, device=dev),
+               "dB": torch.empty((Bt, L, N), dtype=torch.float32, device=dev),
+               "dC": torch.empty((Bt, L, N), dtype=torch.float32, device=dev),
+               "dh0": torch.empty((Bt, D, N), dtype=torch.float32, device=dev) if want_dh0 else None}
+        wsb = int(lib().sscan_backward_workspace_bytes(self._h))
+        ws = torch.empty(wsb, dtype=torch.uint8, device=dev) if wsb else None
+        if stream is None:
+            stream = torch.cuda.current_stream(dev)
+        rc = lib().sscan_backward(self._h, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(h0), _ptr(dy),
+                                  _ptr(dh_final), _ptr(out["du"]), _ptr(out["ddelta"]), _ptr(out["dA"]),
+                                  _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dh0"]), _ptr(ws),
+                                  ctypes.c_void_p(stream.cuda_stream))
+        if rc != OK:
+            raise SscanError(rc, "sscan_backward")
+        return out
 
     def status(self, stream=None) -> int:
         """Synchronise ``stream`` and read (and clear) the plan's device status word."""
