@@ -318,8 +318,34 @@ def run_ours(args, rank, world, local_rank):
         "cpu_baseline": {"value": cpu_value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
     }
+    bwd = time_backward(plan, w, din, dev, stream) if (w.N == 16 and not w.fused) else None
+    if bwd is not None:
+        out["backward"] = bwd
     plan.close()
     return out
+
+
+def time_backward(plan, w, din, dev, stream, reps: int = 5):
+    """The backward pass (sscan_backward) on the same inputs, after the timed forward
+    region: mean of ``reps`` launches (CUDA events), reported beside the forward."""
+    import torch
+    try:
+        dy = torch.ones((w.B, w.L, w.D), dtype=din["u"].dtype, device=dev)
+        f = lambda: plan.backward(din["u"], din["delta"], din["A"], din["B"], din["C"], din["h0"], dy,
+                                  stream=stream)
+        f()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            f()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = a.elapsed_time(b) / reps
+        return {"kernel_ms": ms, "value": w.elements / (ms / 1e3), "unit": UNIT, "launches": reps,
+                "note": "sscan_backward (du, ddelta, dA, dB, dC, dh0; first version), dy = 1"}
+    except Exception as e:  # reported, never fatal for the forward line
+        return {"error": str(e)[:200]}
 
 
 # -------------------------------------------------------- reference arm --
