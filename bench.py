@@ -56,12 +56,13 @@ def load_peaks():
 
 
 def kernel_sources_hash() -> str:
-    """sha256 over the CUDA sources, to tell whether a stored ncu figure is current."""
+    """sha256 over the CUDA sources of the forward kernels and their host code (the
+    backward's own files excluded), to tell whether a stored ncu figure is current."""
     import hashlib
     h = hashlib.sha256()
     cdir = os.path.join(ROOT, "selective_state_space_32_b200", "csrc")
     for name in sorted(os.listdir(cdir)):
-        if name.endswith((".cu", ".cuh")):
+        if name.endswith((".cu", ".cuh")) and "backward" not in name:
             with open(os.path.join(cdir, name), "rb") as f:
                 h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()

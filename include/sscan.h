@@ -145,23 +145,26 @@ SSCAN_API int sscan_forward_gated(sscan_plan_t plan, const void *u, const void *
  * dLoss/dh_final, by the chain rule through h_t = Abar_t h_{t-1} + beta_t u_t,
  * y_t = C_t . h_t, the states recomputed from checkpoints rather than stored
  * ("Selective State-Space Models (Mamba) and Hardware-Aware Scans", section
- * 3, backward-pass recomputation).
- *   u, delta, A, B, C, h0   the forward's inputs (as for sscan_forward)
- *   dy                      [B][L][D], plan dtype
+ * 3, backward-pass recomputation).  Shape-based (no plan):
+ *   B, L, D, N, dtype, flags  as for sscan_plan_create (flags: 0 or SSCAN_ZOH)
+ *   u, delta, A, B_in, C_in, h0  the forward's inputs (as for sscan_forward)
+ *   dy                      [B][L][D], dtype
  *   dh_final                [B][D][N] fp32, or NULL (zero)
- *   du, ddelta              [B][L][D], plan dtype (output)
+ *   du, ddelta              [B][L][D], dtype (output)
  *   dA                      [D][N] fp32 (output; summed over batch and time)
  *   dB, dC                  [B][L][N] fp32 (output; summed over channels)
  *   dh0                     [B][D][N] fp32 (output), or NULL to skip it
- *   workspace               sscan_backward_workspace_bytes(plan) bytes
+ *   workspace               sscan_backward_workspace_bytes(B, L, D, N) bytes
  *                           (the state checkpoints), 16-byte aligned
- * dA, dB and dC are accumulated with fp32 atomics, so their last bits depend
- * on the order of arrival.  Returns SSCAN_ERR_UNSUPPORTED for N != 16 or a plan
- * with SSCAN_DELTA_SOFTPLUS; the other errors as for sscan_forward. */
-SSCAN_API size_t sscan_backward_workspace_bytes(sscan_plan_t plan);
-SSCAN_API int sscan_backward(sscan_plan_t plan, const void *u, const void *delta, const float *A, const void *B,
-                   const void *C, const float *h0, const void *dy, const float *dh_final, void *du,
-                   void *ddelta, float *dA, float *dB, float *dC, float *dh0, void *workspace, void *stream);
+ * All pointers are caller-owned device memory; nothing is retained.  dA, dB
+ * and dC are accumulated with fp32 atomics, so their last bits depend on the
+ * order of arrival.  Returns SSCAN_ERR_UNSUPPORTED for N != 16 or
+ * SSCAN_DELTA_SOFTPLUS; the other errors as for sscan_forward. */
+SSCAN_API size_t sscan_backward_workspace_bytes(int64_t B, int64_t L, int64_t D, int64_t N);
+SSCAN_API int sscan_backward(int64_t B, int64_t L, int64_t D, int64_t N, int dtype, uint32_t flags, const void *u,
+                   const void *delta, const float *A, const void *B_in, const void *C_in, const float *h0,
+                   const void *dy, const float *dh_final, void *du, void *ddelta, float *dA, float *dB, float *dC,
+                   float *dh0, void *workspace, void *stream);
 
 /* Wait for `stream`, then read and clear the plan's device status word.
  * Returns SSCAN_OK, SSCAN_ERR_TIMEOUT, or SSCAN_ERR_CUDA. */

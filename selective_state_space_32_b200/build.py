@@ -13,7 +13,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = [os.path.join(HERE, "csrc", "sscan.cu")]
+SOURCES = [os.path.join(HERE, "csrc", "sscan.cu"), os.path.join(HERE, "csrc", "sscan_backward.cu")]
 HEADERS = [os.path.join(ROOT, "include", "sscan.h")] + [
     os.path.join(HERE, "csrc", f) for f in ("device_utils.cuh", "kernel_chained.cuh", "kernel_generic.cuh",
                                             "kernel_backward.cuh")]

@@ -31,7 +31,6 @@
 
 #include "device_utils.cuh"
 #include "kernel_chained.cuh"
-#include "kernel_backward.cuh"
 #include "kernel_generic.cuh"
 #include "sscan.h"
 
@@ -459,24 +458,6 @@ int noalloc_scratch(int dev, unsigned char **out) {
 
 }  // namespace
 
-// ------------------------------------------------------- backward helpers
-
-namespace {
-int64_t bwd_dpad(const sscan_plan *p) { return ceil_div(p->D, int64_t(kBwdThreads)) * kBwdThreads; }
-// Opt each backward kernel into its dynamic shared memory once (per instantiation).
-template <class IO, bool ZOH>
-cudaError_t bwd_attr() {
-    static std::once_flag once;
-    static cudaError_t err = cudaSuccess;
-    std::call_once(once, [] {
-        err = cudaFuncSetAttribute(sscan_backward_kernel<IO, ZOH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   kBwdSmem);
-    });
-    return err;
-}
-int64_t bwd_chunks(const sscan_plan *p) { return ceil_div(p->L, int64_t(kChunk)); }
-}  // namespace
-
 extern "C" {
 
 int sscan_version(void) { return SSCAN_VERSION; }
@@ -623,76 +604,6 @@ int sscan_forward_gated(sscan_plan_t plan, const void *u, const void *delta, con
         p->dtype == SSCAN_F32 ? launch_generic<float>(p, u, delta, A, B, C, h0, y, h_final, fu, s)
                               : launch_generic<uint16_t>(p, u, delta, A, B, C, h0, y, h_final, fu, s);
     return e == cudaSuccess ? SSCAN_OK : SSCAN_ERR_CUDA;
-}
-
-// ------------------------------------------------------------------ backward
-
-
-size_t sscan_backward_workspace_bytes(sscan_plan_t plan) {
-    if (!plan || plan->N != 16 || plan->L == 0) return 0;
-    return align_up(size_t(plan->B) * size_t(bwd_dpad(plan)) * size_t(bwd_chunks(plan)) * 16 * sizeof(float), 256);
-}
-
-int sscan_backward(sscan_plan_t plan, const void *u, const void *delta, const float *A, const void *B,
-                   const void *C, const float *h0, const void *dy, const float *dh_final, void *du,
-                   void *ddelta, float *dA, float *dB, float *dC, float *dh0, void *workspace, void *stream) {
-    if (!plan) return SSCAN_ERR_INVALID;
-    sscan_plan *p = plan;
-    if (p->N != 16 || (p->flags & SSCAN_DELTA_SOFTPLUS)) return SSCAN_ERR_UNSUPPORTED;
-    const size_t es = p->dtype == SSCAN_F32 ? 4 : 2;
-    const size_t n_bld = static_cast<size_t>(p->B * p->L * p->D), n_bln = static_cast<size_t>(p->B * p->L * p->N);
-    const size_t n_dn = static_cast<size_t>(p->D * p->N), n_bdn = static_cast<size_t>(p->B * p->D * p->N);
-    if (!A || !dA) return SSCAN_ERR_INVALID;
-    if (n_bld && (!u || !delta || !B || !C || !dy || !du || !ddelta || !dB || !dC)) return SSCAN_ERR_INVALID;
-    const void *ptrs[] = {u, delta, A, B, C, h0, dy, dh_final, du, ddelta, dA, dB, dC, dh0, workspace};
-    for (const void *q : ptrs)
-        if (q && !aligned16(q)) return SSCAN_ERR_ALIGN;
-    // outputs must not overlap inputs or each other
-    const void *ins[] = {u, delta, A, B, C, h0, dy, dh_final};
-    const size_t insz[] = {n_bld * es, n_bld * es, n_dn * 4, n_bln * es, n_bln * es, n_bdn * 4, n_bld * es, n_bdn * 4};
-    const void *outs[] = {du, ddelta, dA, dB, dC, dh0};
-    const size_t outsz[] = {n_bld * es, n_bld * es, n_dn * 4, n_bln * 4, n_bln * 4, n_bdn * 4};
-    for (int i = 0; i < 6; ++i) {
-        for (int k = 0; k < 8; ++k)
-            if (overlaps(outs[i], outsz[i], ins[k], insz[k])) return SSCAN_ERR_INVALID;
-        for (int k = i + 1; k < 6; ++k)
-            if (overlaps(outs[i], outsz[i], outs[k], outsz[k])) return SSCAN_ERR_INVALID;
-    }
-    const size_t ws = sscan_backward_workspace_bytes(plan);
-    if (ws && !workspace) return SSCAN_ERR_WORKSPACE;
-    for (int k = 0; k < 8; ++k)
-        if (ws && overlaps(workspace, ws, ins[k], insz[k])) return SSCAN_ERR_WORKSPACE;
-    for (int i = 0; i < 6; ++i)
-        if (ws && overlaps(workspace, ws, outs[i], outsz[i])) return SSCAN_ERR_WORKSPACE;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // dA, dB, dC are accumulated with atomics
-    if (cudaMemsetAsync(dA, 0, n_dn * 4, s) != cudaSuccess) return SSCAN_ERR_CUDA;
-    if (n_bln && (cudaMemsetAsync(dB, 0, n_bln * 4, s) != cudaSuccess ||
-                  cudaMemsetAsync(dC, 0, n_bln * 4, s) != cudaSuccess))
-        return SSCAN_ERR_CUDA;
-    if (p->L == 0) {  // no tokens: dh0 = dh_final
-        if (dh0 && (dh_final ? cudaMemcpyAsync(dh0, dh_final, n_bdn * 4, cudaMemcpyDeviceToDevice, s)
-                             : cudaMemsetAsync(dh0, 0, n_bdn * 4, s)) != cudaSuccess)
-            return SSCAN_ERR_CUDA;
-        return SSCAN_OK;
-    }
-    const dim3 grid(static_cast<unsigned>(bwd_dpad(p) / kBwdThreads), static_cast<unsigned>(p->B));
-    auto launch = [&](auto kern, cudaError_t attr, auto io) -> int {
-        using IO = decltype(io);
-        if (attr != cudaSuccess) return SSCAN_ERR_CUDA;
-        kern<<<grid, kBwdThreads, kBwdSmem, s>>>(
-            static_cast<const IO *>(u), static_cast<const IO *>(delta), A, static_cast<const IO *>(B),
-            static_cast<const IO *>(C), h0, static_cast<const IO *>(dy), dh_final, static_cast<IO *>(du),
-            static_cast<IO *>(ddelta), dA, dB, dC, dh0, static_cast<float *>(workspace), p->L, p->D, bwd_dpad(p),
-            bwd_chunks(p));
-        return cudaGetLastError() == cudaSuccess ? SSCAN_OK : SSCAN_ERR_CUDA;
-    };
-    const bool zoh = (p->flags & SSCAN_ZOH) != 0;
-    if (p->dtype == SSCAN_F32)
-        return zoh ? launch(sscan_backward_kernel<float, true>, bwd_attr<float, true>(), float{})
-                   : launch(sscan_backward_kernel<float, false>, bwd_attr<float, false>(), float{});
-    return zoh ? launch(sscan_backward_kernel<uint16_t, true>, bwd_attr<uint16_t, true>(), uint16_t{})
-               : launch(sscan_backward_kernel<uint16_t, false>, bwd_attr<uint16_t, false>(), uint16_t{});
 }
 
 int sscan_get_status(sscan_plan_t plan, void *stream) {

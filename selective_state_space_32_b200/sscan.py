@@ -67,9 +67,9 @@ def lib() -> ctypes.CDLL:
             L.sscan_forward_noalloc.restype = ip
             L.sscan_forward_gated.argtypes = [vp] * 13
             L.sscan_forward_gated.restype = ip
-            L.sscan_backward.argtypes = [vp] * 17
+            L.sscan_backward.argtypes = [i64, i64, i64, i64, ip, u32] + [vp] * 16
             L.sscan_backward.restype = ip
-            L.sscan_backward_workspace_bytes.argtypes = [vp]
+            L.sscan_backward_workspace_bytes.argtypes = [i64, i64, i64, i64]
             L.sscan_backward_workspace_bytes.restype = sz
             _lib = L
     return _lib
@@ -185,11 +185,13 @@ class Plan:
                "dB": torch.empty((Bt, L, N), dtype=torch.float32, device=dev),
                "dC": torch.empty((Bt, L, N), dtype=torch.float32, device=dev),
                "dh0": torch.empty((Bt, D, N), dtype=torch.float32, device=dev) if want_dh0 else None}
-        wsb = int(lib().sscan_backward_workspace_bytes(self._h))
+        wsb = int(lib().sscan_backward_workspace_bytes(Bt, L, D, N))
         ws = torch.empty(wsb, dtype=torch.uint8, device=dev) if wsb else None
         if stream is None:
             stream = torch.cuda.current_stream(dev)
-        rc = lib().sscan_backward(self._h, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(h0), _ptr(dy),
+        flags = (ZOH if self.zoh else 0) | (DELTA_SOFTPLUS if self.delta_softplus else 0)
+        rc = lib().sscan_backward(Bt, L, D, N, _dtype_code(self.dtype), flags,
+                                  _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(h0), _ptr(dy),
                                   _ptr(dh_final), _ptr(out["du"]), _ptr(out["ddelta"]), _ptr(out["dA"]),
                                   _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dh0"]), _ptr(ws),
                                   ctypes.c_void_p(stream.cuda_stream))

@@ -96,13 +96,12 @@ def test_backward_forward_consistency():
 def test_backward_argument_errors():
     import ctypes
     Bt, L, D = 1, 16, 32
-    plan = S.Plan(Bt, L, D, 32, torch.float32, False)  # N = 32: not supported by the backward
     z = torch.zeros(16, device="cuda")
     p = ctypes.c_void_p(z.data_ptr())
-    rc = S.lib().sscan_backward(plan._h, *([p] * 15), None)
-    assert rc == S.ERR_UNSUPPORTED
-    plan.close()
-    plan = S.Plan(Bt, L, D, 16, torch.float32, False, delta_softplus=True)
-    rc = S.lib().sscan_backward(plan._h, *([p] * 15), None)
-    assert rc == S.ERR_UNSUPPORTED
-    plan.close()
+    # N = 32 and the fused softplus flag are not supported by the backward
+    assert S.lib().sscan_backward(Bt, L, D, 32, S.F32, 0, *([p] * 15), None) == S.ERR_UNSUPPORTED
+    assert S.lib().sscan_backward(Bt, L, D, 16, S.F32, S.DELTA_SOFTPLUS, *([p] * 15), None) == S.ERR_UNSUPPORTED
+    # a bad flag bit and a misaligned pointer
+    assert S.lib().sscan_backward(Bt, L, D, 16, S.F32, 1 << 5, *([p] * 15), None) == S.ERR_INVALID
+    q = ctypes.c_void_p(z.data_ptr() + 4)
+    assert S.lib().sscan_backward(Bt, L, D, 16, S.F32, 0, q, *([p] * 14), None) == S.ERR_ALIGN
