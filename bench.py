@@ -55,16 +55,30 @@ def load_peaks():
         return FALLBACK_HBM_GBS, SM_MAX_MHZ, "fallback"
 
 
-def kernel_sources_hash() -> str:
-    """sha256 over the CUDA sources of the forward kernels and their host code (the
-    backward's own files excluded), to tell whether a stored ncu figure is current."""
+def strip_comments(src: str) -> str:
+    """C/C++/CUDA source without comments and blank lines (string literals in these
+    sources hold no comment markers), so that a comment edit keeps the hash."""
+    import re
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
+def kernel_sources_hash(read=None) -> str:
+    """sha256 over the code (comments stripped) of the forward kernels and their host
+    code (the backward's own files excluded), to tell whether a stored ncu figure is
+    current.  ``read(name)`` returns a file's text (default: the working tree)."""
     import hashlib
     h = hashlib.sha256()
     cdir = os.path.join(ROOT, "selective_state_space_32_b200", "csrc")
-    for name in sorted(os.listdir(cdir)):
-        if name.endswith((".cu", ".cuh")) and "backward" not in name:
-            with open(os.path.join(cdir, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    names = [n for n in sorted(os.listdir(cdir)) if n.endswith((".cu", ".cuh")) and "backward" not in n]
+    for name in names:
+        if read is None:
+            with open(os.path.join(cdir, name), encoding="utf-8") as f:
+                text = f.read()
+        else:
+            text = read(name)
+        h.update(name.encode() + b"\0" + strip_comments(text).encode())
     return h.hexdigest()
 
 

@@ -31,11 +31,19 @@
 // (slow) TMA issue never stalls a consumer and the compute loop only reads
 // shared memory.  bf16 B/C tiles are widened once per stage by the warp.
 //
-// Arithmetic per state update: Abar = 2^(delta*A*log2 e) on the MUFU pipe, or
-// for a quarter of the states on the FMA pipe (exp2_fma_pair) to balance the
-// two pipes; Bbar u (Euler or exact ZOH), h = Abar*h + Bbar u and y += C*h on
+// Arithmetic per state update: Abar = 2^(delta*A*log2 e) on the MUFU pipe (an
+// option, POLY, moves a quarter of the states to the FMA pipe, exp2_fma_pair;
+// measured slower with one consumer warp per SM sub-partition, so off by
+// default); Bbar u (Euler or exact ZOH), h = Abar*h + Bbar u and y += C*h on
 // packed f32x2 instructions.  y is reduced over the LPC lanes of a channel
-// with shuffles and stored directly.
+// with shuffles and stored directly (lanes past the last channel store into a
+// sink slot, so no store is guarded).
+//
+// Fused kernels (FUSED): each stage also carries the gate tile z, and the
+// stage's delta' = softplus(delta + bias) and silu(z) are computed once per
+// tile entry into fp32 tiles (fused_tile) -- by a helper warp per consumer on
+// the same SM sub-partition for 4-consumer shapes (help), else by the
+// consumer itself; y is stored multiplied by silu(z).
 #pragma once
 
 #include "device_utils.cuh"
