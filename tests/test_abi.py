@@ -63,3 +63,42 @@ def test_null_plan_is_rejected(lib):
     assert lib.sscan_forward(None, *([None] * 10)) == S.ERR_INVALID
     assert lib.sscan_get_status(None, None) == S.ERR_INVALID
     lib.sscan_plan_destroy(None)
+
+
+def declared_param_counts():
+    """{function: number of parameters} from the header's SSCAN_API declarations."""
+    with open(HEADER) as f:
+        text = f.read()
+    out = {}
+    for m in re.finditer(r"SSCAN_API\s+[\w\s\*]+?\b(sscan_\w+)\s*\(([^)]*)\)", text):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else len(params.split(","))
+    return out
+
+
+def test_binding_argument_counts_match_the_header(lib):
+    counts = declared_param_counts()
+    assert set(counts) == set(S.SYMBOLS)
+    for name, n in counts.items():
+        assert len(getattr(lib, name).argtypes) == n, (name, n, len(getattr(lib, name).argtypes))
+
+
+def test_gated_and_backward_reject_bad_arguments_without_a_device(lib):
+    assert lib.sscan_forward_gated(None, *([None] * 12)) == S.ERR_INVALID
+    p = ctypes.c_void_p(256)  # never dereferenced: every case fails its checks first
+    args16 = [p] * 15 + [None]
+    assert lib.sscan_backward(1, 16, 32, 32, S.F32, 0, *args16) == S.ERR_UNSUPPORTED      # N = 32
+    assert lib.sscan_backward(1, 16, 32, 16, S.F32, S.DELTA_SOFTPLUS, *args16) == S.ERR_UNSUPPORTED
+    assert lib.sscan_backward(0, 16, 32, 16, S.F32, 0, *args16) == S.ERR_INVALID          # B = 0
+    assert lib.sscan_backward(1, 16, 32, 16, 7, 0, *args16) == S.ERR_INVALID              # dtype
+    assert lib.sscan_backward(1, 16, 32, 16, S.F32, 1 << 5, *args16) == S.ERR_INVALID     # flag
+    assert lib.sscan_backward(1, 16, 32, 16, S.F32, 0, *([p] * 6), None, *([p] * 8), None) == S.ERR_INVALID  # no dy
+    assert lib.sscan_backward(1, 16, 32, 16, S.F32, 0, ctypes.c_void_p(260), *([p] * 14), None) == S.ERR_ALIGN
+
+
+def test_backward_workspace_bytes(lib):
+    # state checkpoints: B x ceil(D/128)*128 channels x ceil(L/8) chunks x 16 states x 4 bytes
+    assert lib.sscan_backward_workspace_bytes(8, 2048, 1536, 16) == 8 * 1536 * 256 * 16 * 4
+    assert lib.sscan_backward_workspace_bytes(2, 37, 70, 16) == 2 * 128 * 5 * 16 * 4
+    assert lib.sscan_backward_workspace_bytes(2, 37, 70, 32) == 0
+    assert lib.sscan_backward_workspace_bytes(2, 0, 70, 16) == 0
