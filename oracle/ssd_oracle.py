@@ -71,3 +71,42 @@ def ssd_forward(x, delta, A, B, C, h0=None):
                 y[b, :, h, :] += (C[b] * head[:, None]) @ h0bh
                 hf[b, h] += head[-1] * h0bh if L > 0 else h0bh
     return y, hf
+
+
+def ssd_forward_chunked(x, delta, A, B, C, h0=None, block=64):
+    """The same map computed the way the page's kernel organises it ("Mamba & Mamba-2
+    Architecture", section 3: the sequence cut into blocks, e.g. 64 tokens): per block,
+    the intra-block part (M_blk o C_blk Bbar_blk^T) X_blk, the block's own end state
+    S = sum_s (prod_{k>s in block} a_k) Bbar_s x_s^T, and the state passed in from the
+    earlier blocks, h <- (prod over the block of a) h + S, which reaches the block's
+    outputs as C_t (prod_{k = block start .. t} a_k) h_in.  Same shapes as ssd_forward."""
+    x = np.asarray(x, np.float64)
+    delta = np.asarray(delta, np.float64)
+    A = np.asarray(A, np.float64)
+    B = np.asarray(B, np.float64)
+    C = np.asarray(C, np.float64)
+    Bt, L, H, P = x.shape
+    N = B.shape[2]
+    y = np.zeros((Bt, L, H, P))
+    hf = np.zeros((Bt, H, N, P))
+    for b in range(Bt):
+        for h in range(H):
+            state = np.zeros((N, P)) if h0 is None else np.asarray(h0, np.float64)[b, h].copy()
+            for t0 in range(0, L, block):
+                t1 = min(L, t0 + block)
+                dl = delta[b, t0:t1, h]
+                a = np.exp(dl * A[h])
+                xb = x[b, t0:t1, h, :]
+                # intra-block: the block's own semiseparable matrix
+                y[b, t0:t1, h, :] = ssd_matrix(dl, A[h], B[b, t0:t1], C[b, t0:t1]) @ xb
+                # inter-block: the carried-in state, decayed to each position of the block
+                head = np.cumprod(a)
+                y[b, t0:t1, h, :] += (C[b, t0:t1] * head[:, None]) @ state
+                # the block's own end state, then the state passing
+                tail = np.ones(t1 - t0)
+                for s in range(t1 - t0 - 2, -1, -1):
+                    tail[s] = tail[s + 1] * a[s + 1]
+                S_blk = (B[b, t0:t1] * (dl * tail)[:, None]).T @ xb
+                state = head[-1] * state + S_blk
+            hf[b, h] = state
+    return y, hf

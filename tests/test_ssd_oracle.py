@@ -85,7 +85,8 @@ MUTANTS = {
                                  "np.asarray(B_b, np.float64) @ np.asarray(C_b, np.float64).T"),
     "h0_not_decayed": ("                head = np.cumprod(a)  # prod_{k=0..t} a_k",
                        "                head = np.ones_like(a)"),
-    "final_state_off_by_one": ("                tail[s] = tail[s + 1] * a[s + 1]", "                tail[s] = tail[s + 1] * a[s]"),
+    "final_state_off_by_one": ("            for s in range(L - 2, -1, -1):\n                tail[s] = tail[s + 1] * a[s + 1]",
+                               "            for s in range(L - 2, -1, -1):\n                tail[s] = tail[s + 1] * a[s]"),
 }
 
 
@@ -106,3 +107,14 @@ def test_ssd_mutants_are_caught():
             except AssertionError:
                 caught.append(pin.__name__)
         assert caught, f"no SSD pin catches mutant {name}"
+
+
+def test_chunked_ssd_equals_the_quadratic_form():
+    # block sizes that divide L, do not divide it, and exceed it
+    rng = np.random.default_rng(74)
+    x, delta, A, B, C, h0 = _problem(rng, Bt=2, L=37, H=2, P=3, N=4)
+    y, hf = S.ssd_forward(x, delta, A, B, C, h0)
+    for block in (1, 8, 16, 64):
+        yc, hc = S.ssd_forward_chunked(x, delta, A, B, C, h0, block=block)
+        assert np.abs(yc - y).max() <= 1e-12 * (1 + np.abs(y).max()), block
+        assert np.abs(hc - hf).max() <= 1e-12 * (1 + np.abs(hf).max()), block
