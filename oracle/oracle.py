@@ -191,3 +191,35 @@ def backward(u, delta, A, B, C, h0=None, zoh=False, dy=None, dh_final=None, nthr
     if rc != 0:
         raise RuntimeError(f"oracle backward failed with code {rc}")
     return out
+
+
+def backward_fused(u, delta_raw, A, B, C, h0=None, zoh=False, dy=None, dh_final=None,
+                   delta_bias=None, softplus=True, z=None, nthreads=None):
+    """Gradients of the fused forward (delta' = softplus(delta_raw + bias), y = scan * silu(z))
+    in fp64, by the chain rule around the plain backward:
+
+        scan output ys = y / silu(z);   dys = dy * silu(z);   dz = dy * ys * silu'(z),
+        silu'(z) = sigmoid(z) (1 + z (1 - sigmoid(z)));
+        d delta_raw = d delta' * sigmoid(delta_raw + bias)   (softplus' = sigmoid; 1 without softplus),
+        d bias[d] = sum over b and t of d delta_raw.
+
+    Returns the plain backward's dict (ddelta replaced by the gradient w.r.t. delta_raw)
+    plus ddelta_bias ([D]) and dz ([Bt, L, D]) when those inputs are given."""
+    u, delta_raw, A, B, C, h0, dy, dh_final, delta_bias, z = map(
+        _f64, (u, delta_raw, A, B, C, h0, dy, dh_final, delta_bias, z))
+    s = delta_raw if delta_bias is None else delta_raw + delta_bias[None, None, :]
+    dprime = (np.maximum(s, 0.0) + np.log1p(np.exp(-np.abs(s)))) if softplus else s
+    dys = dy
+    out_extra = {}
+    if z is not None:
+        sig = 1.0 / (1.0 + np.exp(-z))
+        ys, _ = forward(u, dprime, A, B, C, h0, zoh, nthreads=nthreads)
+        dys = dy * z * sig
+        out_extra["dz"] = dy * ys * sig * (1.0 + z * (1.0 - sig))
+    g = backward(u, dprime, A, B, C, h0, zoh, dys, dh_final, nthreads=nthreads)
+    if softplus:
+        g["ddelta"] = g["ddelta"] / (1.0 + np.exp(-s))
+    if delta_bias is not None:
+        out_extra["ddelta_bias"] = g["ddelta"].sum(axis=(0, 1))
+    g.update(out_extra)
+    return g

@@ -135,3 +135,31 @@ def test_backward_mutant_is_caught(name, tmp_path):
         except AssertionError:
             caught = True
     assert caught, f"no pin catches backward mutant {name}"
+
+
+def test_fused_backward_matches_finite_differences():
+    # delta' = softplus(delta_raw + bias), y = scan(delta') * silu(z): every gradient,
+    # including the raw step, the bias and the gate, against central differences of
+    # the (pinned) fused forward oracle
+    rng = np.random.default_rng(49)
+    u, delta, A, B, C, h0, dy, dhf = _problem(rng)
+    raw = rng.normal(-1.0, 1.0, delta.shape)
+    bias = rng.normal(0.0, 0.5, delta.shape[2])
+    z = rng.normal(0.0, 1.5, u.shape)
+    for zoh in (False, True):
+        g = O.backward_fused(u, raw, A, B, C, h0, zoh, dy, dhf, delta_bias=bias, softplus=True, z=z)
+
+        def loss(uu=u, rr=raw, AA=A, BB=B, CC=C, hh=h0, bb=bias, zz=z):
+            y, hf = O.forward(uu, rr, AA, BB, CC, hh, zoh, delta_bias=bb, softplus=True, z=zz)
+            return float(np.sum(y * dy) + np.sum(hf * dhf))
+
+        eps = 1e-6
+        for name, key, x in (("du", "uu", u), ("ddelta", "rr", raw), ("dA", "AA", A), ("dB", "BB", B),
+                             ("dC", "CC", C), ("dh0", "hh", h0), ("ddelta_bias", "bb", bias), ("dz", "zz", z)):
+            num = np.zeros_like(x)
+            for idx in np.ndindex(x.shape):
+                xp = x.copy(); xp[idx] += eps
+                xm = x.copy(); xm[idx] -= eps
+                num[idx] = (loss(**{key: xp}) - loss(**{key: xm})) / (2 * eps)
+            err = np.abs(g[name] - num).max()
+            assert err <= 1e-6 * (1 + np.abs(num).max()), (name, zoh, err)
