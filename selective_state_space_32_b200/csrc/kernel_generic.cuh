@@ -5,9 +5,11 @@
 // their partial y with shuffles.  u/delta are read with plain loads (adjacent
 // lanes -> adjacent channels) through an 8-token register prefetch ring; B/C
 // rows come from L1.  It accepts any D and any 16-byte aligned pointers and
-// is used where the chained TMA kernel does not apply (D*element size not a
-// multiple of 16 bytes, an empty sequence, or too few channels to fill the GPU
-// without splitting the sequence).
+// is used where the chained TMA kernel does not apply: D*element size not a
+// multiple of 16 bytes, sequences shorter than 64 tokens (decode steps
+// included), or a fused call on a shape whose fused stage ring does not fit
+// shared memory.  It also applies the fused prologue (delta + bias, softplus)
+// and the silu(z) gate per token.
 #pragma once
 
 #include "device_utils.cuh"
