@@ -41,9 +41,10 @@ SM_MAX_MHZ = 1965.0
 # 128 FP32 FMA-pipe lanes.  An update needs one 2^x and four FMA-pipe ops
 # (delta*A, B*(delta*u), Abar*h + Bbar u, y += C*h); a 2^x can instead be
 # computed on the FMA pipe with eight ops (range reduction + degree-5
-# polynomial).  Balancing the two pipes: f = 4/15 of the exps in software gives
-# 16 / (1 - 4/15) = 21.8 updates per SM per clock.
-ALU_UPDATES_PER_SM_CLK = 16.0 / (1.0 - 4.0 / 15.0)
+# polynomial).  With a fraction f of the exponents in software the MUFU pipe
+# allows 16 / (1 - f) updates per clock and the FMA pipe 128 / (4 + 8 f); the
+# two are equal at f = 1/4, i.e. 16 / (3/4) = 21.33 updates per SM per clock.
+ALU_UPDATES_PER_SM_CLK = 16.0 / (1.0 - 0.25)
 
 
 def load_peaks():
@@ -161,21 +162,31 @@ def cpu_oracle_rate(g, w, min_seconds=10.0, max_seconds=30.0):
     """Time the fp64 oracle as it stands on this host's cores: full passes over the
     workload until at least ``min_seconds`` elapsed.  Returns (elements/s, cores, sample)."""
     from oracle import oracle as O
-    v = {k: (None if g.get(k) is None else W.as_f32(g[k], g["dtype"]).astype(np.float64))
-         for k in ("u", "delta", "B", "C", "z")}
-    A = g["A"].astype(np.float64)
-    h0 = None if g["h0"] is None else g["h0"].astype(np.float64)
-    bias = None if g.get("delta_bias") is None else g["delta_bias"].astype(np.float64)
+    v = _oracle_values(g, w)
     cores = O.host_threads()
     n, t0 = 0, time.perf_counter()
     while True:
-        O.forward(v["u"], v["delta"], A, v["B"], v["C"], h0, w.zoh, nthreads=cores,
-                  delta_bias=bias, softplus=w.fused, z=v["z"])
+        O.forward(v["u"], v["delta"], v["A"], v["B"], v["C"], v["h0"], w.zoh, nthreads=cores,
+                  delta_bias=v["delta_bias"], softplus=w.fused, z=v["z"])
         n += 1
         el = time.perf_counter() - t0
         if el >= min_seconds or el + el / n > max_seconds:
             break
     return n * w.elements / el, cores, f"{n} full pass(es) over the workload ({w.elements} elements each) in {el:.2f} s"
+
+
+def workload_config(w, world: int) -> dict:
+    """The ``config`` object of a JSON line: the same keys for both arms, so a line of
+    ours and a reference line of the same workload compare as the same configuration."""
+    alg_bytes = w.algorithmic_bytes()
+    return {"workload": f"{w.name}: B={w.B} L={w.L} D={w.D} N={w.N} io={w.dtype} "
+                        f"{'ZOH' if w.zoh else 'Euler'} h0={'yes' if w.h0_std else 'no'}"
+                        f"{' resets=' + str(w.reset_frac) if w.reset_frac else ''}"
+                        f"{' fused softplus(delta+bias), y*silu(z)' if w.fused else ''}",
+            "B": w.B, "L": w.L, "D": w.D, "N": w.N, "io_dtype": w.dtype,
+            "parallelism": f"dp{world} (independent batch-row shards, no collective)",
+            "l2": f"inputs larger than L2 ({alg_bytes / 1e6:.0f} MB per step vs "
+                  f"{L2_BYTES / 2**20:.0f} MiB L2); no flush"}
 
 
 # ------------------------------------------------------- multi-rank logic --
@@ -309,13 +320,7 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": f"{w.name}: B={w.B} L={w.L} D={w.D} N={w.N} io={w.dtype} "
-                               f"{'ZOH' if w.zoh else 'Euler'} h0={'yes' if w.h0_std else 'no'}"
-                               f"{' fused softplus(delta+bias), y*silu(z)' if w.fused else ''}",
-                   "B": w.B, "L": w.L, "D": w.D, "N": w.N, "io_dtype": w.dtype,
-                   "parallelism": f"dp{world} (independent batch-row shards, no collective)",
-                   "l2": f"inputs larger than L2 ({alg_bytes / 1e6:.0f} MB per step vs "
-                         f"{L2_BYTES / 2**20:.0f} MiB L2); no flush"},
+        "config": workload_config(w, world),
         "roofline": {"bound": "alu", "achieved": upd_rate, "peak": alu_peak,
                      "unit": "Gupdates/s", "frac": upd_rate / alu_peak, "traffic": traffic,
                      "kernel": kernel_name, "schedule": plan.describe(),
@@ -333,10 +338,75 @@ def run_ours(args, rank, world, local_rank):
         "cpu_baseline": {"value": cpu_value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
     }
+    if args.per_config:
+        others = [n for n in W.ORDER[1:] if n != args.workload]
+        out["per_config"] = time_other_configs(others, dev, stream, sm_max, hbm_peak)
     bwd = time_backward(plan, w, din, dev, stream) if (w.N == 16 and not w.fused) else None
     if bwd is not None:
         out["backward"] = bwd
     plan.close()
+    return out
+
+
+def to_device(g, dev):
+    """Generated arrays -> CUDA tensors in their storage dtype (bf16 bit patterns -> bfloat16)."""
+    import torch
+
+    def t(x, dt):
+        if x is None:
+            return None
+        if dt == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(dev)
+    dt = g["dtype"]
+    return {"u": t(g["u"], dt), "delta": t(g["delta"], dt), "A": t(g["A"], "f32"), "B": t(g["B"], dt),
+            "C": t(g["C"], dt), "h0": t(g["h0"], "f32"), "delta_bias": t(g.get("delta_bias"), "f32"),
+            "z": t(g.get("z"), dt)}
+
+
+def time_other_configs(names, dev, stream, sm_max, hbm_peak, launches: int = 20, warmup: int = 3):
+    """Kernel time of each named workload in this run (CUDA events around each launch on
+    the launching stream, inputs resident in HBM), with its element rate and its HBM and
+    ALU roofline fractions.  A figure per configuration beside the headline line."""
+    import torch
+    from selective_state_space_32_b200 import sscan as S
+    out = {}
+    alu_peak = ALU_UPDATES_PER_SM_CLK * SM_COUNT * sm_max * 1e6 / 1e9
+    for name in names:
+        w = W.WORKLOADS[name]
+        try:
+            d = to_device(W.make_inputs(w), dev)
+            tdt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+            plan = S.Plan(w.B, w.L, w.D, w.N, tdt, w.zoh, delta_softplus=w.fused)
+            ws = plan.new_workspace(dev)
+            y = torch.empty((w.B, w.L, w.D), dtype=tdt, device=dev)
+            hf = torch.empty((w.B, w.D, w.N), dtype=torch.float32, device=dev)
+            step = lambda: plan.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"], y=y, h_final=hf,
+                                        workspace=ws, stream=stream, delta_bias=d["delta_bias"], z=d["z"])
+            for _ in range(warmup):
+                step()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(launches)]
+            torch.cuda.synchronize(dev)
+            for a, b in ev:
+                a.record(stream)
+                step()
+                b.record(stream)
+            torch.cuda.synchronize(dev)
+            if plan.status(stream) != S.OK:
+                raise RuntimeError("device status word reported an error")
+            ms = sum(a.elapsed_time(b) for a, b in ev) / launches
+            gbs = w.algorithmic_bytes() / (ms / 1e3) / 1e9
+            upd = w.updates / (ms / 1e3) / 1e9
+            out[name] = {"kernel_ms": ms, "elements_per_s": w.elements / (ms / 1e3),
+                         "hbm_gbs": gbs, "hbm_frac": gbs / hbm_peak, "alu_frac": upd / alu_peak,
+                         "mufu_only_frac": upd / (16.0 * SM_COUNT * sm_max * 1e6 / 1e9),
+                         "launches": launches, "schedule": plan.describe()}
+            plan.close()
+            del d, y, hf, ws
+            torch.cuda.empty_cache()
+        except Exception as e:  # reported, never fatal for the headline line
+            out[name] = {"error": str(e)[:200]}
     return out
 
 
@@ -365,47 +435,69 @@ def time_backward(plan, w, din, dev, stream, reps: int = 5):
 
 # -------------------------------------------------------- reference arm --
 
+def _oracle_values(g, w):
+    """The workload's inputs as the fp64 values the oracle reads (bf16 widened exactly)."""
+    v = {k: (None if g.get(k) is None else W.as_f32(g[k], g["dtype"]).astype(np.float64))
+         for k in ("u", "delta", "B", "C", "z")}
+    v["A"] = g["A"].astype(np.float64)
+    v["h0"] = None if g["h0"] is None else g["h0"].astype(np.float64)
+    v["delta_bias"] = None if g.get("delta_bias") is None else g["delta_bias"].astype(np.float64)
+    return v
+
+
+def _sub_problem(v, nb: int, nd: int) -> dict:
+    """Batch rows [0, nb) and channels [0, nd) of the workload as contiguous arrays (rows
+    are independent, so this is an exact sub-problem of the same workload)."""
+    cut = lambda x: None if x is None else np.ascontiguousarray(x[:nb, :, :nd])
+    return {"u": cut(v["u"]), "delta": cut(v["delta"]), "z": cut(v["z"]),
+            "B": np.ascontiguousarray(v["B"][:nb]), "C": np.ascontiguousarray(v["C"][:nb]),
+            "A": np.ascontiguousarray(v["A"][:nd]),
+            "h0": None if v["h0"] is None else np.ascontiguousarray(v["h0"][:nb, :nd]),
+            "delta_bias": None if v["delta_bias"] is None else np.ascontiguousarray(v["delta_bias"][:nd])}
+
+
 def run_reference(args):
+    """The reference arm: the fp64 oracle (the only reference: the pages ship no runnable
+    code) on the host cores, as it stands.  Every step is one ``O.forward`` over the same
+    contiguous sub-problem of the workload (leading batch rows and channels, prepared
+    before the timed region), sized so that warm-up and timed steps together take about
+    ``--ref-seconds``; the value is the sub-problem's elements per second."""
     w = W.WORKLOADS[args.workload]
     g = W.make_inputs(w)
     from oracle import oracle as O
-    v = {k: (None if g.get(k) is None else W.as_f32(g[k], g["dtype"]).astype(np.float64))
-         for k in ("u", "delta", "B", "C", "z")}
-    A = g["A"].astype(np.float64)
-    h0 = None if g["h0"] is None else g["h0"].astype(np.float64)
-    fk = {"delta_bias": None if g.get("delta_bias") is None else g["delta_bias"].astype(np.float64),
-          "softplus": w.fused, "z": v["z"]}
+    v = _oracle_values(g, w)
     cores = O.host_threads()
-    # each step: a bounded sample of the workload's rows (rows are independent)
-    target = max(1.0, args.ref_step_seconds)
-    rows_all = [(b, d) for b in range(w.B) for d in range(w.D)]
-    probe = rows_all[: max(1, len(rows_all) // 64)]
+    run = lambda p: O.forward(p["u"], p["delta"], p["A"], p["B"], p["C"], p["h0"], w.zoh,
+                              nthreads=cores, delta_bias=p["delta_bias"], softplus=w.fused, z=p["z"])
+    # probe: one batch row, a slice of channels, to size the step
+    nd0 = max(1, min(w.D, 2 * cores))
+    probe = _sub_problem(v, 1, nd0)
     t0 = time.perf_counter()
-    O.forward_rows(probe, v["u"], v["delta"], A, v["B"], v["C"], h0, w.zoh, nthreads=cores, **fk)
-    per_row = (time.perf_counter() - t0) / len(probe)
-    nrows = int(min(len(rows_all), max(1, target / max(per_row, 1e-9))))
-    rng = np.random.default_rng(0)
-    sel = [rows_all[i] for i in sorted(rng.choice(len(rows_all), nrows, replace=False))]
+    run(probe)
+    per_elem = (time.perf_counter() - t0) / (w.L * nd0)
+    per_step = max(0.05, args.ref_seconds / (args.steps + args.warmup))
+    want = max(1, int(per_step / max(per_elem, 1e-12) / w.L))  # (b, d) rows per step
+    nb = max(1, min(w.B, want // w.D))
+    nd = w.D if nb > 1 else max(1, min(w.D, want))
+    sub = _sub_problem(v, nb, nd)
     for _ in range(args.warmup):
-        O.forward_rows(sel[: max(1, nrows // 8)], v["u"], v["delta"], A, v["B"], v["C"], h0,
-                       w.zoh, nthreads=cores, **fk)
+        run(sub)
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
-        O.forward_rows(sel, v["u"], v["delta"], A, v["B"], v["C"], h0, w.zoh, nthreads=cores, **fk)
+        run(sub)
         times.append(time.perf_counter() - t0)
     tot = sum(times)
-    value = nrows * w.L * args.steps / tot
-    sample = f"{nrows} of {len(rows_all)} (b,d) rows x {w.L} tokens per step"
+    elems = nb * w.L * nd
+    value = elems * args.steps / tot
+    sample = (f"batch rows [0, {nb}) x channels [0, {nd}) of the workload ({elems} of {w.elements} "
+              f"elements) per step, one oracle call each")
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": f"{w.name}: B={w.B} L={w.L} D={w.D} N={w.N} io={w.dtype} "
-                               f"{'ZOH' if w.zoh else 'Euler'} h0={'yes' if w.h0_std else 'no'}"
-                               f"{' fused softplus(delta+bias), y*silu(z)' if w.fused else ''}",
-                   "B": w.B, "L": w.L, "D": w.D, "N": w.N, "io_dtype": w.dtype},
+        "config": workload_config(w, 1),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -417,12 +509,14 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="mamba130m_f32", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--workload", default="longseq_bf16", choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--per-config", type=int, default=1,
+                    help="also time the kernel on the other configurations (rank 0, outside the timed region)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="minimum host time spent timing the CPU oracle baseline")
-    ap.add_argument("--ref-step-seconds", type=float, default=2.0,
-                    help="host time per step of the reference (oracle) arm")
+    ap.add_argument("--ref-seconds", type=float, default=120.0,
+                    help="host time of the reference (oracle) arm's warm-up and timed steps together")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -204,11 +204,21 @@ SSCAN_API int sscan_version(void);
  * the parts that must start at zero are cleared on the caller's stream at the
  * start of each call, and calls whose work overlaps on the GPU (other streams,
  * other host threads) race on it.  The return value reports argument and
- * launch errors; the device status word is reset per call and not returned. */
+ * launch errors; what only the device can see (a bounded wait that gave up,
+ * leaving part of y and h_final unwritten) is latched in a status word inside
+ * the array, which each call clears at its start: read it with
+ * sscan_noalloc_status after the call and before the next one. */
 SSCAN_API int sscan_forward_noalloc(int64_t B, int64_t L, int64_t D, int64_t N, int dtype,
                                     uint32_t flags, const void *u, const void *delta, const float *A,
                                     const void *B_in, const void *C_in, const float *h0, void *y,
                                     float *h_final, void *stream);
+
+/* Status of the last sscan_forward_noalloc call on the current device: waits for
+ * `stream` (the stream that call used), reads and clears the device status word
+ * in the library's fixed array.  Allocates nothing.  Returns SSCAN_OK,
+ * SSCAN_ERR_TIMEOUT (a device wait of that call gave up: its y and h_final are
+ * incomplete) or SSCAN_ERR_CUDA. */
+SSCAN_API int sscan_noalloc_status(void *stream);
 
 #ifdef __cplusplus
 }

@@ -2,21 +2,25 @@
 
     python -m selective_state_space_32_b200.build [--force]
 
-The library is written next to this file, so it travels with the source tree
-and is found by ``sscan.py`` without any install step.
+Each translation unit under ``csrc/`` is compiled to an object of its own (in
+parallel, and only when it or a header it includes changed), then the objects
+are linked into ``libsscan.so`` next to this file, so the library travels with
+the source tree and is found by ``sscan.py`` without any install step.
 """
 from __future__ import annotations
 
 import os
+import re
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = [os.path.join(HERE, "csrc", "sscan.cu"), os.path.join(HERE, "csrc", "sscan_backward.cu")]
-HEADERS = [os.path.join(ROOT, "include", "sscan.h")] + [
-    os.path.join(HERE, "csrc", f) for f in ("device_utils.cuh", "kernel_chained.cuh", "kernel_generic.cuh",
-                                            "kernel_backward.cuh")]
+CSRC = os.path.join(HERE, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+SOURCES = sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cu"))
+OBJ_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsscan.so")
 
 NVCC_FLAGS = [
@@ -33,24 +37,62 @@ def nvcc() -> str:
     return cand if os.path.exists(cand) else "nvcc"
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def dependencies(path: str, seen=None) -> set:
+    """The file and every local header it includes (transitively), by `#include "..."`."""
+    seen = set() if seen is None else seen
+    if path in seen or not os.path.exists(path):
+        return seen
+    seen.add(path)
+    with open(path, encoding="utf-8") as f:
+        for name in re.findall(r'^\s*#\s*include\s+"([^"]+)"', f.read(), flags=re.M):
+            for d in (os.path.dirname(path), CSRC, INCLUDE):
+                cand = os.path.join(d, name)
+                if os.path.exists(cand):
+                    dependencies(cand, seen)
+                    break
+    return seen
+
+
+def obj_path(src: str) -> str:
+    return os.path.join(OBJ_DIR, os.path.splitext(os.path.basename(src))[0] + ".o")
+
+
+def stale(target: str, deps) -> bool:
+    if not os.path.exists(target):
         return True
-    t = os.path.getmtime(LIB)
-    return any(os.path.getmtime(f) > t for f in SOURCES + HEADERS + [__file__])
+    t = os.path.getmtime(target)
+    return any(os.path.getmtime(f) > t for f in list(deps) + [__file__])
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not (force or stale()):
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-shared",
-           "-o", tmp, *SOURCES]
+def _compile(src: str, verbose: bool) -> str:
+    out = obj_path(src)
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-c", "-o", tmp, src]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if verbose or r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed ({r.returncode}): {' '.join(cmd)}")
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    todo = [s for s in SOURCES if force or stale(obj_path(s), dependencies(s))]
+    if todo:
+        with ThreadPoolExecutor(max_workers=len(todo)) as ex:
+            list(ex.map(lambda s: _compile(s, verbose), todo))
+    objs = [obj_path(s) for s in SOURCES]
+    if not (force or todo or stale(LIB, objs)):
+        return LIB
+    tmp = LIB + f".tmp{os.getpid()}"
+    cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if verbose or r.returncode != 0:
+        sys.stderr.write(r.stdout + r.stderr)
+    if r.returncode != 0:
+        raise RuntimeError(f"nvcc link failed ({r.returncode}): {' '.join(cmd)}")
     os.replace(tmp, LIB)
     return LIB
 

@@ -6,9 +6,27 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 namespace sscan {
+
+// Opt kernel KERN into `bytes` of dynamic shared memory (above the 48 KB default).
+// The attribute belongs to the device that is current when it is set, so it is
+// set once per (kernel, device): one bit per device ordinal below 64, and every
+// call on a higher ordinal sets it again.
+template <auto KERN>
+inline cudaError_t smem_opt_in(int bytes) {
+    static std::atomic<unsigned long long> done{0};
+    int dev = 0;
+    const cudaError_t g = cudaGetDevice(&dev);
+    if (g != cudaSuccess) return g;
+    const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(KERN, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
 
 // ------------------------------------------------------------ packed fp32 pairs
 

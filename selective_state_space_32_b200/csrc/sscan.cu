@@ -315,12 +315,8 @@ int launch_chained_t(sscan_plan *p, const void *u, const void *dl, const float *
     constexpr int smem_bytes = help ? Cfg::kSmemH : (FUSED ? Cfg::kSmemF : Cfg::kSmem);
     constexpr int threads = help ? Cfg::kThreadsH : Cfg::kThreads;
     auto kern = sscan_chained_kernel<IO, Cfg, ZOH, POLY, SPLIT, FUSED>;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [&] {
-        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
-    });
-    if (attr_err != cudaSuccess) return SSCAN_ERR_CUDA;
+    if (smem_opt_in<sscan_chained_kernel<IO, Cfg, ZOH, POLY, SPLIT, FUSED>>(smem_bytes) != cudaSuccess)
+        return SSCAN_ERR_CUDA;
 
     const int es = sizeof(IO);
     const void *ptrs[5] = {u, dl, Bm, Cm, fu.z};
@@ -613,6 +609,20 @@ int sscan_get_status(sscan_plan_t plan, void *stream) {
     if (cudaMemcpyAsync(&v, plan->d_status, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
         cudaMemsetAsync(plan->d_status, 0, sizeof(int), s) != cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess)
+        return SSCAN_ERR_CUDA;
+    return v == 0 ? SSCAN_OK : SSCAN_ERR_TIMEOUT;
+}
+
+int sscan_noalloc_status(void *stream) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SSCAN_ERR_UNSUPPORTED;
+    unsigned char *scratch = nullptr;
+    const int rc = noalloc_scratch(dev, &scratch);
+    if (rc != SSCAN_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int v = 0;
+    if (cudaMemcpyAsync(&v, scratch, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemsetAsync(scratch, 0, sizeof(int), s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
         return SSCAN_ERR_CUDA;
     return v == 0 ? SSCAN_OK : SSCAN_ERR_TIMEOUT;
 }

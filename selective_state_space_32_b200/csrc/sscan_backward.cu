@@ -7,7 +7,6 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <mutex>
 
 #include "device_utils.cuh"
 #include "kernel_backward.cuh"
@@ -27,23 +26,11 @@ int64_t div_up(int64_t a, int64_t b) { return (a + b - 1) / b; }
 int64_t bwd_dpad(int64_t D) { return div_up(D, kBwdThreads) * kBwdThreads; }
 int64_t bwd_chunks(int64_t L) { return div_up(L, kChunk); }
 
-// Opt each backward kernel into its dynamic shared memory once (per instantiation).
-template <class IO, bool ZOH>
-cudaError_t bwd_attr() {
-    static std::once_flag once;
-    static cudaError_t err = cudaSuccess;
-    std::call_once(once, [] {
-        err = cudaFuncSetAttribute(sscan_backward_kernel<IO, ZOH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   kBwdSmem);
-    });
-    return err;
-}
-
 template <class IO, bool ZOH>
 int launch_backward(int64_t B, int64_t L, int64_t D, const void *u, const void *delta, const float *A,
                     const void *Bm, const void *Cm, const float *h0, const void *dy, const float *dhf, void *du,
                     void *ddelta, float *dA, float *dB, float *dC, float *dh0, void *ws, cudaStream_t s) {
-    if (bwd_attr<IO, ZOH>() != cudaSuccess) return SSCAN_ERR_CUDA;
+    if (smem_opt_in<sscan_backward_kernel<IO, ZOH>>(kBwdSmem) != cudaSuccess) return SSCAN_ERR_CUDA;
     const dim3 grid(static_cast<unsigned>(bwd_dpad(D) / kBwdThreads), static_cast<unsigned>(B));
     sscan_backward_kernel<IO, ZOH><<<grid, kBwdThreads, kBwdSmem, s>>>(
         static_cast<const IO *>(u), static_cast<const IO *>(delta), A, static_cast<const IO *>(Bm),

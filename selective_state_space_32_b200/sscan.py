@@ -23,7 +23,8 @@ OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPAC
 
 SYMBOLS = ("sscan_plan_create", "sscan_plan_destroy", "sscan_workspace_bytes", "sscan_forward",
            "sscan_get_status", "sscan_status_string", "sscan_plan_describe", "sscan_version",
-           "sscan_forward_noalloc", "sscan_forward_gated", "sscan_backward", "sscan_backward_workspace_bytes")
+           "sscan_forward_noalloc", "sscan_noalloc_status", "sscan_forward_gated", "sscan_backward",
+           "sscan_backward_workspace_bytes")
 
 
 class SscanError(RuntimeError):
@@ -65,6 +66,8 @@ def lib() -> ctypes.CDLL:
             L.sscan_version.restype = ip
             L.sscan_forward_noalloc.argtypes = [i64, i64, i64, i64, ip, u32] + [vp] * 9
             L.sscan_forward_noalloc.restype = ip
+            L.sscan_noalloc_status.argtypes = [vp]
+            L.sscan_noalloc_status.restype = ip
             L.sscan_forward_gated.argtypes = [vp] * 13
             L.sscan_forward_gated.restype = ip
             L.sscan_backward.argtypes = [i64, i64, i64, i64, ip, u32] + [vp] * 16
