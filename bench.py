@@ -341,6 +341,18 @@ def run_ours(args, rank, world, local_rank):
     if args.per_config:
         others = [n for n in W.ORDER[1:] if n != args.workload]
         out["per_config"] = time_other_configs(others, dev, stream, sm_max, hbm_peak)
+        for name, sw in W.SSD_WORKLOADS.items():
+            if name == "ssd_small":
+                continue
+            try:
+                _, sd = ssd_to_device(W.make_ssd_inputs(sw), dev)
+                ms = time_ssd(sw, sd, dev, stream, 20, 3)
+                km = sum(ms) / len(ms)
+                out["per_config"][name] = {"kernel_ms": km, "elements_per_s": sw.elements / (km / 1e3),
+                                           **ssd_roofline(sw, km, hbm_peak, read_peaks())}
+                del sd
+            except Exception as e:
+                out["per_config"][name] = {"error": str(e)[:200]}
     bwd = time_backward(plan, w, din, dev, stream) if (w.N == 16 and not w.fused) else None
     if bwd is not None:
         out["backward"] = bwd
@@ -433,6 +445,189 @@ def time_backward(plan, w, din, dev, stream, reps: int = 5):
         return {"error": str(e)[:200]}
 
 
+# ------------------------------------------------------------- SSD arm --
+
+def ssd_config(w, world: int) -> dict:
+    """``config`` of an SSD line (the same keys for both arms)."""
+    alg = w.algorithmic_bytes()
+    return {"workload": f"{w.name}: Mamba-2 SSD B={w.B} L={w.L} H={w.H} P={w.P} N={w.N} io=bf16 "
+                        f"(delta fp32) h0={'yes' if w.h0_std else 'no'}",
+            "B": w.B, "L": w.L, "H": w.H, "P": w.P, "N": w.N, "io_dtype": "bf16",
+            "parallelism": f"dp{world} (independent batch-row shards, no collective)",
+            "l2": f"inputs larger than L2 ({alg / 1e6:.0f} MB per step vs {L2_BYTES / 2**20:.0f} MiB L2); no flush"}
+
+
+def ssd_to_device(g, dev):
+    import torch
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+    f32 = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a, np.float32))
+    host = {"x": bf(g["x"]), "delta": f32(g["delta"]), "A": f32(g["A"]), "B": bf(g["B"]), "C": bf(g["C"]),
+            "h0": f32(g["h0"])}
+    return host, {k: (None if v is None else v.to(dev)) for k, v in host.items()}
+
+
+def ssd_oracle_values(g):
+    w = lambda a: W.bf16_bits_to_f32(a).astype(np.float64)
+    return (w(g["x"]), g["delta"].astype(np.float64), g["A"].astype(np.float64), w(g["B"]), w(g["C"]),
+            None if g["h0"] is None else g["h0"].astype(np.float64))
+
+
+def ssd_oracle_rate(g, w, pairs: int):
+    """The fp64 SSD oracle (block-chunked form, pinned to the quadratic form) as it stands,
+    single-threaded, on ``pairs`` (batch row, head) sequences of the workload (each is an
+    independent problem).  Returns (elements/s, sample description)."""
+    from oracle import ssd_oracle as O
+    x, dl, A, Bm, Cm, h0 = ssd_oracle_values(g)
+    sel = [(i % w.B, (7 * i) % w.H) for i in range(pairs)]
+    subs = [(np.ascontiguousarray(x[b:b + 1, :, h:h + 1]), np.ascontiguousarray(dl[b:b + 1, :, h:h + 1]),
+             A[h:h + 1], np.ascontiguousarray(Bm[b:b + 1]), np.ascontiguousarray(Cm[b:b + 1]),
+             None if h0 is None else np.ascontiguousarray(h0[b:b + 1, h:h + 1])) for b, h in sel]
+    t0 = time.perf_counter()
+    for sub in subs:
+        O.ssd_forward_chunked(*sub, block=64)
+    el = time.perf_counter() - t0
+    return pairs * w.L * w.P / el, f"{pairs} of {w.B * w.H} (batch row, head) sequences, one core, {el:.2f} s"
+
+
+def time_ssd(w, d, dev, stream, launches: int, warmup: int, status=None):
+    """Mean kernel time (ms) of sscan_ssd_forward over ``launches`` launches, CUDA events on
+    the launching stream around each launch, inputs resident in HBM."""
+    import torch
+    from selective_state_space_32_b200 import sscan as S
+    y = torch.empty((w.B, w.L, w.H, w.P), dtype=torch.bfloat16, device=dev)
+    hf = torch.empty((w.B, w.H, w.N, w.P), dtype=torch.float32, device=dev)
+    step = lambda: S.ssd_forward(d["x"], d["delta"], d["A"], d["B"], d["C"], d["h0"], y=y, h_final=hf,
+                                 status=status, stream=stream)
+    for _ in range(warmup):
+        step()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(launches)]
+    torch.cuda.synchronize(dev)
+    for a, b in ev:
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def ssd_roofline(w, kms, hbm_peak, peaks):
+    gbs = w.algorithmic_bytes() / (kms / 1e3) / 1e9
+    tfl = w.flops() / (kms / 1e3) / 1e12
+    bf16 = peaks.get("bf16_tflops", 1590.0)
+    return {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+            "kernel": "ssd_forward_kernel", "tensor": {"achieved_tflops": tfl, "peak_tflops": bf16,
+                                                       "frac": tfl / bf16,
+                                                       "flops_per_step": w.flops()}}
+
+
+def run_ours_ssd(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from selective_state_space_32_b200 import sscan as S
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = W.SSD_WORKLOADS[args.workload]
+    g = W.generate_ssd(w.B, w.L, w.H, w.P, w.N, w.h0_std, seed=W.SEED_BASE + w.index + 1000 * rank)
+    hin, din = ssd_to_device(g, dev)
+    hin = {k: (None if v is None else v.pin_memory()) for k, v in hin.items()}
+    stream = torch.cuda.current_stream(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    y = torch.empty((w.B, w.L, w.H, w.P), dtype=torch.bfloat16, device=dev)
+    hf = torch.empty((w.B, w.H, w.N, w.P), dtype=torch.float32, device=dev)
+    step = lambda: S.ssd_forward(din["x"], din["delta"], din["A"], din["B"], din["C"], din["h0"], y=y, h_final=hf,
+                                 status=status, stream=stream)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    kern_ms = [a.elapsed_time(b) for a, b in ev]
+    if int(status.item()) != 0:
+        raise RuntimeError("SSD kernel reported a wait that gave up")
+    # end to end: pinned host buffers, copies in and out inside the timed region
+    out_h = (torch.empty(y.shape, dtype=y.dtype).pin_memory(), torch.empty(hf.shape, dtype=hf.dtype).pin_memory())
+    e2e_steps = max(1, min(args.steps, 20))
+
+    def e2e_step():
+        dv = {k: (None if v is None else v.to(dev, non_blocking=True)) for k, v in hin.items()}
+        yy, hh = S.ssd_forward(dv["x"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["h0"], stream=stream)
+        out_h[0].copy_(yy, non_blocking=True)
+        out_h[1].copy_(hh, non_blocking=True)
+        torch.cuda.current_stream(dev).synchronize()
+
+    for _ in range(min(args.warmup, 3)):
+        e2e_step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    elapsed_ms, e2e_ms = max_over_ranks([elapsed_ms, e2e_ms], world, dev)
+    if rank != 0:
+        return None
+    hbm_peak, sm_max, peak_src = load_peaks()
+    kmean = sum(kern_ms) / len(kern_ms)
+    cpu_value, sample = ssd_oracle_rate(g, w, args.ssd_oracle_pairs)
+    h2d = sum(v.numel() * v.element_size() for v in hin.values() if v is not None)
+    d2h = sum(v.numel() * v.element_size() for v in out_h)
+    return {
+        "metric": METRIC, "value": w.elements * args.steps * world / (elapsed_ms / 1e3), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 (fp32 accumulate)",
+        "data": "synthetic", "config": ssd_config(w, world),
+        "roofline": ssd_roofline(w, kmean, hbm_peak, read_peaks()),
+        "kernel_ms": {"mean": kmean, "min": min(kern_ms), "max": max(kern_ms)},
+        "e2e": {"value": w.elements * e2e_steps * world / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": args.steps, "clocks": clk.summary(),
+        "cpu_baseline": {"value": cpu_value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+    }
+
+
+def run_reference_ssd(args):
+    w = W.SSD_WORKLOADS[args.workload]
+    g = W.make_ssd_inputs(w)
+    pairs = max(1, args.ssd_oracle_pairs)
+    for _ in range(args.warmup):
+        ssd_oracle_rate(g, w, 1)
+    rates = [ssd_oracle_rate(g, w, pairs)[0] for _ in range(args.steps)]
+    value = len(rates) / sum(1.0 / r for r in rates)
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * pairs * w.L * w.P / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": ssd_config(w, 1),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"{pairs} (batch row, head) sequences per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def read_peaks() -> dict:
+    try:
+        with open(PEAKS_FILE) as f:
+            return json.load(f)
+    except Exception:
+        return {}
+
+
 # -------------------------------------------------------- reference arm --
 
 def _oracle_values(g, w):
@@ -509,7 +704,11 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="longseq_bf16", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--workload", default="longseq_bf16", choices=sorted(W.WORKLOADS) + sorted(W.SSD_WORKLOADS))
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch rows (small cases for profiling); 0 keeps it")
+    ap.add_argument("--ssd-oracle-pairs", type=int, default=4,
+                    help="(batch row, head) sequences the SSD oracle baseline times")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--per-config", type=int, default=1,
                     help="also time the kernel on the other configurations (rank 0, outside the timed region)")
@@ -526,9 +725,16 @@ def main():
     if world != args.gpus:
         if world == 1 and args.gpus > 1:
             ap.error("--gpus > 1 needs one process per GPU (torch.distributed.run)")
+    if args.batch > 0:
+        import dataclasses
+        if args.workload in W.SSD_WORKLOADS:
+            W.SSD_WORKLOADS[args.workload] = dataclasses.replace(W.SSD_WORKLOADS[args.workload], B=args.batch)
+        else:
+            W.WORKLOADS[args.workload] = dataclasses.replace(W.WORKLOADS[args.workload], B=args.batch)
+    is_ssd = args.workload in W.SSD_WORKLOADS
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(run_reference(args)), flush=True)
+            print(json.dumps(run_reference_ssd(args) if is_ssd else run_reference(args)), flush=True)
         return
     if world > 1:
         import datetime
@@ -538,7 +744,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        out = run_ours(args, rank, world, local_rank)
+        out = (run_ours_ssd if is_ssd else run_ours)(args, rank, world, local_rank)
         if out is not None:
             print(json.dumps(out), flush=True)
     finally:

@@ -166,6 +166,39 @@ SSCAN_API int sscan_backward(int64_t B, int64_t L, int64_t D, int64_t N, int dty
                    const void *dy, const float *dh_final, void *du, void *ddelta, float *dA, float *dB, float *dC,
                    float *dh0, void *workspace, void *stream);
 
+/* Mamba-2 state-space-duality (SSD) forward ("Mamba & Mamba-2 Architecture",
+ * section 3, "Mamba-2 and State Space Duality (SSD)"): one scalar transition
+ * per head, a_t = exp(delta[b,t,h] * A[h]); B and C shared by all heads; per
+ * batch row b and head h, with Bbar_s = delta[b,s,h] * B[b,s,:],
+ *
+ *     y[b,t,h,:]    = sum_{s <= t} (C[b,t,:] . Bbar_s) (prod_{k=s+1..t} a_k) x[b,s,h,:]
+ *                     + (prod_{k <= t} a_k) C[b,t,:] h0[b,h]          (Y = (M o C Bbar^T) X)
+ *     h_final[b,h]  = sum_s (prod_{k > s} a_k) Bbar_s^T x[b,s,h,:] + (prod_k a_k) h0[b,h]
+ *
+ * computed block by block (128 tokens) on the tensor cores: the intra-block
+ * matrix times X, the inter-block term from the carried state, and the state
+ * passing between blocks.  Shape-based (no plan, no workspace):
+ *   B, L, H     batch rows, tokens, heads (B, H >= 1; L >= 0)
+ *   P, N        head dimension and state size; P = 64, N = 128 are compiled in
+ *               (others: SSCAN_ERR_UNSUPPORTED)
+ *   x           [B][L][H][P] bf16
+ *   delta       [B][L][H] fp32, the step after softplus (>= 0)
+ *   A           [H] fp32 (A <= 0, the decay per unit step)
+ *   B_in, C_in  [B][L][N] bf16
+ *   h0          [B][H][N][P] fp32, or NULL for a zero initial state
+ *   y           [B][L][H][P] bf16 (output; round to nearest even)
+ *   h_final     [B][H][N][P] fp32 (output), or NULL; may be the same buffer as h0
+ *   status      a device int the kernel ORs error bits into when one of its
+ *               bounded waits gives up (y and h_final then incomplete), or NULL
+ * Every pointer is caller-owned device memory, 16-byte aligned (status: 4);
+ * nothing is retained and nothing is allocated.  Asynchronous on `stream`.
+ * Arithmetic: bf16 MMA operands (x, B, C as given; the intra-block matrix, the
+ * carried state and the decay-weighted x rounded to bf16 as operands), fp32
+ * accumulation, fp32 state and decays.  Errors as for sscan_forward. */
+SSCAN_API int sscan_ssd_forward(int64_t B, int64_t L, int64_t H, int64_t P, int64_t N, const void *x,
+                                const float *delta, const float *A, const void *B_in, const void *C_in,
+                                const float *h0, void *y, float *h_final, int *status, void *stream);
+
 /* Wait for `stream`, then read and clear the plan's device status word.
  * Returns SSCAN_OK, SSCAN_ERR_TIMEOUT, or SSCAN_ERR_CUDA. */
 SSCAN_API int sscan_get_status(sscan_plan_t plan, void *stream);

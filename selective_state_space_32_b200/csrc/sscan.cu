@@ -11,8 +11,11 @@
 // Two kernels:
 //  * chained (kernel_chained.cuh): persistent, cooperative, one warp per
 //    chain segment, TMA-staged inputs, exactly balanced work per warp;
+//  * step (kernel_step.cuh): four states per thread, shaped for the state's
+//    HBM round trip; sequences shorter than the chained kernel's minimum,
+//    the single-token decode step in particular;
 //  * generic (kernel_generic.cuh): one thread per (channel, state group),
-//    plain loads; for shapes the chained kernel cannot take.
+//    plain loads; for the longer shapes the chained kernel cannot take.
 // Both keep every (b,d) state row in registers; the [B,L,D,N] tensors never
 // reach memory.  The path is ALU bound on B200 (one 2^x and four FMA-pipe
 // operations per state update against 1-3 bytes of HBM traffic), so there are
@@ -32,6 +35,7 @@
 #include "device_utils.cuh"
 #include "kernel_chained.cuh"
 #include "kernel_generic.cuh"
+#include "kernel_step.cuh"
 #include "sscan.h"
 
 #define SSCAN_VERSION 200  // 0.2.0
@@ -40,7 +44,7 @@ using namespace sscan;
 
 namespace {
 
-enum Mode { kGeneric = 0, kChained = 1 };
+enum Mode { kGeneric = 0, kChained = 1, kStep = 2 };
 
 // Chained-kernel shapes compiled into the library.  NL states per lane, T
 // tokens per pipeline stage, STAGES stages per warp, WPC warps per block.
@@ -79,7 +83,7 @@ constexpr int kMaxSmem = 227 * 1024;  // dynamic shared memory per block on B200
 // launch ends with its slowest warp; they get 3x fewer chain-steps and the others
 // x more, x = S * kLightPermille / 1000, which evens out the finishing times.
 constexpr int kLightPermille = 10;
-constexpr int64_t kMinChainedL = 64;  // shorter sequences use the generic kernel
+constexpr int64_t kMinChainedL = 64;  // shorter sequences use the step kernel
 
 // Shared memory of a chained-kernel shape (mirrors ChainedCfg::kSmem; a fused call on a
 // shape whose larger ChainedCfg::kSmemF does not fit runs the generic kernel).
@@ -184,13 +188,15 @@ void choose_schedule(sscan_plan *p) {
     const int blocks = (sms > 0 && sms < p->sm_count) ? sms : p->sm_count;
     // the FMA-pipe exponent measured slower than MUFU alone at every occupancy: off unless asked
     p->poly = (p->flags & SSCAN_ZOH) ? false : (poly == 1);
-    if (want == -1) return;
-    // the chained kernel needs TMA-compatible rows and int32 TMA row coordinates; very
-    // short sequences (e.g. one decode step, L = 1) are better served by the generic
-    // kernel than by a persistent grid with a TMA pipeline
-    if (p->L < kMinChainedL || (p->D * es) % 16 != 0 || p->B * p->L >= (int64_t(1) << 31) ||
-        p->L >= (int64_t(1) << 32))
+    // very short sequences (e.g. one decode step, L = 1) are a stream over the state:
+    // the step kernel, not a persistent grid with a TMA pipeline
+    if (p->L < kMinChainedL && want != -1) {
+        p->mode = kStep;
         return;
+    }
+    if (want == -1) return;
+    // the chained kernel needs TMA-compatible rows and int32 TMA row coordinates
+    if ((p->D * es) % 16 != 0 || p->B * p->L >= (int64_t(1) << 31) || p->L >= (int64_t(1) << 32)) return;
     // 1) chained: enough chains that each is cut at most once (segment >= L)
     // 2) split: fewer chains than warps; cut them into pieces scanned concurrently
     for (int pass = force_split ? 1 : 0; pass < 2; ++pass) {
@@ -275,6 +281,32 @@ cudaError_t launch_generic(const sscan_plan *p, const void *u, const void *dl, c
         case 16: return launch_generic_t<IO, 8, 2>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s);
         case 32: return launch_generic_t<IO, 16, 2>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s);
         default: return launch_generic_t<IO, 16, 4>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s);
+    }
+}
+
+// --------------------------------------------------------------- step launch
+
+template <class IO, int N>
+cudaError_t launch_step_t(const sscan_plan *p, const void *u, const void *dl, const float *A, const void *Bm,
+                          const void *Cm, const float *h0, void *y, float *hf, const Fused &fu, cudaStream_t s) {
+    constexpr int per_block = kStepThreads / (N / 4) * kStepItems;  // channels per block
+    const int64_t channels = p->B * p->D;
+    const dim3 grid(static_cast<unsigned>(ceil_div(channels, per_block)));
+    auto kern = (p->flags & SSCAN_ZOH) ? sscan_step_kernel<IO, N, true> : sscan_step_kernel<IO, N, false>;
+    kern<<<grid, kStepThreads, 0, s>>>(static_cast<const IO *>(u), static_cast<const IO *>(dl), A,
+                                       static_cast<const IO *>(Bm), static_cast<const IO *>(Cm), h0,
+                                       static_cast<IO *>(y), hf, p->L, p->D, channels, fu.bias,
+                                       static_cast<const IO *>(fu.z), fu.softplus ? 1 : 0);
+    return cudaGetLastError();
+}
+
+template <class IO>
+cudaError_t launch_step(const sscan_plan *p, const void *u, const void *dl, const float *A, const void *Bm,
+                        const void *Cm, const float *h0, void *y, float *hf, const Fused &fu, cudaStream_t s) {
+    switch (p->N) {
+        case 16: return launch_step_t<IO, 16>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s);
+        case 32: return launch_step_t<IO, 32>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s);
+        default: return launch_step_t<IO, 64>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s);
     }
 }
 
@@ -421,6 +453,14 @@ int launch_chained(sscan_plan *p, const void *u, const void *dl, const float *A,
 
 }  // namespace
 
+// No tokens: the final state is the initial one (zero without h0).
+int step_empty(const sscan_plan *p, const float *h0, float *hf, cudaStream_t s) {
+    if (hf == nullptr || hf == h0) return SSCAN_OK;
+    const size_t bytes = static_cast<size_t>(p->B * p->D * p->N) * sizeof(float);
+    const cudaError_t e = h0 ? cudaMemcpyAsync(hf, h0, bytes, cudaMemcpyDeviceToDevice, s) : cudaMemsetAsync(hf, 0, bytes, s);
+    return e == cudaSuccess ? SSCAN_OK : SSCAN_ERR_CUDA;
+}
+
 // ------------------------------------------------ allocation-free entry point
 
 namespace {
@@ -535,6 +575,13 @@ int sscan_plan_describe(sscan_plan_t plan, char *buf, size_t len) {
                      plan->split ? 1 : 0,
                      (long long)plan->chains, (long long)plan->workers, (long long)plan->seg, (long long)plan->seg_shift, plan->ws_bytes,
                      plan->sm_count);
+    } else if (plan->mode == kStep) {
+        n = snprintf(tmp, sizeof tmp,
+                     "kernel=step B=%lld L=%lld D=%lld N=%lld dtype=%s zoh=%d states_per_thread=4 "
+                     "threads_per_channel=%lld channels_per_thread=%d block=%d sms=%d",
+                     (long long)plan->B, (long long)plan->L, (long long)plan->D, (long long)plan->N,
+                     plan->dtype == SSCAN_F32 ? "f32" : "bf16", (plan->flags & SSCAN_ZOH) ? 1 : 0,
+                     (long long)(plan->N / 4), kStepItems, kStepThreads, plan->sm_count);
     } else {
         n = snprintf(tmp, sizeof tmp,
                      "kernel=generic B=%lld L=%lld D=%lld N=%lld dtype=%s zoh=%d states_per_thread=%d "
@@ -595,6 +642,13 @@ int sscan_forward_gated(sscan_plan_t plan, const void *u, const void *delta, con
         return p->dtype == SSCAN_F32
                    ? launch_chained<float>(p, u, delta, A, B, C, h0, y, h_final, workspace, fu, s)
                    : launch_chained<uint16_t>(p, u, delta, A, B, C, h0, y, h_final, workspace, fu, s);
+    }
+    if (p->mode == kStep) {
+        if (p->L == 0) return step_empty(p, h0, h_final, s);
+        const cudaError_t e =
+            p->dtype == SSCAN_F32 ? launch_step<float>(p, u, delta, A, B, C, h0, y, h_final, fu, s)
+                                  : launch_step<uint16_t>(p, u, delta, A, B, C, h0, y, h_final, fu, s);
+        return e == cudaSuccess ? SSCAN_OK : SSCAN_ERR_CUDA;
     }
     const cudaError_t e =
         p->dtype == SSCAN_F32 ? launch_generic<float>(p, u, delta, A, B, C, h0, y, h_final, fu, s)

@@ -24,7 +24,7 @@ OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPAC
 SYMBOLS = ("sscan_plan_create", "sscan_plan_destroy", "sscan_workspace_bytes", "sscan_forward",
            "sscan_get_status", "sscan_status_string", "sscan_plan_describe", "sscan_version",
            "sscan_forward_noalloc", "sscan_noalloc_status", "sscan_forward_gated", "sscan_backward",
-           "sscan_backward_workspace_bytes")
+           "sscan_backward_workspace_bytes", "sscan_ssd_forward")
 
 
 class SscanError(RuntimeError):
@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
             L.sscan_backward.restype = ip
             L.sscan_backward_workspace_bytes.argtypes = [i64, i64, i64, i64]
             L.sscan_backward_workspace_bytes.restype = sz
+            L.sscan_ssd_forward.argtypes = [i64, i64, i64, i64, i64] + [vp] * 10
+            L.sscan_ssd_forward.restype = ip
             _lib = L
     return _lib
 
@@ -280,3 +282,37 @@ def forward_host(u, delta, A, B, C, h0=None, zoh: bool = False, device="cuda", o
     for st in streams:
         st.synchronize()
     return out
+
+
+def ssd_forward(x, delta, A, B, C, h0=None, y=None, h_final=None, want_final: bool = True,
+                status=None, stream=None):
+    """Mamba-2 SSD forward (``sscan_ssd_forward``) on CUDA tensors.
+
+    x: [B, L, H, P] bfloat16; delta: [B, L, H] float32; A: [H] float32; B, C:
+    [B, L, N] bfloat16; h0: [B, H, N, P] float32 or None; status: a CUDA int32
+    tensor of one element the kernel ORs error bits into, or None.
+    Returns (y [B, L, H, P] bfloat16, h_final [B, H, N, P] float32 or None)."""
+    Bt, L, H, P = x.shape
+    N = B.shape[-1]
+    dev = x.device
+    if y is None:
+        y = torch.empty((Bt, L, H, P), dtype=torch.bfloat16, device=dev)
+    if h_final is None and want_final:
+        h_final = torch.empty((Bt, H, N, P), dtype=torch.float32, device=dev)
+    for name, t, shape, dt in (("x", x, (Bt, L, H, P), torch.bfloat16), ("delta", delta, (Bt, L, H), torch.float32),
+                               ("A", A, (H,), torch.float32), ("B", B, (Bt, L, N), torch.bfloat16),
+                               ("C", C, (Bt, L, N), torch.bfloat16), ("h0", h0, (Bt, H, N, P), torch.float32),
+                               ("y", y, (Bt, L, H, P), torch.bfloat16),
+                               ("h_final", h_final, (Bt, H, N, P), torch.float32),
+                               ("status", status, (1,), torch.int32)):
+        if t is None:
+            continue
+        if tuple(t.shape) != shape or t.dtype != dt or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name}: want contiguous CUDA {dt} {shape}, got {t.dtype} {tuple(t.shape)} on {t.device}")
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    rc = lib().sscan_ssd_forward(Bt, L, H, P, N, _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(h0),
+                                 _ptr(y), _ptr(h_final), _ptr(status), ctypes.c_void_p(stream.cuda_stream))
+    if rc != OK:
+        raise SscanError(rc, "sscan_ssd_forward")
+    return y, h_final

@@ -197,3 +197,87 @@ def make_inputs(w: Workload) -> dict:
     """Inputs of a named workload, seeded with SEED_BASE + its index."""
     return generate(w.B, w.L, w.D, w.N, w.dtype, w.h0_std, w.reset_frac, SEED_BASE + w.index,
                     fused=w.fused)
+
+
+# --------------------------------------------------------------------------
+# Mamba-2 SSD form ("Mamba & Mamba-2 Architecture", section 3): one scalar
+# transition per head, B and C shared by the heads.
+
+@dataclasses.dataclass(frozen=True)
+class SsdWorkload:
+    name: str
+    B: int
+    L: int
+    H: int
+    P: int
+    N: int
+    h0_std: float
+    index: int
+
+    @property
+    def elements(self) -> int:
+        """Scanned elements B*L*H*P (the heads' channels, as B*L*D for the selective scan)."""
+        return self.B * self.L * self.H * self.P
+
+    def algorithmic_bytes(self) -> int:
+        """x and y (bf16), delta (fp32, [B,L,H]), B and C (bf16), A, h_final and h0 (fp32)."""
+        return (2 * 2 * self.B * self.L * self.H * self.P + 4 * self.B * self.L * self.H
+                + 2 * 2 * self.B * self.L * self.N + 4 * self.H
+                + 4 * self.B * self.H * self.N * self.P * (1 + (self.h0_std > 0)))
+
+    def flops(self) -> int:
+        """Useful multiply-adds x 2 of the block algorithm with 128-token blocks: per block
+        and head, C B^T (Q*Q*N; counted once per batch row and block, shared by the heads),
+        the causal half of (S o L) X (Q*(Q+1)/2*P), C h_in and B^T (w X) (Q*N*P each)."""
+        q = 128
+        nblk = -(-self.L // q)
+        per_bh = nblk * (q * (q + 1) // 2 * self.P + 2 * q * self.N * self.P)
+        return 2 * (self.B * self.H * per_bh + self.B * nblk * q * q * self.N)
+
+
+SSD_WORKLOADS = {
+    # parity-sized: two full blocks and a ragged one, a nonzero initial state
+    "ssd_small": SsdWorkload("ssd_small", 2, 300, 4, 64, 128, 0.1, 20),
+    # a Mamba-2 1.3B-like layer (d_model 2048, expand 2 -> 4096 channels = 64 heads of 64,
+    # state 128, one group), 8 sequences of 2048 tokens
+    "ssd_mamba2_1p3b": SsdWorkload("ssd_mamba2_1p3b", 8, 2048, 64, 64, 128, 0.0, 21),
+}
+
+
+def generate_ssd(B: int, L: int, H: int, P: int, N: int, h0_std: float = 0.0, seed: int = SEED_BASE,
+                 reset_frac: float = 0.0, A_zero: bool = False) -> dict:
+    """Seeded inputs of the SSD form.
+
+    Draw order from PCG64(seed), fp64: dt[h] log-uniform in [1e-3, 1e-1] per head;
+    A_log[h] = log(U[1, 16]) (A = -exp(A_log) in [-16, -1], the Mamba-2 range);
+    the reset mask (reset_frac > 0: round(reset_frac * L) positions per batch row get
+    delta + 3, the others delta * 0.01, as for the long-sequence selective scan);
+    z ~ N(0, 1) [B, L, H] -> delta = softplus(0.5 z + softplus^-1(dt[h])) kept in fp32;
+    x ~ N(0, 1) [B, L, H, P]; B, C ~ N(0, 1) [B, L, N]; h0 ~ N(0, h0_std^2)
+    [B, H, N, P] fp32 when h0_std > 0.  x, B, C are rounded to bf16 (uint16 bit
+    patterns).  A_zero sets A = 0 (every decay 1: causal linear attention)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    dt = np.exp(rng.uniform(math.log(1e-3), math.log(1e-1), size=H))
+    A_log = np.log(rng.uniform(1.0, 16.0, size=H))
+    reset = None
+    if reset_frac > 0:
+        k = int(round(reset_frac * L))
+        reset = np.zeros((B, L), dtype=bool)
+        for b in range(B):
+            reset[b, rng.permutation(L)[:k]] = True
+    z = rng.standard_normal((B, L, H))
+    delta = _softplus(0.5 * z + _inv_softplus(dt)[None, None, :])
+    if reset is not None:
+        delta = np.where(reset[:, :, None], delta + 3.0, delta * 0.01)
+    x = _store(rng.standard_normal(B * L * H * P), "bf16").reshape(B, L, H, P)
+    Bm = _store(rng.standard_normal(B * L * N), "bf16").reshape(B, L, N)
+    Cm = _store(rng.standard_normal(B * L * N), "bf16").reshape(B, L, N)
+    h0 = None
+    if h0_std > 0:
+        h0 = (h0_std * rng.standard_normal(B * H * N * P)).astype(np.float32).reshape(B, H, N, P)
+    A = np.zeros(H, np.float32) if A_zero else (-np.exp(A_log)).astype(np.float32)
+    return {"x": x, "delta": delta.astype(np.float32), "A": A, "B": Bm, "C": Cm, "h0": h0}
+
+
+def make_ssd_inputs(w: SsdWorkload) -> dict:
+    return generate_ssd(w.B, w.L, w.H, w.P, w.N, w.h0_std, SEED_BASE + w.index)

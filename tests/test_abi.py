@@ -102,3 +102,12 @@ def test_backward_workspace_bytes(lib):
     assert lib.sscan_backward_workspace_bytes(2, 37, 70, 16) == 2 * 128 * 5 * 16 * 4
     assert lib.sscan_backward_workspace_bytes(2, 37, 70, 32) == 0
     assert lib.sscan_backward_workspace_bytes(2, 0, 70, 16) == 0
+
+
+def test_ssd_rejects_bad_shapes_without_a_device(lib):
+    # size checks come before any CUDA call (no pointer is touched)
+    assert lib.sscan_ssd_forward(1, 64, 2, 32, 128, *([None] * 10)) == S.ERR_UNSUPPORTED   # P = 32
+    assert lib.sscan_ssd_forward(1, 64, 2, 64, 16, *([None] * 10)) == S.ERR_UNSUPPORTED    # N = 16
+    assert lib.sscan_ssd_forward(0, 64, 2, 64, 128, *([None] * 10)) == S.ERR_INVALID       # B = 0
+    assert lib.sscan_ssd_forward(1, -1, 2, 64, 128, *([None] * 10)) == S.ERR_INVALID       # L < 0
+    assert lib.sscan_ssd_forward(1, 64, 2, 64, 128, *([None] * 10)) == S.ERR_INVALID       # no A

@@ -124,21 +124,23 @@ def test_fused_split_forced(case, monkeypatch):
 
 
 GENERIC = [
-    # (B, L, D, N, dtype, zoh): shapes the generic kernel takes
-    (2, 100, 70, 16, "f32", False),     # D * 4 % 16 != 0
-    (3, 37, 96, 16, "bf16", False),     # L < 64
-    (2, 50, 44, 32, "bf16", True),      # ZOH, N = 32, D * 2 % 16 != 0
-    (1, 45, 20, 64, "f32", True),       # N = 64
+    # (B, L, D, N, dtype, zoh, kernel): shapes the chained kernel does not take
+    (2, 100, 70, 16, "f32", False, "generic"),    # D * 4 % 16 != 0
+    (2, 80, 44, 32, "bf16", True, "generic"),     # ZOH, N = 32, D * 2 % 16 != 0
+    (1, 70, 22, 64, "f32", True, "generic"),      # N = 64, D * 4 % 16 != 0
+    (3, 37, 96, 16, "bf16", False, "step"),       # L < 64
+    (2, 50, 44, 32, "bf16", True, "step"),        # ZOH, N = 32, ragged D
+    (1, 45, 20, 64, "f32", True, "step"),         # N = 64
 ]
 
 
-@pytest.mark.parametrize("case", GENERIC, ids=[f"B{c[0]}L{c[1]}D{c[2]}N{c[3]}{c[4]}{'_zoh' if c[5] else ''}"
+@pytest.mark.parametrize("case", GENERIC, ids=[f"B{c[0]}L{c[1]}D{c[2]}N{c[3]}{c[4]}{'_zoh' if c[5] else ''}_{c[6]}"
                                                 for c in GENERIC])
-def test_fused_generic(case):
-    Bt, L, D, N, dt, zoh = case
+def test_fused_generic_and_step(case):
+    Bt, L, D, N, dt, zoh, kernel = case
     g = W.generate(Bt, L, D, N, dt, 0.1, seed=7000 + L + D, A_jitter=0.3, fused=True)
     plan = S.Plan(Bt, L, D, N, _tdt(dt), zoh, delta_softplus=True)
-    assert "kernel=generic" in plan.describe(), plan.describe()
+    assert f"kernel={kernel}" in plan.describe(), plan.describe()
     y, hf, _ = _run_plan(plan, g)
     yr, hr = P.run_oracle(g, zoh, softplus=True)
     P.check(y.float().cpu().numpy(), yr, dt, "y")

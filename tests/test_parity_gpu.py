@@ -37,6 +37,11 @@ SMALL = [
     (1, 200, 40, 64, "bf16", False, True, 0.0),
     (2, 64, 200, 32, "bf16", True, True, 0.5),
     (1, 1000, 64, 16, "f32", True, True, 0.0),      # long-ish horizon, exact ZOH in fp32
+    # short sequences (the step kernel): ragged channel counts, every N, both I/O types
+    (5, 33, 50, 32, "bf16", True, True, 0.3),
+    (7, 1, 300, 64, "f32", True, False, 0.3),
+    (3, 63, 129, 16, "bf16", False, False, 0.0),
+    (130, 1, 77, 16, "f32", True, True, 0.3),       # many rows, several blocks, ragged last block
 ]
 
 
@@ -228,7 +233,7 @@ def test_decode_steps_match_one_forward(dt, zoh):
     y_full, h_full = S.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"], zoh=zoh)
     tdt = torch.float32 if dt == "f32" else torch.bfloat16
     plan = S.get_plan(Bt, 1, D, N, tdt, zoh)
-    assert "kernel=generic" in plan.describe()
+    assert "kernel=step" in plan.describe()
     state = d["h0"].clone()
     ys = []
     for t in range(L):
@@ -288,7 +293,8 @@ def _sample_rows(w, k, seed):
 
 
 @pytest.mark.parametrize("name,k", [("mamba130m_f32", 256), ("mamba1p4b_bf16", 128),
-                                    ("longseq_bf16", 48), ("zoh_n64_bf16", 192)])
+                                    ("longseq_bf16", 48), ("zoh_n64_bf16", 192),
+                                    ("decode_b256_f32", 2048)])
 def test_full_workload_sampled_rows(name, k):
     w = W.WORKLOADS[name]
     g = W.make_inputs(w)
