@@ -353,9 +353,8 @@ def run_ours(args, rank, world, local_rank):
                 del sd
             except Exception as e:
                 out["per_config"][name] = {"error": str(e)[:200]}
-    bwd = time_backward(plan, w, din, dev, stream) if (w.N == 16 and not w.fused) else None
-    if bwd is not None:
-        out["backward"] = bwd
+    if args.per_config:
+        out["backward"] = time_backward(dev, stream)
     plan.close()
     return out
 
@@ -422,12 +421,18 @@ def time_other_configs(names, dev, stream, sm_max, hbm_peak, launches: int = 20,
     return out
 
 
-def time_backward(plan, w, din, dev, stream, reps: int = 5):
-    """The backward pass (sscan_backward) on the same inputs, after the timed forward
-    region: mean of ``reps`` launches (CUDA events), reported beside the forward."""
+def time_backward(dev, stream, name: str = "mamba130m_f32", reps: int = 5):
+    """The backward pass (sscan_backward) on the named workload's inputs (a fixed
+    shape, whatever the headline workload is), dy = 1: mean of ``reps`` launches
+    (CUDA events), reported beside the forward."""
     import torch
+    from selective_state_space_32_b200 import sscan as S
     try:
-        dy = torch.ones((w.B, w.L, w.D), dtype=din["u"].dtype, device=dev)
+        w = W.WORKLOADS[name]
+        din = to_device(W.make_inputs(w), dev)
+        tdt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+        plan = S.Plan(w.B, w.L, w.D, w.N, tdt, w.zoh)
+        dy = torch.ones((w.B, w.L, w.D), dtype=tdt, device=dev)
         f = lambda: plan.backward(din["u"], din["delta"], din["A"], din["B"], din["C"], din["h0"], dy,
                                   stream=stream)
         f()
@@ -439,8 +444,11 @@ def time_backward(plan, w, din, dev, stream, reps: int = 5):
         b.record(stream)
         torch.cuda.synchronize(dev)
         ms = a.elapsed_time(b) / reps
-        return {"kernel_ms": ms, "value": w.elements / (ms / 1e3), "unit": UNIT, "launches": reps,
-                "note": "sscan_backward (du, ddelta, dA, dB, dC, dh0; first version), dy = 1"}
+        plan.close()
+        return {"workload": name, "kernel_ms": ms, "value": w.elements / (ms / 1e3), "unit": UNIT,
+                "launches": reps, "note": "sscan_backward (du, ddelta, dA, dB, dC, dh0), dy = 1; "
+                "3 exponentials per state update (forward checkpoints, recompute, reverse)",
+                "mufu_only_frac": 3 * w.updates / (ms / 1e3) / (16.0 * SM_COUNT * SM_MAX_MHZ * 1e6)}
     except Exception as e:  # reported, never fatal for the forward line
         return {"error": str(e)[:200]}
 

@@ -140,17 +140,20 @@ SSCAN_API int sscan_forward_gated(sscan_plan_t plan, const void *u, const void *
                         const void *B, const void *C, const float *h0, const float *delta_bias,
                         const void *z, void *y, float *h_final, void *workspace, void *stream);
 
-/* Backward pass of the plain forward (no fused prologue / epilogue; N = 16):
- * gradients of a loss given dy = dLoss/dy and optionally dh_final =
- * dLoss/dh_final, by the chain rule through h_t = Abar_t h_{t-1} + beta_t u_t,
- * y_t = C_t . h_t, the states recomputed from checkpoints rather than stored
- * ("Selective State-Space Models (Mamba) and Hardware-Aware Scans", section
- * 3, backward-pass recomputation).  Shape-based (no plan):
- *   B, L, D, N, dtype, flags  as for sscan_plan_create (flags: 0 or SSCAN_ZOH)
- *   u, delta, A, B_in, C_in, h0  the forward's inputs (as for sscan_forward)
+/* Backward pass of the forward: gradients of a loss given dy = dLoss/dy and
+ * optionally dh_final = dLoss/dh_final, by the chain rule through
+ * h_t = Abar_t h_{t-1} + beta_t u_t, y_t = C_t . h_t, the states recomputed
+ * from checkpoints rather than stored ("Selective State-Space Models (Mamba)
+ * and Hardware-Aware Scans", section 3, backward-pass recomputation).
+ * Shape-based (no plan):
+ *   B, L, D, N, dtype, flags  as for sscan_plan_create (N = 16, 32 or 64; flags
+ *                           SSCAN_ZOH and SSCAN_DELTA_SOFTPLUS as in the forward)
+ *   u, delta, A, B_in, C_in, h0  the forward's inputs (as for sscan_forward;
+ *                           delta is the raw step when SSCAN_DELTA_SOFTPLUS is set)
  *   dy                      [B][L][D], dtype
  *   dh_final                [B][D][N] fp32, or NULL (zero)
- *   du, ddelta              [B][L][D], dtype (output)
+ *   du, ddelta              [B][L][D], dtype (output; ddelta is the gradient of
+ *                           the delta passed in, i.e. of the raw step when fused)
  *   dA                      [D][N] fp32 (output; summed over batch and time)
  *   dB, dC                  [B][L][N] fp32 (output; summed over channels)
  *   dh0                     [B][D][N] fp32 (output), or NULL to skip it
@@ -158,13 +161,36 @@ SSCAN_API int sscan_forward_gated(sscan_plan_t plan, const void *u, const void *
  *                           (the state checkpoints), 16-byte aligned
  * All pointers are caller-owned device memory; nothing is retained.  dA, dB
  * and dC are accumulated with fp32 atomics, so their last bits depend on the
- * order of arrival.  Returns SSCAN_ERR_UNSUPPORTED for N != 16 or
- * SSCAN_DELTA_SOFTPLUS; the other errors as for sscan_forward. */
+ * order of arrival.  Errors as for sscan_forward (SSCAN_ERR_UNSUPPORTED for N
+ * outside {16, 32, 64}).  sscan_backward is sscan_backward_gated without a
+ * bias and a gate. */
 SSCAN_API size_t sscan_backward_workspace_bytes(int64_t B, int64_t L, int64_t D, int64_t N);
 SSCAN_API int sscan_backward(int64_t B, int64_t L, int64_t D, int64_t N, int dtype, uint32_t flags, const void *u,
                    const void *delta, const float *A, const void *B_in, const void *C_in, const float *h0,
                    const void *dy, const float *dh_final, void *du, void *ddelta, float *dA, float *dB, float *dC,
                    float *dh0, void *workspace, void *stream);
+
+/* Backward pass of sscan_forward_gated (the fused prologue delta' =
+ * softplus(delta + delta_bias) and gate y' = y silu(z)): the arguments of
+ * sscan_backward plus
+ *   delta_bias              [D] fp32 as passed to the forward, or NULL
+ *   z                       [B][L][D], dtype, the forward's gate, or NULL
+ *   ddelta_bias             [D] fp32 (output, summed over batch and time;
+ *                           required when delta_bias is given, else NULL)
+ *   dz                      [B][L][D], dtype (output; required when z is given)
+ * dy is the gradient of the gated output y'; ddelta the gradient of the raw
+ * delta.  By the chain rule around the plain backward: the scan's output
+ * gradient is dy silu(z), dz = dy ys silu'(z) with ys the scan's output
+ * (recomputed), ddelta_raw = ddelta' sigmoid(delta + delta_bias) under
+ * softplus ("Selective State-Space Models (Mamba) and Hardware-Aware Scans",
+ * section 4, the gate; "tm_ssm_selective", "The mechanism: parameters as
+ * functions of the input", the softplus step). */
+SSCAN_API int sscan_backward_gated(int64_t B, int64_t L, int64_t D, int64_t N, int dtype, uint32_t flags,
+                                   const void *u, const void *delta, const float *A, const void *B_in,
+                                   const void *C_in, const float *h0, const float *delta_bias, const void *z,
+                                   const void *dy, const float *dh_final, void *du, void *ddelta, float *dA,
+                                   float *dB, float *dC, float *dh0, float *ddelta_bias, void *dz,
+                                   void *workspace, void *stream);
 
 /* Mamba-2 state-space-duality (SSD) forward ("Mamba & Mamba-2 Architecture",
  * section 3, "Mamba-2 and State Space Duality (SSD)"): one scalar transition

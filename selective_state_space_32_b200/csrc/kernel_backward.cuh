@@ -1,4 +1,6 @@
-// kernel_backward.cuh -- backward pass of the selective scan (N = 16).
+// kernel_backward.cuh -- backward pass of the selective scan (N = 16, 32, 64),
+// with the fused prologue (delta' = softplus(delta + bias)) and gate
+// (y' = y silu(z)) of the forward.
 //
 // Gradients of a loss through h_t = Abar_t h_{t-1} + beta_t u_t,
 // y_t = sum_n C_t[n] h_t[n], Abar_t = exp(delta_t A), beta_t = delta_t B_t
@@ -10,94 +12,116 @@
 //   dB_t += g_t u_t dbeta/dB        dC_t += dy_t h_t          (summed over channels d)
 //   dh0 = Abar_0 g_0
 //
+// and, for the fused layer, with s = delta_raw + bias and ys the scan's output:
+//   dy_scan = dy silu(z),   dz = dy ys silu'(z),   silu'(z) = sig(z) (1 + z (1 - sig(z))),
+//   ddelta_raw = ddelta' sig(s) (softplus' = sigmoid; 1 without softplus),
+//   dbias[d] = sum over b and t of ddelta_raw.
+//
 // "Selective State-Space Models (Mamba) and Hardware-Aware Scans", section 3:
 // the backward pass recomputes the states instead of reading a stored
-// [B, L, D, N] tensor.  Here a first pass runs the recurrence forward and keeps
-// the state every kChunk tokens (a checkpoint per channel, in the workspace);
-// the reverse sweep then takes the chunks last to first, recomputes each
-// chunk's kChunk states from its checkpoint into shared memory, and runs the
-// reverse recurrence over them.
+// [B, L, D, N] tensor.  A forward pass keeps the state entering every chunk of
+// KC tokens (a checkpoint per channel, in the workspace); the reverse sweep
+// takes the chunks last to first, recomputes each chunk's states from its
+// checkpoint into registers and runs the reverse recurrence over them.
 //
-// Mapping: one lane per channel holding all 16 states, a warp = 32 consecutive
-// channels of one batch row, so du, ddelta and dA need no cross-lane work.  dB
-// and dC are sums over channels: per token each lane's 16 values are
-// reduce-scattered over the warp (16 + 16 shuffles), and 16 lanes add one value
-// each into the fp32 output with an atomic (outputs zeroed by the host).
+// Mapping: each lane holds four states of one channel (LPC = N/4 adjacent lanes
+// per channel, CPW = 32/LPC channels per warp), so du, ddelta and the gate's
+// ys are summed over LPC lanes (log2 LPC shuffles) and dA needs none; a block
+// of four warps covers 4 CPW consecutive channels of one batch row and walks
+// the same chunks in the same order, so dB and dC (sums over channels) are
+// summed over the warp by shuffles, over the block in shared memory once per
+// chunk, and added to the fp32 outputs with one 16-byte atomic per four
+// states and token (outputs zeroed by the host).
 #pragma once
 
 #include "device_utils.cuh"
 
 namespace sscan {
 
-constexpr int kBwdThreads = 128;  // 4 warps = 128 channels of one batch row
-constexpr int kChunk = 8;         // tokens per recomputed chunk
-constexpr int kBwdSmem = kChunk * 16 * kBwdThreads * 4;  // dynamic shared memory (64 KB)
+constexpr int kBwdWarps = 4;
+constexpr int kBwdThreads = 32 * kBwdWarps;
+constexpr int kChunk = 16;  // tokens per recomputed chunk
 
-// Sum 16 per-lane values over the 32 lanes of the warp; afterwards lane l
-// (l < 16) holds the total of value l (lanes 16..31 hold duplicates).
-__device__ __forceinline__ float warp_sum16(float (&v)[16], int lane) {
-    // levels 16, 8, 4, 2: each lane keeps the half of its values its partner does not
+// channels a backward block covers
+__host__ __device__ constexpr int bwd_block_channels(int N) { return kBwdWarps * (32 / (N / 4)); }
+
+struct BwdParams {
+    const void *u, *delta, *Bm, *Cm, *dy, *z;
+    const float *A, *h0, *dhf, *bias;
+    void *du, *ddelta, *dz;
+    float *dA, *dB, *dC, *dh0, *dbias;
+    float *ckpt;           // [B][Dpad][nchunks][N]
+    int64_t L, D, Dpad, nchunks;
+    int softplus;
+};
+
+template <class IO> __device__ __forceinline__ float4 bwd_ld4(const IO *p);
+template <> __device__ __forceinline__ float4 bwd_ld4<float>(const float *p) {
+    return __ldg(reinterpret_cast<const float4 *>(p));
+}
+template <> __device__ __forceinline__ float4 bwd_ld4<uint16_t>(const uint16_t *p) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2 *>(p));
+    return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u), __uint_as_float(v.y << 16),
+                       __uint_as_float(v.y & 0xffff0000u));
+}
+__device__ __forceinline__ float f4_at(const float4 &v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
+
+template <class IO, int N, bool ZOH, bool FUSED>
+__global__ void __launch_bounds__(kBwdThreads)
+sscan_backward_kernel(const BwdParams P) {
+    constexpr int LPC = N / 4, CPW = 32 / LPC, CPB = kBwdWarps * CPW, KC = kChunk;
+    __shared__ float4 s_db[kBwdWarps][KC][N / 4], s_dc[kBwdWarps][KC][N / 4];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cl = lane / LPC, g = lane % LPC, n0 = 4 * g;
+    const int64_t L = P.L, D = P.D;
+    const int64_t b = blockIdx.y;
+    const int64_t d = static_cast<int64_t>(blockIdx.x) * CPB + warp * CPW + cl;
+    const bool valid = d < D;
+    const int64_t dc = valid ? d : D - 1;  // past the last channel: compute on a real one, add nothing
+    const IO *u = static_cast<const IO *>(P.u) + b * L * D + dc;
+    const IO *dl_in = static_cast<const IO *>(P.delta) + b * L * D + dc;
+    const IO *dyp = static_cast<const IO *>(P.dy) + b * L * D + dc;
+    const IO *zp = FUSED && P.z ? static_cast<const IO *>(P.z) + b * L * D + dc : nullptr;
+    const IO *Bp = static_cast<const IO *>(P.Bm) + b * L * N + n0;
+    const IO *Cp = static_cast<const IO *>(P.Cm) + b * L * N + n0;
+    float *ck = P.ckpt + (b * P.Dpad + d) * P.nchunks * N + n0;  // own slot even past D
+
+    float a1[4], a2[4], ia[4];
+    {
+        const float4 a = __ldg(reinterpret_cast<const float4 *>(P.A + dc * N + n0));
 #pragma unroll
-    for (int m = 16, cnt = 16; m >= 2; m >>= 1, cnt >>= 1) {
-        const bool up = (lane & m) != 0;
-#pragma unroll
-        for (int i = 0; i < cnt / 2; ++i) {
-            const float send = up ? v[i] : v[i + cnt / 2];
-            const float keep = up ? v[i + cnt / 2] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        for (int i = 0; i < 4; ++i) {
+            a1[i] = f4_at(a, i);
+            a2[i] = static_cast<float>(static_cast<double>(a1[i]) * 1.4426950408889634);
+            ia[i] = a1[i] != 0.0f ? 1.0f / a1[i] : 0.0f;
         }
     }
-    // one value left: the value index is the lane's bits 4, 3, 2, 1 (halves kept at
-    // each level), summed over those bits; the last level sums over bit 0
-    return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
-}
-
-// Value index held by lane l after warp_sum16's first four levels.
-__device__ __forceinline__ int warp_sum16_index(int lane) {
-    return ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
-}
-
-template <class IO, bool ZOH>
-__global__ void __launch_bounds__(kBwdThreads)
-sscan_backward_kernel(const IO *__restrict__ u, const IO *__restrict__ delta, const float *__restrict__ A,
-                      const IO *__restrict__ Bm, const IO *__restrict__ Cm, const float *__restrict__ h0,
-                      const IO *__restrict__ dy, const float *__restrict__ dhf, IO *__restrict__ du,
-                      IO *__restrict__ ddelta, float *__restrict__ dA, float *__restrict__ dB,
-                      float *__restrict__ dC, float *__restrict__ dh0, float *__restrict__ ckpt,
-                      int64_t L, int64_t D, int64_t Dpad, int64_t nchunks) {
-    constexpr int N = 16;
-    extern __shared__ float hs[];  // [kChunk][N][kBwdThreads]: the current chunk's states
-    const int lane = threadIdx.x & 31;
-    const int64_t b = blockIdx.y;
-    const int64_t d = static_cast<int64_t>(blockIdx.x) * kBwdThreads + threadIdx.x;
-    const bool valid = d < D;
-    const int64_t dc = valid ? d : D - 1;  // past the last channel: compute on a real one, store nothing
-
-    float a2[N], a1[N], ia[N];
-#pragma unroll
-    for (int n = 0; n < N; ++n) {
-        const float an = __ldg(A + dc * N + n);
-        a2[n] = static_cast<float>(static_cast<double>(an) * 1.4426950408889634);
-        a1[n] = an;
-        ia[n] = an != 0.0f ? 1.0f / an : 0.0f;
-    }
-    const IO *up = u + b * L * D + dc;
-    const IO *dp = delta + b * L * D + dc;
-    const IO *gp = dy + b * L * D + dc;
-    const IO *bp = Bm + b * L * N;
-    const IO *cp = Cm + b * L * N;
-    float *ck = ckpt + (b * Dpad + d) * nchunks * N;  // this lane's checkpoints (own slot even past D)
-
-    // beta and its derivatives for one state
-    auto coefs = [&](int n, float dl, float abar, float Bn, float &beta, float &dbdl, float &dbda, float &dbdb) {
+    const float biasv = FUSED && P.bias ? __ldg(P.bias + dc) : 0.0f;
+    // the step the scan uses, and (fused) softplus' = sigmoid of its argument
+    auto step = [&](int64_t t, float &sig) {
+        const float raw = Io<IO>::widen(Io<IO>::ld(dl_in + t * D));
+        if (!FUSED) {
+            sig = 1.0f;
+            return raw;
+        }
+        const float s = raw + biasv;
+        if (!P.softplus) {
+            sig = 1.0f;
+            return s;
+        }
+        sig = 1.0f / (1.0f + ex2(-s * 1.4426950408889634f));
+        return softplus_f(s);
+    };
+    // beta and its derivatives for state i
+    auto coefs = [&](int i, float dl, float abar, float Bn, float &beta, float &dbdl, float &dbda, float &dbdb) {
         if (!ZOH) {
             beta = dl * Bn; dbdl = Bn; dbda = 0.0f; dbdb = dl;
-        } else if (a1[n] != 0.0f) {
-            const float z = dl * a1[n];
-            // (e^z - 1)/A: the small-|z| form keeps the relative accuracy of e^z - 1
+        } else if (a1[i] != 0.0f) {
+            const float z = dl * a1[i];
+            // (e^z - 1)/A: the small-|z| series keeps the relative accuracy of e^z - 1
             const float em1 = fabsf(z) < 0.25f ? z * (1.0f + z * (0.5f + z * (1.0f / 6.0f + z * (1.0f / 24.0f + z * (1.0f / 120.0f)))))
                                               : abar - 1.0f;
-            dbdb = em1 * ia[n];
+            dbdb = em1 * ia[i];
             beta = dbdb * Bn;
             dbdl = abar * Bn;
             // (delta abar A - (abar - 1)) / A^2 = delta^2 sum_{k>=2} z^(k-2) (k-1)/k!: the series
@@ -105,7 +129,7 @@ sscan_backward_kernel(const IO *__restrict__ u, const IO *__restrict__ delta, co
             // form cancels; the direct form beyond
             const float ser = 0.5f + z * (1.0f / 3.0f + z * (0.125f + z * (1.0f / 30.0f + z * (1.0f / 144.0f +
                               z * (1.0f / 840.0f + z * (1.0f / 5760.0f + z * (1.0f / 45360.0f + z * (1.0f / 403200.0f))))))));
-            const float num = fabsf(z) < 1.0f ? dl * dl * ser : (dl * abar * a1[n] - em1) * ia[n] * ia[n];
+            const float num = fabsf(z) < 1.0f ? dl * dl * ser : (dl * abar * a1[i] - em1) * ia[i] * ia[i];
             dbda = Bn * num;
         } else {
             beta = dl * Bn; dbdl = Bn; dbda = 0.5f * dl * dl * Bn; dbdb = dl;
@@ -113,107 +137,163 @@ sscan_backward_kernel(const IO *__restrict__ u, const IO *__restrict__ delta, co
     };
 
     // ---- pass 1: forward, keeping the state entering every chunk ----
-    float h[N];
-#pragma unroll
-    for (int n = 0; n < N; ++n) h[n] = h0 != nullptr ? h0[(b * D + dc) * N + n] : 0.0f;
+    float h[4];
+    {
+        const float4 v = P.h0 ? *reinterpret_cast<const float4 *>(P.h0 + (b * D + dc) * N + n0)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        h[0] = v.x; h[1] = v.y; h[2] = v.z; h[3] = v.w;
+    }
     for (int64_t t = 0; t < L; ++t) {
-        if (t % kChunk == 0) {
-            float *dst = ck + (t / kChunk) * N;
+        if (t % KC == 0)
+            *reinterpret_cast<float4 *>(ck + (t / KC) * N) = make_float4(h[0], h[1], h[2], h[3]);
+        float sg;
+        const float dl = step(t, sg);
+        const float x = Io<IO>::widen(Io<IO>::ld(u + t * D));
+        const float4 Bv = bwd_ld4<IO>(Bp + t * N);
 #pragma unroll
-            for (int n = 0; n < N; n += 4) *reinterpret_cast<float4 *>(dst + n) = make_float4(h[n], h[n + 1], h[n + 2], h[n + 3]);
-        }
-        const float x = Io<IO>::widen(Io<IO>::ld(up + t * D));
-        const float dl = Io<IO>::widen(Io<IO>::ld(dp + t * D));
-#pragma unroll
-        for (int n = 0; n < N; ++n) {
-            const float abar = ex2(dl * a2[n]);
+        for (int i = 0; i < 4; ++i) {
+            const float abar = ex2(dl * a2[i]);
             float beta, q0, q1, q2;
-            coefs(n, dl, abar, Io<IO>::widen(Io<IO>::ld(bp + t * N + n)), beta, q0, q1, q2);
-            h[n] = fmaf(abar, h[n], beta * x);
+            coefs(i, dl, abar, f4_at(Bv, i), beta, q0, q1, q2);
+            h[i] = fmaf(abar, h[i], beta * x);
         }
     }
 
     // ---- pass 2: reverse sweep over the chunks ----
-    float g[N], dacc[N];
-#pragma unroll
-    for (int n = 0; n < N; ++n) {
-        g[n] = dhf != nullptr ? dhf[(b * D + dc) * N + n] : 0.0f;
-        dacc[n] = 0.0f;
+    float gs[4], dacc[4];
+    {
+        const float4 v = (P.dhf && valid) ? *reinterpret_cast<const float4 *>(P.dhf + (b * D + dc) * N + n0)
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+        gs[0] = v.x; gs[1] = v.y; gs[2] = v.z; gs[3] = v.w;
     }
-    const int vi = warp_sum16_index(lane);
-    for (int64_t c = nchunks - 1; c >= 0; --c) {
-        const int64_t t0 = c * kChunk;
-        const int nt = static_cast<int>(L - t0 < kChunk ? L - t0 : kChunk);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dacc[i] = 0.0f;
+    float dbias_acc = 0.0f;
+    for (int64_t c = P.nchunks - 1; c >= 0; --c) {
+        const int64_t t0 = c * KC;
+        const int nt = static_cast<int>(L - t0 < KC ? L - t0 : KC);
         // recompute the chunk's states h_{t0 .. t0+nt-1} from its checkpoint
-        float hc[N];
-        const float *src = ck + c * N;
-#pragma unroll
-        for (int n = 0; n < N; n += 4) {
-            const float4 v = *reinterpret_cast<const float4 *>(src + n);
-            hc[n] = v.x; hc[n + 1] = v.y; hc[n + 2] = v.z; hc[n + 3] = v.w;
+        float h_in[4], hk[KC][4];
+        {
+            const float4 v = *reinterpret_cast<const float4 *>(ck + c * N);
+            h_in[0] = v.x; h_in[1] = v.y; h_in[2] = v.z; h_in[3] = v.w;
         }
-        for (int k = 0; k < nt; ++k) {
-            const int64_t t = t0 + k;
-            const float x = Io<IO>::widen(Io<IO>::ld(up + t * D));
-            const float dl = Io<IO>::widen(Io<IO>::ld(dp + t * D));
+        {
+            float hc[4] = {h_in[0], h_in[1], h_in[2], h_in[3]};
 #pragma unroll
-            for (int n = 0; n < N; ++n) {
-                const float abar = ex2(dl * a2[n]);
-                float beta, q0, q1, q2;
-                coefs(n, dl, abar, Io<IO>::widen(Io<IO>::ld(bp + t * N + n)), beta, q0, q1, q2);
-                hc[n] = fmaf(abar, hc[n], beta * x);
-                hs[(k * N + n) * kBwdThreads + threadIdx.x] = hc[n];
+            for (int k = 0; k < KC; ++k) {
+                if (k < nt) {
+                    const int64_t t = t0 + k;
+                    float sg;
+                    const float dl = step(t, sg);
+                    const float x = Io<IO>::widen(Io<IO>::ld(u + t * D));
+                    const float4 Bv = bwd_ld4<IO>(Bp + t * N);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float abar = ex2(dl * a2[i]);
+                        float beta, q0, q1, q2;
+                        coefs(i, dl, abar, f4_at(Bv, i), beta, q0, q1, q2);
+                        hc[i] = fmaf(abar, hc[i], beta * x);
+                        hk[k][i] = hc[i];
+                    }
+                }
             }
         }
         // reverse over the chunk's tokens
-        for (int k = nt - 1; k >= 0; --k) {
-            const int64_t t = t0 + k;
-            const float x = Io<IO>::widen(Io<IO>::ld(up + t * D));
-            const float dl = Io<IO>::widen(Io<IO>::ld(dp + t * D));
-            const float dyt = valid ? Io<IO>::widen(Io<IO>::ld(gp + t * D)) : 0.0f;  // idle lanes add nothing
-            float vb[N], vc[N];
-            float dut = 0.0f, ddt = 0.0f;
 #pragma unroll
-            for (int n = 0; n < N; ++n) {
-                // h_{t-1}: the previous token of this chunk, or the chunk's checkpoint
-                const float hprev = k > 0 ? hs[((k - 1) * N + n) * kBwdThreads + threadIdx.x] : ck[c * N + n];
-                const float ht = hs[(k * N + n) * kBwdThreads + threadIdx.x];
-                const float Bn = Io<IO>::widen(Io<IO>::ld(bp + t * N + n));
-                const float Cn = Io<IO>::widen(Io<IO>::ld(cp + t * N + n));
-                const float abar = ex2(dl * a2[n]);
-                float beta, dbdl, dbda, dbdb;
-                coefs(n, dl, abar, Bn, beta, dbdl, dbda, dbdb);
-                g[n] = fmaf(Cn, dyt, g[n]);
-                dut = fmaf(g[n], beta, dut);
-                ddt = fmaf(g[n], fmaf(hprev * a1[n], abar, x * dbdl), ddt);
-                dacc[n] = fmaf(g[n], fmaf(hprev * dl, abar, x * dbda), dacc[n]);
-                vb[n] = g[n] * x * dbdb;
-                vc[n] = dyt * ht;
-                g[n] *= abar;
-            }
-            if (valid) {
-                Io<IO>::st(du + (b * L + t) * D + d, dut);
-                Io<IO>::st(ddelta + (b * L + t) * D + d, ddt);
-            } else {
+        for (int k = KC - 1; k >= 0; --k) {
+            float4 vb4 = make_float4(0.f, 0.f, 0.f, 0.f), vc4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (k < nt) {
+                const int64_t t = t0 + k;
+                float sg;
+                const float dl = step(t, sg);
+                const float x = Io<IO>::widen(Io<IO>::ld(u + t * D));
+                float dyt = valid ? Io<IO>::widen(Io<IO>::ld(dyp + t * D)) : 0.0f;  // idle lanes add nothing
+                const float4 Bv = bwd_ld4<IO>(Bp + t * N);
+                const float4 Cv = bwd_ld4<IO>(Cp + t * N);
+                float dzt = 0.0f;
+                if (FUSED && zp != nullptr) {
+                    // the gate: the scan's own output ys = C . h_t, summed over the channel's lanes
+                    float ys = 0.0f;
 #pragma unroll
-                for (int n = 0; n < N; ++n) vb[n] = 0.0f;  // idle lanes add nothing to dB
+                    for (int i = 0; i < 4; ++i) ys = fmaf(f4_at(Cv, i), hk[k][i], ys);
+#pragma unroll
+                    for (int o = 1; o < LPC; o <<= 1) ys += __shfl_xor_sync(0xffffffffu, ys, o);
+                    const float zt = Io<IO>::widen(Io<IO>::ld(zp + t * D));
+                    const float sz = 1.0f / (1.0f + ex2(-zt * 1.4426950408889634f));
+                    dzt = dyt * ys * sz * fmaf(zt, 1.0f - sz, 1.0f);
+                    dyt *= zt * sz;
+                }
+                float dut = 0.0f, ddt = 0.0f;
+                float vb[4], vc[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float hprev = k > 0 ? hk[k > 0 ? k - 1 : 0][i] : h_in[i];
+                    const float abar = ex2(dl * a2[i]);
+                    float beta, dbdl, dbda, dbdb;
+                    coefs(i, dl, abar, f4_at(Bv, i), beta, dbdl, dbda, dbdb);
+                    gs[i] = fmaf(f4_at(Cv, i), dyt, gs[i]);
+                    dut = fmaf(gs[i], beta, dut);
+                    ddt = fmaf(gs[i], fmaf(hprev * a1[i], abar, x * dbdl), ddt);
+                    dacc[i] = fmaf(gs[i], fmaf(hprev * dl, abar, x * dbda), dacc[i]);
+                    vb[i] = gs[i] * x * dbdb;
+                    vc[i] = dyt * hk[k][i];
+                    gs[i] *= abar;
+                }
+#pragma unroll
+                for (int o = 1; o < LPC; o <<= 1) {
+                    dut += __shfl_xor_sync(0xffffffffu, dut, o);
+                    ddt += __shfl_xor_sync(0xffffffffu, ddt, o);
+                }
+                ddt *= sg;  // the gradient of the raw step (softplus' = sigmoid)
+                if (valid) {
+                    dbias_acc += ddt;
+                    if (g == 0) {
+                        const int64_t idx = (b * L + t) * D + d;
+                        Io<IO>::st(static_cast<IO *>(P.du) + idx, dut);
+                        Io<IO>::st(static_cast<IO *>(P.ddelta) + idx, ddt);
+                        if (FUSED && zp != nullptr) Io<IO>::st(static_cast<IO *>(P.dz) + idx, dzt);
+                    }
+                }
+                // sums over the warp's channels (lanes with the same state group)
+#pragma unroll
+                for (int o = LPC; o < 32; o <<= 1) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        vb[i] += __shfl_xor_sync(0xffffffffu, vb[i], o);
+                        vc[i] += __shfl_xor_sync(0xffffffffu, vc[i], o);
+                    }
+                }
+                vb4 = make_float4(vb[0], vb[1], vb[2], vb[3]);
+                vc4 = make_float4(vc[0], vc[1], vc[2], vc[3]);
             }
-            const float sb = warp_sum16(vb, lane);
-            const float sc = warp_sum16(vc, lane);
-            if ((lane & 1) == 0) {  // one of the two lanes holding each total
-                atomicAdd(dB + (b * L + t) * N + vi, sb);
-                atomicAdd(dC + (b * L + t) * N + vi, sc);
+            if (cl == 0) {
+                s_db[warp][k][g] = vb4;
+                s_dc[warp][k][g] = vc4;
             }
         }
+        __syncthreads();
+        // sum over the block's warps; one 16-byte atomic per four states and token
+        constexpr int kEntries = KC * (N / 4);
+        for (int e = threadIdx.x; e < 2 * kEntries; e += kBwdThreads) {
+            const int which = e / kEntries, r = e % kEntries, k = r / (N / 4), q = r % (N / 4);
+            if (k >= nt) continue;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int w = 0; w < kBwdWarps; ++w) {
+                const float4 v = which ? s_dc[w][k][q] : s_db[w][k][q];
+                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+            }
+            float *dst = (which ? P.dC : P.dB) + (b * L + t0 + k) * N + 4 * q;
+            atomicAdd(reinterpret_cast<float4 *>(dst), acc);
+        }
+        __syncthreads();
     }
     if (valid) {
-        if (dh0 != nullptr) {
-#pragma unroll
-            for (int n = 0; n < N; n += 4)
-                *reinterpret_cast<float4 *>(dh0 + (b * D + d) * N + n) = make_float4(g[n], g[n + 1], g[n + 2], g[n + 3]);
-        }
-#pragma unroll
-        for (int n = 0; n < N; ++n) atomicAdd(dA + d * N + n, dacc[n]);
+        if (P.dh0 != nullptr)
+            *reinterpret_cast<float4 *>(P.dh0 + (b * D + d) * N + n0) = make_float4(gs[0], gs[1], gs[2], gs[3]);
+        atomicAdd(reinterpret_cast<float4 *>(P.dA + d * N + n0), make_float4(dacc[0], dacc[1], dacc[2], dacc[3]));
+        if (FUSED && P.dbias != nullptr && g == 0) atomicAdd(P.dbias + d, dbias_acc);
     }
 }
 

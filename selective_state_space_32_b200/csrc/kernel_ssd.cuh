@@ -22,29 +22,33 @@
 // of 128 tokens (the page's "e.g. block size 64" names a size, not a rule; 128
 // is the tcgen05 MMA's natural M, and any block size gives the same result).
 //
-// Work unit and schedule.  One CTA per (b, h) walks the blocks in order (the
-// state passing is sequential, but it is only the cheap last line above: the
-// MMAs of a block depend on the previous block only through h_in in MMA 3).
-// Two CTAs share an SM (97 KB of shared memory and 256 of the 512 TMEM columns
-// each), so one CTA's CUDA-core epilogue overlaps the other's MMAs and loads.
+// Work unit.  One CTA per (b, h) walks the blocks in order; the state passing
+// is sequential, but it is only the cheap last line above, so the blocks are
+// pipelined: block c+2 is being loaded and the MMAs of block c+1 run while the
+// CUDA cores finish block c.  One CTA per SM (211 KB of shared memory, 448 of
+// the 512 TMEM columns).
 //
-// Roles.  Warp 4, lane 0 issues the TMA loads (C, B: two 64-state boxes each;
-// X: one box) and every tcgen05.mma and commit.  Warps 0-3 (thread i = TMEM
-// lane i = token row i, state row i) compute the decay factors, P (read from
-// TMEM, written back into TMEM as the bf16 A operand of MMA 2), the weighted
-// w X (in place of X in shared memory, after MMA 2 has consumed X), y, and
-// the fp32 state.
+// Roles (9 warps).
+//   warp 8, lane 0  TMA loads (C, B: two 64-state boxes each; X: one box) into
+//                   two stages, and every tcgen05.mma and commit;
+//   warps 0-3 (P)   decays of the block, then P from S (TMEM) back into TMEM as
+//                   the bf16 A operand of MMA 2 (over S's first 64 columns);
+//   warps 4-7 (Y)   w X (bf16, shared memory) for MMA 4, the fp32 state h and
+//                   its bf16 copy h_in for MMA 3 (two buffers), and y.
+// Thread i of a warpgroup is TMEM lane i: token row i of S, P and Y, state row
+// i of S_blk and h.  Each warpgroup scans the block's steps itself.
+//
+// Tensor memory (512 columns allocated, 448 used; lanes x 32-bit columns):
+// S of even blocks [0, 128), of odd blocks [128, 256) (P over the first 64 of
+// them); P X [256, 320); C h_in [320, 384); S_blk [384, 448).
 //
 // Precision.  bf16 operands, fp32 accumulation; P, h_in and w X are rounded
 // to bf16 as MMA operands, the state and the decays stay fp32.
 //
-// Tensor memory (256 columns x 128 lanes of 32 bits): [0, 128) S, then P
-// (packed bf16 pairs, columns 0-63) and S_blk (columns 64-127); [128, 192) the
-// P X accumulator; [192, 256) the C h_in accumulator.
-//
 // Every wait is bounded; a wait that gives up sets an abort flag that every
-// other wait of the CTA checks, latches a bit in the caller's status word and
-// the CTA drains its last MMA, releases its tensor memory and exits.
+// other wait of the CTA checks, latches a bit in the caller's status word, and
+// the CTA drains its last MMAs, releases its tensor memory and exits.  Every
+// thread of a warpgroup runs the same named barriers whatever happens.
 #pragma once
 
 #include "device_utils.cuh"
@@ -55,30 +59,43 @@ namespace ssd {
 constexpr int kQ = 128;          // tokens per block (M of the MMAs over tokens)
 constexpr int kN = 128;          // state size
 constexpr int kP = 64;           // head dimension
-constexpr int kEpi = 128;        // epilogue threads (warps 0-3)
-constexpr int kThreads = kEpi + 32;
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0, kColSblk = 64, kColY1 = 128, kColY2 = 192;
+constexpr int kWG = 128;         // threads per warpgroup
+constexpr int kThreads = 2 * kWG + 32;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColY1 = 256, kColY2 = 320, kColSblk = 384;  // S of block c at kColS + 128 (c & 1)
 
 // Shared memory, from a 1024-byte aligned base (the 128-byte swizzle atom).
 constexpr int kBox = kQ * 128;                 // one TMA box: 128 rows x 128 bytes
-constexpr int kOffC = 0;                       // C: 2 boxes (states 0-63, 64-127)
-constexpr int kOffB = kOffC + 2 * kBox;        // B: 2 boxes
-constexpr int kOffX = kOffB + 2 * kBox;        // X, then w X: 1 box (head dim 0-63)
-constexpr int kOffH = kOffX + kBox;            // h_in as bf16, [state n][head dim p]
-constexpr int kOffCs = kOffH + kBox;           // float cs2[128]: cumulative delta*A*log2(e)
-constexpr int kOffDt = kOffCs + 512;           // float delta[128]
-constexpr int kOffColf = kOffDt + 512;         // float column factors[128]
-constexpr int kOffWarp = kOffColf + 512;       // float warp totals of the scan[4]
+constexpr int kStage = 5 * kBox;               // C (2 boxes), B (2 boxes), X
+constexpr int kOffStage = 0;                   // 2 stages
+constexpr int kOffWX = 2 * kStage;             // w X, [token s][head dim p]
+constexpr int kOffH = kOffWX + kBox;           // h_in as bf16, [state n][head dim p], 2 buffers
+constexpr int kOffCs = kOffH + 2 * kBox;       // warpgroup P: float cs2[128] (cumulative delta*A*log2 e)
+constexpr int kOffDt = kOffCs + 512;           //              float delta[128]
+constexpr int kOffColf = kOffDt + 512;         //              float column factors[128]
+constexpr int kOffWarp = kOffColf + 512;       // float scan totals [2 warpgroups][4 warps]
 constexpr int kOffBars = kOffWarp + 64;        // mbarriers
-constexpr int kNumBars = 7;
+constexpr int kNumBars = 13;
 constexpr int kOffTmem = kOffBars + 8 * kNumBars;
 constexpr int kOffAbort = kOffTmem + 4;
 constexpr int kSmemUsed = kOffAbort + 4;
 constexpr int kSmemBytes = kSmemUsed + 1024;   // + slack to align the base
-constexpr uint32_t kLoadBytes = 5 * kBox;      // C, B (2 boxes each) and X per block
+constexpr uint32_t kLoadBytes = kStage;        // C, B and X per block
+constexpr int kOffC = 0, kOffB = 2 * kBox, kOffX = 4 * kBox;  // within a stage
 
-enum { BAR_LD = 0, BAR_S, BAR_P, BAR_M2, BAR_WX, BAR_MM, BAR_FREE };
+// mbarriers; a per-stage barrier completes once per two blocks, the others once per block
+enum {
+    BAR_FULL = 0,      // [2] TMA of a stage landed                      (count 1 + bytes)
+    BAR_SDONE = 2,     // [2] MMA 1 of the stage's block done             (commit)
+    BAR_PREADY = 4,    // [2] P of the stage's block in TMEM              (warpgroup P)
+    BAR_WXREADY = 6,   // w X of the block written                        (warpgroup Y)
+    BAR_M4 = 7,        // MMA 4 of the block done: S_blk ready, w X free  (commit)
+    BAR_SBLKFREE = 8,  // S_blk of the block read                         (warpgroup Y)
+    BAR_HREADY = 9,    // h_in of the next block written                  (warpgroup Y)
+    BAR_YREADY = 10,   // MMAs 2 and 3 of the block done (and everything before them)
+    BAR_YFREE = 11,    // P X and C h_in of the block read                (warpgroup Y)
+    BAR_DRAIN = 12,    // every MMA of the CTA done (before the tensor memory is released)
+};
 
 struct Params {
     const float *dt;       // [B][L][H] step delta (after softplus)
@@ -230,7 +247,29 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, vo
 
 // --------------------------------------------------------------- the kernel
 
-__global__ void __launch_bounds__(kThreads, 2)
+// Inclusive scan of v over the 128 threads of a warpgroup (named barrier `bar_id`,
+// warp totals in tot4[4]); returns the thread's prefix and the block total.
+__device__ __forceinline__ float wg_scan(float v, int wl, int lane, float *tot4, int bar_id, float &total) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+    }
+    if (lane == 31) tot4[wl] = v;
+    asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
+    float pre = 0.0f, tot = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float wt = tot4[i];
+        pre += i < wl ? wt : 0.0f;
+        tot += wt;
+    }
+    asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");  // totals read before the next block's scan
+    total = tot;
+    return v + pre;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
 ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                    const __grid_constant__ CUtensorMap tm_c, const Params prm) {
     extern __shared__ unsigned char smem_raw[];
@@ -243,280 +282,312 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kOffBars);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + kOffTmem);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + kOffAbort);
-    float *s_cs = reinterpret_cast<float *>(sm + kOffCs);
-    float *s_dt = reinterpret_cast<float *>(sm + kOffDt);
-    float *s_colf = reinterpret_cast<float *>(sm + kOffColf);
-    float *s_warp = reinterpret_cast<float *>(sm + kOffWarp);
 
     if (threadIdx.x == 0) {
-        mbar_init(&bars[BAR_LD], 1);
-        mbar_init(&bars[BAR_S], 1);
-        mbar_init(&bars[BAR_P], kEpi);
-        mbar_init(&bars[BAR_M2], 1);
-        mbar_init(&bars[BAR_WX], kEpi);
-        mbar_init(&bars[BAR_MM], 1);
-        mbar_init(&bars[BAR_FREE], kEpi);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars[BAR_FULL + i], 1);
+            mbar_init(&bars[BAR_SDONE + i], 1);
+            mbar_init(&bars[BAR_PREADY + i], kWG);
+        }
+        mbar_init(&bars[BAR_WXREADY], kWG);
+        mbar_init(&bars[BAR_M4], 1);
+        mbar_init(&bars[BAR_SBLKFREE], kWG);
+        mbar_init(&bars[BAR_HREADY], kWG);
+        mbar_init(&bars[BAR_YREADY], 1);
+        mbar_init(&bars[BAR_YFREE], kWG);
+        mbar_init(&bars[BAR_DRAIN], 1);
         *abort_flag = 0;
         mbar_fence_init();
     }
-    if (warp == 4) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    if (warp == 8) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
     const int nb = prm.nblocks;
+    const float a2 = __ldg(prm.A + h) * 1.4426950408889634f;  // A_h log2(e): decays as powers of 2
 
-    if (warp == 4) {
+    if (warp == 8) {
         if (lane == 0) {
-            // ------------------------------------------ TMA and MMA issue
+            // ------------------------------------------------ TMA and MMA issue
             tma_prefetch_desc(&tm_x);
             tma_prefetch_desc(&tm_b);
             tma_prefetch_desc(&tm_c);
             constexpr uint32_t id_s = idesc_bf16(kQ, kQ, 0, 0);    // C (K-major) x B^T (K-major)
             constexpr uint32_t id_y = idesc_bf16(kQ, kP, 0, 1);    // P or C (K-major) x X or h (MN-major)
             constexpr uint32_t id_st = idesc_bf16(kN, kP, 1, 1);   // B^T (MN-major) x wX (MN-major)
-            const uint32_t sC = sbase + kOffC, sB = sbase + kOffB, sX = sbase + kOffX, sH = sbase + kOffH;
-            uint64_t *last_bar = nullptr;
-            uint32_t last_par = 0;
-            for (int c = 0; c < nb; ++c) {
-                const uint32_t par = c & 1, prev = (c - 1) & 1;
-                if (c > 0 && !wait_or_abort(&bars[BAR_MM], prev, abort_flag, prm.status, 16)) break;
+            const uint32_t sWX = sbase + kOffWX;
+            auto load = [&](int c) {  // block c into stage c & 1
+                const uint32_t st = sbase + kOffStage + (c & 1) * kStage;
+                uint64_t *bar = &bars[BAR_FULL + (c & 1)];
                 const int t0 = c * kQ;
-                mbar_expect_tx(&bars[BAR_LD], kLoadBytes);
-                tma_load_3d(sC, &tm_c, 0, t0, b, &bars[BAR_LD]);
-                tma_load_3d(sC + kBox, &tm_c, 64, t0, b, &bars[BAR_LD]);
-                tma_load_3d(sB, &tm_b, 0, t0, b, &bars[BAR_LD]);
-                tma_load_3d(sB + kBox, &tm_b, 64, t0, b, &bars[BAR_LD]);
-                tma_load_4d(sX, &tm_x, 0, h, t0, b, &bars[BAR_LD]);
-                if (!wait_or_abort(&bars[BAR_LD], par, abort_flag, prm.status, 16)) break;
-                if (c > 0 && !wait_or_abort(&bars[BAR_FREE], prev, abort_flag, prm.status, 16)) break;
+                mbar_expect_tx(bar, kLoadBytes);
+                tma_load_3d(st + kOffC, &tm_c, 0, t0, b, bar);
+                tma_load_3d(st + kOffC + kBox, &tm_c, 64, t0, b, bar);
+                tma_load_3d(st + kOffB, &tm_b, 0, t0, b, bar);
+                tma_load_3d(st + kOffB + kBox, &tm_b, 64, t0, b, bar);
+                tma_load_4d(st + kOffX, &tm_x, 0, h, t0, b, bar);
+            };
+            auto wait = [&](int bar, uint32_t parity) {
+                return wait_or_abort(&bars[bar], parity, abort_flag, prm.status, 16);
+            };
+            bool issued = false;
+            load(0);
+            if (nb > 1) load(1);
+            for (int c = 0; c < nb; ++c) {
+                const int s = c & 1;
+                const uint32_t ps = (c >> 1) & 1, pc = c & 1, pp = (c - 1) & 1;
+                const uint32_t st = sbase + kOffStage + s * kStage;
+                const uint32_t sC = st + kOffC, sB = st + kOffB, sX = st + kOffX;
+                const uint32_t sH = sbase + kOffH + s * kBox;  // h_in of this block
+                const uint32_t tS = tbase + kColS + 128 * s;
+                if (!wait(BAR_FULL + s, ps)) break;
                 tc_fence_after();
-                // MMA 1: S = C B^T, K = N in 8 steps of 16 states (4 per 64-state box)
+                // MMA 1: S = C B^T, K = N in 8 steps of 16 states (4 per 64-state box).  S of
+                // this stage was last read (as P) by MMA 2 of block c-2, done: see below.
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const uint32_t off = (k >> 2) * kBox + (k & 3) * 32;
-                    mma_ss(tbase + kColS, sdesc_sw128(sC + off, 16, 1024), sdesc_sw128(sB + off, 16, 1024), id_s,
-                           k > 0);
+                    mma_ss(tS, sdesc_sw128(sC + off, 16, 1024), sdesc_sw128(sB + off, 16, 1024), id_s, k > 0);
                 }
-                mma_commit(&bars[BAR_S]);
-                last_bar = &bars[BAR_S];
-                last_par = par;
-                if (!wait_or_abort(&bars[BAR_P], par, abort_flag, prm.status, 16)) break;
+                mma_commit(&bars[BAR_SDONE + s]);
+                issued = true;
+                // block c+1 reuses the stage of block c-1: free once MMAs 2-4 of c-1 are done
+                if (c >= 1 && c + 1 < nb) {
+                    if (!wait(BAR_YREADY, pp)) break;
+                    load(c + 1);
+                }
+                // MMA 4: S_blk = B^T (w X), M = N (two 64-state chunks kBox apart), K = Q
+                if (!wait(BAR_WXREADY, pc)) break;
+                if (c > 0 && !wait(BAR_SBLKFREE, pp)) break;
                 tc_fence_after();
-                // MMA 2: Y1 = P X (P: TMEM columns 8k.. of packed pairs), K = Q in 8 steps of 16 tokens
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    mma_ts(tbase + kColY1, tbase + kColS + 8 * k, sdesc_sw128(sX + k * 2048, kBox, 1024), id_y,
-                           k > 0);
-                // MMA 3: Y2 = C h_in, K = N
+                    mma_ss(tbase + kColSblk, sdesc_sw128(sB + k * 2048, kBox, 1024),
+                           sdesc_sw128(sWX + k * 2048, kBox, 1024), id_st, k > 0);
+                mma_commit(&bars[BAR_M4]);
+                // MMA 2: Y1 = P X (P: TMEM columns 8k.. of packed pairs), MMA 3: Y2 = C h_in
+                if (!wait(BAR_PREADY + s, ps)) break;
+                if (!wait(BAR_HREADY, pc)) break;
+                if (c > 0 && !wait(BAR_YFREE, pp)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_ts(tbase + kColY1, tS + 8 * k, sdesc_sw128(sX + k * 2048, kBox, 1024), id_y, k > 0);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const uint32_t off = (k >> 2) * kBox + (k & 3) * 32;
                     mma_ss(tbase + kColY2, sdesc_sw128(sC + off, 16, 1024), sdesc_sw128(sH + k * 2048, kBox, 1024),
                            id_y, k > 0);
                 }
-                mma_commit(&bars[BAR_M2]);
-                last_bar = &bars[BAR_M2];
-                last_par = par;
-                if (!wait_or_abort(&bars[BAR_WX], par, abort_flag, prm.status, 16)) break;
-                tc_fence_after();
-                // MMA 4: S_blk = B^T (w X), M = N (two 64-state chunks kBox apart), K = Q
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_ss(tbase + kColSblk, sdesc_sw128(sB + k * 2048, kBox, 1024),
-                           sdesc_sw128(sX + k * 2048, kBox, 1024), id_st, k > 0);
-                mma_commit(&bars[BAR_MM]);
-                last_bar = &bars[BAR_MM];
-                last_par = par;
+                mma_commit(&bars[BAR_YREADY]);
             }
-            // the tensor memory is released below: let the last committed MMAs finish
-            // first (a commit tracks every earlier MMA of this thread; bounded)
-            if (last_bar != nullptr)
+            // the tensor memory is released below: every MMA issued must be done first.  A
+            // commit tracks all earlier MMAs of this thread: one more on its own barrier,
+            // waited for with a bound (also after an abort)
+            if (issued) {
+                mma_commit(&bars[BAR_DRAIN]);
                 for (uint32_t i = 0; i < kSpinLimit; ++i)
-                    if (mbar_try_wait(last_bar, last_par)) break;
+                    if (mbar_try_wait(&bars[BAR_DRAIN], 0)) break;
+            }
         }
         __syncwarp();
     } else {
-        // ---------------------------------------------- epilogue warps
-        const int t = threadIdx.x;  // token row of the block, state row n of h
-        const uint32_t lane_base = tbase + (uint32_t(warp * 32) << 16);
-        const float a2 = __ldg(prm.A + h) * 1.4426950408889634f;
-        float hs[kP];  // state row n = t, fp32
-        {
-            const float *src = prm.h0 ? prm.h0 + ((int64_t(b) * prm.H + h) * kN + t) * kP : nullptr;
-#pragma unroll
-            for (int j = 0; j < kP; j += 4) {
-                const float4 v = src ? __ldg(reinterpret_cast<const float4 *>(src + j)) : make_float4(0, 0, 0, 0);
-                hs[j] = v.x;
-                hs[j + 1] = v.y;
-                hs[j + 2] = v.z;
-                hs[j + 3] = v.w;
-            }
-        }
-        auto write_h = [&]() {  // h_in row n = t as bf16 into the swizzled [n][p] tile
-            unsigned char *row = sm + kOffH;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint4 v;
-                v.x = pack_bf16(hs[8 * c + 0], hs[8 * c + 1]);
-                v.y = pack_bf16(hs[8 * c + 2], hs[8 * c + 3]);
-                v.z = pack_bf16(hs[8 * c + 4], hs[8 * c + 5]);
-                v.w = pack_bf16(hs[8 * c + 6], hs[8 * c + 7]);
-                *reinterpret_cast<uint4 *>(row + sw128(t, c)) = v;
-            }
-        };
-        write_h();
-        // Every thread runs every block's named barriers; once a wait has failed (ok
-        // false, the same in the whole warp) the work between them is skipped.
+        // ------------------------------------------------ the two warpgroups
+        const bool is_p = warp < 4;
+        const int wl = warp & 3;               // warp within the warpgroup
+        const int t = threadIdx.x & 127;       // TMEM lane = token row = state row
+        const uint32_t lane_base = tbase + (uint32_t(wl * 32) << 16);
+        float *tot4 = reinterpret_cast<float *>(sm + kOffWarp) + (is_p ? 0 : 4);
+        const int bar_id = is_p ? 1 : 2;
         bool ok = true;
         auto wait_warp = [&](int bar, uint32_t parity) {
             const bool r = ok && wait_or_abort(&bars[bar], parity, abort_flag, prm.status, 32);
             return __all_sync(0xffffffffu, r);
         };
-        for (int c = 0; c < nb; ++c) {
-            const uint32_t par = c & 1;
-            const int64_t tok = int64_t(c) * kQ + t;
-            // ---- cumulative decay of the block: inclusive scan of delta*A*log2(e)
-            const float dt = tok < L ? __ldg(prm.dt + (int64_t(b) * L + tok) * prm.H + h) : 0.0f;
-            float v = dt * a2;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float u = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += u;
-            }
-            if (lane == 31) s_warp[warp] = v;
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            float pre = 0.0f, tot = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float wt = s_warp[i];
-                pre += i < warp ? wt : 0.0f;
-                tot += wt;
-            }
-            const float cs = v + pre;  // log2 of prod_{k <= t} a_k within the block
-            s_cs[t] = cs;
-            s_dt[t] = dt;
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            // column factor of token s = t for the 16-token group it belongs to:
-            // delta_s 2^(r_g - cs_s), r_g = cs at the group's last token (<= 1 for A <= 0)
-            s_colf[t] = dt * ex2(s_cs[(t & ~15) + 15] - cs);
-            const float wv = dt * ex2(tot - cs);  // w_s of the block end state
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+        const float *dtp = prm.dt + int64_t(b) * L * prm.H + h;
+        float dt_next = t < L ? __ldg(dtp + int64_t(t) * prm.H) : 0.0f;
 
-            // ---- P = S o L into TMEM (packed bf16 pairs over S's first 64 columns)
-            ok = wait_warp(BAR_S, par);
-            if (ok) {
-                tc_fence_after();
+        if (is_p) {
+            // ============================================ warpgroup P
+            float *s_cs = reinterpret_cast<float *>(sm + kOffCs);
+            float *s_dt = reinterpret_cast<float *>(sm + kOffDt);
+            float *s_colf = reinterpret_cast<float *>(sm + kOffColf);
+            for (int c = 0; c < nb; ++c) {
+                const int s = c & 1;
+                const uint32_t ps = (c >> 1) & 1;
+                const float dt = dt_next;
+                const int64_t nxt = int64_t(c + 1) * kQ + t;
+                dt_next = nxt < L ? __ldg(dtp + nxt * prm.H) : 0.0f;  // next block's step, in flight
+                float tot;
+                const float cs = wg_scan(dt * a2, wl, lane, tot4, bar_id, tot);
+                s_cs[t] = cs;
+                s_dt[t] = dt;
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                // column factor of token s = t for its 16-token group: delta_s 2^(r_g - cs_s),
+                // r_g = cs at the group's last token (<= 1 for A <= 0)
+                s_colf[t] = dt * ex2(s_cs[(t & ~15) + 15] - cs);
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                // P = S o L into TMEM (packed bf16 pairs over S's first 64 columns)
+                ok = wait_warp(BAR_SDONE + s, ps);
+                if (ok) {
+                    tc_fence_after();
+                    const uint32_t tS = lane_base + kColS + 128 * s;
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {  // columns 32kk .. 32kk+31 (groups 2kk, 2kk+1)
-                    uint32_t pk[16];
-                    if (kk < warp) {
-                        // groups entirely before this warp's rows: 2^(cs_t - cs_s) = 2^(cs_t - r_g) 2^(r_g - cs_s)
-                        uint32_t s_raw[32];
-                        tmem_ld32(lane_base + kColS + 32 * kk, s_raw);
-                        const float rf0 = ex2(cs - s_cs[32 * kk + 15]);
-                        const float rf1 = ex2(cs - s_cs[32 * kk + 31]);
+                    for (int kk = 0; kk < 4; ++kk) {  // columns 32kk .. 32kk+31 (groups 2kk, 2kk+1)
+                        uint32_t pk[16];
+                        if (kk < wl) {
+                            // groups entirely before this warp's rows: 2^(cs_t - cs_s) = 2^(cs_t - r_g) 2^(r_g - cs_s)
+                            uint32_t s_raw[32];
+                            tmem_ld32(tS + 32 * kk, s_raw);
+                            const float rf0 = ex2(cs - s_cs[32 * kk + 15]);
+                            const float rf1 = ex2(cs - s_cs[32 * kk + 31]);
 #pragma unroll
-                        for (int j = 0; j < 32; j += 2) {
-                            const float rf = j < 16 ? rf0 : rf1;
-                            const float p0 = __uint_as_float(s_raw[j]) * s_colf[32 * kk + j] * rf;
-                            const float p1 = __uint_as_float(s_raw[j + 1]) * s_colf[32 * kk + j + 1] * rf;
-                            pk[j / 2] = pack_bf16(p0, p1);
+                            for (int j = 0; j < 32; j += 2) {
+                                const float rf = j < 16 ? rf0 : rf1;
+                                const float p0 = __uint_as_float(s_raw[j]) * s_colf[32 * kk + j] * rf;
+                                const float p1 = __uint_as_float(s_raw[j + 1]) * s_colf[32 * kk + j + 1] * rf;
+                                pk[j / 2] = pack_bf16(p0, p1);
+                            }
+                        } else if (kk == wl) {
+                            // the groups holding this warp's diagonal: 2^(cs_t - cs_s) directly, 0 above it
+                            uint32_t s_raw[32];
+                            tmem_ld32(tS + 32 * kk, s_raw);
+#pragma unroll
+                            for (int j = 0; j < 32; j += 2) {
+                                const int s0 = 32 * kk + j;
+                                const float p0 =
+                                    s0 <= t ? __uint_as_float(s_raw[j]) * s_dt[s0] * ex2(cs - s_cs[s0]) : 0.0f;
+                                const float p1 = s0 + 1 <= t ? __uint_as_float(s_raw[j + 1]) * s_dt[s0 + 1] *
+                                                                   ex2(cs - s_cs[s0 + 1])
+                                                             : 0.0f;
+                                pk[j / 2] = pack_bf16(p0, p1);
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) pk[j] = 0u;
                         }
-                    } else if (kk == warp) {
-                        // the groups holding this warp's diagonal: 2^(cs_t - cs_s) directly, 0 above it
-                        uint32_t s_raw[32];
-                        tmem_ld32(lane_base + kColS + 32 * kk, s_raw);
-#pragma unroll
-                        for (int j = 0; j < 32; j += 2) {
-                            const int s0 = 32 * kk + j;
-                            const float p0 =
-                                s0 <= t ? __uint_as_float(s_raw[j]) * s_dt[s0] * ex2(cs - s_cs[s0]) : 0.0f;
-                            const float p1 = s0 + 1 <= t
-                                                 ? __uint_as_float(s_raw[j + 1]) * s_dt[s0 + 1] * ex2(cs - s_cs[s0 + 1])
-                                                 : 0.0f;
-                            pk[j / 2] = pack_bf16(p0, p1);
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) pk[j] = 0u;
+                        tmem_st16(tS + 16 * kk, pk);
                     }
-                    tmem_st16(lane_base + kColS + 16 * kk, pk);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(&bars[BAR_PREADY + s]);
                 }
-                tmem_wait_st();
-                fence_proxy_async_smem();  // h_in rows written by this thread -> the MMA's operand reads
-                tc_fence_before();
-                mbar_arrive(&bars[BAR_P]);
             }
-
-            // ---- w X in place of X, once MMA 2 has read X; then y
-            ok = wait_warp(BAR_LD, par);
-            ok = wait_warp(BAR_M2, par);
-            if (ok) {
-                tc_fence_after();
-                unsigned char *row = sm + kOffX;
+        } else {
+            // ============================================ warpgroup Y
+            float hs[kP];  // state row n = t, fp32
+            {
+                const float *src = prm.h0 ? prm.h0 + ((int64_t(b) * prm.H + h) * kN + t) * kP : nullptr;
+#pragma unroll
+                for (int j = 0; j < kP; j += 4) {
+                    const float4 v = src ? __ldg(reinterpret_cast<const float4 *>(src + j)) : make_float4(0, 0, 0, 0);
+                    hs[j] = v.x;
+                    hs[j + 1] = v.y;
+                    hs[j + 2] = v.z;
+                    hs[j + 3] = v.w;
+                }
+            }
+            auto write_h = [&](int buf) {  // h_in row n = t as bf16 into the swizzled [n][p] tile
+                unsigned char *row = sm + kOffH + buf * kBox;
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    uint4 *p = reinterpret_cast<uint4 *>(row + sw128(t, q));
-                    uint4 v4 = *p;
-                    v4.x = pack_bf16(bf16_lo(v4.x) * wv, bf16_hi(v4.x) * wv);
-                    v4.y = pack_bf16(bf16_lo(v4.y) * wv, bf16_hi(v4.y) * wv);
-                    v4.z = pack_bf16(bf16_lo(v4.z) * wv, bf16_hi(v4.z) * wv);
-                    v4.w = pack_bf16(bf16_lo(v4.w) * wv, bf16_hi(v4.w) * wv);
-                    *p = v4;
+                    uint4 v;
+                    v.x = pack_bf16(hs[8 * q + 0], hs[8 * q + 1]);
+                    v.y = pack_bf16(hs[8 * q + 2], hs[8 * q + 3]);
+                    v.z = pack_bf16(hs[8 * q + 4], hs[8 * q + 5]);
+                    v.w = pack_bf16(hs[8 * q + 6], hs[8 * q + 7]);
+                    *reinterpret_cast<uint4 *>(row + sw128(t, q)) = v;
                 }
-                fence_proxy_async_smem();
-                mbar_arrive(&bars[BAR_WX]);
-                // y = P X + 2^cs (C h_in), rows inside the sequence only
-                const float e = ex2(cs);
-                uint16_t *dst = prm.y + ((int64_t(b) * L + tok) * prm.H + h) * kP;
+                fence_proxy_async_smem();  // generic writes -> the MMA's operand reads
+            };
+            write_h(0);
+            mbar_arrive(&bars[BAR_HREADY]);
+            for (int c = 0; c < nb; ++c) {
+                const int s = c & 1;
+                const uint32_t ps = (c >> 1) & 1, pc = c & 1;
+                const float dt = dt_next;
+                const int64_t tok = int64_t(c) * kQ + t;
+                const int64_t nxt = tok + kQ;
+                dt_next = nxt < L ? __ldg(dtp + nxt * prm.H) : 0.0f;
+                float tot;
+                const float cs = wg_scan(dt * a2, wl, lane, tot4, bar_id, tot);
+                // ---- w X for MMA 4: X of this block landed; w X's buffer was freed by MMA 4 of
+                // block c-1 (waited below in the previous block)
+                ok = wait_warp(BAR_FULL + s, ps);
+                if (ok) {
+                    const float wv = dt * ex2(tot - cs);  // w_s of the block end state, s = t
+                    const unsigned char *xr = sm + kOffStage + s * kStage + kOffX;
+                    unsigned char *wr = sm + kOffWX;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t y1[32], y2[32];
-                    tmem_ld32(lane_base + kColY1 + 32 * half, y1);
-                    tmem_ld32(lane_base + kColY2 + 32 * half, y2);
-                    uint32_t o[16];
+                    for (int q = 0; q < 8; ++q) {
+                        uint4 v4 = *reinterpret_cast<const uint4 *>(xr + sw128(t, q));
+                        v4.x = pack_bf16(bf16_lo(v4.x) * wv, bf16_hi(v4.x) * wv);
+                        v4.y = pack_bf16(bf16_lo(v4.y) * wv, bf16_hi(v4.y) * wv);
+                        v4.z = pack_bf16(bf16_lo(v4.z) * wv, bf16_hi(v4.z) * wv);
+                        v4.w = pack_bf16(bf16_lo(v4.w) * wv, bf16_hi(v4.w) * wv);
+                        *reinterpret_cast<uint4 *>(wr + sw128(t, q)) = v4;
+                    }
+                    fence_proxy_async_smem();
+                    mbar_arrive(&bars[BAR_WXREADY]);
+                }
+                // ---- state passing: h = 2^cs_end h + S_blk (row n = t); then h_in of block c+1
+                ok = wait_warp(BAR_M4, pc);
+                if (ok) {
+                    tc_fence_after();
+                    const float aend = ex2(tot);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        o[j] = pack_bf16(fmaf(e, __uint_as_float(y2[2 * j]), __uint_as_float(y1[2 * j])),
-                                         fmaf(e, __uint_as_float(y2[2 * j + 1]), __uint_as_float(y1[2 * j + 1])));
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t sb[32];
+                        tmem_ld32(lane_base + kColSblk + 32 * half, sb);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            hs[32 * half + j] = fmaf(aend, hs[32 * half + j], __uint_as_float(sb[j]));
+                    }
+                    tc_fence_before();
+                    mbar_arrive(&bars[BAR_SBLKFREE]);
+                    // buffer (c+1)&1 was last read by MMA 3 of block c-1, waited below in block c-1
+                    write_h((c + 1) & 1);
+                    mbar_arrive(&bars[BAR_HREADY]);
+                }
+                // ---- y = P X + 2^cs (C h_in), rows inside the sequence only
+                ok = wait_warp(BAR_YREADY, pc);
+                if (ok) {
+                    tc_fence_after();
+                    const float e = ex2(cs);
+                    uint32_t o[2][16];
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t y1[32], y2[32];
+                        tmem_ld32(lane_base + kColY1 + 32 * half, y1);
+                        tmem_ld32(lane_base + kColY2 + 32 * half, y2);
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            o[half][j] = pack_bf16(fmaf(e, __uint_as_float(y2[2 * j]), __uint_as_float(y1[2 * j])),
+                                                   fmaf(e, __uint_as_float(y2[2 * j + 1]), __uint_as_float(y1[2 * j + 1])));
+                    }
+                    tc_fence_before();
+                    mbar_arrive(&bars[BAR_YFREE]);
                     if (tok < L) {
-                        uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * half);
+                        uint4 *d4 = reinterpret_cast<uint4 *>(prm.y + ((int64_t(b) * L + tok) * prm.H + h) * kP);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            d4[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+                        for (int q = 0; q < 8; ++q)
+                            d4[q] = make_uint4(o[q >> 2][4 * (q & 3)], o[q >> 2][4 * (q & 3) + 1],
+                                               o[q >> 2][4 * (q & 3) + 2], o[q >> 2][4 * (q & 3) + 3]);
                     }
                 }
             }
-
-            // ---- state passing: h = 2^cs_end h + S_blk (row n = t)
-            ok = wait_warp(BAR_MM, par);
-            if (ok) {
-                tc_fence_after();
-                const float aend = ex2(tot);
+            if (ok && prm.h_final) {
+                float *dst = prm.h_final + ((int64_t(b) * prm.H + h) * kN + t) * kP;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t sb[32];
-                    tmem_ld32(lane_base + kColSblk + 32 * half, sb);
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        hs[32 * half + j] = fmaf(aend, hs[32 * half + j], __uint_as_float(sb[j]));
-                }
-                tc_fence_before();
-                mbar_arrive(&bars[BAR_FREE]);
-                write_h();
+                for (int j = 0; j < kP; j += 4)
+                    *reinterpret_cast<float4 *>(dst + j) = make_float4(hs[j], hs[j + 1], hs[j + 2], hs[j + 3]);
             }
-        }
-        if (ok && prm.h_final) {
-            float *dst = prm.h_final + ((int64_t(b) * prm.H + h) * kN + t) * kP;
-#pragma unroll
-            for (int j = 0; j < kP; j += 4)
-                *reinterpret_cast<float4 *>(dst + j) = make_float4(hs[j], hs[j + 1], hs[j + 2], hs[j + 3]);
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == 8) {
         tc_fence_after();
         tmem_dealloc(tbase, kTmemCols);
     }

@@ -225,8 +225,19 @@ void choose_schedule(sscan_plan *p) {
             p->cfg = i;
             p->chains_per_row = cpr;
             p->chains = chains;
+            if (p->split) {
+                // the same whole number of pieces for every chain, so that neighbouring
+                // chains (which share the 64-byte L2 lines of their u and delta rows) are
+                // cut at nearly the same tokens and scanned there at the same time; with
+                // a fractional count their pieces drift apart and each line is fetched
+                // from DRAM once per chain (1.6x the input bytes measured on B200)
+                const int64_t pieces = workers / chains;
+                p->seg = ceil_div(p->L, pieces);
+                workers = ceil_div(chains * pieces, k.WPC) * k.WPC;  // whole blocks; trailing warps idle
+            } else {
+                p->seg = ceil_div(chains * p->L, workers);
+            }
             p->workers = workers;
-            p->seg = ceil_div(chains * p->L, workers);
             // split mode indexes pieces by equal segments; the chained mode balances time
             p->seg_shift = p->split ? 0 : p->seg * (light >= 0 ? light : kLightPermille) / 1000;
             if (p->split) {

@@ -24,7 +24,7 @@ OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPAC
 SYMBOLS = ("sscan_plan_create", "sscan_plan_destroy", "sscan_workspace_bytes", "sscan_forward",
            "sscan_get_status", "sscan_status_string", "sscan_plan_describe", "sscan_version",
            "sscan_forward_noalloc", "sscan_noalloc_status", "sscan_forward_gated", "sscan_backward",
-           "sscan_backward_workspace_bytes", "sscan_ssd_forward")
+           "sscan_backward_workspace_bytes", "sscan_ssd_forward", "sscan_backward_gated")
 
 
 class SscanError(RuntimeError):
@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
             L.sscan_backward_workspace_bytes.restype = sz
             L.sscan_ssd_forward.argtypes = [i64, i64, i64, i64, i64] + [vp] * 10
             L.sscan_ssd_forward.restype = ip
+            L.sscan_backward_gated.argtypes = [i64, i64, i64, i64, ip, u32] + [vp] * 20
+            L.sscan_backward_gated.restype = ip
             _lib = L
     return _lib
 
@@ -179,9 +181,11 @@ class Plan:
             raise SscanError(rc, what)
         return y, h_final
 
-    def backward(self, u, delta, A, B, C, h0, dy, dh_final=None, want_dh0: bool = True, stream=None) -> dict:
-        """Gradients of the plain forward (N = 16): returns a dict with du, ddelta (plan dtype),
-        dA, dB, dC and dh0 (fp32) given dy (and optionally dh_final)."""
+    def backward(self, u, delta, A, B, C, h0, dy, dh_final=None, want_dh0: bool = True, stream=None,
+                 delta_bias=None, z=None) -> dict:
+        """Gradients of this plan's forward: returns a dict with du, ddelta (plan dtype), dA,
+        dB, dC and dh0 (fp32) given dy (and optionally dh_final); with delta_bias and z
+        (the fused layer, ``sscan_backward_gated``) also ddelta_bias (fp32) and dz."""
         Bt, L, D, N = self.shape
         dev = u.device
         out = {"du": torch.empty((Bt, L, D), dtype=self.dtype, device=dev),
@@ -189,19 +193,22 @@ class Plan:
                "dA": torch.empty((D, N), dtype=torch.float32, device=dev),
                "dB": torch.empty((Bt, L, N), dtype=torch.float32, device=dev),
                "dC": torch.empty((Bt, L, N), dtype=torch.float32, device=dev),
-               "dh0": torch.empty((Bt, D, N), dtype=torch.float32, device=dev) if want_dh0 else None}
+               "dh0": torch.empty((Bt, D, N), dtype=torch.float32, device=dev) if want_dh0 else None,
+               "ddelta_bias": torch.empty((D,), dtype=torch.float32, device=dev) if delta_bias is not None else None,
+               "dz": torch.empty((Bt, L, D), dtype=self.dtype, device=dev) if z is not None else None}
         wsb = int(lib().sscan_backward_workspace_bytes(Bt, L, D, N))
         ws = torch.empty(wsb, dtype=torch.uint8, device=dev) if wsb else None
         if stream is None:
             stream = torch.cuda.current_stream(dev)
         flags = (ZOH if self.zoh else 0) | (DELTA_SOFTPLUS if self.delta_softplus else 0)
-        rc = lib().sscan_backward(Bt, L, D, N, _dtype_code(self.dtype), flags,
-                                  _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(h0), _ptr(dy),
-                                  _ptr(dh_final), _ptr(out["du"]), _ptr(out["ddelta"]), _ptr(out["dA"]),
-                                  _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dh0"]), _ptr(ws),
-                                  ctypes.c_void_p(stream.cuda_stream))
+        rc = lib().sscan_backward_gated(Bt, L, D, N, _dtype_code(self.dtype), flags,
+                                        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(h0),
+                                        _ptr(delta_bias), _ptr(z), _ptr(dy), _ptr(dh_final), _ptr(out["du"]),
+                                        _ptr(out["ddelta"]), _ptr(out["dA"]), _ptr(out["dB"]), _ptr(out["dC"]),
+                                        _ptr(out["dh0"]), _ptr(out["ddelta_bias"]), _ptr(out["dz"]), _ptr(ws),
+                                        ctypes.c_void_p(stream.cuda_stream))
         if rc != OK:
-            raise SscanError(rc, "sscan_backward")
+            raise SscanError(rc, "sscan_backward_gated")
         return out
 
     def status(self, stream=None) -> int:

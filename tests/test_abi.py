@@ -84,23 +84,34 @@ def test_binding_argument_counts_match_the_header(lib):
 
 
 def test_gated_and_backward_reject_bad_arguments_without_a_device(lib):
+    # every case below fails an argument check before any CUDA call; none may reach a
+    # launch, so none uses a supported shape with all its pointers present and aligned
     assert lib.sscan_forward_gated(None, *([None] * 12)) == S.ERR_INVALID
     p = ctypes.c_void_p(256)  # never dereferenced: every case fails its checks first
     args16 = [p] * 15 + [None]
-    assert lib.sscan_backward(1, 16, 32, 32, S.F32, 0, *args16) == S.ERR_UNSUPPORTED      # N = 32
-    assert lib.sscan_backward(1, 16, 32, 16, S.F32, S.DELTA_SOFTPLUS, *args16) == S.ERR_UNSUPPORTED
+    assert lib.sscan_backward(1, 16, 32, 24, S.F32, 0, *args16) == S.ERR_UNSUPPORTED      # N = 24
+    assert lib.sscan_backward(1, 16, 32, 128, S.F32, 0, *args16) == S.ERR_UNSUPPORTED     # N = 128
     assert lib.sscan_backward(0, 16, 32, 16, S.F32, 0, *args16) == S.ERR_INVALID          # B = 0
     assert lib.sscan_backward(1, 16, 32, 16, 7, 0, *args16) == S.ERR_INVALID              # dtype
     assert lib.sscan_backward(1, 16, 32, 16, S.F32, 1 << 5, *args16) == S.ERR_INVALID     # flag
     assert lib.sscan_backward(1, 16, 32, 16, S.F32, 0, *([p] * 6), None, *([p] * 8), None) == S.ERR_INVALID  # no dy
     assert lib.sscan_backward(1, 16, 32, 16, S.F32, 0, ctypes.c_void_p(260), *([p] * 14), None) == S.ERR_ALIGN
+    # the gated backward: a gate without its gradient output, a bias without its gradient
+    a = [p] * 6  # u, delta, A, B, C, h0
+    assert lib.sscan_backward_gated(1, 16, 32, 16, S.F32, 0, *a, None, p, p, None, p, p, p, p, p, p, None, None,
+                                    p, None) == S.ERR_INVALID
+    assert lib.sscan_backward_gated(1, 16, 32, 16, S.F32, 0, *a, p, None, p, None, p, p, p, p, p, p, None, None,
+                                    p, None) == S.ERR_INVALID
 
 
 def test_backward_workspace_bytes(lib):
-    # state checkpoints: B x ceil(D/128)*128 channels x ceil(L/8) chunks x 16 states x 4 bytes
-    assert lib.sscan_backward_workspace_bytes(8, 2048, 1536, 16) == 8 * 1536 * 256 * 16 * 4
-    assert lib.sscan_backward_workspace_bytes(2, 37, 70, 16) == 2 * 128 * 5 * 16 * 4
-    assert lib.sscan_backward_workspace_bytes(2, 37, 70, 32) == 0
+    # state checkpoints: B x channels padded to a block (4 warps x 32/(N/4) channels) x
+    # ceil(L/16) chunks x N states x 4 bytes, rounded up to 256 bytes
+    assert lib.sscan_backward_workspace_bytes(8, 2048, 1536, 16) == 8 * 1536 * 128 * 16 * 4
+    assert lib.sscan_backward_workspace_bytes(2, 37, 70, 16) == 2 * 96 * 3 * 16 * 4
+    assert lib.sscan_backward_workspace_bytes(2, 37, 70, 32) == 2 * 80 * 3 * 32 * 4
+    assert lib.sscan_backward_workspace_bytes(2, 37, 70, 64) == 2 * 72 * 3 * 64 * 4
+    assert lib.sscan_backward_workspace_bytes(2, 37, 70, 24) == 0
     assert lib.sscan_backward_workspace_bytes(2, 0, 70, 16) == 0
 
 

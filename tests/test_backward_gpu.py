@@ -1,13 +1,19 @@
 """Parity of the CUDA backward pass with the fp64 oracle's backward (B200).
 
-The oracle's backward is pinned by finite differences of the forward oracle
-(tests/test_oracle_backward.py).  Cases cover Euler and ZOH (with some A = 0,
-the limit branch), fp32 and bf16 I/O, a ragged channel count (D not a multiple
-of the 128-channel block) and ragged sequence (L not a multiple of the 8-token
-recompute chunk), with and without h0 and dh_final.  dA, dB, dC are fp32 sums
-over many terms accumulated with atomics; the tolerances are those of the
-forward (fp32: relative L2 1e-5; bf16 inputs: 5e-3).
+The oracle's backward, plain and fused, is pinned by finite differences of the
+forward oracle (tests/test_oracle_backward.py).  Cases cover N = 16, 32 and 64,
+Euler and ZOH (with some A = 0, the limit branch), fp32 and bf16 I/O, ragged
+channel counts (D not a multiple of a block's channels) and ragged sequences
+(L not a multiple of the 16-token recompute chunk), with and without h0 and
+dh_final, and the fused layer (softplus(delta + bias) and the silu(z) gate:
+gradients of the raw delta, the bias and z).  Tolerances are those of the
+forward: fp32 relative L2 <= 1e-5 and |err| <= 1e-4 (1 + |ref|) elementwise on
+every gradient; bf16 inputs relative L2 <= 5e-3.  dA, dB, dC and the bias
+gradient are fp32 sums over many terms accumulated with atomics, well inside
+those bounds.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -35,6 +41,25 @@ def _rel(got, ref):
     return float(np.linalg.norm(got - ref) / den) if den > 0 else float(np.linalg.norm(got))
 
 
+def _check(got, ref, keys, dt):
+    for k in keys:
+        gv = got[k].float().cpu().numpy().astype(np.float64)
+        assert np.all(np.isfinite(gv)), k
+        r = _rel(gv, ref[k])
+        if dt == "f32":
+            assert r <= 1e-5, f"{k}: rel L2 {r:.3e} > 1e-5"
+            m = float((np.abs(gv - ref[k]) / (1.0 + np.abs(ref[k]))).max()) if gv.size else 0.0
+            assert m <= 1e-4, f"{k}: max |err|/(1+|ref|) {m:.3e} > 1e-4"
+        else:
+            assert r <= 5e-3, f"{k}: rel L2 {r:.3e} > 5e-3"
+
+
+def _dy(shape, dt, seed):
+    rng = np.random.default_rng(seed)
+    dy32 = rng.standard_normal(shape).astype(np.float32)
+    return dy32 if dt == "f32" else W.f32_to_bf16_bits(dy32)
+
+
 CASES = [
     # (B, L, D, N, dtype, h0, dhf, zoh, zero_a)
     (2, 37, 70, 16, "f32", True, True, False, False),     # ragged D and L
@@ -44,21 +69,23 @@ CASES = [
     (2, 100, 96, 16, "bf16", True, True, False, False),
     (1, 80, 64, 16, "bf16", True, False, True, False),
     (1, 1, 32, 16, "f32", True, True, False, False),       # a single token
+    (2, 75, 44, 32, "f32", True, True, True, False),       # N = 32, ZOH
+    (2, 130, 36, 32, "bf16", True, True, False, False),
+    (2, 50, 21, 64, "f32", True, True, True, True),        # N = 64, ZOH with A = 0, ragged D
+    (1, 200, 40, 64, "bf16", False, True, True, False),
 ]
 
 
-@pytest.mark.parametrize("case", CASES, ids=[f"B{c[0]}L{c[1]}D{c[2]}{c[4]}{'_zoh' if c[7] else ''}"
+@pytest.mark.parametrize("case", CASES, ids=[f"B{c[0]}L{c[1]}D{c[2]}N{c[3]}{c[4]}{'_zoh' if c[7] else ''}"
                                               f"{'_a0' if c[8] else ''}{'_h0' if c[5] else ''}{'_dhf' if c[6] else ''}"
                                               for c in CASES])
 def test_backward_matches_oracle(case):
     Bt, L, D, N, dt, with_h0, with_dhf, zoh, zero_a = case
-    g = W.generate(Bt, L, D, N, dt, 0.1 if with_h0 else 0.0, seed=8000 + L + D, A_jitter=0.3)
+    g = W.generate(Bt, L, D, N, dt, 0.1 if with_h0 else 0.0, seed=8000 + L + D + N, A_jitter=0.3)
     if zero_a:
         g["A"][::7, 3] = 0.0
-    rng = np.random.default_rng(L + D)
-    dy32 = rng.standard_normal((Bt, L, D)).astype(np.float32)
-    dy = dy32 if dt == "f32" else W.f32_to_bf16_bits(dy32)
-    dhf = rng.standard_normal((Bt, D, N)).astype(np.float32) if with_dhf else None
+    dy = _dy((Bt, L, D), dt, L + D)
+    dhf = np.random.default_rng(N).standard_normal((Bt, D, N)).astype(np.float32) if with_dhf else None
     d = P.to_device(g)
     tdt = torch.float32 if dt == "f32" else torch.bfloat16
     dy_d = P.to_device({**g, "u": dy})["u"]
@@ -68,11 +95,46 @@ def test_backward_matches_oracle(case):
     torch.cuda.synchronize()
     v = P.host_values(g)
     ref = O.backward(v["u"], v["delta"], v["A"], v["B"], v["C"], v["h0"], zoh, W.as_f32(dy, dt), dhf)
-    tol = 1e-5 if dt == "f32" else 5e-3
-    for k in ("du", "ddelta", "dA", "dB", "dC", "dh0"):
-        r = _rel(got[k].float().cpu().numpy(), ref[k])
-        assert np.all(np.isfinite(got[k].float().cpu().numpy())), k
-        assert r <= tol, f"{k}: rel L2 {r:.3e} > {tol}"
+    _check(got, ref, ("du", "ddelta", "dA", "dB", "dC", "dh0"), dt)
+    plan.close()
+
+
+FUSED = [
+    # (B, L, D, N, dtype, zoh, softplus, bias, gate)
+    (2, 70, 64, 16, "f32", False, True, True, True),
+    (2, 45, 40, 32, "f32", True, True, True, True),
+    (1, 66, 24, 64, "f32", False, True, False, True),
+    (2, 90, 96, 16, "bf16", False, True, True, True),
+    (2, 40, 48, 16, "f32", False, False, True, False),      # bias only, no softplus, no gate
+    (1, 33, 16, 16, "f32", False, True, True, False),       # softplus + bias, no gate
+]
+
+
+@pytest.mark.parametrize("case", FUSED, ids=[f"B{c[0]}L{c[1]}D{c[2]}N{c[3]}{c[4]}{'_zoh' if c[5] else ''}"
+                                              f"{'_sp' if c[6] else ''}{'_bias' if c[7] else ''}{'_gate' if c[8] else ''}"
+                                              for c in FUSED])
+def test_fused_backward_matches_oracle(case):
+    Bt, L, D, N, dt, zoh, sp, with_bias, with_gate = case
+    g = W.generate(Bt, L, D, N, dt, 0.1, seed=8500 + L + D + N, A_jitter=0.3, fused=True)
+    if not with_bias:
+        g["delta_bias"] = None
+    if not with_gate:
+        g["z"] = None
+    dy = _dy((Bt, L, D), dt, 3 * L + D)
+    dhf = np.random.default_rng(D).standard_normal((Bt, D, N)).astype(np.float32)
+    d = P.to_device(g)
+    tdt = torch.float32 if dt == "f32" else torch.bfloat16
+    dy_d = P.to_device({**g, "u": dy})["u"]
+    plan = S.Plan(Bt, L, D, N, tdt, zoh, delta_softplus=sp)
+    got = plan.backward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"], dy_d, torch.from_numpy(dhf).cuda(),
+                        delta_bias=d["delta_bias"], z=d["z"])
+    torch.cuda.synchronize()
+    v = P.host_values(g)
+    ref = O.backward_fused(v["u"], v["delta"], v["A"], v["B"], v["C"], v["h0"], zoh, W.as_f32(dy, dt), dhf,
+                           delta_bias=v["delta_bias"], softplus=sp, z=v["z"])
+    keys = ["du", "ddelta", "dA", "dB", "dC", "dh0"] + (["ddelta_bias"] if with_bias else []) + \
+        (["dz"] if with_gate else [])
+    _check(got, ref, keys, dt)
     plan.close()
 
 
@@ -94,14 +156,24 @@ def test_backward_forward_consistency():
 
 
 def test_backward_argument_errors():
-    import ctypes
-    Bt, L, D = 1, 16, 32
-    z = torch.zeros(16, device="cuda")
-    p = ctypes.c_void_p(z.data_ptr())
-    # N = 32 and the fused softplus flag are not supported by the backward
-    assert S.lib().sscan_backward(Bt, L, D, 32, S.F32, 0, *([p] * 15), None) == S.ERR_UNSUPPORTED
-    assert S.lib().sscan_backward(Bt, L, D, 16, S.F32, S.DELTA_SOFTPLUS, *([p] * 15), None) == S.ERR_UNSUPPORTED
-    # a bad flag bit and a misaligned pointer
-    assert S.lib().sscan_backward(Bt, L, D, 16, S.F32, 1 << 5, *([p] * 15), None) == S.ERR_INVALID
-    q = ctypes.c_void_p(z.data_ptr() + 4)
-    assert S.lib().sscan_backward(Bt, L, D, 16, S.F32, 0, q, *([p] * 14), None) == S.ERR_ALIGN
+    """Every call below fails a check before any launch; the buffers are real and large
+    enough for the stated shape, so a check that wrongly passed could not make a kernel
+    touch memory it does not own."""
+    Bt, L, D, N = 1, 16, 32, 16
+    lib = S.lib()
+    buf = [torch.zeros(Bt * L * D * N + 64, device="cuda") for _ in range(16)]
+    p = [ctypes.c_void_p(t.data_ptr()) for t in buf]
+    # u, delta, A, B, C, h0, dy, dh_final, du, ddelta, dA, dB, dC, dh0, workspace
+    ok_args = p[:15]
+    assert lib.sscan_backward(Bt, L, D, 24, S.F32, 0, *ok_args, None) == S.ERR_UNSUPPORTED   # N = 24
+    assert lib.sscan_backward(Bt, L, D, N, S.F32, 1 << 5, *ok_args, None) == S.ERR_INVALID   # bad flag
+    q = ctypes.c_void_p(buf[0].data_ptr() + 4)
+    assert lib.sscan_backward(Bt, L, D, N, S.F32, 0, q, *ok_args[1:], None) == S.ERR_ALIGN
+    bad = list(ok_args)
+    bad[8] = p[0]                                                                        # du over u
+    assert lib.sscan_backward(Bt, L, D, N, S.F32, 0, *bad, None) == S.ERR_INVALID
+    # gated: a bias without its gradient output, a gate without dz
+    g = p[:6] + [p[15], None] + p[6:14] + [None, None, p[14], None]
+    assert lib.sscan_backward_gated(Bt, L, D, N, S.F32, 0, *g) == S.ERR_INVALID
+    g = p[:6] + [None, p[15]] + p[6:14] + [None, None, p[14], None]
+    assert lib.sscan_backward_gated(Bt, L, D, N, S.F32, 0, *g) == S.ERR_INVALID
