@@ -357,9 +357,13 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                     if (!wait(BAR_YREADY, pp)) break;
                     load(c + 1);
                 }
-                // MMA 4: S_blk = B^T (w X), M = N (two 64-state chunks kBox apart), K = Q
+                // MMA 4: S_blk = B^T (w X), M = N (two 64-state chunks kBox apart), K = Q.
+                // h_in of this block is waited for here, before MMA 4: warpgroup Y arrives
+                // for the next block's h_in as soon as MMA 4 is done, and a phase-parity
+                // wait must never fall two phases behind its barrier.
                 if (!wait(BAR_WXREADY, pc)) break;
                 if (c > 0 && !wait(BAR_SBLKFREE, pp)) break;
+                if (!wait(BAR_HREADY, pc)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
@@ -368,7 +372,6 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                 mma_commit(&bars[BAR_M4]);
                 // MMA 2: Y1 = P X (P: TMEM columns 8k.. of packed pairs), MMA 3: Y2 = C h_in
                 if (!wait(BAR_PREADY + s, ps)) break;
-                if (!wait(BAR_HREADY, pc)) break;
                 if (c > 0 && !wait(BAR_YFREE, pp)) break;
                 tc_fence_after();
 #pragma unroll
