@@ -715,6 +715,8 @@ def main():
     ap.add_argument("--workload", default="longseq_bf16", choices=sorted(W.WORKLOADS) + sorted(W.SSD_WORKLOADS))
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch rows (small cases for profiling); 0 keeps it")
+    ap.add_argument("--length", type=int, default=0,
+                    help="override the workload's sequence length (small cases for profiling); 0 keeps it")
     ap.add_argument("--ssd-oracle-pairs", type=int, default=4,
                     help="(batch row, head) sequences the SSD oracle baseline times")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -733,12 +735,11 @@ def main():
     if world != args.gpus:
         if world == 1 and args.gpus > 1:
             ap.error("--gpus > 1 needs one process per GPU (torch.distributed.run)")
-    if args.batch > 0:
+    if args.batch > 0 or args.length > 0:
         import dataclasses
-        if args.workload in W.SSD_WORKLOADS:
-            W.SSD_WORKLOADS[args.workload] = dataclasses.replace(W.SSD_WORKLOADS[args.workload], B=args.batch)
-        else:
-            W.WORKLOADS[args.workload] = dataclasses.replace(W.WORKLOADS[args.workload], B=args.batch)
+        table = W.SSD_WORKLOADS if args.workload in W.SSD_WORKLOADS else W.WORKLOADS
+        w0 = table[args.workload]
+        table[args.workload] = dataclasses.replace(w0, B=args.batch or w0.B, L=args.length or w0.L)
     is_ssd = args.workload in W.SSD_WORKLOADS
     if args.impl == "reference":
         if rank == 0:

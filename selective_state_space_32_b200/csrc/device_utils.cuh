@@ -89,28 +89,31 @@ __device__ __forceinline__ f2 exp2_fma_pair(f2 dd, f2 a) {
     return pack2(__uint_as_float(r0), __uint_as_float(r1));
 }
 
-// phi(z) = (exp(z) - 1) / z for |z| <= 1/4: degree-4 polynomial fitted for
-// minimax relative error (csrc/gen_phi_poly.py; 1.5e-7 max relative error in
-// fp32), constant term exactly 1 so that phi(0) = 1.
-__device__ __forceinline__ f2 phi2(f2 z) {
-    f2 q = fma2(splat2(8.333330042660236e-03f), z, splat2(4.177515208721161e-02f));
-    q = fma2(q, z, splat2(1.666673868894577e-01f));
-    q = fma2(q, z, splat2(4.999983012676239e-01f));
-    return fma2(q, z, splat2(1.0f));
+// psi(e) = phi(e ln 2), phi(z) = (exp(z) - 1) / z, for |e| <= 1/(8 ln 2), i.e.
+// |z| <= 1/8, in the variable e = z / ln 2 = delta * A * log2(e) that the
+// exponential 2^e already needs: a degree-3 polynomial fitted for minimax
+// relative error (csrc/gen_phi_poly.py 3 0.125 --log2; 3.3e-7 max relative
+// error of the fp32 Horner evaluation).
+__device__ __forceinline__ f2 psi2(f2 e) {
+    f2 q = fma2(splat2(1.387602649629116e-02f), e, splat2(8.013805747032166e-02f));
+    q = fma2(q, e, splat2(3.4657374024391174e-01f));
+    return fma2(q, e, splat2(9.999997615814209e-01f));
 }
 
-// Exact ZOH coefficient (exp(z) - 1) / A for a pair, z = d*A: d*phi(z) when
-// |z| <= 1/4 (also exact at A = 0), (abar - 1) * (1/A) otherwise (there
-// |abar - 1| >= 0.22, so the 2^-22 relative error of abar stays below ~1.1e-6).
-__device__ __forceinline__ f2 zoh_coef_pair(f2 dd, f2 a1, f2 ia, f2 abar) {
-    const f2 z = mul2(dd, a1);
-    const f2 small = mul2(dd, phi2(z));
-    const f2 big = mul2(add2(abar, splat2(-1.0f)), ia);
-    float z0, z1, s0, s1, g0, g1;
-    unpack2(z, z0, z1);
+// Exact ZOH coefficient (exp(z) - 1) / A for a pair, z = d*A, from e = d*A*log2(e)
+// (the exponent of abar = 2^e), ia = 1/A and nia = -1/A: d*psi(e) when |z| <= 1/8
+// (also at A = 0, where ia is not finite and the other branch is not taken),
+// abar*(1/A) - 1/A otherwise (there |abar - 1| >= 0.117, so the 2^-22 relative
+// error of abar stays below ~2e-6).
+__device__ __forceinline__ f2 zoh_coef_pair(f2 dd, f2 e, f2 ia, f2 nia, f2 abar) {
+    const f2 small = mul2(dd, psi2(e));
+    const f2 big = fma2(abar, ia, nia);
+    float e0, e1, s0, s1, g0, g1;
+    unpack2(e, e0, e1);
     unpack2(small, s0, s1);
     unpack2(big, g0, g1);
-    return pack2(fabsf(z0) <= 0.25f ? s0 : g0, fabsf(z1) <= 0.25f ? s1 : g1);
+    constexpr float kLim = 0.18033688011112042f;  // 1/8 / ln 2
+    return pack2(fabsf(e0) <= kLim ? s0 : g0, fabsf(e1) <= kLim ? s1 : g1);
 }
 
 // softplus(s) = log(1 + e^s) for the fused prologue.  s itself above 20 (the

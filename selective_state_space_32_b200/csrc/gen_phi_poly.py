@@ -5,18 +5,27 @@ against phi on [-Z, Z], in float64 (phi > 0 there).  Prints the coefficients
 (lowest first) as fp32 values and the error of the fp32 Horner evaluation
 (fused multiply-add, as on the GPU) against float64.
 
-    python selective_state_space_32_b200/csrc/gen_phi_poly.py [DEG] [Z]
+    python selective_state_space_32_b200/csrc/gen_phi_poly.py [DEG] [Z] [--log2]
+
+With --log2 the polynomial's variable is e = z / ln 2 (the exponent of 2^e =
+exp(z) that the kernels already compute), i.e. the fit is of phi(e ln 2) on
+|e| <= Z / ln 2.
 """
 import sys
 
 import numpy as np
 
-DEG = int(sys.argv[1]) if len(sys.argv) > 1 else 4
-Z = float(sys.argv[2]) if len(sys.argv) > 2 else 0.25
+ARGS = [a for a in sys.argv[1:] if not a.startswith("--")]
+DEG = int(ARGS[0]) if len(ARGS) > 0 else 4
+Z = float(ARGS[1]) if len(ARGS) > 1 else 0.25
+LOG2 = "--log2" in sys.argv
+SCALE = np.log(2.0) if LOG2 else 1.0  # z = SCALE * variable
+if LOG2:
+    Z = Z / np.log(2.0)
 
 
-def phi(z):
-    z = np.asarray(z, dtype=np.float64)
+def phi(v):
+    z = np.asarray(v, dtype=np.float64) * SCALE
     out = np.ones_like(z)
     nz = np.abs(z) > 1e-12
     out[nz] = np.expm1(z[nz]) / z[nz]
@@ -58,6 +67,6 @@ p = np.full_like(g, c32[DEG])
 for k in range(DEG - 1, -1, -1):
     p = (p.astype(np.float64) * g.astype(np.float64) + np.float64(c32[k])).astype(np.float32)
 rel = np.abs(p.astype(np.float64) - phi(g.astype(np.float64))) / phi(g.astype(np.float64))
-print(f"degree {DEG} on |z| <= {Z}: minimax relative error {e:.3e} (float64), fp32 Horner max {rel.max():.3e}")
+print(f"degree {DEG} on |{'e' if LOG2 else 'z'}| <= {Z:.8f}: minimax relative error {e:.3e} (float64), fp32 Horner max {rel.max():.3e}")
 for k, v in enumerate(c32):
     print(f"c{k} = {float(v)!r:>24}  ({np.float32(v).view(np.uint32):#010x})")

@@ -95,7 +95,13 @@ struct ChainedCfg {
     static constexpr int kU = T * CPW * ES;                 // one u or delta tile
     static constexpr int kB = T * N * ES;                   // one B or C tile
     static constexpr int kStage = 2 * kU + 2 * kB;          // TMA bytes per stage
-    static constexpr int kConv = ES == 2 ? 2 * T * N * 4 : 0;  // widened B, C (bf16 I/O)
+    // widened B, C (bf16 I/O): fp32 rows of N states; with 16 states per lane each
+    // lane's group is followed by 4 floats of padding, so that the LPC groups a warp
+    // reads with one 16-byte load per lane fall on disjoint banks (unpadded, groups
+    // 64 bytes apart pair up on the same banks)
+    static constexpr int kPadG = (ES == 2 && NL >= 16) ? 4 : 0;
+    static constexpr int kRowW = N + LPC * kPadG;             // floats per widened row
+    static constexpr int kConv = ES == 2 ? 2 * T * kRowW * 4 : 0;
     static constexpr int kWarp = ((STAGES * kStage + kConv) + 127) / 128 * 128;
     static constexpr int kBars = (2 * WPC * STAGES * 8 + 127) / 128 * 128;  // full + empty per slot
     static constexpr int kSmem = WPC * kWarp + kBars;
@@ -127,7 +133,7 @@ struct ChainedCfg {
 // token's parity; it selects which pairs take 2^x on the FMA pipe (a quarter
 // of all pairs across two tokens).
 template <int NP, bool ZOH, bool POLY, int PAR>
-__device__ __forceinline__ void discretize(f2 (&ab)[NP], f2 (&bu)[NP], const f2 (&A2)[NP], const f2 (&A1)[NP],
+__device__ __forceinline__ void discretize(f2 (&ab)[NP], f2 (&bu)[NP], const f2 (&A2)[NP], const f2 (&nA)[NP],
                                            const f2 (&iA)[NP], float cap, float x, float dl,
                                            const float *Bs) {
     const f2 dd = splat2(dl);
@@ -145,15 +151,16 @@ __device__ __forceinline__ void discretize(f2 (&ab)[NP], f2 (&bu)[NP], const f2 
         for (int q = 0; q < 2; ++q) {
             const int p = 2 * i + q;
             const f2 bp = q ? b23 : b01;
+            const f2 e = mul2(dd, A2[p]);
             if (POLY && ((PAR * NP + p) % 4 == 3)) {
                 ab[p] = exp2_fma_pair(ddc, A2[p]);
             } else {
                 float e0, e1;
-                unpack2(mul2(dd, A2[p]), e0, e1);
+                unpack2(e, e0, e1);
                 ab[p] = pack2(ex2(e0), ex2(e1));
             }
             if (ZOH)
-                bu[p] = mul2(zoh_coef_pair(dd, A1[p], iA[p], ab[p]), mul2(bp, xx));
+                bu[p] = mul2(zoh_coef_pair(dd, e, iA[p], nA[p], ab[p]), mul2(bp, xx));
             else
                 bu[p] = mul2(bp, du2);
         }
@@ -626,7 +633,7 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
     constexpr int kStageB = FUSED ? Cfg::kStageF : Cfg::kStage;  // bytes of one stage
     unsigned char *wbase = smem + warp * kWarpB;
     float *convB = reinterpret_cast<float *>(wbase + STAGES * kStageB);
-    float *convC = convB + T * N;
+    float *convC = convB + T * Cfg::kRowW;
     float *dsf0 = reinterpret_cast<float *>(wbase + STAGES * kStageB + Cfg::kConv);  // FUSED: delta'
     float *gsf0 = dsf0 + (HELP ? STAGES : 1) * T * CPW;                               // FUSED: silu(z)
     uint64_t *full = bars + warp * STAGES;
@@ -651,6 +658,10 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
     const int cl = lane / LPC;   // channel within the chain
     const int g = lane % LPC;    // state group
     const int n0 = g * NL;
+    // B, C tiles: row stride and this lane's group offset (TMA tiles for fp32 I/O,
+    // padded widened tiles for bf16)
+    constexpr int RS = Cfg::ES == 4 ? N : Cfg::kRowW;
+    const int gofs = Cfg::ES == 4 ? n0 : g * (NL + Cfg::kPadG);
     int64_t consumed = 0;
     bool failed = false;
 
@@ -671,8 +682,8 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
             A2[p] = pack2(static_cast<float>(static_cast<double>(a0) * 1.4426950408889634),
                           static_cast<float>(static_cast<double>(a1) * 1.4426950408889634));
             if (ZOH) {
-                A1[p] = pack2(a0, a1);
                 iA[p] = pack2(1.0f / a0, 1.0f / a1);
+                A1[p] = pack2(-1.0f / a0, -1.0f / a1);  // -1/A for the ZOH coefficient
             }
             if (POLY && (p % 2 == 1)) {  // pairs that may take the FMA-pipe exponent
                 float x0, x1;
@@ -761,7 +772,7 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
                 Bs = reinterpret_cast<const float *>(tile_b(s));
                 Cs = reinterpret_cast<const float *>(tile_c(s));
             } else {
-                // widen the stage's B and C tiles to fp32 once for all lanes
+                // widen the stage's B and C tiles to fp32 once for all lanes (padded rows)
                 constexpr int kChunks = T * N / 8;  // 8 bf16 per 16-byte chunk
                 const uint4 *rb = reinterpret_cast<const uint4 *>(tile_b(s));
                 const uint4 *rc = reinterpret_cast<const uint4 *>(tile_c(s));
@@ -770,8 +781,10 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
                     const uint4 vb = rb[q], vc = rc[q];
                     const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
                     const uint32_t wc[4] = {vc.x, vc.y, vc.z, vc.w};
-                    float4 *ob = reinterpret_cast<float4 *>(convB + 8 * q);
-                    float4 *oc = reinterpret_cast<float4 *>(convC + 8 * q);
+                    const int col = (8 * q) % N, row = (8 * q) / N;  // a chunk never spans two groups
+                    const int dst = row * Cfg::kRowW + (col / NL) * (NL + Cfg::kPadG) + col % NL;
+                    float4 *ob = reinterpret_cast<float4 *>(convB + dst);
+                    float4 *oc = reinterpret_cast<float4 *>(convC + dst);
                     ob[0] = make_float4(__uint_as_float(wb[0] << 16), __uint_as_float(wb[0] & 0xffff0000u),
                                         __uint_as_float(wb[1] << 16), __uint_as_float(wb[1] & 0xffff0000u));
                     ob[1] = make_float4(__uint_as_float(wb[2] << 16), __uint_as_float(wb[2] & 0xffff0000u),
@@ -824,7 +837,7 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
                 float yv[G];
 #pragma unroll
                 for (int q = 0; q < G; ++q)
-                    yv[q] = advance_euler<NP>(h, ab[q], duv[q], Bs + (j0 + q) * N + n0, Cs + (j0 + q) * N + n0);
+                    yv[q] = advance_euler<NP>(h, ab[q], duv[q], Bs + (j0 + q) * RS + gofs, Cs + (j0 + q) * RS + gofs);
                 const int base = reduce_scatter<LPC, G>(yv, g);
                 if (FUSED) {
 #pragma unroll
@@ -849,13 +862,13 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
                         dmin = fminf(dmin, dl);
                     }
                     if (q & 1)
-                        discretize<NP, ZOH, POLY, 1>(ab[q], bu[q], A2, A1, iA, cap, x, dl, Bs + (j0 + q) * N + n0);
+                        discretize<NP, ZOH, POLY, 1>(ab[q], bu[q], A2, A1, iA, cap, x, dl, Bs + (j0 + q) * RS + gofs);
                     else
-                        discretize<NP, ZOH, POLY, 0>(ab[q], bu[q], A2, A1, iA, cap, x, dl, Bs + (j0 + q) * N + n0);
+                        discretize<NP, ZOH, POLY, 0>(ab[q], bu[q], A2, A1, iA, cap, x, dl, Bs + (j0 + q) * RS + gofs);
                 }
                 float yv[G];
 #pragma unroll
-                for (int q = 0; q < G; ++q) yv[q] = advance<NP>(h, ab[q], bu[q], Cs + (j0 + q) * N + n0);
+                for (int q = 0; q < G; ++q) yv[q] = advance<NP>(h, ab[q], bu[q], Cs + (j0 + q) * RS + gofs);
                 const int base = reduce_scatter<LPC, G>(yv, g);
                 if (FUSED) {
 #pragma unroll
@@ -891,8 +904,8 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
                     ssum += dl;
                     dmin = fminf(dmin, dl);
                 }
-                discretize<NP, ZOH, POLY, 0>(ab, bu, A2, A1, iA, cap, x, dl, Bs + j * N + n0);
-                float yv = advance<NP>(h, ab, bu, Cs + j * N + n0);
+                discretize<NP, ZOH, POLY, 0>(ab, bu, A2, A1, iA, cap, x, dl, Bs + j * RS + gofs);
+                float yv = advance<NP>(h, ab, bu, Cs + j * RS + gofs);
 #pragma unroll
                 for (int o = 1; o < LPC; o <<= 1) yv += __shfl_xor_sync(0xffffffffu, yv, o);
                 if (FUSED) yv *= gsf[j * CPW + cl];

@@ -40,7 +40,7 @@ sscan_generic_kernel(const IO *__restrict__ u, const IO *__restrict__ delta,
     const int64_t dc = valid ? d : D - 1;  // ragged tail: read a real channel, store nothing
     const int n0 = g * NL;
 
-    // per-thread constants: A*log2(e) (Abar = 2^(delta*A2)); ZOH also needs A and 1/A
+    // per-thread constants: A*log2(e) (Abar = 2^(delta*A2)); ZOH also needs 1/A and -1/A
     f2 A2[NP], A1[NP], iA[NP];
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
@@ -48,7 +48,7 @@ sscan_generic_kernel(const IO *__restrict__ u, const IO *__restrict__ delta,
         A2[p] = pack2(static_cast<float>(static_cast<double>(a0) * 1.4426950408889634),
                       static_cast<float>(static_cast<double>(a1) * 1.4426950408889634));
         if (ZOH) {
-            A1[p] = pack2(a0, a1);
+            A1[p] = pack2(-1.0f / a0, -1.0f / a1);  // -1/A for the ZOH coefficient
             iA[p] = pack2(1.0f / a0, 1.0f / a1);
         }
     }
@@ -108,13 +108,14 @@ sscan_generic_kernel(const IO *__restrict__ u, const IO *__restrict__ delta,
 #pragma unroll
                 for (int p = 0; p < NP; ++p) {
                     float e0, e1;
-                    unpack2(mul2(dd, A2[p]), e0, e1);
+                    const f2 e = mul2(dd, A2[p]);
+                    unpack2(e, e0, e1);
                     const f2 abar = pack2(ex2(e0), ex2(e1));
                     f2 bu;
                     if (!ZOH) {
                         bu = mul2(Bp[p], du2);
                     } else {
-                        bu = mul2(zoh_coef_pair(dd, A1[p], iA[p], abar), mul2(Bp[p], xx));
+                        bu = mul2(zoh_coef_pair(dd, e, iA[p], A1[p], abar), mul2(Bp[p], xx));
                     }
                     h[p] = fma2(abar, h[p], bu);
                     if (p & 1)

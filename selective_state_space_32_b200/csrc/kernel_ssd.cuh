@@ -332,31 +332,35 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                 return wait_or_abort(&bars[bar], parity, abort_flag, prm.status, 16);
             };
             bool issued = false;
+            auto mma1 = [&](int c) {  // S of block c = C B^T, K = N in 8 steps of 16 states
+                const uint32_t st = sbase + kOffStage + (c & 1) * kStage;
+                const uint32_t sC = st + kOffC, sB = st + kOffB;
+                const uint32_t tS = tbase + kColS + 128 * (c & 1);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t off = (k >> 2) * kBox + (k & 3) * 32;
+                    mma_ss(tS, sdesc_sw128(sC + off, 16, 1024), sdesc_sw128(sB + off, 16, 1024), id_s, k > 0);
+                }
+                mma_commit(&bars[BAR_SDONE + (c & 1)]);
+                issued = true;
+            };
+            // Issue order: MMA 1 of block c+1 goes ahead of MMAs 2 and 3 of block c, so that
+            // warpgroup P forms P of block c+1 while they run.  The S buffer of block c+1 last
+            // held block c-1's P, read by its MMA 2: done once BAR_YREADY of c-1 was seen.
             load(0);
             if (nb > 1) load(1);
-            for (int c = 0; c < nb; ++c) {
+            bool run = wait(BAR_FULL, 0);
+            if (run) {
+                tc_fence_after();
+                mma1(0);
+            }
+            for (int c = 0; run && c < nb; ++c) {
                 const int s = c & 1;
                 const uint32_t ps = (c >> 1) & 1, pc = c & 1, pp = (c - 1) & 1;
                 const uint32_t st = sbase + kOffStage + s * kStage;
                 const uint32_t sC = st + kOffC, sB = st + kOffB, sX = st + kOffX;
                 const uint32_t sH = sbase + kOffH + s * kBox;  // h_in of this block
                 const uint32_t tS = tbase + kColS + 128 * s;
-                if (!wait(BAR_FULL + s, ps)) break;
-                tc_fence_after();
-                // MMA 1: S = C B^T, K = N in 8 steps of 16 states (4 per 64-state box).  S of
-                // this stage was last read (as P) by MMA 2 of block c-2, done: see below.
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint32_t off = (k >> 2) * kBox + (k & 3) * 32;
-                    mma_ss(tS, sdesc_sw128(sC + off, 16, 1024), sdesc_sw128(sB + off, 16, 1024), id_s, k > 0);
-                }
-                mma_commit(&bars[BAR_SDONE + s]);
-                issued = true;
-                // block c+1 reuses the stage of block c-1: free once MMAs 2-4 of c-1 are done
-                if (c >= 1 && c + 1 < nb) {
-                    if (!wait(BAR_YREADY, pp)) break;
-                    load(c + 1);
-                }
                 // MMA 4: S_blk = B^T (w X), M = N (two 64-state chunks kBox apart), K = Q.
                 // h_in of this block is waited for here, before MMA 4: warpgroup Y arrives
                 // for the next block's h_in as soon as MMA 4 is done, and a phase-parity
@@ -370,6 +374,12 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                     mma_ss(tbase + kColSblk, sdesc_sw128(sB + k * 2048, kBox, 1024),
                            sdesc_sw128(sWX + k * 2048, kBox, 1024), id_st, k > 0);
                 mma_commit(&bars[BAR_M4]);
+                // MMA 1 of the next block
+                if (c + 1 < nb) {
+                    if (!wait(BAR_FULL + (s ^ 1), ((c + 1) >> 1) & 1)) break;
+                    tc_fence_after();
+                    mma1(c + 1);
+                }
                 // MMA 2: Y1 = P X (P: TMEM columns 8k.. of packed pairs), MMA 3: Y2 = C h_in
                 if (!wait(BAR_PREADY + s, ps)) break;
                 if (c > 0 && !wait(BAR_YFREE, pp)) break;
@@ -384,6 +394,11 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                            id_y, k > 0);
                 }
                 mma_commit(&bars[BAR_YREADY]);
+                // block c+2 goes into this stage once every MMA of block c is done
+                if (c + 2 < nb) {
+                    if (!wait(BAR_YREADY, pc)) break;
+                    load(c + 2);
+                }
             }
             // the tensor memory is released below: every MMA issued must be done first.  A
             // commit tracks all earlier MMAs of this thread: one more on its own barrier,
@@ -436,7 +451,7 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                 if (ok) {
                     tc_fence_after();
                     const uint32_t tS = lane_base + kColS + 128 * s;
-#pragma unroll
+#pragma unroll 1
                     for (int kk = 0; kk < 4; ++kk) {  // columns 32kk .. 32kk+31 (groups 2kk, 2kk+1)
                         uint32_t pk[16];
                         if (kk < wl) {
@@ -506,17 +521,47 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
             };
             write_h(0);
             mbar_arrive(&bars[BAR_HREADY]);
+            // y of block c: P X + 2^cs (C h_in), rows inside the sequence only
+            auto emit_y = [&](int c, float cs) {
+                ok = wait_warp(BAR_YREADY, c & 1);
+                if (!ok) return;
+                tc_fence_after();
+                const float e = ex2(cs);
+                uint32_t o[2][16];
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t y1[32], y2[32];
+                    tmem_ld32(lane_base + kColY1 + 32 * half, y1);
+                    tmem_ld32(lane_base + kColY2 + 32 * half, y2);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        o[half][j] = pack_bf16(fmaf(e, __uint_as_float(y2[2 * j]), __uint_as_float(y1[2 * j])),
+                                               fmaf(e, __uint_as_float(y2[2 * j + 1]), __uint_as_float(y1[2 * j + 1])));
+                }
+                tc_fence_before();
+                mbar_arrive(&bars[BAR_YFREE]);
+                const int64_t tok = int64_t(c) * kQ + t;
+                if (tok < L) {
+                    uint4 *d4 = reinterpret_cast<uint4 *>(prm.y + ((int64_t(b) * L + tok) * prm.H + h) * kP);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        d4[q] = make_uint4(o[q >> 2][4 * (q & 3)], o[q >> 2][4 * (q & 3) + 1],
+                                           o[q >> 2][4 * (q & 3) + 2], o[q >> 2][4 * (q & 3) + 3]);
+                }
+            };
+            // Per block c: w X of block c first (MMA 4 of block c can start at once),
+            // then y of block c-1 (while MMA 4 runs), then the state passing of block c.
+            float cs_prev = 0.0f;
             for (int c = 0; c < nb; ++c) {
                 const int s = c & 1;
                 const uint32_t ps = (c >> 1) & 1, pc = c & 1;
                 const float dt = dt_next;
-                const int64_t tok = int64_t(c) * kQ + t;
-                const int64_t nxt = tok + kQ;
+                const int64_t nxt = int64_t(c + 1) * kQ + t;
                 dt_next = nxt < L ? __ldg(dtp + nxt * prm.H) : 0.0f;
                 float tot;
                 const float cs = wg_scan(dt * a2, wl, lane, tot4, bar_id, tot);
-                // ---- w X for MMA 4: X of this block landed; w X's buffer was freed by MMA 4 of
-                // block c-1 (waited below in the previous block)
+                // ---- w X for MMA 4: X of this block landed; w X's buffer was freed by MMA 4
+                // of block c-1 (waited for in the state step of the previous block)
                 ok = wait_warp(BAR_FULL + s, ps);
                 if (ok) {
                     const float wv = dt * ex2(tot - cs);  // w_s of the block end state, s = t
@@ -534,7 +579,10 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                     fence_proxy_async_smem();
                     mbar_arrive(&bars[BAR_WXREADY]);
                 }
-                // ---- state passing: h = 2^cs_end h + S_blk (row n = t); then h_in of block c+1
+                if (c > 0) emit_y(c - 1, cs_prev);
+                cs_prev = cs;
+                // ---- state passing: h = 2^cs_end h + S_blk (row n = t); then h_in of block c+1,
+                // into the buffer MMA 3 of block c-1 read (done: its y was just emitted)
                 ok = wait_warp(BAR_M4, pc);
                 if (ok) {
                     tc_fence_after();
@@ -549,37 +597,11 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                     }
                     tc_fence_before();
                     mbar_arrive(&bars[BAR_SBLKFREE]);
-                    // buffer (c+1)&1 was last read by MMA 3 of block c-1, waited below in block c-1
                     write_h((c + 1) & 1);
                     mbar_arrive(&bars[BAR_HREADY]);
                 }
-                // ---- y = P X + 2^cs (C h_in), rows inside the sequence only
-                ok = wait_warp(BAR_YREADY, pc);
-                if (ok) {
-                    tc_fence_after();
-                    const float e = ex2(cs);
-                    uint32_t o[2][16];
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        uint32_t y1[32], y2[32];
-                        tmem_ld32(lane_base + kColY1 + 32 * half, y1);
-                        tmem_ld32(lane_base + kColY2 + 32 * half, y2);
-#pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            o[half][j] = pack_bf16(fmaf(e, __uint_as_float(y2[2 * j]), __uint_as_float(y1[2 * j])),
-                                                   fmaf(e, __uint_as_float(y2[2 * j + 1]), __uint_as_float(y1[2 * j + 1])));
-                    }
-                    tc_fence_before();
-                    mbar_arrive(&bars[BAR_YFREE]);
-                    if (tok < L) {
-                        uint4 *d4 = reinterpret_cast<uint4 *>(prm.y + ((int64_t(b) * L + tok) * prm.H + h) * kP);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            d4[q] = make_uint4(o[q >> 2][4 * (q & 3)], o[q >> 2][4 * (q & 3) + 1],
-                                               o[q >> 2][4 * (q & 3) + 2], o[q >> 2][4 * (q & 3) + 3]);
-                    }
-                }
             }
+            if (nb > 0) emit_y(nb - 1, cs_prev);
             if (ok && prm.h_final) {
                 float *dst = prm.h_final + ((int64_t(b) * prm.H + h) * kN + t) * kP;
 #pragma unroll

@@ -67,11 +67,11 @@ sscan_step_kernel(const IO *__restrict__ u, const IO *__restrict__ delta, const 
                          static_cast<float>(static_cast<double>(a.y) * 1.4426950408889634));
         A2[k][1] = pack2(static_cast<float>(static_cast<double>(a.z) * 1.4426950408889634),
                          static_cast<float>(static_cast<double>(a.w) * 1.4426950408889634));
-        if (ZOH) {
-            A1[k][0] = pack2(a.x, a.y);
-            A1[k][1] = pack2(a.z, a.w);
+        if (ZOH) {  // 1/A and -1/A for the ZOH coefficient
             iA[k][0] = pack2(1.0f / a.x, 1.0f / a.y);
             iA[k][1] = pack2(1.0f / a.z, 1.0f / a.w);
+            A1[k][0] = pack2(-1.0f / a.x, -1.0f / a.y);
+            A1[k][1] = pack2(-1.0f / a.z, -1.0f / a.w);
         }
         if (h0 != nullptr) {
             const float4 v = *reinterpret_cast<const float4 *>(h0 + (b[k] * D + d[k]) * N + n0);
@@ -103,10 +103,11 @@ sscan_step_kernel(const IO *__restrict__ u, const IO *__restrict__ delta, const 
 #pragma unroll
             for (int p = 0; p < 2; ++p) {
                 float e0, e1;
-                unpack2(mul2(dd, A2[k][p]), e0, e1);
+                const f2 e = mul2(dd, A2[k][p]);
+                unpack2(e, e0, e1);
                 const f2 abar = pack2(ex2(e0), ex2(e1));
                 const f2 bp = p ? b23 : b01;
-                const f2 bu = ZOH ? mul2(zoh_coef_pair(dd, A1[k][p], iA[k][p], abar), mul2(bp, splat2(x[k])))
+                const f2 bu = ZOH ? mul2(zoh_coef_pair(dd, e, iA[k][p], A1[k][p], abar), mul2(bp, splat2(x[k])))
                                   : mul2(bp, splat2(dv * x[k]));
                 h[k][p] = fma2(abar, h[k][p], bu);
                 ya = fma2(p ? pack2(Cv[k].z, Cv[k].w) : pack2(Cv[k].x, Cv[k].y), h[k][p], ya);

@@ -90,7 +90,8 @@ constexpr int64_t kMinChainedL = 64;  // shorter sequences use the step kernel
 int chained_smem_bytes(const KCfg &k, int es) {
     const int lpc = k.N / k.NL, cpw = 32 / lpc;
     const int kU = k.T * cpw * es, kB = k.T * k.N * es;
-    const int stage = 2 * kU + 2 * kB, conv = es == 2 ? 2 * k.T * k.N * 4 : 0;
+    const int rowW = k.N + ((es == 2 && k.NL >= 16) ? 4 * lpc : 0);  // ChainedCfg::kRowW
+    const int stage = 2 * kU + 2 * kB, conv = es == 2 ? 2 * k.T * rowW * 4 : 0;
     const int warp = (k.STAGES * stage + conv + 127) / 128 * 128;
     const int bars = (2 * k.WPC * k.STAGES * 8 + 127) / 128 * 128;
     return k.WPC * warp + bars;
