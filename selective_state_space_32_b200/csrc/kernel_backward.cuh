@@ -29,9 +29,9 @@
 // ys are summed over LPC lanes (log2 LPC shuffles) and dA needs none; a block
 // of four warps covers 4 CPW consecutive channels of one batch row and walks
 // the same chunks in the same order, so dB and dC (sums over channels) are
-// summed over the warp by shuffles, over the block in shared memory once per
-// chunk, and added to the fp32 outputs with one 16-byte atomic per four
-// states and token (outputs zeroed by the host).
+// summed over the warp by a reduce-scatter of shuffles, over the block in
+// shared memory once per chunk, and added to the fp32 outputs with one 16-byte
+// atomic per four states and token (outputs zeroed by the host).
 #pragma once
 
 #include "device_utils.cuh"
@@ -66,11 +66,40 @@ template <> __device__ __forceinline__ float4 bwd_ld4<uint16_t>(const uint16_t *
 }
 __device__ __forceinline__ float f4_at(const float4 &v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
 
+// Sum the four per-lane values over the lanes that share a state group (the
+// warp's channels: lane bits LPC, 2 LPC, ... 16), as a reduce-scatter: while a
+// lane holds more than one value it keeps half and sends the other half to its
+// partner, then whole values are summed.  Afterwards v[0 .. V) hold the totals
+// of the group's states jbase .. jbase + V - 1, V = 4 >> min(levels, 2); lanes
+// that differ only in the bits above the first two levels hold the same totals.
+template <int LPC>
+__device__ __forceinline__ int channel_scatter4(float (&v)[4], int lane, int &V) {
+    int jbase = 0, cnt = 4;
+#pragma unroll
+    for (int m = LPC; m < 32; m <<= 1) {
+        if (cnt >= 2) {
+            const bool up = (lane & m) != 0;
+#pragma unroll
+            for (int i = 0; i < cnt / 2; ++i) {
+                const float send = up ? v[i] : v[i + cnt / 2];
+                const float keep = up ? v[i + cnt / 2] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+            }
+            if (up) jbase += cnt / 2;
+            cnt /= 2;
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
+        }
+    }
+    V = cnt;
+    return jbase;
+}
+
 template <class IO, int N, bool ZOH, bool FUSED>
 __global__ void __launch_bounds__(kBwdThreads)
 sscan_backward_kernel(const BwdParams P) {
     constexpr int LPC = N / 4, CPW = 32 / LPC, CPB = kBwdWarps * CPW, KC = kChunk;
-    __shared__ float4 s_db[kBwdWarps][KC][N / 4], s_dc[kBwdWarps][KC][N / 4];
+    __shared__ __align__(16) float s_db[kBwdWarps][KC][N], s_dc[kBwdWarps][KC][N];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cl = lane / LPC, g = lane % LPC, n0 = 4 * g;
     const int64_t L = P.L, D = P.D;
@@ -137,25 +166,40 @@ sscan_backward_kernel(const BwdParams P) {
     };
 
     // ---- pass 1: forward, keeping the state entering every chunk ----
+    // (chunk by chunk: a chunk's loads sit in one straight-line block, ahead of its
+    // dependent updates)
     float h[4];
     {
         const float4 v = P.h0 ? *reinterpret_cast<const float4 *>(P.h0 + (b * D + dc) * N + n0)
                               : make_float4(0.f, 0.f, 0.f, 0.f);
         h[0] = v.x; h[1] = v.y; h[2] = v.z; h[3] = v.w;
     }
-    for (int64_t t = 0; t < L; ++t) {
-        if (t % KC == 0)
-            *reinterpret_cast<float4 *>(ck + (t / KC) * N) = make_float4(h[0], h[1], h[2], h[3]);
-        float sg;
-        const float dl = step(t, sg);
-        const float x = Io<IO>::widen(Io<IO>::ld(u + t * D));
-        const float4 Bv = bwd_ld4<IO>(Bp + t * N);
+    for (int64_t c = 0; c < P.nchunks; ++c) {
+        const int64_t t0 = c * KC;
+        const int nt = static_cast<int>(L - t0 < KC ? L - t0 : KC);
+        *reinterpret_cast<float4 *>(ck + c * N) = make_float4(h[0], h[1], h[2], h[3]);
+        float xs[KC], ds[KC];
+        float4 Bs[KC];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float abar = ex2(dl * a2[i]);
-            float beta, q0, q1, q2;
-            coefs(i, dl, abar, f4_at(Bv, i), beta, q0, q1, q2);
-            h[i] = fmaf(abar, h[i], beta * x);
+        for (int k = 0; k < KC; ++k) {
+            if (k < nt) {
+                float sg;
+                ds[k] = step(t0 + k, sg);
+                xs[k] = Io<IO>::widen(Io<IO>::ld(u + (t0 + k) * D));
+                Bs[k] = bwd_ld4<IO>(Bp + (t0 + k) * N);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < KC; ++k) {
+            if (k < nt) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float abar = ex2(ds[k] * a2[i]);
+                    float beta, q0, q1, q2;
+                    coefs(i, ds[k], abar, f4_at(Bs[k], i), beta, q0, q1, q2);
+                    h[i] = fmaf(abar, h[i], beta * xs[k]);
+                }
+            }
         }
     }
 
@@ -202,7 +246,6 @@ sscan_backward_kernel(const BwdParams P) {
         // reverse over the chunk's tokens
 #pragma unroll
         for (int k = KC - 1; k >= 0; --k) {
-            float4 vb4 = make_float4(0.f, 0.f, 0.f, 0.f), vc4 = make_float4(0.f, 0.f, 0.f, 0.f);
             if (k < nt) {
                 const int64_t t = t0 + k;
                 float sg;
@@ -256,20 +299,17 @@ sscan_backward_kernel(const BwdParams P) {
                     }
                 }
                 // sums over the warp's channels (lanes with the same state group)
+                int V;
+                const int jb = channel_scatter4<LPC>(vb, lane, V);
+                channel_scatter4<LPC>(vc, lane, V);
+                if (lane < 4 * LPC) {  // one of the lanes holding each total
 #pragma unroll
-                for (int o = LPC; o < 32; o <<= 1) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        vb[i] += __shfl_xor_sync(0xffffffffu, vb[i], o);
-                        vc[i] += __shfl_xor_sync(0xffffffffu, vc[i], o);
-                    }
+                    for (int i = 0; i < 4; ++i)
+                        if (i < V) {
+                            s_db[warp][k][n0 + jb + i] = vb[i];
+                            s_dc[warp][k][n0 + jb + i] = vc[i];
+                        }
                 }
-                vb4 = make_float4(vb[0], vb[1], vb[2], vb[3]);
-                vc4 = make_float4(vc[0], vc[1], vc[2], vc[3]);
-            }
-            if (cl == 0) {
-                s_db[warp][k][g] = vb4;
-                s_dc[warp][k][g] = vc4;
             }
         }
         __syncthreads();
@@ -281,7 +321,7 @@ sscan_backward_kernel(const BwdParams P) {
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int w = 0; w < kBwdWarps; ++w) {
-                const float4 v = which ? s_dc[w][k][q] : s_db[w][k][q];
+                const float4 v = *reinterpret_cast<const float4 *>(which ? &s_dc[w][k][4 * q] : &s_db[w][k][4 * q]);
                 acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
             }
             float *dst = (which ? P.dC : P.dB) + (b * L + t0 + k) * N + 4 * q;

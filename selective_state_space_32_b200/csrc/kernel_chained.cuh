@@ -879,62 +879,7 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
                     for (int q = 0; q < KEEP; ++q) Io<IO>::st(yp + (j0 + base + q) * ystr, yv[q]);
                 }
             };
-            // Euler with 8 states per lane, full stage: software-pipelined 8-token groups.
-            // The exponentials of group gi+1 (MUFU, independent of the state) are placed
-            // with the state updates of group gi (FMA pipe), so one warp keeps both pipes
-            // busy instead of alternating between an exponential phase and an update phase;
-            // the two 8-token buffers take the registers of one 16-token group.
-            constexpr int GP = 8;
-            constexpr bool PIPE = !ZOH && NL == 8 && T % GP == 0 && T / GP >= 2;
-            auto disc_p = [&](int j0, f2 (&abx)[GP][NP], float (&dux)[GP]) {
-#pragma unroll
-                for (int q = 0; q < GP; ++q) {
-                    const float x = Io<IO>::widen(us[(j0 + q) * CPW + cl]);
-                    const float dl = delta_at((j0 + q) * CPW + cl);
-                    if (SPLIT) {
-                        ssum += dl;
-                        dmin = fminf(dmin, dl);
-                    }
-                    dux[q] = dl * x;
-                    if (q & 1)
-                        discretize_abar<NP, POLY, 1>(abx[q], A2, cap, dl);
-                    else
-                        discretize_abar<NP, POLY, 0>(abx[q], A2, cap, dl);
-                }
-            };
-            auto adv_p = [&](int j0, f2 (&abx)[GP][NP], float (&dux)[GP]) {
-                constexpr int KP = GP / LPC > 0 ? GP / LPC : 1;
-                const bool store = LPC <= GP || (g & (LPC / GP - 1)) == 0;
-                float yv[GP];
-#pragma unroll
-                for (int q = 0; q < GP; ++q)
-                    yv[q] = advance_euler<NP>(h, abx[q], dux[q], Bs + (j0 + q) * RS + gofs, Cs + (j0 + q) * RS + gofs);
-                const int base = reduce_scatter<LPC, GP>(yv, g);
-                if (FUSED) {
-#pragma unroll
-                    for (int q = 0; q < KP; ++q) yv[q] *= gsf[(j0 + base + q) * CPW + cl];
-                }
-                if (store) {
-#pragma unroll
-                    for (int q = 0; q < KP; ++q) Io<IO>::st(yp + (j0 + base + q) * ystr, yv[q]);
-                }
-            };
-            if (PIPE && nsteps == T) {
-                f2 abA[GP][NP], abB[GP][NP];
-                float duA[GP], duB[GP];
-                disc_p(0, abA, duA);
-#pragma unroll
-                for (int gi = 0; gi < T / GP; ++gi) {
-                    if (gi % 2 == 0) {
-                        if (gi + 1 < T / GP) disc_p((gi + 1) * GP, abB, duB);
-                        adv_p(gi * GP, abA, duA);
-                    } else {
-                        if (gi + 1 < T / GP) disc_p((gi + 1) * GP, abA, duA);
-                        adv_p(gi * GP, abB, duB);
-                    }
-                }
-                j = T;
-            } else if (!ZOH) {
+            if (!ZOH) {
                 if (nsteps == T) {
 #pragma unroll
                     for (int j0 = 0; j0 < T; j0 += G) group_euler(j0);

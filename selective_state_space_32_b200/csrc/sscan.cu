@@ -226,18 +226,13 @@ void choose_schedule(sscan_plan *p) {
             p->cfg = i;
             p->chains_per_row = cpr;
             p->chains = chains;
-            if (p->split) {
-                // the same whole number of pieces for every chain, so that neighbouring
-                // chains (which share the 64-byte L2 lines of their u and delta rows) are
-                // cut at nearly the same tokens and scanned there at the same time; with
-                // a fractional count their pieces drift apart and each line is fetched
-                // from DRAM once per chain (1.6x the input bytes measured on B200)
-                const int64_t pieces = workers / chains;
-                p->seg = ceil_div(p->L, pieces);
-                workers = ceil_div(chains * pieces, k.WPC) * k.WPC;  // whole blocks; trailing warps idle
-            } else {
-                p->seg = ceil_div(chains * p->L, workers);
-            }
+            // Segments are equal over the whole grid, in split mode too.  Cutting every chain
+            // into the same whole number of pieces would line up the pieces of neighbouring
+            // chains (which share the 64-byte L2 lines of their u and delta rows) and read
+            // each input byte from DRAM once instead of 1.6 times, but leaves warps idle
+            // (1152 of 1184 on the 131072-token sequence) and measured 3 % slower on B200:
+            // the kernel is bound by its ALUs, not by DRAM.
+            p->seg = ceil_div(chains * p->L, workers);
             p->workers = workers;
             // split mode indexes pieces by equal segments; the chained mode balances time
             p->seg_shift = p->split ? 0 : p->seg * (light >= 0 ? light : kLightPermille) / 1000;
