@@ -182,12 +182,11 @@ sscan_backward_kernel(const BwdParams P) {
         float4 Bs[KC];
 #pragma unroll
         for (int k = 0; k < KC; ++k) {
-            if (k < nt) {
-                float sg;
-                ds[k] = step(t0 + k, sg);
-                xs[k] = Io<IO>::widen(Io<IO>::ld(u + (t0 + k) * D));
-                Bs[k] = bwd_ld4<IO>(Bp + (t0 + k) * N);
-            }
+            const int64_t t = t0 + (k < nt ? k : nt - 1);
+            float sg;
+            ds[k] = step(t, sg);
+            xs[k] = Io<IO>::widen(Io<IO>::ld(u + t * D));
+            Bs[k] = bwd_ld4<IO>(Bp + t * N);
         }
 #pragma unroll
         for (int k = 0; k < KC; ++k) {
@@ -226,12 +225,12 @@ sscan_backward_kernel(const BwdParams P) {
             float hc[4] = {h_in[0], h_in[1], h_in[2], h_in[3]};
 #pragma unroll
             for (int k = 0; k < KC; ++k) {
+                const int64_t t = t0 + (k < nt ? k : nt - 1);  // loads need not wait behind work
+                float sg;
+                const float dl = step(t, sg);
+                const float x = Io<IO>::widen(Io<IO>::ld(u + t * D));
+                const float4 Bv = bwd_ld4<IO>(Bp + t * N);
                 if (k < nt) {
-                    const int64_t t = t0 + k;
-                    float sg;
-                    const float dl = step(t, sg);
-                    const float x = Io<IO>::widen(Io<IO>::ld(u + t * D));
-                    const float4 Bv = bwd_ld4<IO>(Bp + t * N);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const float abar = ex2(dl * a2[i]);
@@ -246,14 +245,17 @@ sscan_backward_kernel(const BwdParams P) {
         // reverse over the chunk's tokens
 #pragma unroll
         for (int k = KC - 1; k >= 0; --k) {
+            // the token's inputs are loaded unconditionally (past the sequence's end: its last
+            // token, unused), so the loads need not wait behind the previous token's work
+            const int64_t t = t0 + (k < nt ? k : nt - 1);
+            float sg;
+            const float dl = step(t, sg);
+            const float x = Io<IO>::widen(Io<IO>::ld(u + t * D));
+            float dyt = valid ? Io<IO>::widen(Io<IO>::ld(dyp + t * D)) : 0.0f;  // idle lanes add nothing
+            const float4 Bv = bwd_ld4<IO>(Bp + t * N);
+            const float4 Cv = bwd_ld4<IO>(Cp + t * N);
+            const float zraw = (FUSED && zp != nullptr) ? Io<IO>::widen(Io<IO>::ld(zp + t * D)) : 0.0f;
             if (k < nt) {
-                const int64_t t = t0 + k;
-                float sg;
-                const float dl = step(t, sg);
-                const float x = Io<IO>::widen(Io<IO>::ld(u + t * D));
-                float dyt = valid ? Io<IO>::widen(Io<IO>::ld(dyp + t * D)) : 0.0f;  // idle lanes add nothing
-                const float4 Bv = bwd_ld4<IO>(Bp + t * N);
-                const float4 Cv = bwd_ld4<IO>(Cp + t * N);
                 float dzt = 0.0f;
                 if (FUSED && zp != nullptr) {
                     // the gate: the scan's own output ys = C . h_t, summed over the channel's lanes
@@ -262,7 +264,7 @@ sscan_backward_kernel(const BwdParams P) {
                     for (int i = 0; i < 4; ++i) ys = fmaf(f4_at(Cv, i), hk[k][i], ys);
 #pragma unroll
                     for (int o = 1; o < LPC; o <<= 1) ys += __shfl_xor_sync(0xffffffffu, ys, o);
-                    const float zt = Io<IO>::widen(Io<IO>::ld(zp + t * D));
+                    const float zt = zraw;
                     const float sz = 1.0f / (1.0f + ex2(-zt * 1.4426950408889634f));
                     dzt = dyt * ys * sz * fmaf(zt, 1.0f - sz, 1.0f);
                     dyt *= zt * sz;

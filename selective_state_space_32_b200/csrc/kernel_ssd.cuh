@@ -68,14 +68,14 @@ constexpr uint32_t kColS = 0, kColY1 = 256, kColY2 = 320, kColSblk = 384;  // S 
 constexpr int kBox = kQ * 128;                 // one TMA box: 128 rows x 128 bytes
 constexpr int kStage = 5 * kBox;               // C (2 boxes), B (2 boxes), X
 constexpr int kOffStage = 0;                   // 2 stages
-constexpr int kOffWX = 2 * kStage;             // w X, [token s][head dim p], 2 buffers (block parity)
-constexpr int kOffH = kOffWX + 2 * kBox;       // h_in as bf16, [state n][head dim p], 2 buffers
+constexpr int kOffWX = 2 * kStage;             // w X, [token s][head dim p]
+constexpr int kOffH = kOffWX + kBox;           // h_in as bf16, [state n][head dim p], 2 buffers
 constexpr int kOffCs = kOffH + 2 * kBox;       // warpgroup P: float cs2[128] (cumulative delta*A*log2 e)
 constexpr int kOffDt = kOffCs + 512;           //              float delta[128]
 constexpr int kOffColf = kOffDt + 512;         //              float column factors[128]
 constexpr int kOffWarp = kOffColf + 512;       // float scan totals [2 warpgroups][4 warps]
 constexpr int kOffBars = kOffWarp + 64;        // mbarriers
-constexpr int kNumBars = 15;
+constexpr int kNumBars = 13;
 constexpr int kOffTmem = kOffBars + 8 * kNumBars;
 constexpr int kOffAbort = kOffTmem + 4;
 constexpr int kSmemUsed = kOffAbort + 4;
@@ -88,18 +88,14 @@ enum {
     BAR_FULL = 0,      // [2] TMA of a stage landed                      (count 1 + bytes)
     BAR_SDONE = 2,     // [2] MMA 1 of the stage's block done             (commit)
     BAR_PREADY = 4,    // [2] P of the stage's block in TMEM              (warpgroup P)
-    BAR_WXREADY = 6,   // [2] w X of a block written into buffer (block parity)   (warpgroup Y)
-    BAR_HREADY = 8,    // [2] h_in of a block written into buffer (block parity)  (warpgroup Y)
-    BAR_M4 = 10,       // MMA 4 of the block done: S_blk ready, its w X buffer free (commit)
-    BAR_SBLKFREE = 11, // S_blk of the block read                         (warpgroup Y)
-    BAR_YREADY = 12,   // MMAs 2 and 3 of the block done (and everything before them)
-    BAR_YFREE = 13,    // P X and C h_in of the block read                (warpgroup Y)
-    BAR_DRAIN = 14,    // every MMA of the CTA done (before the tensor memory is released)
+    BAR_WXREADY = 6,   // w X of the block written                        (warpgroup Y)
+    BAR_M4 = 7,        // MMA 4 of the block done: S_blk ready, w X free  (commit)
+    BAR_SBLKFREE = 8,  // S_blk of the block read                         (warpgroup Y)
+    BAR_HREADY = 9,    // h_in of the next block written                  (warpgroup Y)
+    BAR_YREADY = 10,   // MMAs 2 and 3 of the block done (and everything before them)
+    BAR_YFREE = 11,    // P X and C h_in of the block read                (warpgroup Y)
+    BAR_DRAIN = 12,    // every MMA of the CTA done (before the tensor memory is released)
 };
-// A barrier that completes once per block is waited for with the block's parity; one
-// per buffer or stage (two blocks use it alternately) with parity (block >> 1) & 1.
-// Every wait below was checked to be ordered before the barrier's next-but-one
-// phase can complete (a parity wait two phases behind would never return).
 
 struct Params {
     const float *dt;       // [B][L][H] step delta (after softplus)
@@ -292,11 +288,11 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
             mbar_init(&bars[BAR_FULL + i], 1);
             mbar_init(&bars[BAR_SDONE + i], 1);
             mbar_init(&bars[BAR_PREADY + i], kWG);
-            mbar_init(&bars[BAR_WXREADY + i], kWG);
-            mbar_init(&bars[BAR_HREADY + i], kWG);
         }
+        mbar_init(&bars[BAR_WXREADY], kWG);
         mbar_init(&bars[BAR_M4], 1);
         mbar_init(&bars[BAR_SBLKFREE], kWG);
+        mbar_init(&bars[BAR_HREADY], kWG);
         mbar_init(&bars[BAR_YREADY], 1);
         mbar_init(&bars[BAR_YFREE], kWG);
         mbar_init(&bars[BAR_DRAIN], 1);
@@ -312,37 +308,29 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
     const float a2 = __ldg(prm.A + h) * 1.4426950408889634f;  // A_h log2(e): decays as powers of 2
 
     if (warp == 8) {
-        constexpr uint32_t id_s = idesc_bf16(kQ, kQ, 0, 0);    // C (K-major) x B^T (K-major)
-        constexpr uint32_t id_y = idesc_bf16(kQ, kP, 0, 1);    // P or C (K-major) x X or h (MN-major)
-        constexpr uint32_t id_st = idesc_bf16(kN, kP, 1, 1);   // B^T (MN-major) x wX (MN-major)
-        auto wait = [&](int bar, uint32_t parity) {
-            return wait_or_abort(&bars[bar], parity, abort_flag, prm.status, 16);
-        };
-        auto load = [&](int c) {  // block c into stage c & 1
-            const uint32_t st = sbase + kOffStage + (c & 1) * kStage;
-            uint64_t *bar = &bars[BAR_FULL + (c & 1)];
-            const int t0 = c * kQ;
-            mbar_expect_tx(bar, kLoadBytes);
-            tma_load_3d(st + kOffC, &tm_c, 0, t0, b, bar);
-            tma_load_3d(st + kOffC + kBox, &tm_c, 64, t0, b, bar);
-            tma_load_3d(st + kOffB, &tm_b, 0, t0, b, bar);
-            tma_load_3d(st + kOffB + kBox, &tm_b, 64, t0, b, bar);
-            tma_load_4d(st + kOffX, &tm_x, 0, h, t0, b, bar);
-        };
-        if (lane == 1) {
-            // ------------------------------------------------ TMA producer
-            // Block c goes into the stage block c-2 used, once every MMA of c-2 is done.
+        if (lane == 0) {
+            // ------------------------------------------------ TMA and MMA issue
             tma_prefetch_desc(&tm_x);
             tma_prefetch_desc(&tm_b);
             tma_prefetch_desc(&tm_c);
-            load(0);
-            if (nb > 1) load(1);
-            for (int c = 2; c < nb; ++c) {
-                if (!wait(BAR_YREADY, (c - 2) & 1)) break;
-                load(c);
-            }
-        } else if (lane == 0) {
-            // ------------------------------------------------ MMA issue
+            constexpr uint32_t id_s = idesc_bf16(kQ, kQ, 0, 0);    // C (K-major) x B^T (K-major)
+            constexpr uint32_t id_y = idesc_bf16(kQ, kP, 0, 1);    // P or C (K-major) x X or h (MN-major)
+            constexpr uint32_t id_st = idesc_bf16(kN, kP, 1, 1);   // B^T (MN-major) x wX (MN-major)
+            const uint32_t sWX = sbase + kOffWX;
+            auto load = [&](int c) {  // block c into stage c & 1
+                const uint32_t st = sbase + kOffStage + (c & 1) * kStage;
+                uint64_t *bar = &bars[BAR_FULL + (c & 1)];
+                const int t0 = c * kQ;
+                mbar_expect_tx(bar, kLoadBytes);
+                tma_load_3d(st + kOffC, &tm_c, 0, t0, b, bar);
+                tma_load_3d(st + kOffC + kBox, &tm_c, 64, t0, b, bar);
+                tma_load_3d(st + kOffB, &tm_b, 0, t0, b, bar);
+                tma_load_3d(st + kOffB + kBox, &tm_b, 64, t0, b, bar);
+                tma_load_4d(st + kOffX, &tm_x, 0, h, t0, b, bar);
+            };
+            auto wait = [&](int bar, uint32_t parity) {
+                return wait_or_abort(&bars[bar], parity, abort_flag, prm.status, 16);
+            };
             bool issued = false;
             auto mma1 = [&](int c) {  // S of block c = C B^T, K = N in 8 steps of 16 states
                 const uint32_t st = sbase + kOffStage + (c & 1) * kStage;
@@ -356,11 +344,11 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                 mma_commit(&bars[BAR_SDONE + (c & 1)]);
                 issued = true;
             };
-            // Issue order per block c: MMA 4(c), MMA 1(c+1), MMAs 2-3(c).  MMA 4 waits only
-            // for w X of block c (prepared a block ahead) and for S_blk of block c-1 to be
-            // read; MMA 1 of block c+1 goes ahead of MMAs 2-3 of block c so that P of block
-            // c+1 is formed while they run; its S buffer last held block c-1's P, read by
-            // MMA 2 of c-1: done once BAR_YREADY of c-1 is seen.
+            // Issue order: MMA 1 of block c+1 goes ahead of MMAs 2 and 3 of block c, so that
+            // warpgroup P forms P of block c+1 while they run.  The S buffer of block c+1 last
+            // held block c-1's P, read by its MMA 2: done once BAR_YREADY of c-1 was seen.
+            load(0);
+            if (nb > 1) load(1);
             bool run = wait(BAR_FULL, 0);
             if (run) {
                 tc_fence_after();
@@ -368,15 +356,18 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
             }
             for (int c = 0; run && c < nb; ++c) {
                 const int s = c & 1;
-                const uint32_t ps = (c >> 1) & 1, pp = (c - 1) & 1;
+                const uint32_t ps = (c >> 1) & 1, pc = c & 1, pp = (c - 1) & 1;
                 const uint32_t st = sbase + kOffStage + s * kStage;
                 const uint32_t sC = st + kOffC, sB = st + kOffB, sX = st + kOffX;
-                const uint32_t sH = sbase + kOffH + s * kBox;    // h_in of this block
-                const uint32_t sWX = sbase + kOffWX + s * kBox;  // w X of this block
+                const uint32_t sH = sbase + kOffH + s * kBox;  // h_in of this block
                 const uint32_t tS = tbase + kColS + 128 * s;
-                // MMA 4: S_blk = B^T (w X), M = N (two 64-state chunks kBox apart), K = Q
-                if (!wait(BAR_WXREADY + s, ps)) break;
+                // MMA 4: S_blk = B^T (w X), M = N (two 64-state chunks kBox apart), K = Q.
+                // h_in of this block is waited for here, before MMA 4: warpgroup Y arrives
+                // for the next block's h_in as soon as MMA 4 is done, and a phase-parity
+                // wait must never fall two phases behind its barrier.
+                if (!wait(BAR_WXREADY, pc)) break;
                 if (c > 0 && !wait(BAR_SBLKFREE, pp)) break;
+                if (!wait(BAR_HREADY, pc)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
@@ -385,14 +376,12 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                 mma_commit(&bars[BAR_M4]);
                 // MMA 1 of the next block
                 if (c + 1 < nb) {
-                    if (c >= 1 && !wait(BAR_YREADY, pp)) break;
                     if (!wait(BAR_FULL + (s ^ 1), ((c + 1) >> 1) & 1)) break;
                     tc_fence_after();
                     mma1(c + 1);
                 }
                 // MMA 2: Y1 = P X (P: TMEM columns 8k.. of packed pairs), MMA 3: Y2 = C h_in
                 if (!wait(BAR_PREADY + s, ps)) break;
-                if (!wait(BAR_HREADY + s, ps)) break;
                 if (c > 0 && !wait(BAR_YFREE, pp)) break;
                 tc_fence_after();
 #pragma unroll
@@ -405,6 +394,11 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                            id_y, k > 0);
                 }
                 mma_commit(&bars[BAR_YREADY]);
+                // block c+2 goes into this stage once every MMA of block c is done
+                if (c + 2 < nb) {
+                    if (!wait(BAR_YREADY, pc)) break;
+                    load(c + 2);
+                }
             }
             // the tensor memory is released below: every MMA issued must be done first.  A
             // commit tracks all earlier MMAs of this thread: one more on its own barrier,
@@ -525,25 +519,6 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                 }
                 fence_proxy_async_smem();  // generic writes -> the MMA's operand reads
             };
-            // w X of block c into buffer c & 1 (free once MMA 4 of block c-2 is done)
-            auto make_wx = [&](int c, float dt, float cs, float tot) {
-                ok = wait_warp(BAR_FULL + (c & 1), (c >> 1) & 1);  // X of block c landed
-                if (!ok) return;
-                const float wv = dt * ex2(tot - cs);  // w_s of the block end state, s = t
-                const unsigned char *xr = sm + kOffStage + (c & 1) * kStage + kOffX;
-                unsigned char *wr = sm + kOffWX + (c & 1) * kBox;
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    uint4 v4 = *reinterpret_cast<const uint4 *>(xr + sw128(t, q));
-                    v4.x = pack_bf16(bf16_lo(v4.x) * wv, bf16_hi(v4.x) * wv);
-                    v4.y = pack_bf16(bf16_lo(v4.y) * wv, bf16_hi(v4.y) * wv);
-                    v4.z = pack_bf16(bf16_lo(v4.z) * wv, bf16_hi(v4.z) * wv);
-                    v4.w = pack_bf16(bf16_lo(v4.w) * wv, bf16_hi(v4.w) * wv);
-                    *reinterpret_cast<uint4 *>(wr + sw128(t, q)) = v4;
-                }
-                fence_proxy_async_smem();
-                mbar_arrive(&bars[BAR_WXREADY + (c & 1)]);
-            };
             write_h(0);
             mbar_arrive(&bars[BAR_HREADY]);
             // y of block c: P X + 2^cs (C h_in), rows inside the sequence only
@@ -574,34 +549,44 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                                            o[q >> 2][4 * (q & 3) + 2], o[q >> 2][4 * (q & 3) + 3]);
                 }
             };
-            // Per block c: w X of block c+1 (so MMA 4 of block c+1 waits for nothing but
-            // S_blk of block c being read), y of block c-1 (while MMA 4 of block c runs), then
-            // the state passing of block c and h_in of block c+1.
-            float tot_c;
-            float cs_c = wg_scan(dt_next * a2, wl, lane, tot4, bar_id, tot_c);  // block 0
-            {
-                const float dt0 = dt_next;
-                dt_next = int64_t(kQ) + t < L ? __ldg(dtp + (int64_t(kQ) + t) * prm.H) : 0.0f;
-                make_wx(0, dt0, cs_c, tot_c);
-            }
+            // Per block c: w X of block c first (MMA 4 of block c can start at once),
+            // then y of block c-1 (while MMA 4 runs), then the state passing of block c.
             float cs_prev = 0.0f;
             for (int c = 0; c < nb; ++c) {
-                float cs_n = 0.0f, tot_n = 0.0f;
-                if (c + 1 < nb) {
-                    const float dt = dt_next;
-                    const int64_t nxt = int64_t(c + 2) * kQ + t;
-                    dt_next = nxt < L ? __ldg(dtp + nxt * prm.H) : 0.0f;
-                    cs_n = wg_scan(dt * a2, wl, lane, tot4, bar_id, tot_n);
-                    // buffer (c+1) & 1 was read by MMA 4 of block c-1: waited for in block c-1
-                    make_wx(c + 1, dt, cs_n, tot_n);
+                const int s = c & 1;
+                const uint32_t ps = (c >> 1) & 1, pc = c & 1;
+                const float dt = dt_next;
+                const int64_t nxt = int64_t(c + 1) * kQ + t;
+                dt_next = nxt < L ? __ldg(dtp + nxt * prm.H) : 0.0f;
+                float tot;
+                const float cs = wg_scan(dt * a2, wl, lane, tot4, bar_id, tot);
+                // ---- w X for MMA 4: X of this block landed; w X's buffer was freed by MMA 4
+                // of block c-1 (waited for in the state step of the previous block)
+                ok = wait_warp(BAR_FULL + s, ps);
+                if (ok) {
+                    const float wv = dt * ex2(tot - cs);  // w_s of the block end state, s = t
+                    const unsigned char *xr = sm + kOffStage + s * kStage + kOffX;
+                    unsigned char *wr = sm + kOffWX;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        uint4 v4 = *reinterpret_cast<const uint4 *>(xr + sw128(t, q));
+                        v4.x = pack_bf16(bf16_lo(v4.x) * wv, bf16_hi(v4.x) * wv);
+                        v4.y = pack_bf16(bf16_lo(v4.y) * wv, bf16_hi(v4.y) * wv);
+                        v4.z = pack_bf16(bf16_lo(v4.z) * wv, bf16_hi(v4.z) * wv);
+                        v4.w = pack_bf16(bf16_lo(v4.w) * wv, bf16_hi(v4.w) * wv);
+                        *reinterpret_cast<uint4 *>(wr + sw128(t, q)) = v4;
+                    }
+                    fence_proxy_async_smem();
+                    mbar_arrive(&bars[BAR_WXREADY]);
                 }
                 if (c > 0) emit_y(c - 1, cs_prev);
-                // ---- state passing: h = 2^cs_end h + S_blk (row n = t); then h_in of block
-                // c+1, into the buffer MMA 3 of block c-1 read (done: its y was just emitted)
-                ok = wait_warp(BAR_M4, c & 1);
+                cs_prev = cs;
+                // ---- state passing: h = 2^cs_end h + S_blk (row n = t); then h_in of block c+1,
+                // into the buffer MMA 3 of block c-1 read (done: its y was just emitted)
+                ok = wait_warp(BAR_M4, pc);
                 if (ok) {
                     tc_fence_after();
-                    const float aend = ex2(tot_c);
+                    const float aend = ex2(tot);
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
                         uint32_t sb[32];
@@ -613,11 +598,8 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                     tc_fence_before();
                     mbar_arrive(&bars[BAR_SBLKFREE]);
                     write_h((c + 1) & 1);
-                    mbar_arrive(&bars[BAR_HREADY + ((c + 1) & 1)]);
+                    mbar_arrive(&bars[BAR_HREADY]);
                 }
-                cs_prev = cs_c;
-                cs_c = cs_n;
-                tot_c = tot_n;
             }
             if (nb > 0) emit_y(nb - 1, cs_prev);
             if (ok && prm.h_final) {
