@@ -339,7 +339,7 @@ def run_ours(args, rank, world, local_rank):
                          "sample": sample},
     }
     if args.per_config:
-        others = [n for n in W.ORDER[1:] if n != args.workload]
+        others = [n for n in W.ORDER[1:] + ["decode_b256_f32"] if n != args.workload]
         out["per_config"] = time_other_configs(others, dev, stream, sm_max, hbm_peak)
         for name, sw in W.SSD_WORKLOADS.items():
             if name == "ssd_small":

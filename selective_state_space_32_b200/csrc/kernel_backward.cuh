@@ -24,6 +24,10 @@
 // takes the chunks last to first, recomputes each chunk's states from its
 // checkpoint into registers and runs the reverse recurrence over them.
 //
+// Occupancy: three blocks per SM (registers capped at 170 per thread; with
+// 8-token chunks nothing spills), so the 384 blocks of a 8 x 1536-channel layer
+// run in one wave.
+//
 // Mapping: each lane holds four states of one channel (LPC = N/4 adjacent lanes
 // per channel, CPW = 32/LPC channels per warp), so du, ddelta and the gate's
 // ys are summed over LPC lanes (log2 LPC shuffles) and dA needs none; a block
@@ -40,7 +44,7 @@ namespace sscan {
 
 constexpr int kBwdWarps = 4;
 constexpr int kBwdThreads = 32 * kBwdWarps;
-constexpr int kChunk = 16;  // tokens per recomputed chunk
+constexpr int kChunk = 8;   // tokens per recomputed chunk
 
 // channels a backward block covers
 __host__ __device__ constexpr int bwd_block_channels(int N) { return kBwdWarps * (32 / (N / 4)); }
@@ -96,7 +100,7 @@ __device__ __forceinline__ int channel_scatter4(float (&v)[4], int lane, int &V)
 }
 
 template <class IO, int N, bool ZOH, bool FUSED>
-__global__ void __launch_bounds__(kBwdThreads)
+__global__ void __launch_bounds__(kBwdThreads, 3)
 sscan_backward_kernel(const BwdParams P) {
     constexpr int LPC = N / 4, CPW = 32 / LPC, CPB = kBwdWarps * CPW, KC = kChunk;
     __shared__ __align__(16) float s_db[kBwdWarps][KC][N], s_dc[kBwdWarps][KC][N];

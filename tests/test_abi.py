@@ -106,11 +106,11 @@ def test_gated_and_backward_reject_bad_arguments_without_a_device(lib):
 
 def test_backward_workspace_bytes(lib):
     # state checkpoints: B x channels padded to a block (4 warps x 32/(N/4) channels) x
-    # ceil(L/16) chunks x N states x 4 bytes, rounded up to 256 bytes
-    assert lib.sscan_backward_workspace_bytes(8, 2048, 1536, 16) == 8 * 1536 * 128 * 16 * 4
-    assert lib.sscan_backward_workspace_bytes(2, 37, 70, 16) == 2 * 96 * 3 * 16 * 4
-    assert lib.sscan_backward_workspace_bytes(2, 37, 70, 32) == 2 * 80 * 3 * 32 * 4
-    assert lib.sscan_backward_workspace_bytes(2, 37, 70, 64) == 2 * 72 * 3 * 64 * 4
+    # ceil(L/8) chunks x N states x 4 bytes, rounded up to 256 bytes
+    assert lib.sscan_backward_workspace_bytes(8, 2048, 1536, 16) == 8 * 1536 * 256 * 16 * 4
+    assert lib.sscan_backward_workspace_bytes(2, 37, 70, 16) == 2 * 96 * 5 * 16 * 4
+    assert lib.sscan_backward_workspace_bytes(2, 37, 70, 32) == 2 * 80 * 5 * 32 * 4
+    assert lib.sscan_backward_workspace_bytes(2, 37, 70, 64) == 2 * 72 * 5 * 64 * 4
     assert lib.sscan_backward_workspace_bytes(2, 37, 70, 24) == 0
     assert lib.sscan_backward_workspace_bytes(2, 0, 70, 16) == 0
 

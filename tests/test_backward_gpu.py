@@ -4,7 +4,7 @@ The oracle's backward, plain and fused, is pinned by finite differences of the
 forward oracle (tests/test_oracle_backward.py).  Cases cover N = 16, 32 and 64,
 Euler and ZOH (with some A = 0, the limit branch), fp32 and bf16 I/O, ragged
 channel counts (D not a multiple of a block's channels) and ragged sequences
-(L not a multiple of the 16-token recompute chunk), with and without h0 and
+(L not a multiple of the 8-token recompute chunk), with and without h0 and
 dh_final, and the fused layer (softplus(delta + bias) and the silu(z) gate:
 gradients of the raw delta, the bias and z).  Tolerances are those of the
 forward: fp32 relative L2 <= 1e-5 and |err| <= 1e-4 (1 + |ref|) elementwise on
