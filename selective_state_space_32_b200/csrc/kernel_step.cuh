@@ -35,29 +35,28 @@ template <> __device__ __forceinline__ float4 ld4<uint16_t>(const uint16_t *p) {
                        __uint_as_float(v.y & 0xffff0000u));
 }
 
-// Thread (channel slot k of ITEMS, lane group g): states 4g .. 4g+3 of channel
-// ch = (blockIdx.x * ITEMS + k) * CPB + threadIdx.x / LPC over the B*D channels
-// (row-major [b][d]); LPC = N/4 adjacent lanes share a channel.
+// Batch row b = blockIdx.y; thread (channel slot k of ITEMS, lane group g): states
+// 4g .. 4g+3 of channel d = (blockIdx.x * ITEMS + k) * CPB + threadIdx.x / LPC;
+// LPC = N/4 adjacent lanes share a channel.  (A 2-D grid: no index division.)
 template <class IO, int N, bool ZOH>
 __global__ void __launch_bounds__(kStepThreads)
 sscan_step_kernel(const IO *__restrict__ u, const IO *__restrict__ delta, const float *__restrict__ A,
                   const IO *__restrict__ Bm, const IO *__restrict__ Cm, const float *h0, IO *__restrict__ y,
-                  float *h_final, int64_t L, int64_t D, int64_t channels, const float *__restrict__ delta_bias,
+                  float *h_final, int64_t L, int64_t D, const float *__restrict__ delta_bias,
                   const IO *__restrict__ z, int softplus) {
     constexpr int LPC = N / 4;
     constexpr int CPB = kStepThreads / LPC;  // channels per block slice
     const int g = threadIdx.x % LPC;
     const int n0 = 4 * g;
-    int64_t ch[kStepItems], b[kStepItems], d[kStepItems];
+    int64_t b[kStepItems], d[kStepItems];
     bool valid[kStepItems];
     f2 A2[kStepItems][2], A1[kStepItems][2], iA[kStepItems][2], h[kStepItems][2];
 #pragma unroll
     for (int k = 0; k < kStepItems; ++k) {
-        ch[k] = (static_cast<int64_t>(blockIdx.x) * kStepItems + k) * CPB + threadIdx.x / LPC;
-        valid[k] = ch[k] < channels;
-        const int64_t c = valid[k] ? ch[k] : channels - 1;  // ragged tail: read a real channel, store nothing
-        b[k] = c / D;
-        d[k] = c - b[k] * D;
+        const int64_t dd = (static_cast<int64_t>(blockIdx.x) * kStepItems + k) * CPB + threadIdx.x / LPC;
+        valid[k] = dd < D;
+        b[k] = blockIdx.y;
+        d[k] = valid[k] ? dd : D - 1;  // ragged tail: read a real channel, store nothing
     }
     // every independent load first: A rows, states, then the per-token inputs
 #pragma unroll

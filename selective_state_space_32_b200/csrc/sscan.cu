@@ -297,12 +297,11 @@ template <class IO, int N>
 cudaError_t launch_step_t(const sscan_plan *p, const void *u, const void *dl, const float *A, const void *Bm,
                           const void *Cm, const float *h0, void *y, float *hf, const Fused &fu, cudaStream_t s) {
     constexpr int per_block = kStepThreads / (N / 4) * kStepItems;  // channels per block
-    const int64_t channels = p->B * p->D;
-    const dim3 grid(static_cast<unsigned>(ceil_div(channels, per_block)));
+    const dim3 grid(static_cast<unsigned>(ceil_div(p->D, per_block)), static_cast<unsigned>(p->B));
     auto kern = (p->flags & SSCAN_ZOH) ? sscan_step_kernel<IO, N, true> : sscan_step_kernel<IO, N, false>;
     kern<<<grid, kStepThreads, 0, s>>>(static_cast<const IO *>(u), static_cast<const IO *>(dl), A,
                                        static_cast<const IO *>(Bm), static_cast<const IO *>(Cm), h0,
-                                       static_cast<IO *>(y), hf, p->L, p->D, channels, fu.bias,
+                                       static_cast<IO *>(y), hf, p->L, p->D, fu.bias,
                                        static_cast<const IO *>(fu.z), fu.softplus ? 1 : 0);
     return cudaGetLastError();
 }
