@@ -282,7 +282,7 @@ def run_ours(args, rank, world, local_rank):
     def e2e_step():
         S.forward_host(hin["u"], hin["delta"], hin["A"], hin["B"], hin["C"], hin["h0"],
                        zoh=w.zoh, device=dev, out=out_h, delta_bias=hin["delta_bias"],
-                       delta_softplus=w.fused, z=hin["z"])
+                       delta_softplus=w.fused, z=hin["z"], stream=stream)
 
     for _ in range(min(args.warmup, 3)):
         e2e_step()

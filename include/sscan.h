@@ -140,6 +140,39 @@ SSCAN_API int sscan_forward_gated(sscan_plan_t plan, const void *u, const void *
                         const void *B, const void *C, const float *h0, const float *delta_bias,
                         const void *z, void *y, float *h_final, void *workspace, void *stream);
 
+/* Bytes of device workspace sscan_forward_host needs for this plan (always
+ * > 0; 0 only when plan is NULL or host memory ran out).  The workspace must
+ * be 256-byte aligned.  It holds two buffer slots of one piece's inputs and
+ * output (the slot for z is reserved whether or not a call passes z), A, the
+ * bias, the carried state and the pieces' scan workspaces. */
+SSCAN_API size_t sscan_host_workspace_bytes(sscan_plan_t plan);
+
+/* sscan_forward_gated on HOST buffers: the arguments and their layouts are
+ * those of sscan_forward_gated, except that u, delta, A, B, C, h0,
+ * delta_bias, z, y and h_final live in host memory (page-locked memory lets
+ * the copies overlap; any memory cudaMemcpy accepts works), need no
+ * alignment, and `workspace` is device memory of
+ * sscan_host_workspace_bytes(plan) bytes.  The call cuts the sequence into
+ * at most 8 pieces along L (multiples of 64 tokens, the last one shorter)
+ * and, for each piece, copies its inputs to the device, scans it (the state
+ * carried between pieces in the workspace: a piece's h_final is the next
+ * piece's h0, exactly the split-call resume of sscan_forward) and copies its
+ * y back; with two buffer slots, the host-to-device copy of piece k+1 and the
+ * device-to-host copy of piece k-1 run while piece k is scanned.  The
+ * results equal one sscan_forward_gated call on the whole sequence.
+ * Streams: the work starts after what is already queued on `stream`, and
+ * `stream` waits for all of it (copies included) before anything queued
+ * later, so synchronising `stream` makes y and h_final readable; the call
+ * itself returns without synchronising.  The plan creates two internal
+ * streams and a few events on its first host call (freed with the plan).
+ * Ownership and errors as for sscan_forward_gated (the aliasing rules apply
+ * to the host buffers; a workspace that overlaps one gives
+ * SSCAN_ERR_WORKSPACE); device-side waits of the pieces are latched in the
+ * plan's status word (sscan_get_status). */
+SSCAN_API int sscan_forward_host(sscan_plan_t plan, const void *u, const void *delta, const float *A,
+                                 const void *B, const void *C, const float *h0, const float *delta_bias,
+                                 const void *z, void *y, float *h_final, void *workspace, void *stream);
+
 /* Backward pass of the forward: gradients of a loss given dy = dLoss/dy and
  * optionally dh_final = dLoss/dh_final, by the chain rule through
  * h_t = Abar_t h_{t-1} + beta_t u_t, y_t = C_t . h_t, the states recomputed

@@ -24,7 +24,8 @@ OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPAC
 SYMBOLS = ("sscan_plan_create", "sscan_plan_destroy", "sscan_workspace_bytes", "sscan_forward",
            "sscan_get_status", "sscan_status_string", "sscan_plan_describe", "sscan_version",
            "sscan_forward_noalloc", "sscan_noalloc_status", "sscan_forward_gated", "sscan_backward",
-           "sscan_backward_workspace_bytes", "sscan_ssd_forward", "sscan_backward_gated")
+           "sscan_backward_workspace_bytes", "sscan_ssd_forward", "sscan_backward_gated",
+           "sscan_host_workspace_bytes", "sscan_forward_host")
 
 
 class SscanError(RuntimeError):
@@ -78,6 +79,10 @@ def lib() -> ctypes.CDLL:
             L.sscan_ssd_forward.restype = ip
             L.sscan_backward_gated.argtypes = [i64, i64, i64, i64, ip, u32] + [vp] * 20
             L.sscan_backward_gated.restype = ip
+            L.sscan_host_workspace_bytes.argtypes = [vp]
+            L.sscan_host_workspace_bytes.restype = sz
+            L.sscan_forward_host.argtypes = [vp] * 13
+            L.sscan_forward_host.restype = ip
             _lib = L
     return _lib
 
@@ -181,6 +186,46 @@ class Plan:
             raise SscanError(rc, what)
         return y, h_final
 
+    def host_workspace_bytes(self) -> int:
+        n = int(lib().sscan_host_workspace_bytes(self._h))
+        if n == 0:
+            raise SscanError(ERR_INVALID, "sscan_host_workspace_bytes")
+        return n
+
+    def forward_host(self, u, delta, A, B, C, h0, y, h_final, delta_bias=None, z=None, stream=None,
+                     workspace=None):
+        """Enqueue ``sscan_forward_host`` on ``stream``: every tensor a contiguous CPU
+        tensor (pinned for overlapped copies), the device workspace allocated here
+        unless given.  Returns without waiting; synchronise ``stream`` before
+        reading y and h_final."""
+        Bt, L, D, N = self.shape
+        for name, t, shape, dt in (("u", u, (Bt, L, D), self.dtype),
+                                   ("delta", delta, (Bt, L, D), self.dtype),
+                                   ("A", A, (D, N), torch.float32),
+                                   ("B", B, (Bt, L, N), self.dtype),
+                                   ("C", C, (Bt, L, N), self.dtype),
+                                   ("h0", h0, (Bt, D, N), torch.float32),
+                                   ("y", y, (Bt, L, D), self.dtype),
+                                   ("h_final", h_final, (Bt, D, N), torch.float32),
+                                   ("delta_bias", delta_bias, (D,), torch.float32),
+                                   ("z", z, (Bt, L, D), self.dtype)):
+            if t is None:
+                continue
+            if tuple(t.shape) != shape or t.dtype != dt or t.is_cuda or not t.is_contiguous():
+                raise ValueError(f"{name}: want contiguous host {dt} {shape}, got "
+                                 f"{t.dtype} {tuple(t.shape)} on {t.device}")
+        if stream is None:
+            stream = torch.cuda.current_stream()
+        if workspace is None:
+            workspace = torch.empty(self.host_workspace_bytes(), dtype=torch.uint8, device=stream.device)
+        rc = lib().sscan_forward_host(self._h, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(h0),
+                                      _ptr(delta_bias), _ptr(z), _ptr(y), _ptr(h_final), _ptr(workspace),
+                                      ctypes.c_void_p(stream.cuda_stream))
+        if rc != OK:
+            raise SscanError(rc, "sscan_forward_host")
+        workspace.record_stream(stream)
+        return y, h_final
+
     def backward(self, u, delta, A, B, C, h0, dy, dh_final=None, want_dh0: bool = True, stream=None,
                  delta_bias=None, z=None) -> dict:
         """Gradients of this plan's forward: returns a dict with du, ddelta (plan dtype), dA,
@@ -246,48 +291,26 @@ def forward(u, delta, A, B, C, h0=None, zoh: bool = False, want_final: bool = Tr
 
 
 def forward_host(u, delta, A, B, C, h0=None, zoh: bool = False, device="cuda", out=None,
-                 chunks: int = 2, delta_bias=None, delta_softplus: bool = False, z=None):
-    """Forward on host (CPU) tensors: copies the inputs to the device, runs the scan
-    and copies y and h_final back, then waits for the copies.
-
-    Batch rows are independent, so the batch is cut into ``chunks`` pieces that
-    flow through two streams: a piece's host-to-device copy overlaps the previous
-    piece's scan and device-to-host copy (the transfer, not the scan, bounds this
-    path).  Pinned host tensors are needed for the copies to be asynchronous;
-    ``out`` = (y_host, h_final_host) reuses output buffers; delta_bias, delta_softplus
-    and z select the fused prologue / epilogue (z is cut like u).
-    Returns (y_host, h_final_host)."""
+                 delta_bias=None, delta_softplus: bool = False, z=None, stream=None):
+    """Forward on host (CPU) tensors through ``sscan_forward_host``: the library
+    copies the inputs to the device piece by piece, scans, and copies y and
+    h_final back, the copies of neighbouring pieces overlapping the scan.
+    Page-locked (pinned) host tensors let the copies run asynchronously;
+    ``out`` = (y_host, h_final_host) reuses output buffers; delta_bias,
+    delta_softplus and z select the fused prologue / epilogue.  Waits for the
+    stream before returning.  Returns (y_host, h_final_host)."""
     dev = torch.device(device)
     Bt, L, D = u.shape
     N = A.shape[1]
+    plan = get_plan(Bt, L, D, N, u.dtype, zoh, delta_softplus)
     if out is None:
         pin = u.is_pinned()
         out = (torch.empty((Bt, L, D), dtype=u.dtype, pin_memory=pin),
                torch.empty((Bt, D, N), dtype=torch.float32, pin_memory=pin))
-    n = max(1, min(int(chunks), Bt))
-    bounds = [Bt * i // n for i in range(n + 1)]
-    main = torch.cuda.current_stream(dev)
-    streams = [torch.cuda.Stream(dev) for _ in range(min(2, n))]
-    A_d = A.to(dev, non_blocking=True)
-    bias_d = None if delta_bias is None else delta_bias.to(dev, non_blocking=True)
-    for st in streams:
-        st.wait_stream(main)
-    for i in range(n):
-        b0, b1 = bounds[i], bounds[i + 1]
-        st = streams[i % len(streams)]
-        with torch.cuda.stream(st):
-            dv = [None if t is None else t[b0:b1].to(dev, non_blocking=True)
-                  for t in (u, delta, B, C, h0, z)]
-            plan = get_plan(b1 - b0, L, D, N, u.dtype, zoh, delta_softplus)
-            y, hf = plan.forward(dv[0], dv[1], A_d, dv[2], dv[3], dv[4], stream=st,
-                                 delta_bias=bias_d, z=dv[5])
-            out[0][b0:b1].copy_(y, non_blocking=True)
-            out[1][b0:b1].copy_(hf, non_blocking=True)
-            for t in (*dv, y, hf, bias_d):  # keep the caching allocator from reusing them early
-                if t is not None:
-                    t.record_stream(st)
-    for st in streams:
-        st.synchronize()
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    plan.forward_host(u, delta, A, B, C, h0, out[0], out[1], delta_bias=delta_bias, z=z, stream=stream)
+    stream.synchronize()
     return out
 
 

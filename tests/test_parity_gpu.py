@@ -5,6 +5,8 @@ the full-size workloads run the exact launch the benchmark times and compare a
 seeded sample of (b, d) rows, each recomputed by the oracle row by row (rows
 are independent, so a sampled row is an exact reference).
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -208,19 +210,91 @@ def test_split_call_resume_matches_one_call():
     assert torch.allclose(torch.cat([y1, y2], 1), y, rtol=1e-5, atol=1e-6)
 
 
-def test_forward_host_chunked_matches_device_path():
-    g = W.generate(6, 300, 256, 16, "bf16", 0.1, seed=9)
-    d = P.to_device(g)
-    y_dev, hf_dev = S.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"])
-    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in d.items()}
-    for chunks in (1, 4):
-        y_h, hf_h = S.forward_host(host["u"], host["delta"], host["A"], host["B"], host["C"],
-                                   host["h0"], chunks=chunks)
-        assert y_h.dtype == torch.bfloat16 and not y_h.is_cuda
-        yr, hr = P.run_oracle(g)
-        P.check(y_h.float().numpy(), yr, "bf16", f"y host chunks={chunks}")
-        P.check(hf_h.numpy(), hr, "bf16", f"h_final host chunks={chunks}")
-        assert torch.allclose(hf_h, hf_dev.cpu(), rtol=1e-5, atol=1e-6)
+HOST = [
+    # (B, L, D, N, dtype, h0, zoh, fused): sscan_forward_host, pieces of ceil(L/8) rounded up to 64 tokens
+    (6, 300, 256, 16, "bf16", True, False, False),   # 5 pieces of 64 + a last piece of 44
+    (3, 1000, 96, 32, "f32", True, True, False),     # 8 pieces of 128, the last one 104
+    (2, 2048, 64, 16, "f32", False, False, True),    # 8 equal pieces; softplus(delta + bias), silu(z) gate
+    (4, 700, 40, 64, "bf16", True, True, True),
+    (5, 1, 300, 16, "f32", True, False, False),      # one token: a single piece
+    (2, 50, 33, 16, "f32", False, True, False),      # shorter than one piece alignment: one piece
+]
+
+
+@pytest.mark.parametrize("case", HOST, ids=[f"B{c[0]}L{c[1]}D{c[2]}N{c[3]}{c[4]}{'_h0' if c[5] else ''}"
+                                             f"{'_zoh' if c[6] else ''}{'_fused' if c[7] else ''}" for c in HOST])
+def test_forward_host_matches_oracle(case):
+    """The host-buffer entry point (pinned host inputs and outputs, pieces along L with
+    the state carried on the device) against the oracle, every element."""
+    Bt, L, D, N, dt, with_h0, zoh, fused = case
+    g = W.generate(Bt, L, D, N, dt, 0.1 if with_h0 else 0.0, seed=9000 + L + D + N, A_jitter=0.3,
+                   fused=fused)
+    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in P.to_device(g).items()}
+    y_h, hf_h = S.forward_host(host["u"], host["delta"], host["A"], host["B"], host["C"], host["h0"],
+                               zoh=zoh, delta_bias=host["delta_bias"], delta_softplus=fused, z=host["z"])
+    assert not y_h.is_cuda and y_h.dtype == host["u"].dtype
+    yr, hr = P.run_oracle(g, zoh, softplus=fused)
+    P.check(y_h.float().numpy(), yr, dt, "y host")
+    P.check(hf_h.numpy(), hr, dt, "h_final host")
+    plan = S.get_plan(Bt, L, D, N, host["u"].dtype, zoh, fused)
+    assert plan.status() == S.OK
+
+
+def test_forward_host_empty_and_no_final():
+    """L = 0 returns h0 (or zeros) as h_final; h_final may be skipped; the same plan
+    runs again with other buffers and gives the same result."""
+    Bt, D, N = 3, 48, 16
+    h0 = torch.randn(Bt, D, N).pin_memory()
+    plan = S.Plan(Bt, 0, D, N, torch.float32)
+    A = -torch.rand(D, N).pin_memory()
+    e = torch.empty(Bt, 0, D).pin_memory()
+    en = torch.empty(Bt, 0, N).pin_memory()
+    hf = torch.full((Bt, D, N), 7.0).pin_memory()
+    plan.forward_host(e, e, A, en, en, h0, e, hf)
+    torch.cuda.current_stream().synchronize()
+    assert torch.equal(hf, h0)
+    plan.forward_host(e, e, A, en, en, None, e, hf)
+    torch.cuda.current_stream().synchronize()
+    assert float(hf.abs().max()) == 0.0
+    plan.close()
+    g = W.generate(2, 333, 64, 16, "f32", 0.1, seed=21)
+    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in P.to_device(g).items()}
+    plan = S.Plan(2, 333, 64, 16, torch.float32)
+    y1 = torch.empty(2, 333, 64).pin_memory()
+    y2 = torch.empty(2, 333, 64).pin_memory()
+    plan.forward_host(host["u"], host["delta"], host["A"], host["B"], host["C"], host["h0"], y1, None)
+    plan.forward_host(host["u"], host["delta"], host["A"], host["B"], host["C"], host["h0"], y2, None)
+    torch.cuda.current_stream().synchronize()
+    yr, _ = P.run_oracle(g)
+    P.check(y1.numpy(), yr, "f32", "y host, no h_final")
+    assert torch.equal(y1, y2)
+    plan.close()
+
+
+def test_forward_host_argument_errors():
+    """Checks made before anything is queued: every buffer is real and of the stated size."""
+    Bt, L, D, N = 2, 100, 32, 16
+    lib = S.lib()
+    plan = S.Plan(Bt, L, D, N, torch.float32)
+    n = int(lib.sscan_host_workspace_bytes(plan._h))
+    assert n > 0
+    ws = torch.empty(n + 512, dtype=torch.uint8, device="cuda")
+    bld = [torch.zeros(Bt, L, D).pin_memory() for _ in range(3)]
+    bln = [torch.zeros(Bt, L, N).pin_memory() for _ in range(2)]
+    A = torch.zeros(D, N).pin_memory()
+    hf = torch.zeros(Bt, D, N).pin_memory()
+    S_ = torch.cuda.current_stream().cuda_stream
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    args = lambda u, y, w: [plan._h, p(u), p(bld[1]), p(A), p(bln[0]), p(bln[1]), None, None, None, p(y), p(hf),
+                            w, ctypes.c_void_p(S_)]
+    assert lib.sscan_forward_host(*args(bld[0], bld[0], p(ws))) == S.ERR_INVALID        # y over u
+    assert lib.sscan_forward_host(*args(bld[0], bld[2], None)) == S.ERR_WORKSPACE         # no workspace
+    mis = ctypes.c_void_p(ws.data_ptr() + 16)
+    assert lib.sscan_forward_host(*args(bld[0], bld[2], mis)) == S.ERR_WORKSPACE          # not 256-aligned
+    a = args(bld[0], bld[2], p(ws))
+    a[3] = None
+    assert lib.sscan_forward_host(*a) == S.ERR_INVALID                                     # no A
+    plan.close()
 
 
 @pytest.mark.parametrize("dt,zoh", [("f32", False), ("bf16", True)])
