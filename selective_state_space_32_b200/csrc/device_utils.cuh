@@ -250,6 +250,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
         if (mbar_try_wait(bar, parity)) return true;
     return false;
 }
+// mbar_wait for a waiter that is expected to wait: each try suspends the thread
+// for up to kSleepHintNs (it resumes as soon as the phase completes) instead of
+// spinning through issue slots the other warps need.  Bounded by kSleepLimit tries.
+constexpr uint32_t kSleepHintNs = 20000;
+constexpr uint32_t kSleepLimit = 1u << 16;
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity) {
+    if (mbar_test_wait(bar, parity)) return true;
+    for (uint32_t i = 0; i < kSleepLimit; ++i) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity), "r"(kSleepHintNs)
+            : "memory");
+        if (ok) return true;
+    }
+    return false;
+}
 // 2-D tiled TMA load (no multicast) of box {x, y} into shared memory, completing on bar.
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
     asm volatile(

@@ -35,6 +35,7 @@
 
 #include "device_utils.cuh"
 #include "kernel_chained.cuh"
+#include "kernel_decode.cuh"
 #include "kernel_generic.cuh"
 #include "kernel_step.cuh"
 #include "sscan.h"
@@ -127,6 +128,9 @@ struct sscan_plan {
     bool tm_valid;
     // generic kernel
     int g_nl, g_lpc;
+    // decode kernel (L = 1 with a state)
+    bool decode;
+    int dec_grid;  // persistent grid, set on the first launch
     // sscan_forward_host: piece schedule, sub-plans and streams (made on first use)
     HostPipe *host;
 };
@@ -165,14 +169,16 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // head skip publishing the carried state (failure-detection tests: the
 // bounded waits of the warps running the tails must give up and report it),
 // light=<per mille> sets how much shorter the segments of the warps that share
-// an SM sub-partition with the producer warp are (see kLightPermille).
-void read_tune(int &cfg, int &poly, int &sms, int &split, int &nopublish, int &light) {
+// an SM sub-partition with the producer warp are (see kLightPermille), decode=0
+// runs a decode step (L = 1) on the step kernel instead of the decode kernel.
+void read_tune(int &cfg, int &poly, int &sms, int &split, int &nopublish, int &light, int &decode) {
     cfg = -2;
     poly = -1;
     sms = 0;
     split = 0;
     nopublish = 0;
     light = -1;
+    decode = 1;
     const char *s = getenv("SSCAN_TUNE");
     if (!s) return;
     if (const char *c = strstr(s, "cfg=")) cfg = atoi(c + 4);
@@ -181,6 +187,7 @@ void read_tune(int &cfg, int &poly, int &sms, int &split, int &nopublish, int &l
     if (const char *c = strstr(s, "split=")) split = atoi(c + 6);
     if (const char *c = strstr(s, "nopublish=")) nopublish = atoi(c + 10);
     if (const char *c = strstr(s, "light=")) light = atoi(c + 6);
+    if (const char *c = strstr(s, "decode=")) decode = atoi(c + 7);
 }
 
 void choose_schedule(sscan_plan *p) {
@@ -188,8 +195,8 @@ void choose_schedule(sscan_plan *p) {
     p->mode = kGeneric;
     p->g_nl = p->N == 16 ? 8 : 16;
     p->g_lpc = static_cast<int>(p->N) / p->g_nl;
-    int want = -2, poly = -1, sms = 0, force_split = 0, nopublish = 0, light = -1;
-    read_tune(want, poly, sms, force_split, nopublish, light);
+    int want = -2, poly = -1, sms = 0, force_split = 0, nopublish = 0, light = -1, decode = 1;
+    read_tune(want, poly, sms, force_split, nopublish, light, decode);
     p->drop_publish = nopublish != 0;
     const int blocks = (sms > 0 && sms < p->sm_count) ? sms : p->sm_count;
     // the FMA-pipe exponent measured slower than MUFU alone at every occupancy: off unless asked
@@ -198,6 +205,9 @@ void choose_schedule(sscan_plan *p) {
     // the step kernel, not a persistent grid with a TMA pipeline
     if (p->L < kMinChainedL && want != -1) {
         p->mode = kStep;
+        // one token with every bulk copy a multiple of 16 bytes: the decode kernel
+        // (calls with a state; without one the step kernel runs)
+        p->decode = p->L == 1 && p->D % 8 == 0 && decode != 0;
         return;
     }
     if (want == -1) return;
@@ -318,6 +328,44 @@ cudaError_t launch_step(const sscan_plan *p, const void *u, const void *dl, cons
         case 16: return launch_step_t<IO, 16>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s);
         case 32: return launch_step_t<IO, 32>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s);
         default: return launch_step_t<IO, 64>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s);
+    }
+}
+
+template <class IO, int N, bool ZOH>
+int launch_decode_t(sscan_plan *p, const void *u, const void *dl, const float *A, const void *Bm, const void *Cm,
+                    const float *h0, void *y, float *hf, const Fused &fu, cudaStream_t s) {
+    using Cfg = DecodeCfg<IO, N>;
+    auto kern = sscan_decode_kernel<IO, N, ZOH>;
+    if (smem_opt_in<sscan_decode_kernel<IO, N, ZOH>>(Cfg::kSmem) != cudaSuccess) return SSCAN_ERR_CUDA;
+    if (p->dec_grid == 0) {
+        int occ = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kDecThreads, Cfg::kSmem) != cudaSuccess)
+            return SSCAN_ERR_CUDA;
+        // the walk of sscan_decode_kernel: with R channel ranges and at most `slots` resident
+        // blocks, K = min(B, slots / R) blocks per range (grid K * R), else one block per slot
+        const int64_t R = ceil_div(p->D, Cfg::TD);
+        const int64_t slots = static_cast<int64_t>(occ > 0 ? occ : 1) * p->sm_count;
+        const int64_t K = std::min<int64_t>(p->B, slots / R);
+        p->dec_grid = static_cast<int>(R <= slots ? K * R : slots);
+    }
+    kern<<<p->dec_grid, kDecThreads, Cfg::kSmem, s>>>(
+        static_cast<const IO *>(u), static_cast<const IO *>(dl), A, static_cast<const IO *>(Bm),
+        static_cast<const IO *>(Cm), h0, static_cast<IO *>(y), hf, p->B, p->D, fu.bias,
+        static_cast<const IO *>(fu.z), fu.softplus ? 1 : 0, p->d_status);
+    return cudaGetLastError() == cudaSuccess ? SSCAN_OK : SSCAN_ERR_CUDA;
+}
+
+template <class IO>
+int launch_decode(sscan_plan *p, const void *u, const void *dl, const float *A, const void *Bm, const void *Cm,
+                  const float *h0, void *y, float *hf, const Fused &fu, cudaStream_t s) {
+    const bool zoh = (p->flags & SSCAN_ZOH) != 0;
+    switch (p->N) {
+        case 16: return zoh ? launch_decode_t<IO, 16, true>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s)
+                            : launch_decode_t<IO, 16, false>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s);
+        case 32: return zoh ? launch_decode_t<IO, 32, true>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s)
+                            : launch_decode_t<IO, 32, false>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s);
+        default: return zoh ? launch_decode_t<IO, 64, true>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s)
+                            : launch_decode_t<IO, 64, false>(p, u, dl, A, Bm, Cm, h0, y, hf, fu, s);
     }
 }
 
@@ -722,6 +770,14 @@ int sscan_plan_describe(sscan_plan_t plan, char *buf, size_t len) {
                      plan->split ? 1 : 0,
                      (long long)plan->chains, (long long)plan->workers, (long long)plan->seg, (long long)plan->seg_shift, plan->ws_bytes,
                      plan->sm_count);
+    } else if (plan->mode == kStep && plan->decode) {
+        n = snprintf(tmp, sizeof tmp,
+                     "kernel=decode B=%lld L=%lld D=%lld N=%lld dtype=%s zoh=%d states_per_thread=4 "
+                     "threads_per_channel=%lld stages=%d tile_state_bytes=%d threads=%d sms=%d "
+                     "(the step kernel when h0 is NULL)",
+                     (long long)plan->B, (long long)plan->L, (long long)plan->D, (long long)plan->N,
+                     plan->dtype == SSCAN_F32 ? "f32" : "bf16", (plan->flags & SSCAN_ZOH) ? 1 : 0,
+                     (long long)(plan->N / 4), kDecStages, kDecTileStateBytes, kDecThreads, plan->sm_count);
     } else if (plan->mode == kStep) {
         n = snprintf(tmp, sizeof tmp,
                      "kernel=step B=%lld L=%lld D=%lld N=%lld dtype=%s zoh=%d states_per_thread=4 "
@@ -792,6 +848,9 @@ int sscan_forward_gated(sscan_plan_t plan, const void *u, const void *delta, con
     }
     if (p->mode == kStep) {
         if (p->L == 0) return step_empty(p, h0, h_final, s);
+        if (p->decode && h0 != nullptr)
+            return p->dtype == SSCAN_F32 ? launch_decode<float>(p, u, delta, A, B, C, h0, y, h_final, fu, s)
+                                         : launch_decode<uint16_t>(p, u, delta, A, B, C, h0, y, h_final, fu, s);
         const cudaError_t e =
             p->dtype == SSCAN_F32 ? launch_step<float>(p, u, delta, A, B, C, h0, y, h_final, fu, s)
                                   : launch_step<uint16_t>(p, u, delta, A, B, C, h0, y, h_final, fu, s);

@@ -307,7 +307,7 @@ def test_decode_steps_match_one_forward(dt, zoh):
     y_full, h_full = S.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"], zoh=zoh)
     tdt = torch.float32 if dt == "f32" else torch.bfloat16
     plan = S.get_plan(Bt, 1, D, N, tdt, zoh)
-    assert "kernel=step" in plan.describe()
+    assert "kernel=decode" in plan.describe()
     state = d["h0"].clone()
     ys = []
     for t in range(L):
@@ -321,6 +321,42 @@ def test_decode_steps_match_one_forward(dt, zoh):
     P.check(state.cpu().numpy(), hr, dt, "decoded state")
     assert torch.allclose(torch.cat(ys, 1).float(), y_full.float(), rtol=2e-2 if dt == "bf16" else 1e-5,
                           atol=1e-2 if dt == "bf16" else 1e-5)
+
+
+DECODE = [
+    # (B, D, N, dtype, zoh, fused, in_place): one token with a state (the decode kernel when D % 8 == 0)
+    (4, 256, 16, "f32", False, False, True),
+    (3, 200, 16, "bf16", True, False, False),     # ragged last tile (128 + 72 channels)
+    (600, 1024, 16, "f32", False, False, True),   # 4800 tiles: every block's stage ring wraps
+    (5, 136, 32, "f32", True, False, True),       # N = 32: 64-channel tiles, ragged
+    (7, 72, 64, "bf16", False, True, True),       # N = 64: 32-channel tiles; softplus(delta + bias), gate
+    (9, 520, 16, "f32", True, True, False),
+    (2, 100, 16, "f32", False, False, True),      # D % 8 != 0: the step kernel
+]
+
+
+@pytest.mark.parametrize("case", DECODE, ids=[f"B{c[0]}D{c[1]}N{c[2]}{c[3]}{'_zoh' if c[4] else ''}"
+                                               f"{'_fused' if c[5] else ''}{'_inplace' if c[6] else ''}"
+                                               for c in DECODE])
+def test_decode_kernel_matches_oracle(case):
+    Bt, D, N, dt, zoh, fused, in_place = case
+    g = W.generate(Bt, 1, D, N, dt, 0.5, seed=9500 + Bt + D + N, A_jitter=0.3, fused=fused)
+    d = P.to_device(g)
+    tdt = torch.float32 if dt == "f32" else torch.bfloat16
+    plan = S.Plan(Bt, 1, D, N, tdt, zoh, delta_softplus=fused)
+    assert ("kernel=decode" if D % 8 == 0 else "kernel=step") in plan.describe()
+    h = d["h0"].clone()
+    hf = h if in_place else torch.empty_like(h)
+    y, _ = plan.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], h0=h, h_final=hf,
+                        delta_bias=d["delta_bias"], z=d["z"])
+    torch.cuda.synchronize()
+    assert plan.status() == S.OK
+    yr, hr = P.run_oracle(g, zoh, softplus=fused)
+    P.check(y.float().cpu().numpy(), yr, dt, "y")
+    P.check(hf.cpu().numpy(), hr, dt, "h_final")
+    if not in_place:
+        assert torch.equal(h, d["h0"])  # the input state is not written
+    plan.close()
 
 
 def test_h_final_may_alias_h0():
