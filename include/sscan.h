@@ -191,10 +191,12 @@ SSCAN_API int sscan_forward_host(sscan_plan_t plan, const void *u, const void *d
  *   dB, dC                  [B][L][N] fp32 (output; summed over channels)
  *   dh0                     [B][D][N] fp32 (output), or NULL to skip it
  *   workspace               sscan_backward_workspace_bytes(B, L, D, N) bytes
- *                           (the state checkpoints), 16-byte aligned
- * All pointers are caller-owned device memory; nothing is retained.  dA, dB
- * and dC are accumulated with fp32 atomics, so their last bits depend on the
- * order of arrival.  Errors as for sscan_forward (SSCAN_ERR_UNSUPPORTED for N
+ *                           (the state checkpoints and the per-block partial
+ *                           sums of dB and dC), 16-byte aligned
+ * All pointers are caller-owned device memory; nothing is retained.  dA and
+ * the bias gradient are accumulated with fp32 atomics, so their last bits
+ * depend on the order of arrival; dB and dC are sums in a fixed order.  Two
+ * kernels are enqueued.  Errors as for sscan_forward (SSCAN_ERR_UNSUPPORTED for N
  * outside {16, 32, 64}).  sscan_backward is sscan_backward_gated without a
  * bias and a gate. */
 SSCAN_API size_t sscan_backward_workspace_bytes(int64_t B, int64_t L, int64_t D, int64_t N);

@@ -24,18 +24,21 @@
 // takes the chunks last to first, recomputes each chunk's states from its
 // checkpoint into registers and runs the reverse recurrence over them.
 //
-// Occupancy: three blocks per SM (registers capped at 170 per thread; with
-// 8-token chunks nothing spills), so the 384 blocks of a 8 x 1536-channel layer
-// run in one wave.
-//
-// Mapping: each lane holds four states of one channel (LPC = N/4 adjacent lanes
-// per channel, CPW = 32/LPC channels per warp), so du, ddelta and the gate's
-// ys are summed over LPC lanes (log2 LPC shuffles) and dA needs none; a block
-// of four warps covers 4 CPW consecutive channels of one batch row and walks
-// the same chunks in the same order, so dB and dC (sums over channels) are
-// summed over the warp by a reduce-scatter of shuffles, over the block in
-// shared memory once per chunk, and added to the fp32 outputs with one 16-byte
-// atomic per four states and token (outputs zeroed by the host).
+// Mapping: each lane holds S consecutive states of one channel (S = 4, 2 or 1;
+// LPC = N/S adjacent lanes per channel, CPW = 32/LPC channels per warp); a block
+// of four warps covers CPB = 4 CPW consecutive channels of one batch row, and
+// its warps walk the same chunks in the same order.  The reverse sweep over a
+// chunk keeps every cross-lane sum out of the token loop: each lane writes its
+// per-token partials (its states' share of du, ddelta and the gate's ys, and
+// its contributions to dB and dC) to shared memory; after the chunk the block's
+// threads reduce them data-parallel: du, ddelta (and dz) of each (token,
+// channel) over the channel's LPC lanes, stored with coalesced writes, and dB,
+// dC of each (token, four states) over the block's channels, stored in the
+// block's own plane of a workspace array.  A second kernel sums the planes
+// into dB and dC: the blocks of a batch row walk the same tokens at the same
+// time, so atomics on dB and dC would all meet on the same few lines.  dA
+// needs no cross-lane sum (one atomic per lane at the end).  The recompute
+// keeps each token's Abar in registers for the reverse sweep.
 #pragma once
 
 #include "device_utils.cuh"
@@ -46,8 +49,13 @@ constexpr int kBwdWarps = 4;
 constexpr int kBwdThreads = 32 * kBwdWarps;
 constexpr int kChunk = 8;   // tokens per recomputed chunk
 
-// channels a backward block covers
-__host__ __device__ constexpr int bwd_block_channels(int N) { return kBwdWarps * (32 / (N / 4)); }
+// channels a backward block covers with S states per lane
+__host__ __device__ constexpr int bwd_block_channels_s(int N, int S) { return kBwdWarps * (32 / (N / S)); }
+// channel padding of the checkpoint workspace: the widest block (S = 4), a
+// multiple of every block width
+__host__ __device__ constexpr int bwd_block_channels(int N) { return bwd_block_channels_s(N, 4); }
+// blocks per SM the register budget is set for
+template <int S> constexpr int bwd_min_blocks() { return S == 4 ? 3 : S == 2 ? 6 : 10; }
 
 struct BwdParams {
     const void *u, *delta, *Bm, *Cm, *dy, *z;
@@ -55,57 +63,86 @@ struct BwdParams {
     void *du, *ddelta, *dz;
     float *dA, *dB, *dC, *dh0, *dbias;
     float *ckpt;           // [B][Dpad][nchunks][N]
+    float *part;           // [Dpad / CPB][B][L][2][N]: each block's dB, dC sums over its channels
     int64_t L, D, Dpad, nchunks;
     int softplus;
 };
 
-template <class IO> __device__ __forceinline__ float4 bwd_ld4(const IO *p);
-template <> __device__ __forceinline__ float4 bwd_ld4<float>(const float *p) {
-    return __ldg(reinterpret_cast<const float4 *>(p));
-}
-template <> __device__ __forceinline__ float4 bwd_ld4<uint16_t>(const uint16_t *p) {
-    const uint2 v = __ldg(reinterpret_cast<const uint2 *>(p));
-    return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u), __uint_as_float(v.y << 16),
-                       __uint_as_float(v.y & 0xffff0000u));
-}
-__device__ __forceinline__ float f4_at(const float4 &v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
-
-// Sum the four per-lane values over the lanes that share a state group (the
-// warp's channels: lane bits LPC, 2 LPC, ... 16), as a reduce-scatter: while a
-// lane holds more than one value it keeps half and sends the other half to its
-// partner, then whole values are summed.  Afterwards v[0 .. V) hold the totals
-// of the group's states jbase .. jbase + V - 1, V = 4 >> min(levels, 2); lanes
-// that differ only in the bits above the first two levels hold the same totals.
-template <int LPC>
-__device__ __forceinline__ int channel_scatter4(float (&v)[4], int lane, int &V) {
-    int jbase = 0, cnt = 4;
-#pragma unroll
-    for (int m = LPC; m < 32; m <<= 1) {
-        if (cnt >= 2) {
-            const bool up = (lane & m) != 0;
-#pragma unroll
-            for (int i = 0; i < cnt / 2; ++i) {
-                const float send = up ? v[i] : v[i + cnt / 2];
-                const float keep = up ? v[i + cnt / 2] : v[i];
-                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-            }
-            if (up) jbase += cnt / 2;
-            cnt /= 2;
-        } else {
-            v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
-        }
+// S consecutive fp32 values (S = 4, 2, 1): load (read-only path or plain), store, atomic add
+template <int S> __device__ __forceinline__ void ldv(const float *p, float (&v)[S], bool ro = true) {
+    if constexpr (S == 4) {
+        const float4 t = ro ? __ldg(reinterpret_cast<const float4 *>(p)) : *reinterpret_cast<const float4 *>(p);
+        v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+    } else if constexpr (S == 2) {
+        const float2 t = ro ? __ldg(reinterpret_cast<const float2 *>(p)) : *reinterpret_cast<const float2 *>(p);
+        v[0] = t.x; v[1] = t.y;
+    } else {
+        v[0] = ro ? __ldg(p) : *p;
     }
-    V = cnt;
-    return jbase;
+}
+template <int S> __device__ __forceinline__ void stv(float *p, const float (&v)[S]) {
+    if constexpr (S == 4) *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    else if constexpr (S == 2) *reinterpret_cast<float2 *>(p) = make_float2(v[0], v[1]);
+    else *p = v[0];
+}
+template <int S> __device__ __forceinline__ void atomic_addv(float *p, const float (&v)[S]) {
+    if constexpr (S == 4) atomicAdd(reinterpret_cast<float4 *>(p), make_float4(v[0], v[1], v[2], v[3]));
+    else if constexpr (S == 2) atomicAdd(reinterpret_cast<float2 *>(p), make_float2(v[0], v[1]));
+    else atomicAdd(p, v[0]);
+}
+// S consecutive values of a B or C row in the I/O type, widened to fp32
+template <class IO, int S> __device__ __forceinline__ void ldv_io(const IO *p, float (&v)[S]) {
+    if constexpr (sizeof(IO) == 4) {
+        ldv<S>(reinterpret_cast<const float *>(p), v);
+    } else if constexpr (S == 4) {
+        const uint2 t = __ldg(reinterpret_cast<const uint2 *>(p));
+        v[0] = __uint_as_float(t.x << 16); v[1] = __uint_as_float(t.x & 0xffff0000u);
+        v[2] = __uint_as_float(t.y << 16); v[3] = __uint_as_float(t.y & 0xffff0000u);
+    } else if constexpr (S == 2) {
+        const uint32_t t = __ldg(reinterpret_cast<const unsigned int *>(p));
+        v[0] = __uint_as_float(t << 16); v[1] = __uint_as_float(t & 0xffff0000u);
+    } else {
+        v[0] = __uint_as_float(static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short *>(p))) << 16);
+    }
 }
 
-template <class IO, int N, bool ZOH, bool FUSED>
-__global__ void __launch_bounds__(kBwdThreads, 3)
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+__device__ __forceinline__ void prefetch_l1(const void *p) {
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
+// Sum of LPC consecutive floats in shared memory (16-byte aligned when LPC >= 4).
+template <int LPC> __device__ __forceinline__ float sum_lanes(const float *p) {
+    float acc = 0.0f;
+    if constexpr (LPC >= 4) {
+#pragma unroll
+        for (int i = 0; i < LPC; i += 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(p + i);
+            acc += (v.x + v.y) + (v.z + v.w);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < LPC; ++i) acc += p[i];
+    }
+    return acc;
+}
+
+template <class IO, int N, int S, bool ZOH, bool FUSED>
+__global__ void __launch_bounds__(kBwdThreads, bwd_min_blocks<S>())
 sscan_backward_kernel(const BwdParams P) {
-    constexpr int LPC = N / 4, CPW = 32 / LPC, CPB = kBwdWarps * CPW, KC = kChunk;
-    __shared__ __align__(16) float s_db[kBwdWarps][KC][N], s_dc[kBwdWarps][KC][N];
+    constexpr int LPC = N / S, CPW = 32 / LPC, CPB = kBwdWarps * CPW, KC = kChunk;
+    // keep each token's Abar from the recompute for the reverse sweep (S = 4), or
+    // take it again from the MUFU pipe there (fewer registers: S = 2, 1)
+    constexpr bool kKeepAbar = S >= 4;
+    constexpr int KA = kKeepAbar ? KC : 1;
+    // per chunk: each lane's partials of du, ddelta (of the raw step) and the gate's ys per
+    // token, and its S contributions to dB and dC per token ([k][channel][N] order)
+    __shared__ __align__(16) float s_tok[3][KC][kBwdThreads];
+    __shared__ __align__(16) float s_vb[KC][kBwdThreads * S], s_vc[KC][kBwdThreads * S];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int cl = lane / LPC, g = lane % LPC, n0 = 4 * g;
+    const int cl = lane / LPC, g = lane % LPC, n0 = S * g;
     const int64_t L = P.L, D = P.D;
     const int64_t b = blockIdx.y;
     const int64_t d = static_cast<int64_t>(blockIdx.x) * CPB + warp * CPW + cl;
@@ -119,15 +156,12 @@ sscan_backward_kernel(const BwdParams P) {
     const IO *Cp = static_cast<const IO *>(P.Cm) + b * L * N + n0;
     float *ck = P.ckpt + (b * P.Dpad + d) * P.nchunks * N + n0;  // own slot even past D
 
-    float a1[4], a2[4], ia[4];
-    {
-        const float4 a = __ldg(reinterpret_cast<const float4 *>(P.A + dc * N + n0));
+    float a1[S], a2[S], ia[S];
+    ldv<S>(P.A + dc * N + n0, a1);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            a1[i] = f4_at(a, i);
-            a2[i] = static_cast<float>(static_cast<double>(a1[i]) * 1.4426950408889634);
-            ia[i] = a1[i] != 0.0f ? 1.0f / a1[i] : 0.0f;
-        }
+    for (int i = 0; i < S; ++i) {
+        a2[i] = static_cast<float>(static_cast<double>(a1[i]) * 1.4426950408889634);
+        ia[i] = a1[i] != 0.0f ? 1.0f / a1[i] : 0.0f;
     }
     const float biasv = FUSED && P.bias ? __ldg(P.bias + dc) : 0.0f;
     // the step the scan uses, and (fused) softplus' = sigmoid of its argument
@@ -169,37 +203,62 @@ sscan_backward_kernel(const BwdParams P) {
         }
     };
 
+    // The rows a chunk reads (delta, u, dy, z of this warp's channels, B and C) are
+    // prefetched ahead of it: into L1 one chunk ahead, into L2 two chunks ahead; lane
+    // l takes token l % KC of row kind l / KC.  Prefetches are hints: addresses stay
+    // inside the tensors (tokens clamped to the sequence).
+    auto prefetch_chunk = [&](int64_t c, bool l1, bool with_dy) {
+        if (c < 0 || c >= P.nchunks) return;
+        const int64_t t = c * KC + lane % KC < L ? c * KC + lane % KC : L - 1;
+        const void *a;
+        switch (lane / KC) {
+            case 0: a = dl_in + t * D; break;
+            case 1: a = u + t * D; break;
+            case 2: a = with_dy ? static_cast<const void *>(dyp + t * D) : static_cast<const void *>(Bp + t * N); break;
+            default: a = (with_dy && zp) ? static_cast<const void *>(zp + t * D) : static_cast<const void *>(Cp + t * N); break;
+        }
+        if (l1) prefetch_l1(a); else prefetch_l2(a);
+        if (with_dy && lane / KC >= 2) {  // B and C rows too
+            const void *bc = lane / KC == 2 ? static_cast<const void *>(Bp + t * N) : static_cast<const void *>(Cp + t * N);
+            if (l1) prefetch_l1(bc); else prefetch_l2(bc);
+        }
+    };
+
     // ---- pass 1: forward, keeping the state entering every chunk ----
     // (chunk by chunk: a chunk's loads sit in one straight-line block, ahead of its
     // dependent updates)
-    float h[4];
-    {
-        const float4 v = P.h0 ? *reinterpret_cast<const float4 *>(P.h0 + (b * D + dc) * N + n0)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-        h[0] = v.x; h[1] = v.y; h[2] = v.z; h[3] = v.w;
+    float h[S];
+    if (P.h0) {
+        ldv<S>(P.h0 + (b * D + dc) * N + n0, h, false);
+    } else {
+#pragma unroll
+        for (int i = 0; i < S; ++i) h[i] = 0.0f;
     }
+    prefetch_chunk(0, true, false);
+    prefetch_chunk(1, false, false);
     for (int64_t c = 0; c < P.nchunks; ++c) {
         const int64_t t0 = c * KC;
         const int nt = static_cast<int>(L - t0 < KC ? L - t0 : KC);
-        *reinterpret_cast<float4 *>(ck + c * N) = make_float4(h[0], h[1], h[2], h[3]);
-        float xs[KC], ds[KC];
-        float4 Bs[KC];
+        prefetch_chunk(c + 1, true, false);
+        prefetch_chunk(c + 2, false, false);
+        stv<S>(ck + c * N, h);
+        float xs[KC], ds[KC], Bs[KC][S];
 #pragma unroll
         for (int k = 0; k < KC; ++k) {
             const int64_t t = t0 + (k < nt ? k : nt - 1);
             float sg;
             ds[k] = step(t, sg);
             xs[k] = Io<IO>::widen(Io<IO>::ld(u + t * D));
-            Bs[k] = bwd_ld4<IO>(Bp + t * N);
+            ldv_io<IO, S>(Bp + t * N, Bs[k]);
         }
 #pragma unroll
         for (int k = 0; k < KC; ++k) {
             if (k < nt) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
+                for (int i = 0; i < S; ++i) {
                     const float abar = ex2(ds[k] * a2[i]);
                     float beta, q0, q1, q2;
-                    coefs(i, ds[k], abar, f4_at(Bs[k], i), beta, q0, q1, q2);
+                    coefs(i, ds[k], abar, Bs[k][i], beta, q0, q1, q2);
                     h[i] = fmaf(abar, h[i], beta * xs[k]);
                 }
             }
@@ -207,42 +266,46 @@ sscan_backward_kernel(const BwdParams P) {
     }
 
     // ---- pass 2: reverse sweep over the chunks ----
-    float gs[4], dacc[4];
-    {
-        const float4 v = (P.dhf && valid) ? *reinterpret_cast<const float4 *>(P.dhf + (b * D + dc) * N + n0)
-                                          : make_float4(0.f, 0.f, 0.f, 0.f);
-        gs[0] = v.x; gs[1] = v.y; gs[2] = v.z; gs[3] = v.w;
+    float gs[S], dacc[S];
+    if (P.dhf && valid) {
+        ldv<S>(P.dhf + (b * D + dc) * N + n0, gs, false);
+    } else {
+#pragma unroll
+        for (int i = 0; i < S; ++i) gs[i] = 0.0f;
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) dacc[i] = 0.0f;
+    for (int i = 0; i < S; ++i) dacc[i] = 0.0f;
     float dbias_acc = 0.0f;
+    prefetch_chunk(P.nchunks - 1, true, true);
     for (int64_t c = P.nchunks - 1; c >= 0; --c) {
         const int64_t t0 = c * KC;
         const int nt = static_cast<int>(L - t0 < KC ? L - t0 : KC);
-        // recompute the chunk's states h_{t0 .. t0+nt-1} from its checkpoint
-        float h_in[4], hk[KC][4];
+        prefetch_chunk(c - 1, true, true);
+        prefetch_chunk(c - 2, false, true);
+        if (c >= 1) prefetch_l1(ck + (c - 1) * N);
+        // recompute the chunk's states h_{t0 .. t0+nt-1} (and each token's Abar) from its checkpoint
+        float h_in[S], hk[KC][S], ab[KA][S];
+        ldv<S>(ck + c * N, h_in, false);
         {
-            const float4 v = *reinterpret_cast<const float4 *>(ck + c * N);
-            h_in[0] = v.x; h_in[1] = v.y; h_in[2] = v.z; h_in[3] = v.w;
-        }
-        {
-            float hc[4] = {h_in[0], h_in[1], h_in[2], h_in[3]};
+            float hc[S];
+#pragma unroll
+            for (int i = 0; i < S; ++i) hc[i] = h_in[i];
 #pragma unroll
             for (int k = 0; k < KC; ++k) {
                 const int64_t t = t0 + (k < nt ? k : nt - 1);  // loads need not wait behind work
                 float sg;
                 const float dl = step(t, sg);
                 const float x = Io<IO>::widen(Io<IO>::ld(u + t * D));
-                const float4 Bv = bwd_ld4<IO>(Bp + t * N);
-                if (k < nt) {
+                float Bv[S];
+                ldv_io<IO, S>(Bp + t * N, Bv);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float abar = ex2(dl * a2[i]);
-                        float beta, q0, q1, q2;
-                        coefs(i, dl, abar, f4_at(Bv, i), beta, q0, q1, q2);
-                        hc[i] = fmaf(abar, hc[i], beta * x);
-                        hk[k][i] = hc[i];
-                    }
+                for (int i = 0; i < S; ++i) {
+                    const float abar = ex2(dl * a2[i]);
+                    float beta, q0, q1, q2;
+                    coefs(i, dl, abar, Bv[i], beta, q0, q1, q2);
+                    if (k < nt) hc[i] = fmaf(abar, hc[i], beta * x);
+                    hk[k][i] = hc[i];
+                    if constexpr (kKeepAbar) ab[k][i] = abar;
                 }
             }
         }
@@ -256,32 +319,30 @@ sscan_backward_kernel(const BwdParams P) {
             const float dl = step(t, sg);
             const float x = Io<IO>::widen(Io<IO>::ld(u + t * D));
             float dyt = valid ? Io<IO>::widen(Io<IO>::ld(dyp + t * D)) : 0.0f;  // idle lanes add nothing
-            const float4 Bv = bwd_ld4<IO>(Bp + t * N);
-            const float4 Cv = bwd_ld4<IO>(Cp + t * N);
+            float Bv[S], Cv[S];
+            ldv_io<IO, S>(Bp + t * N, Bv);
+            ldv_io<IO, S>(Cp + t * N, Cv);
             const float zraw = (FUSED && zp != nullptr) ? Io<IO>::widen(Io<IO>::ld(zp + t * D)) : 0.0f;
             if (k < nt) {
-                float dzt = 0.0f;
+                float ysp = 0.0f;
                 if (FUSED && zp != nullptr) {
-                    // the gate: the scan's own output ys = C . h_t, summed over the channel's lanes
-                    float ys = 0.0f;
+                    // the gate: this lane's share of the scan's own output ys = C . h_t
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) ys = fmaf(f4_at(Cv, i), hk[k][i], ys);
-#pragma unroll
-                    for (int o = 1; o < LPC; o <<= 1) ys += __shfl_xor_sync(0xffffffffu, ys, o);
-                    const float zt = zraw;
-                    const float sz = 1.0f / (1.0f + ex2(-zt * 1.4426950408889634f));
-                    dzt = dyt * ys * sz * fmaf(zt, 1.0f - sz, 1.0f);
-                    dyt *= zt * sz;
+                    for (int i = 0; i < S; ++i) ysp = fmaf(Cv[i], hk[k][i], ysp);
+                    const float sz = 1.0f / (1.0f + ex2(-zraw * 1.4426950408889634f));
+                    dyt *= zraw * sz;  // dy of the scan = dy silu(z)
                 }
                 float dut = 0.0f, ddt = 0.0f;
-                float vb[4], vc[4];
+                float vb[S], vc[S];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
+                for (int i = 0; i < S; ++i) {
                     const float hprev = k > 0 ? hk[k > 0 ? k - 1 : 0][i] : h_in[i];
-                    const float abar = ex2(dl * a2[i]);
+                    float abar;
+                    if constexpr (kKeepAbar) abar = ab[k][i];
+                    else abar = ex2(dl * a2[i]);
                     float beta, dbdl, dbda, dbdb;
-                    coefs(i, dl, abar, f4_at(Bv, i), beta, dbdl, dbda, dbdb);
-                    gs[i] = fmaf(f4_at(Cv, i), dyt, gs[i]);
+                    coefs(i, dl, abar, Bv[i], beta, dbdl, dbda, dbdb);
+                    gs[i] = fmaf(Cv[i], dyt, gs[i]);
                     dut = fmaf(gs[i], beta, dut);
                     ddt = fmaf(gs[i], fmaf(hprev * a1[i], abar, x * dbdl), ddt);
                     dacc[i] = fmaf(gs[i], fmaf(hprev * dl, abar, x * dbda), dacc[i]);
@@ -289,57 +350,81 @@ sscan_backward_kernel(const BwdParams P) {
                     vc[i] = dyt * hk[k][i];
                     gs[i] *= abar;
                 }
-#pragma unroll
-                for (int o = 1; o < LPC; o <<= 1) {
-                    dut += __shfl_xor_sync(0xffffffffu, dut, o);
-                    ddt += __shfl_xor_sync(0xffffffffu, ddt, o);
-                }
-                ddt *= sg;  // the gradient of the raw step (softplus' = sigmoid)
-                if (valid) {
-                    dbias_acc += ddt;
-                    if (g == 0) {
-                        const int64_t idx = (b * L + t) * D + d;
-                        Io<IO>::st(static_cast<IO *>(P.du) + idx, dut);
-                        Io<IO>::st(static_cast<IO *>(P.ddelta) + idx, ddt);
-                        if (FUSED && zp != nullptr) Io<IO>::st(static_cast<IO *>(P.dz) + idx, dzt);
-                    }
-                }
-                // sums over the warp's channels (lanes with the same state group)
-                int V;
-                const int jb = channel_scatter4<LPC>(vb, lane, V);
-                channel_scatter4<LPC>(vc, lane, V);
-                if (lane < 4 * LPC) {  // one of the lanes holding each total
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        if (i < V) {
-                            s_db[warp][k][n0 + jb + i] = vb[i];
-                            s_dc[warp][k][n0 + jb + i] = vc[i];
-                        }
-                }
+                s_tok[0][k][threadIdx.x] = dut;
+                s_tok[1][k][threadIdx.x] = ddt * sg;  // the gradient of the raw step (softplus' = sigmoid)
+                if (FUSED && zp != nullptr) s_tok[2][k][threadIdx.x] = ysp;
+                stv<S>(&s_vb[k][threadIdx.x * S], vb);
+                stv<S>(&s_vc[k][threadIdx.x * S], vc);
             }
         }
         __syncthreads();
-        // sum over the block's warps; one 16-byte atomic per four states and token
-        constexpr int kEntries = KC * (N / 4);
-        for (int e = threadIdx.x; e < 2 * kEntries; e += kBwdThreads) {
-            const int which = e / kEntries, r = e % kEntries, k = r / (N / 4), q = r % (N / 4);
+        // du, ddelta (and dz) of each (token, channel): the channel's LPC lanes are the
+        // consecutive threads j LPC .. j LPC + LPC - 1
+        for (int e = threadIdx.x; e < KC * CPB; e += kBwdThreads) {
+            const int k = e / CPB, j = e % CPB;
+            const int64_t dj = static_cast<int64_t>(blockIdx.x) * CPB + j;
+            if (k >= nt || dj >= D) continue;
+            const int64_t idx = (b * L + t0 + k) * D + dj;
+            const float dut = sum_lanes<LPC>(&s_tok[0][k][j * LPC]);
+            const float ddt = sum_lanes<LPC>(&s_tok[1][k][j * LPC]);
+            Io<IO>::st(static_cast<IO *>(P.du) + idx, dut);
+            Io<IO>::st(static_cast<IO *>(P.ddelta) + idx, ddt);
+            dbias_acc += ddt;  // this thread's channel is always j = threadIdx.x % CPB
+            if (FUSED && zp != nullptr) {
+                const float ys = sum_lanes<LPC>(&s_tok[2][k][j * LPC]);
+                const float zt = Io<IO>::widen(Io<IO>::ld(static_cast<const IO *>(P.z) + idx));
+                const float dy0 = Io<IO>::widen(Io<IO>::ld(static_cast<const IO *>(P.dy) + idx));
+                const float sz = 1.0f / (1.0f + ex2(-zt * 1.4426950408889634f));
+                Io<IO>::st(static_cast<IO *>(P.dz) + idx, dy0 * ys * sz * fmaf(zt, 1.0f - sz, 1.0f));
+            }
+        }
+        // dB, dC of each (token, four states): summed over the block's channels (the
+        // contributions sit in [k][channel][N] order) into this block's plane
+        constexpr int kQ = N / 4;
+        float *plane = P.part + static_cast<int64_t>(blockIdx.x) * gridDim.y * L * 2 * N;
+        for (int e = threadIdx.x; e < 2 * KC * kQ; e += kBwdThreads) {
+            const int which = e / (KC * kQ), r = e % (KC * kQ), k = r / kQ, q = r % kQ;
             if (k >= nt) continue;
+            const float *src = (which ? &s_vc[k][0] : &s_vb[k][0]) + 4 * q;
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int w = 0; w < kBwdWarps; ++w) {
-                const float4 v = *reinterpret_cast<const float4 *>(which ? &s_dc[w][k][4 * q] : &s_db[w][k][4 * q]);
+#pragma unroll 4
+            for (int j = 0; j < CPB; ++j) {
+                const float4 v = *reinterpret_cast<const float4 *>(src + j * N);
                 acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
             }
-            float *dst = (which ? P.dC : P.dB) + (b * L + t0 + k) * N + 4 * q;
-            atomicAdd(reinterpret_cast<float4 *>(dst), acc);
+            *reinterpret_cast<float4 *>(plane + ((b * L + t0 + k) * 2 + which) * N + 4 * q) = acc;
         }
         __syncthreads();
     }
     if (valid) {
-        if (P.dh0 != nullptr)
-            *reinterpret_cast<float4 *>(P.dh0 + (b * D + d) * N + n0) = make_float4(gs[0], gs[1], gs[2], gs[3]);
-        atomicAdd(reinterpret_cast<float4 *>(P.dA + d * N + n0), make_float4(dacc[0], dacc[1], dacc[2], dacc[3]));
-        if (FUSED && P.dbias != nullptr && g == 0) atomicAdd(P.dbias + d, dbias_acc);
+        if (P.dh0 != nullptr) stv<S>(P.dh0 + (b * D + d) * N + n0, gs);
+        atomic_addv<S>(P.dA + d * N + n0, dacc);
+    }
+    if (FUSED && P.dbias != nullptr && threadIdx.x < KC * CPB) {
+        const int64_t dj = static_cast<int64_t>(blockIdx.x) * CPB + threadIdx.x % CPB;
+        if (dj < D) atomicAdd(P.dbias + dj, dbias_acc);
+    }
+}
+
+// dB and dC: the sum of the backward blocks' planes ([planes][rows][2][N],
+// rows = B L), one thread per four outputs, the planes read with coalesced
+// 16-byte loads.
+__global__ void __launch_bounds__(256)
+sscan_backward_reduce_kernel(const float *__restrict__ part, float *__restrict__ dB, float *__restrict__ dC,
+                             int64_t rows, int N, int64_t planes) {
+    const int64_t per_plane = rows * 2 * (N / 4);
+    for (int64_t q4 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; q4 < per_plane;
+         q4 += static_cast<int64_t>(gridDim.x) * blockDim.x) {  // float4 index within a plane
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 *p = reinterpret_cast<const float4 *>(part) + q4;
+        for (int64_t k = 0; k < planes; ++k) {
+            const float4 v = __ldg(p + k * per_plane);
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+        const int64_t row = q4 / (2 * (N / 4));
+        const int rem = static_cast<int>(q4 % (2 * (N / 4)));
+        const int which = rem / (N / 4), q = rem % (N / 4);
+        *reinterpret_cast<float4 *>((which ? dC : dB) + row * N + 4 * q) = acc;
     }
 }
 

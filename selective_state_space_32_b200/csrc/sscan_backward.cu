@@ -27,26 +27,38 @@ int64_t div_up(int64_t a, int64_t b) { return (a + b - 1) / b; }
 int64_t bwd_dpad(int64_t D, int64_t N) { return div_up(D, bwd_block_channels(static_cast<int>(N))) * bwd_block_channels(static_cast<int>(N)); }
 int64_t bwd_chunks(int64_t L) { return div_up(L, kChunk); }
 
-template <class IO, int N, bool ZOH, bool FUSED>
+// States per lane: 4 for every N (2 and 1, with twice and four times the warps,
+// measured slower: the extra lane-sum work outweighs the latency hidden).
+constexpr int bwd_states(int64_t) { return 4; }
+// backward blocks per batch row (planes of the dB / dC partial sums)
+int64_t bwd_planes(int64_t D, int64_t N) {
+    return bwd_dpad(D, N) / bwd_block_channels_s(static_cast<int>(N), bwd_states(N));
+}
+size_t bwd_ckpt_bytes(int64_t B, int64_t L, int64_t D, int64_t N) {
+    const size_t bytes = size_t(B) * size_t(bwd_dpad(D, N)) * size_t(bwd_chunks(L)) * size_t(N) * sizeof(float);
+    return (bytes + 255) / 256 * 256;
+}
+
+template <class IO, int N, int S, bool ZOH, bool FUSED>
 int launch_backward_t(int64_t B, const BwdParams &prm, cudaStream_t s) {
-    const dim3 grid(static_cast<unsigned>(prm.Dpad / bwd_block_channels(N)), static_cast<unsigned>(B));
-    sscan_backward_kernel<IO, N, ZOH, FUSED><<<grid, kBwdThreads, 0, s>>>(prm);
+    const dim3 grid(static_cast<unsigned>(prm.Dpad / bwd_block_channels_s(N, S)), static_cast<unsigned>(B));
+    sscan_backward_kernel<IO, N, S, ZOH, FUSED><<<grid, kBwdThreads, 0, s>>>(prm);
     return cudaGetLastError() == cudaSuccess ? SSCAN_OK : SSCAN_ERR_CUDA;
 }
 
-template <class IO, int N>
-int launch_backward_n(int64_t B, bool zoh, bool fused, const BwdParams &prm, cudaStream_t s) {
+template <class IO, int N, int S>
+int launch_backward_s(int64_t B, bool zoh, bool fused, const BwdParams &prm, cudaStream_t s) {
     if (fused)
-        return zoh ? launch_backward_t<IO, N, true, true>(B, prm, s) : launch_backward_t<IO, N, false, true>(B, prm, s);
-    return zoh ? launch_backward_t<IO, N, true, false>(B, prm, s) : launch_backward_t<IO, N, false, false>(B, prm, s);
+        return zoh ? launch_backward_t<IO, N, S, true, true>(B, prm, s) : launch_backward_t<IO, N, S, false, true>(B, prm, s);
+    return zoh ? launch_backward_t<IO, N, S, true, false>(B, prm, s) : launch_backward_t<IO, N, S, false, false>(B, prm, s);
 }
 
 template <class IO>
 int launch_backward(int64_t B, int64_t N, bool zoh, bool fused, const BwdParams &prm, cudaStream_t s) {
     switch (N) {
-        case 16: return launch_backward_n<IO, 16>(B, zoh, fused, prm, s);
-        case 32: return launch_backward_n<IO, 32>(B, zoh, fused, prm, s);
-        default: return launch_backward_n<IO, 64>(B, zoh, fused, prm, s);
+        case 16: return launch_backward_s<IO, 16, bwd_states(16)>(B, zoh, fused, prm, s);
+        case 32: return launch_backward_s<IO, 32, bwd_states(32)>(B, zoh, fused, prm, s);
+        default: return launch_backward_s<IO, 64, bwd_states(64)>(B, zoh, fused, prm, s);
     }
 }
 
@@ -56,8 +68,8 @@ extern "C" {
 
 size_t sscan_backward_workspace_bytes(int64_t B, int64_t L, int64_t D, int64_t N) {
     if (B < 1 || D < 1 || L < 1 || (N != 16 && N != 32 && N != 64)) return 0;
-    const size_t bytes = size_t(B) * size_t(bwd_dpad(D, N)) * size_t(bwd_chunks(L)) * size_t(N) * sizeof(float);
-    return (bytes + 255) / 256 * 256;
+    const size_t part = size_t(bwd_planes(D, N)) * size_t(B) * size_t(L) * 2 * size_t(N) * sizeof(float);
+    return bwd_ckpt_bytes(B, L, D, N) + (part + 255) / 256 * 256;
 }
 
 int sscan_backward_gated(int64_t B, int64_t L, int64_t D, int64_t N, int dtype, uint32_t flags, const void *u,
@@ -103,12 +115,9 @@ int sscan_backward_gated(int64_t B, int64_t L, int64_t D, int64_t N, int dtype, 
     for (int i = 0; i < 8; ++i)
         if (ws && overlaps_b(workspace, ws, outs[i], outsz[i])) return SSCAN_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // dA, dB, dC and the bias gradient are accumulated with atomics
+    // dA and the bias gradient are accumulated with atomics (dB and dC are written whole)
     if (cudaMemsetAsync(dA, 0, n_dn * 4, s) != cudaSuccess) return SSCAN_ERR_CUDA;
     if (ddelta_bias && cudaMemsetAsync(ddelta_bias, 0, static_cast<size_t>(D) * 4, s) != cudaSuccess)
-        return SSCAN_ERR_CUDA;
-    if (n_bln && (cudaMemsetAsync(dB, 0, n_bln * 4, s) != cudaSuccess ||
-                  cudaMemsetAsync(dC, 0, n_bln * 4, s) != cudaSuccess))
         return SSCAN_ERR_CUDA;
     if (L == 0) {  // no tokens: dh0 = dh_final
         if (dh0 && (dh_final ? cudaMemcpyAsync(dh0, dh_final, n_bdn * 4, cudaMemcpyDeviceToDevice, s)
@@ -122,11 +131,18 @@ int sscan_backward_gated(int64_t B, int64_t L, int64_t D, int64_t N, int dtype, 
     prm.du = du; prm.ddelta = ddelta; prm.dz = dz;
     prm.dA = dA; prm.dB = dB; prm.dC = dC; prm.dh0 = dh0; prm.dbias = ddelta_bias;
     prm.ckpt = static_cast<float *>(workspace);
+    prm.part = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + bwd_ckpt_bytes(B, L, D, N));
     prm.L = L; prm.D = D; prm.Dpad = bwd_dpad(D, N); prm.nchunks = bwd_chunks(L);
     prm.softplus = softplus ? 1 : 0;
     const bool zoh = (flags & SSCAN_ZOH) != 0;
-    return dtype == SSCAN_F32 ? launch_backward<float>(B, N, zoh, fused, prm, s)
-                              : launch_backward<uint16_t>(B, N, zoh, fused, prm, s);
+    const int rc = dtype == SSCAN_F32 ? launch_backward<float>(B, N, zoh, fused, prm, s)
+                                      : launch_backward<uint16_t>(B, N, zoh, fused, prm, s);
+    if (rc != SSCAN_OK) return rc;
+    const int64_t quads = B * L * 2 * (N / 4);
+    const int64_t rblocks = div_up(quads, 256) < 148 * 64 ? div_up(quads, 256) : 148 * 64;  // grid-stride beyond
+    sscan_backward_reduce_kernel<<<static_cast<unsigned>(rblocks), 256, 0, s>>>(
+        prm.part, dB, dC, B * L, static_cast<int>(N), bwd_planes(D, N));
+    return cudaGetLastError() == cudaSuccess ? SSCAN_OK : SSCAN_ERR_CUDA;
 }
 
 int sscan_backward(int64_t B, int64_t L, int64_t D, int64_t N, int dtype, uint32_t flags, const void *u,

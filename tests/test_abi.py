@@ -106,11 +106,19 @@ def test_gated_and_backward_reject_bad_arguments_without_a_device(lib):
 
 def test_backward_workspace_bytes(lib):
     # state checkpoints: B x channels padded to a block (4 warps x 32/(N/4) channels) x
-    # ceil(L/8) chunks x N states x 4 bytes, rounded up to 256 bytes
-    assert lib.sscan_backward_workspace_bytes(8, 2048, 1536, 16) == 8 * 1536 * 256 * 16 * 4
-    assert lib.sscan_backward_workspace_bytes(2, 37, 70, 16) == 2 * 96 * 5 * 16 * 4
-    assert lib.sscan_backward_workspace_bytes(2, 37, 70, 32) == 2 * 80 * 5 * 32 * 4
-    assert lib.sscan_backward_workspace_bytes(2, 37, 70, 64) == 2 * 72 * 5 * 64 * 4
+    # ceil(L/8) chunks x N states x 4 bytes; then the per-block dB / dC partial sums:
+    # (padded channels / block channels) planes x B x L x 2 N x 4 bytes; each rounded up
+    # to 256 bytes
+    up = lambda v: (v + 255) // 256 * 256
+
+    def want(B, L, D, N):
+        cpb = 4 * (32 // (N // 4))
+        dpad = -(-D // cpb) * cpb
+        return up(B * dpad * -(-L // 8) * N * 4) + up((dpad // cpb) * B * L * 2 * N * 4)
+    assert lib.sscan_backward_workspace_bytes(8, 2048, 1536, 16) == 8 * 1536 * 256 * 16 * 4 + 48 * 8 * 2048 * 32 * 4
+    assert lib.sscan_backward_workspace_bytes(2, 37, 70, 16) == 2 * 96 * 5 * 16 * 4 + 3 * 2 * 37 * 32 * 4
+    for shape in ((2, 37, 70, 32), (2, 37, 70, 64), (3, 1, 5, 16), (1, 1000, 4096, 64)):
+        assert lib.sscan_backward_workspace_bytes(*shape) == want(*shape)
     assert lib.sscan_backward_workspace_bytes(2, 37, 70, 24) == 0
     assert lib.sscan_backward_workspace_bytes(2, 0, 70, 16) == 0
 
