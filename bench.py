@@ -277,15 +277,17 @@ def run_ours(args, rank, world, local_rank):
     with ClockSampler(local_rank) as clk:
         t_start.record(stream)
         for i in range(args.steps):
-            ev[i][0].record(stream)
+            if nsets == 1:  # a step of a few microseconds (rotated sets) is not split by events
+                ev[i][0].record(stream)
             step(i)
-            ev[i][1].record(stream)
+            if nsets == 1:
+                ev[i][1].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    kern_ms = [a.elapsed_time(b) for a, b in ev]
     elapsed_ms = t_start.elapsed_time(t_end)
+    kern_ms = [a.elapsed_time(b) for a, b in ev] if nsets == 1 else [elapsed_ms / args.steps] * args.steps
     if plan.status(stream) != S.OK:
         raise RuntimeError("device status word reported an error in the timed region")
 
@@ -358,7 +360,8 @@ def run_ours(args, rank, world, local_rank):
                          "sample": sample},
     }
     if args.per_config:
-        others = [n for n in W.ORDER[1:] + ["decode_b256_f32"] if n != args.workload]
+        others = [n for n in W.ORDER[1:] + ["mamba130m_fused_f32", "mamba1p4b_fused_bf16", "decode_b256_f32"]
+                  if n != args.workload]
         out["per_config"] = time_other_configs(others, dev, stream, sm_max, hbm_peak)
         for name, sw in W.SSD_WORKLOADS.items():
             if name == "ssd_small":
@@ -423,12 +426,18 @@ def time_other_configs(names, dev, stream, sm_max, hbm_peak, launches: int = 20,
             for i in range(max(warmup, nsets)):
                 step(i)
             ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(launches)]
+                  for _ in range(launches if nsets == 1 else 1)]
             torch.cuda.synchronize(dev)
-            for i, (a, b) in enumerate(ev):
-                a.record(stream)
-                step(i)
-                b.record(stream)
+            if nsets == 1:  # events around every launch
+                for i, (a, b) in enumerate(ev):
+                    a.record(stream)
+                    step(i)
+                    b.record(stream)
+            else:  # steps of a few microseconds: back to back, one pair of events
+                ev[0][0].record(stream)
+                for i in range(launches):
+                    step(i)
+                ev[0][1].record(stream)
             torch.cuda.synchronize(dev)
             if plan.status(stream) != S.OK:
                 raise RuntimeError("device status word reported an error")
@@ -551,6 +560,7 @@ def ssd_roofline(w, kms, hbm_peak, peaks):
     tfl = w.flops() / (kms / 1e3) / 1e12
     bf16 = peaks.get("bf16_tflops", 1590.0)
     return {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+            "traffic": measured_traffic(w.name),
             "kernel": "ssd_forward_kernel", "tensor": {"achieved_tflops": tfl, "peak_tflops": bf16,
                                                        "frac": tfl / bf16,
                                                        "flops_per_step": w.flops()}}

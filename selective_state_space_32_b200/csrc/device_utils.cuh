@@ -56,6 +56,8 @@ __device__ __forceinline__ f2 add2(f2 a, f2 b) {
     return r;
 }
 __device__ __forceinline__ f2 splat2(float v) { return pack2(v, v); }
+// -a for a pair (the two sign bits flipped: integer operations, no FP pipe)
+__device__ __forceinline__ f2 neg2(f2 a) { return a ^ 0x8000000080000000ull; }
 
 // 2^x on the MUFU pipe (ex2.approx; results below 2^-126 flush to zero)
 __device__ __forceinline__ float ex2(float x) {
@@ -114,6 +116,22 @@ __device__ __forceinline__ f2 zoh_coef_pair(f2 dd, f2 e, f2 ia, f2 nia, f2 abar)
     unpack2(big, g0, g1);
     constexpr float kLim = 0.18033688011112042f;  // 1/8 / ln 2
     return pack2(fabsf(e0) <= kLim ? s0 : g0, fabsf(e1) <= kLim ? s1 : g1);
+}
+
+// The ZOH coefficient to the precision of bf16 I/O, in one packed operation and a
+// select: d (the z -> 0 limit: relative error |phi(z) - 1| <= |z|/2) when
+// |z| <= 2^-10.5, abar*(1/A) - 1/A beyond (relative error of abar - 1 about
+// 2^-22 / |z|); both below 3.5e-4 relative, against the 2^-9 rounding of a bf16
+// output and the bf16 tolerance of 5e-3 relative L2.  (A = 0 takes the first
+// form: e = 0 there, and ia is not finite.)
+__device__ __forceinline__ f2 zoh_coef_pair_bf16(f2 dd, f2 e, f2 ia, f2 nia, f2 abar) {
+    const f2 big = fma2(abar, ia, nia);
+    float e0, e1, d0, d1, g0, g1;
+    unpack2(e, e0, e1);
+    unpack2(dd, d0, d1);
+    unpack2(big, g0, g1);
+    constexpr float kLim = 9.9606e-4f;  // 2^-10.5 / ln 2
+    return pack2(fabsf(e0) <= kLim ? d0 : g0, fabsf(e1) <= kLim ? d1 : g1);
 }
 
 // softplus(s) = log(1 + e^s) for the fused prologue.  s itself above 20 (the

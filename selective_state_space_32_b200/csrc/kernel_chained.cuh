@@ -131,8 +131,9 @@ struct ChainedCfg {
 // Independent of the state, so a group of tokens is discretized ahead of the
 // (sequential) state updates and the MUFU latency overlaps them.  PAR is the
 // token's parity; it selects which pairs take 2^x on the FMA pipe (a quarter
-// of all pairs across two tokens).
-template <int NP, bool ZOH, bool POLY, int PAR>
+// of all pairs across two tokens).  COARSE (bf16 I/O) takes the ZOH coefficient
+// to bf16 precision (zoh_coef_pair_bf16).
+template <int NP, bool ZOH, bool POLY, int PAR, bool COARSE = false>
 __device__ __forceinline__ void discretize(f2 (&ab)[NP], f2 (&bu)[NP], const f2 (&A2)[NP], const f2 (&nA)[NP],
                                            const f2 (&iA)[NP], float cap, float x, float dl,
                                            const float *Bs) {
@@ -159,7 +160,9 @@ __device__ __forceinline__ void discretize(f2 (&ab)[NP], f2 (&bu)[NP], const f2 
                 unpack2(e, e0, e1);
                 ab[p] = pack2(ex2(e0), ex2(e1));
             }
-            if (ZOH)
+            if (ZOH && COARSE)  // -1/A from 1/A by its sign bits: no -1/A registers to keep
+                bu[p] = mul2(zoh_coef_pair_bf16(dd, e, iA[p], neg2(iA[p]), ab[p]), mul2(bp, xx));
+            else if (ZOH)
                 bu[p] = mul2(zoh_coef_pair(dd, e, iA[p], nA[p], ab[p]), mul2(bp, xx));
             else
                 bu[p] = mul2(bp, du2);
@@ -862,9 +865,9 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
                         dmin = fminf(dmin, dl);
                     }
                     if (q & 1)
-                        discretize<NP, ZOH, POLY, 1>(ab[q], bu[q], A2, A1, iA, cap, x, dl, Bs + (j0 + q) * RS + gofs);
+                        discretize<NP, ZOH, POLY, 1, sizeof(IO) == 2>(ab[q], bu[q], A2, A1, iA, cap, x, dl, Bs + (j0 + q) * RS + gofs);
                     else
-                        discretize<NP, ZOH, POLY, 0>(ab[q], bu[q], A2, A1, iA, cap, x, dl, Bs + (j0 + q) * RS + gofs);
+                        discretize<NP, ZOH, POLY, 0, sizeof(IO) == 2>(ab[q], bu[q], A2, A1, iA, cap, x, dl, Bs + (j0 + q) * RS + gofs);
                 }
                 float yv[G];
 #pragma unroll
@@ -904,7 +907,7 @@ sscan_chained_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_cons
                     ssum += dl;
                     dmin = fminf(dmin, dl);
                 }
-                discretize<NP, ZOH, POLY, 0>(ab, bu, A2, A1, iA, cap, x, dl, Bs + j * RS + gofs);
+                discretize<NP, ZOH, POLY, 0, sizeof(IO) == 2>(ab, bu, A2, A1, iA, cap, x, dl, Bs + j * RS + gofs);
                 float yv = advance<NP>(h, ab, bu, Cs + j * RS + gofs);
 #pragma unroll
                 for (int o = 1; o < LPC; o <<= 1) yv += __shfl_xor_sync(0xffffffffu, yv, o);
