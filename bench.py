@@ -192,6 +192,24 @@ def workload_config(w, world: int) -> dict:
                    f"used in turn, one per step (as the layers of a model), steps back to back; no flush")}
 
 
+def graph_of_steps(step, count: int, stream, dev):
+    """A CUDA graph of ``count`` calls ``step(i, s)`` captured on a side stream, for steps
+    of a few microseconds whose Python launch cost would otherwise set the pace; None if
+    the capture fails.  Only for schedules without launch epochs (decode, step)."""
+    import torch
+    try:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            for i in range(count):
+                step(i, side)
+        stream.wait_stream(side)
+        return g
+    except Exception:
+        return None
+
+
 def rotating_sets(w) -> int:
     """Distinct input/state sets a workload whose working set fits in L2 is timed over
     (one per step, in turn), so that together they exceed L2 three times over."""
@@ -255,10 +273,10 @@ def run_ours(args, rank, world, local_rank):
     sets = [(din, y, hf)] + [({k: (None if v is None else v.clone()) for k, v in din.items()},
                               torch.empty_like(y), torch.empty_like(hf)) for _ in range(nsets - 1)]
 
-    def step(i=0):
+    def step(i=0, st=None):
         d, yy, hh = sets[i % nsets]
         plan.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"],
-                     y=yy, h_final=hh, workspace=ws, stream=stream,
+                     y=yy, h_final=hh, workspace=ws, stream=st or stream,
                      delta_bias=d["delta_bias"], z=d["z"])
 
     for i in range(max(args.warmup, nsets)):
@@ -266,6 +284,13 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     if plan.status(stream) != S.OK:
         raise RuntimeError("device status word reported an error during warm-up")
+    # steps of a few microseconds (rotated sets; no launch epochs) replay as one CUDA graph
+    graph = (graph_of_steps(step, args.steps, stream, dev)
+             if nsets > 1 and plan.describe().startswith(("kernel=decode", "kernel=step")) else None)
+    if graph is not None:
+        with torch.cuda.stream(stream):
+            graph.replay()  # a warm-up replay
+        torch.cuda.synchronize(dev)
 
     # ---- timed region: K steps, events around every launch (kernel time) ----
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -276,18 +301,24 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     with ClockSampler(local_rank) as clk:
         t_start.record(stream)
-        for i in range(args.steps):
-            if nsets == 1:  # a step of a few microseconds (rotated sets) is not split by events
-                ev[i][0].record(stream)
-            step(i)
-            if nsets == 1:
-                ev[i][1].record(stream)
+        if graph is not None:
+            with torch.cuda.stream(stream):
+                graph.replay()
+        else:
+            for i in range(args.steps):
+                if nsets == 1:  # a step of a few microseconds (rotated sets) is not split by events
+                    ev[i][0].record(stream)
+                step(i)
+                if nsets == 1:
+                    ev[i][1].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
     kern_ms = [a.elapsed_time(b) for a, b in ev] if nsets == 1 else [elapsed_ms / args.steps] * args.steps
+    launch_mode = ("one CUDA graph of the K steps" if graph is not None else
+                   "direct launches, back to back" if nsets > 1 else "direct launches, events around each")
     if plan.status(stream) != S.OK:
         raise RuntimeError("device status word reported an error in the timed region")
 
@@ -337,6 +368,7 @@ def run_ours(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": workload_config(w, world),
+        "timing": launch_mode,
         "roofline": ({"bound": "alu", "achieved": upd_rate, "peak": alu_peak,
                       "unit": "Gupdates/s", "frac": upd_rate / alu_peak, "traffic": traffic,
                       "kernel": kernel_name, "schedule": plan.describe(),
@@ -419,12 +451,17 @@ def time_other_configs(names, dev, stream, sm_max, hbm_peak, launches: int = 20,
             sets = [(d, y, hf)] + [({k: (None if v is None else v.clone()) for k, v in d.items()},
                                     torch.empty_like(y), torch.empty_like(hf)) for _ in range(nsets - 1)]
 
-            def step(i=0):
+            def step(i=0, st=None):
                 dd, yy, hh = sets[i % nsets]
                 plan.forward(dd["u"], dd["delta"], dd["A"], dd["B"], dd["C"], dd["h0"], y=yy, h_final=hh,
-                             workspace=ws, stream=stream, delta_bias=dd["delta_bias"], z=dd["z"])
+                             workspace=ws, stream=st or stream, delta_bias=dd["delta_bias"], z=dd["z"])
             for i in range(max(warmup, nsets)):
                 step(i)
+            graph = (graph_of_steps(step, launches, stream, dev)
+                     if nsets > 1 and plan.describe().startswith(("kernel=decode", "kernel=step")) else None)
+            if graph is not None:
+                with torch.cuda.stream(stream):
+                    graph.replay()
             ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for _ in range(launches if nsets == 1 else 1)]
             torch.cuda.synchronize(dev)
@@ -433,10 +470,14 @@ def time_other_configs(names, dev, stream, sm_max, hbm_peak, launches: int = 20,
                     a.record(stream)
                     step(i)
                     b.record(stream)
-            else:  # steps of a few microseconds: back to back, one pair of events
+            else:  # steps of a few microseconds: back to back (one CUDA graph), one pair of events
                 ev[0][0].record(stream)
-                for i in range(launches):
-                    step(i)
+                if graph is not None:
+                    with torch.cuda.stream(stream):
+                        graph.replay()
+                else:
+                    for i in range(launches):
+                        step(i)
                 ev[0][1].record(stream)
             torch.cuda.synchronize(dev)
             if plan.status(stream) != S.OK:
@@ -449,9 +490,11 @@ def time_other_configs(names, dev, stream, sm_max, hbm_peak, launches: int = 20,
                          "mufu_only_frac": upd / (16.0 * SM_COUNT * sm_max * 1e6 / 1e9),
                          "launches": launches, "schedule": plan.describe(),
                          "l2": (f"{nsets} input/state sets used in turn (working set below L2)" if nsets > 1
-                                else "inputs larger than L2; no flush")}
+                                else "inputs larger than L2; no flush"),
+                         "launch": ("one CUDA graph of the launches" if graph is not None else
+                                    "direct launches" if nsets > 1 else "direct launches, events around each")}
             plan.close()
-            del d, y, hf, ws, sets
+            del d, y, hf, ws, sets, graph
             torch.cuda.empty_cache()
         except Exception as e:  # reported, never fatal for the headline line
             out[name] = {"error": str(e)[:200]}

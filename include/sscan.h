@@ -38,6 +38,13 @@
  * device can see (a bounded wait that gave up) are latched in the plan's
  * status word and read back with sscan_get_status.
  *
+ * CUDA graphs.  A launch of the chained schedule (sscan_plan_describe says
+ * "kernel=chained") tags its carry flags with a tag the host picks per call,
+ * so a graph that captured it would replay the same tag and could read a
+ * carried state left by an earlier replay: do not replay such calls from a
+ * graph.  The decode, step and generic schedules keep no state between
+ * launches and may be captured.
+ *
  * Aliasing.  y must not overlap any input.  h_final may be the same buffer
  * as h0 (each state row is read before it is written, by the same thread).
  *
