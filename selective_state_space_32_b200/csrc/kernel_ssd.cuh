@@ -425,12 +425,42 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
         };
         const float *dtp = prm.dt + int64_t(b) * L * prm.H + h;
         float dt_next = t < L ? __ldg(dtp + int64_t(t) * prm.H) : 0.0f;
+        // y of block c: P X + 2^cs (C h_in), rows inside the sequence only (warpgroup P, after
+        // forming the next block's P; its TMEM reads end before YFREE lets MMAs 2, 3 reuse them)
+        auto emit_y = [&](int c, float cs) {
+            ok = wait_warp(BAR_YREADY, c & 1);
+            if (!ok) return;
+            tc_fence_after();
+            const float e = ex2(cs);
+            uint32_t o[2][16];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t y1[32], y2[32];
+                tmem_ld32(lane_base + kColY1 + 32 * half, y1);
+                tmem_ld32(lane_base + kColY2 + 32 * half, y2);
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    o[half][j] = pack_bf16(fmaf(e, __uint_as_float(y2[2 * j]), __uint_as_float(y1[2 * j])),
+                                           fmaf(e, __uint_as_float(y2[2 * j + 1]), __uint_as_float(y1[2 * j + 1])));
+            }
+            tc_fence_before();
+            mbar_arrive(&bars[BAR_YFREE]);
+            const int64_t tok = int64_t(c) * kQ + t;
+            if (tok < L) {
+                uint4 *d4 = reinterpret_cast<uint4 *>(prm.y + ((int64_t(b) * L + tok) * prm.H + h) * kP);
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    d4[q] = make_uint4(o[q >> 2][4 * (q & 3)], o[q >> 2][4 * (q & 3) + 1],
+                                       o[q >> 2][4 * (q & 3) + 2], o[q >> 2][4 * (q & 3) + 3]);
+            }
+        };
 
         if (is_p) {
             // ============================================ warpgroup P
             float *s_cs = reinterpret_cast<float *>(sm + kOffCs);
             float *s_dt = reinterpret_cast<float *>(sm + kOffDt);
             float *s_colf = reinterpret_cast<float *>(sm + kOffColf);
+            float cs_prev = 0.0f;
             for (int c = 0; c < nb; ++c) {
                 const int s = c & 1;
                 const uint32_t ps = (c >> 1) & 1;
@@ -491,7 +521,10 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                     tc_fence_before();
                     mbar_arrive(&bars[BAR_PREADY + s]);
                 }
+                if (ok && c > 0) emit_y(c - 1, cs_prev);
+                cs_prev = cs;
             }
+            if (ok && nb > 0) emit_y(nb - 1, cs_prev);
         } else {
             // ============================================ warpgroup Y
             float hs[kP];  // state row n = t, fp32
@@ -521,37 +554,10 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
             };
             write_h(0);
             mbar_arrive(&bars[BAR_HREADY]);
-            // y of block c: P X + 2^cs (C h_in), rows inside the sequence only
-            auto emit_y = [&](int c, float cs) {
-                ok = wait_warp(BAR_YREADY, c & 1);
-                if (!ok) return;
-                tc_fence_after();
-                const float e = ex2(cs);
-                uint32_t o[2][16];
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t y1[32], y2[32];
-                    tmem_ld32(lane_base + kColY1 + 32 * half, y1);
-                    tmem_ld32(lane_base + kColY2 + 32 * half, y2);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        o[half][j] = pack_bf16(fmaf(e, __uint_as_float(y2[2 * j]), __uint_as_float(y1[2 * j])),
-                                               fmaf(e, __uint_as_float(y2[2 * j + 1]), __uint_as_float(y1[2 * j + 1])));
-                }
-                tc_fence_before();
-                mbar_arrive(&bars[BAR_YFREE]);
-                const int64_t tok = int64_t(c) * kQ + t;
-                if (tok < L) {
-                    uint4 *d4 = reinterpret_cast<uint4 *>(prm.y + ((int64_t(b) * L + tok) * prm.H + h) * kP);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        d4[q] = make_uint4(o[q >> 2][4 * (q & 3)], o[q >> 2][4 * (q & 3) + 1],
-                                           o[q >> 2][4 * (q & 3) + 2], o[q >> 2][4 * (q & 3) + 3]);
-                }
-            };
-            // Per block c: w X of block c first (MMA 4 of block c can start at once),
-            // then y of block c-1 (while MMA 4 runs), then the state passing of block c.
-            float cs_prev = 0.0f;
+            // Per block c: w X of block c first (MMA 4 of block c can start at once), then
+            // the state passing of block c (warpgroup P emits y).  The h_in buffer written
+            // for block c+1 was read by MMA 3 of block c-1: done once MMA 4 of block c is,
+            // as a commit tracks every earlier MMA of the issuing thread.
             for (int c = 0; c < nb; ++c) {
                 const int s = c & 1;
                 const uint32_t ps = (c >> 1) & 1, pc = c & 1;
@@ -579,10 +585,8 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                     fence_proxy_async_smem();
                     mbar_arrive(&bars[BAR_WXREADY]);
                 }
-                if (c > 0) emit_y(c - 1, cs_prev);
-                cs_prev = cs;
                 // ---- state passing: h = 2^cs_end h + S_blk (row n = t); then h_in of block c+1,
-                // into the buffer MMA 3 of block c-1 read (done: its y was just emitted)
+                // into the buffer MMA 3 of block c-1 read
                 ok = wait_warp(BAR_M4, pc);
                 if (ok) {
                     tc_fence_after();
@@ -601,7 +605,6 @@ ssd_forward_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_consta
                     mbar_arrive(&bars[BAR_HREADY]);
                 }
             }
-            if (nb > 0) emit_y(nb - 1, cs_prev);
             if (ok && prm.h_final) {
                 float *dst = prm.h_final + ((int64_t(b) * prm.H + h) * kN + t) * kP;
 #pragma unroll
