@@ -65,14 +65,23 @@ def strip_comments(src: str) -> str:
     return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
 
 
-def kernel_sources_hash(read=None) -> str:
-    """sha256 over the code (comments stripped) of the forward kernels and their host
-    code (the backward's own files excluded), to tell whether a stored ncu figure is
-    current.  ``read(name)`` returns a file's text (default: the working tree)."""
+SSD_SOURCES = ("kernel_ssd.cuh", "ssd.cu")
+
+
+def kernel_sources_hash(read=None, family: str = "scan") -> str:
+    """sha256 over the code (comments stripped) of one family of forward kernels and
+    their host code, to tell whether a stored ncu figure is current: "scan" (the
+    selective-scan kernels: every CUDA source but the backward's and the SSD form's)
+    or "ssd" (the SSD form's sources and the shared device utilities).  ``read(name)``
+    returns a file's text (default: the working tree)."""
     import hashlib
     h = hashlib.sha256()
     cdir = os.path.join(ROOT, "selective_state_space_32_b200", "csrc")
     names = [n for n in sorted(os.listdir(cdir)) if n.endswith((".cu", ".cuh")) and "backward" not in n]
+    if family == "ssd":
+        names = [n for n in names if n in SSD_SOURCES or n == "device_utils.cuh"]
+    else:
+        names = [n for n in names if n not in SSD_SOURCES]
     for name in names:
         if read is None:
             with open(os.path.join(cdir, name), encoding="utf-8") as f:
@@ -89,7 +98,8 @@ def measured_traffic(workload: str):
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             t = json.load(f)
-        if t.get("kernel_sources_sha256") != kernel_sources_hash():
+        family = "ssd" if workload in W.SSD_WORKLOADS else "scan"
+        if t.get("kernel_sources_sha256", {}).get(family) != kernel_sources_hash(family=family):
             return None
         v = t["workloads"][workload]["dram_bytes_per_launch"]
         return float(v)
