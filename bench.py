@@ -66,18 +66,21 @@ def strip_comments(src: str) -> str:
 
 
 SSD_SOURCES = ("kernel_ssd.cuh", "ssd.cu")
+HOST_ONLY_SOURCES = ("host_pipe.cu",)  # copies and sub-plan calls: no kernel launch of its own
 
 
 def kernel_sources_hash(read=None, family: str = "scan") -> str:
     """sha256 over the code (comments stripped) of one family of forward kernels and
     their host code, to tell whether a stored ncu figure is current: "scan" (the
     selective-scan kernels: every CUDA source but the backward's and the SSD form's)
-    or "ssd" (the SSD form's sources and the shared device utilities).  ``read(name)``
-    returns a file's text (default: the working tree)."""
+    or "ssd" (the SSD form's sources and the shared device utilities); the host-buffer
+    pipeline's file launches nothing itself and is in neither.  ``read(name)`` returns a
+    file's text (default: the working tree)."""
     import hashlib
     h = hashlib.sha256()
     cdir = os.path.join(ROOT, "selective_state_space_32_b200", "csrc")
-    names = [n for n in sorted(os.listdir(cdir)) if n.endswith((".cu", ".cuh")) and "backward" not in n]
+    names = [n for n in sorted(os.listdir(cdir))
+             if n.endswith((".cu", ".cuh")) and "backward" not in n and n not in HOST_ONLY_SOURCES]
     if family == "ssd":
         names = [n for n in names if n in SSD_SOURCES or n == "device_utils.cuh"]
     else:

@@ -150,8 +150,9 @@ SSCAN_API int sscan_forward_gated(sscan_plan_t plan, const void *u, const void *
 /* Bytes of device workspace sscan_forward_host needs for this plan (always
  * > 0; 0 only when plan is NULL or host memory ran out).  The workspace must
  * be 256-byte aligned.  It holds two buffer slots of one piece's inputs and
- * output (the slot for z is reserved whether or not a call passes z), A, the
- * bias, the carried state and the pieces' scan workspaces. */
+ * outputs (the slot for z is reserved whether or not a call passes z), A, the
+ * bias, the state (carried, or the piece's rows') and the pieces' scan
+ * workspaces. */
 SSCAN_API size_t sscan_host_workspace_bytes(sscan_plan_t plan);
 
 /* sscan_forward_gated on HOST buffers: the arguments and their layouts are
@@ -159,14 +160,16 @@ SSCAN_API size_t sscan_host_workspace_bytes(sscan_plan_t plan);
  * delta_bias, z, y and h_final live in host memory (page-locked memory lets
  * the copies overlap; any memory cudaMemcpy accepts works), need no
  * alignment, and `workspace` is device memory of
- * sscan_host_workspace_bytes(plan) bytes.  The call cuts the sequence into
- * at most 8 pieces along L (multiples of 64 tokens, the last one shorter)
- * and, for each piece, copies its inputs to the device, scans it (the state
- * carried between pieces in the workspace: a piece's h_final is the next
- * piece's h0, exactly the split-call resume of sscan_forward) and copies its
- * y back; with two buffer slots, the host-to-device copy of piece k+1 and the
- * device-to-host copy of piece k-1 run while piece k is scanned.  The
- * results equal one sscan_forward_gated call on the whole sequence.
+ * sscan_host_workspace_bytes(plan) bytes.  The call cuts the problem into
+ * pieces: at most 8 along L (multiples of 64 tokens, the last one shorter; the
+ * state carried between pieces in the workspace: a piece's h_final is the
+ * next piece's h0, exactly the split-call resume of sscan_forward) or, when L
+ * is below 512 tokens and B >= 2, 2 along the independent batch rows.  For each
+ * piece it copies the inputs to the device, scans and copies y (and, along B,
+ * the rows' h_final) back; with two buffer slots, the host-to-device copy of
+ * piece k+1 and the device-to-host copy of piece k-1 run while piece k is
+ * scanned.  The results equal one sscan_forward_gated call on the whole
+ * problem.
  * Streams: the work starts after what is already queued on `stream`, and
  * `stream` waits for all of it (copies included) before anything queued
  * later, so synchronising `stream` makes y and h_final readable; the call

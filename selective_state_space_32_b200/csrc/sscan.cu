@@ -1,6 +1,7 @@
 // sscan.cu -- host side of the B200 (sm_100a) selective-scan forward library:
 // plans, schedule choice, TMA descriptors, launches, and the C ABI declared in
-// include/sscan.h.
+// include/sscan.h (the host-buffer entry point is in host_pipe.cu, the
+// backward in sscan_backward.cu, the SSD form in ssd.cu).
 //
 // What is computed ("tm_ssm_selective" (Transformer Math page on selective
 // SSMs), section "Discretization becomes a per-token operation"; the
@@ -38,6 +39,7 @@
 #include "kernel_decode.cuh"
 #include "kernel_generic.cuh"
 #include "kernel_step.cuh"
+#include "plan.cuh"
 #include "sscan.h"
 
 #define SSCAN_VERSION 200  // 0.2.0
@@ -45,8 +47,6 @@
 using namespace sscan;
 
 namespace {
-
-enum Mode { kGeneric = 0, kChained = 1, kStep = 2 };
 
 // Chained-kernel shapes compiled into the library.  NL states per lane, T
 // tokens per pipeline stage, STAGES stages per warp, WPC warps per block.
@@ -100,40 +100,6 @@ int chained_smem_bytes(const KCfg &k, int es) {
 }
 
 }  // namespace
-
-struct HostPipe;
-
-struct sscan_plan {
-    int64_t B, L, D, N;
-    int dtype;
-    uint32_t flags;
-    int device;
-    int sm_count;
-    int *d_status;
-    Mode mode;
-    // chained kernel
-    int cfg;           // index into kChainedCfgs
-    bool poly;         // part of the exponents on the FMA pipe
-    bool split;        // chains cut into concurrently scanned pieces + look-back fix-up
-    bool drop_publish; // failure-detection tests: heads skip publishing (see read_tune)
-    int64_t chains_per_row, chains, workers, seg, max_pieces;
-    int64_t seg_shift;  // segment re-balancing unit x (see ChainedParams::seg_shift)
-    size_t flag_off, flag_bytes;                // flags cleared on a workspace's first use
-    size_t rec_s_off, rec_mono_off, ws_bytes;   // split-mode record arrays (rec_h at 0)
-    size_t sink_off;                            // y sink of lanes past the last channel
-    const void *last_ws;  // workspace whose flags were last cleared
-    // tensor-map cache
-    const void *tm_ptr[5];
-    CUtensorMap tm[5];  // u, delta, B, C, gate z (z: fused calls with a gate; else a copy of u's)
-    bool tm_valid;
-    // generic kernel
-    int g_nl, g_lpc;
-    // decode kernel (L = 1 with a state)
-    bool decode;
-    int dec_grid;  // persistent grid, set on the first launch
-    // sscan_forward_host: piece schedule, sub-plans and streams (made on first use)
-    HostPipe *host;
-};
 
 namespace {
 
@@ -512,6 +478,8 @@ int launch_chained(sscan_plan *p, const void *u, const void *dl, const float *A,
 
 }  // namespace
 
+void sscan_choose_schedule(sscan_plan *p) { choose_schedule(p); }
+
 // No tokens: the final state is the initial one (zero without h0).
 int step_empty(const sscan_plan *p, const float *h0, float *hf, cudaStream_t s) {
     if (hf == nullptr || hf == h0) return SSCAN_OK;
@@ -519,140 +487,6 @@ int step_empty(const sscan_plan *p, const float *h0, float *hf, cudaStream_t s) 
     const cudaError_t e = h0 ? cudaMemcpyAsync(hf, h0, bytes, cudaMemcpyDeviceToDevice, s) : cudaMemsetAsync(hf, 0, bytes, s);
     return e == cudaSuccess ? SSCAN_OK : SSCAN_ERR_CUDA;
 }
-
-// ------------------------------------------------ forward on host buffers
-
-// sscan_forward_host cuts the sequence into pieces along L and runs them as a
-// three-stage pipeline: copy a piece's inputs in (stream s_in), scan it (the
-// caller's stream), copy its y out (stream s_out).  Two buffer slots let the
-// copies of the neighbouring pieces run while a piece is scanned; the state
-// is carried from piece to piece in one device buffer (each piece's h_final is
-// the next one's h0, the split-call resume the scan supports exactly).
-struct HostPipe {
-    int64_t piece_L = 0, pieces = 0;
-    sscan_plan *sub[2] = {};  // plans for a full piece and for a shorter last piece
-    size_t off_ws[2] = {}, off_A = 0, off_bias = 0, off_h = 0, bytes = 0;
-    size_t off_slot[2][6] = {};  // per slot: u, delta, z, B, C, y
-    size_t max_pitch = 0;
-    cudaStream_t s_in = nullptr, s_out = nullptr;
-    cudaEvent_t ev_join = nullptr, ev_in[2] = {}, ev_comp[2] = {}, ev_out[2] = {};
-    bool streams_ready = false;
-};
-
-namespace {
-
-constexpr int64_t kHostPieces = 8;      // a call is cut into at most this many pieces
-constexpr int64_t kHostPieceAlign = 64; // piece lengths are multiples of this many tokens
-
-sscan_plan *host_sub_plan(const sscan_plan *p, int64_t L) {
-    sscan_plan *q = new (std::nothrow) sscan_plan();
-    if (!q) return nullptr;
-    q->B = p->B;
-    q->L = L;
-    q->D = p->D;
-    q->N = p->N;
-    q->dtype = p->dtype;
-    q->flags = p->flags;
-    q->device = p->device;
-    q->sm_count = p->sm_count;
-    q->d_status = p->d_status;  // shared: sscan_get_status on the parent sees the pieces' waits
-    q->last_ws = nullptr;
-    q->tm_valid = false;
-    q->ws_bytes = 0;
-    q->host = nullptr;
-    choose_schedule(q);
-    return q;
-}
-
-void host_pipe_free(HostPipe *h) {
-    if (!h) return;
-    if (h->s_in) cudaStreamDestroy(h->s_in);
-    if (h->s_out) cudaStreamDestroy(h->s_out);
-    cudaEvent_t evs[] = {h->ev_join, h->ev_in[0], h->ev_in[1], h->ev_comp[0], h->ev_comp[1],
-                         h->ev_out[0], h->ev_out[1]};
-    for (cudaEvent_t e : evs)
-        if (e) cudaEventDestroy(e);
-    delete h->sub[0];  // sub-plans own no device memory (the status word is the parent's)
-    delete h->sub[1];
-    delete h;
-}
-
-// Piece schedule and device-workspace layout of sscan_forward_host (host
-// arithmetic only; made once per plan).
-HostPipe *host_layout(sscan_plan *p) {
-    if (p->host) return p->host;
-    HostPipe *h = new (std::nothrow) HostPipe();
-    if (!h) return nullptr;
-    const int64_t L = p->L;
-    int64_t lp = ceil_div(ceil_div(L, kHostPieces), kHostPieceAlign) * kHostPieceAlign;
-    if (lp > L) lp = L;
-    h->piece_L = lp;
-    h->pieces = L == 0 ? 1 : ceil_div(L, lp);
-    const int64_t last = L - (h->pieces - 1) * lp;
-    h->sub[0] = host_sub_plan(p, lp);
-    h->sub[1] = last != lp ? host_sub_plan(p, last) : nullptr;
-    if (!h->sub[0] || (last != lp && !h->sub[1])) {
-        host_pipe_free(h);
-        return nullptr;
-    }
-    const size_t es = p->dtype == SSCAN_F32 ? 4 : 2;
-    size_t o = 0;
-    auto take = [&o](size_t bytes) {
-        const size_t at = o;
-        o = align_up(o + bytes, 256);
-        return at;
-    };
-    h->off_ws[0] = take(h->sub[0]->ws_bytes);
-    h->off_ws[1] = take(h->sub[1] ? h->sub[1]->ws_bytes : 0);
-    h->off_A = take(static_cast<size_t>(p->D * p->N) * 4);
-    h->off_bias = take(static_cast<size_t>(p->D) * 4);
-    h->off_h = take(static_cast<size_t>(p->B * p->D * p->N) * 4);
-    const size_t bld = static_cast<size_t>(p->B * lp * p->D) * es;
-    const size_t bln = static_cast<size_t>(p->B * lp * p->N) * es;
-    for (int j = 0; j < 2; ++j) {
-        const size_t sizes[6] = {bld, bld, bld, bln, bln, bld};
-        for (int i = 0; i < 6; ++i) h->off_slot[j][i] = take(sizes[i]);
-    }
-    h->bytes = o;
-    p->host = h;
-    return h;
-}
-
-int host_streams(HostPipe *h, int dev) {
-    if (h->streams_ready) return SSCAN_OK;
-    int mp = 0;
-    bool ok = cudaDeviceGetAttribute(&mp, cudaDevAttrMaxPitch, dev) == cudaSuccess && mp > 0;
-    h->max_pitch = static_cast<size_t>(mp);
-    if (ok && !h->s_in) ok = cudaStreamCreateWithFlags(&h->s_in, cudaStreamNonBlocking) == cudaSuccess;
-    if (ok && !h->s_out) ok = cudaStreamCreateWithFlags(&h->s_out, cudaStreamNonBlocking) == cudaSuccess;
-    cudaEvent_t *evs[] = {&h->ev_join, &h->ev_in[0], &h->ev_in[1], &h->ev_comp[0], &h->ev_comp[1],
-                          &h->ev_out[0], &h->ev_out[1]};
-    for (cudaEvent_t *e : evs)
-        if (ok && !*e) ok = cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
-    if (!ok) return SSCAN_ERR_CUDA;  // what was made is kept and freed with the plan
-    h->streams_ready = true;
-    return SSCAN_OK;
-}
-
-// `rows` rows of `width` bytes, source rows `spitch` apart, destination rows
-// `dpitch` apart (one 2-D copy; row by row past the device's pitch limit).
-cudaError_t copy_rows(void *dst, size_t dpitch, const void *src, size_t spitch, size_t width,
-                      int64_t rows, size_t max_pitch, cudaStream_t s) {
-    if (width == 0 || rows == 0) return cudaSuccess;
-    if (dpitch == width && spitch == width)
-        return cudaMemcpyAsync(dst, src, width * static_cast<size_t>(rows), cudaMemcpyDefault, s);
-    if (dpitch <= max_pitch && spitch <= max_pitch)
-        return cudaMemcpy2DAsync(dst, dpitch, src, spitch, width, static_cast<size_t>(rows), cudaMemcpyDefault, s);
-    for (int64_t r = 0; r < rows; ++r) {
-        const cudaError_t e = cudaMemcpyAsync(static_cast<char *>(dst) + r * dpitch,
-                                              static_cast<const char *>(src) + r * spitch, width,
-                                              cudaMemcpyDefault, s);
-        if (e != cudaSuccess) return e;
-    }
-    return cudaSuccess;
-}
-
-}  // namespace
 
 // ------------------------------------------------ allocation-free entry point
 
@@ -746,7 +580,7 @@ int sscan_plan_create(sscan_plan_t *plan, int64_t B, int64_t L, int64_t D, int64
 
 void sscan_plan_destroy(sscan_plan_t plan) {
     if (!plan) return;
-    host_pipe_free(plan->host);
+    sscan_host_pipe_free(plan->host);
     if (plan->d_status) cudaFree(plan->d_status);
     delete plan;
 }
@@ -860,111 +694,6 @@ int sscan_forward_gated(sscan_plan_t plan, const void *u, const void *delta, con
         p->dtype == SSCAN_F32 ? launch_generic<float>(p, u, delta, A, B, C, h0, y, h_final, fu, s)
                               : launch_generic<uint16_t>(p, u, delta, A, B, C, h0, y, h_final, fu, s);
     return e == cudaSuccess ? SSCAN_OK : SSCAN_ERR_CUDA;
-}
-
-size_t sscan_host_workspace_bytes(sscan_plan_t plan) {
-    if (!plan) return 0;
-    const HostPipe *h = host_layout(plan);
-    return h ? h->bytes : 0;
-}
-
-int sscan_forward_host(sscan_plan_t plan, const void *u, const void *delta, const float *A,
-                       const void *B, const void *C, const float *h0, const float *delta_bias,
-                       const void *z, void *y, float *h_final, void *workspace, void *stream) {
-    if (!plan) return SSCAN_ERR_INVALID;
-    sscan_plan *p = plan;
-    const size_t es = p->dtype == SSCAN_F32 ? 4 : 2;
-    const size_t n_bld = static_cast<size_t>(p->B * p->L * p->D);
-    const size_t n_bln = static_cast<size_t>(p->B * p->L * p->N);
-    const size_t n_dn = static_cast<size_t>(p->D * p->N);
-    const size_t n_bdn = static_cast<size_t>(p->B * p->D * p->N);
-    if (!A) return SSCAN_ERR_INVALID;
-    if (n_bld && (!u || !delta || !y)) return SSCAN_ERR_INVALID;
-    if (n_bln && (!B || !C)) return SSCAN_ERR_INVALID;
-    // the same aliasing rules as sscan_forward_gated, on the caller's buffers
-    const void *ins[] = {u, delta, A, B, C, delta_bias, z, h0};
-    const size_t insz[] = {n_bld * es, n_bld * es, n_dn * 4, n_bln * es, n_bln * es,
-                           static_cast<size_t>(p->D) * 4, n_bld * es, n_bdn * 4};
-    for (int i = 0; i < 8; ++i) {
-        if (overlaps(y, n_bld * es, ins[i], insz[i])) return SSCAN_ERR_INVALID;
-        if (i < 7 && overlaps(h_final, n_bdn * 4, ins[i], insz[i])) return SSCAN_ERR_INVALID;
-    }
-    if (h0 && h_final && h0 != h_final && overlaps(h_final, n_bdn * 4, h0, n_bdn * 4)) return SSCAN_ERR_INVALID;
-    if (overlaps(h_final, n_bdn * 4, y, n_bld * es)) return SSCAN_ERR_INVALID;
-    HostPipe *h = host_layout(p);
-    if (!h) return SSCAN_ERR_INVALID;
-    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SSCAN_ERR_WORKSPACE;
-    for (int i = 0; i < 8; ++i)
-        if (overlaps(workspace, h->bytes, ins[i], insz[i])) return SSCAN_ERR_WORKSPACE;
-    if (overlaps(workspace, h->bytes, y, n_bld * es) || overlaps(workspace, h->bytes, h_final, n_bdn * 4))
-        return SSCAN_ERR_WORKSPACE;
-    const int src = host_streams(h, p->device);
-    if (src != SSCAN_OK) return src;
-
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    unsigned char *w = static_cast<unsigned char *>(workspace);
-    float *dA = reinterpret_cast<float *>(w + h->off_A);
-    float *dbias = reinterpret_cast<float *>(w + h->off_bias);
-    float *dh = reinterpret_cast<float *>(w + h->off_h);
-    int rc = SSCAN_OK;
-    auto ok = [&rc](cudaError_t e) {
-        if (e != cudaSuccess && rc == SSCAN_OK) rc = SSCAN_ERR_CUDA;
-        return rc == SSCAN_OK;
-    };
-    do {
-        // the internal streams start after the work already queued on `stream`
-        if (!ok(cudaEventRecord(h->ev_join, s)) || !ok(cudaStreamWaitEvent(h->s_in, h->ev_join, 0)) ||
-            !ok(cudaStreamWaitEvent(h->s_out, h->ev_join, 0)))
-            break;
-        if (!ok(cudaMemcpyAsync(dA, A, n_dn * 4, cudaMemcpyDefault, h->s_in))) break;
-        if (delta_bias && !ok(cudaMemcpyAsync(dbias, delta_bias, static_cast<size_t>(p->D) * 4,
-                                              cudaMemcpyDefault, h->s_in)))
-            break;
-        if (h0 && !ok(cudaMemcpyAsync(dh, h0, n_bdn * 4, cudaMemcpyDefault, h->s_in))) break;
-        const size_t pitch_d = static_cast<size_t>(p->L * p->D) * es, pitch_n = static_cast<size_t>(p->L * p->N) * es;
-        for (int64_t k = 0; k < h->pieces && rc == SSCAN_OK; ++k) {
-            const int j = static_cast<int>(k & 1);
-            const int64_t l0 = k * h->piece_L, lk = std::min(h->piece_L, p->L - l0);
-            const int which = lk == h->piece_L ? 0 : 1;
-            sscan_plan *q = h->sub[which];
-            unsigned char *slot[6];
-            for (int i = 0; i < 6; ++i) slot[i] = w + h->off_slot[j][i];
-            const size_t row_d = static_cast<size_t>(lk * p->D) * es, row_n = static_cast<size_t>(lk * p->N) * es;
-            const size_t at_d = static_cast<size_t>(l0 * p->D) * es, at_n = static_cast<size_t>(l0 * p->N) * es;
-            // inputs of piece k into slot j, once the scan of piece k-2 has read it
-            if (k >= 2 && !ok(cudaStreamWaitEvent(h->s_in, h->ev_comp[j], 0))) break;
-            if (!ok(copy_rows(slot[0], row_d, static_cast<const char *>(u) + at_d, pitch_d, row_d, p->B, h->max_pitch, h->s_in)) ||
-                !ok(copy_rows(slot[1], row_d, static_cast<const char *>(delta) + at_d, pitch_d, row_d, p->B, h->max_pitch, h->s_in)) ||
-                (z && !ok(copy_rows(slot[2], row_d, static_cast<const char *>(z) + at_d, pitch_d, row_d, p->B, h->max_pitch, h->s_in))) ||
-                !ok(copy_rows(slot[3], row_n, static_cast<const char *>(B) + at_n, pitch_n, row_n, p->B, h->max_pitch, h->s_in)) ||
-                !ok(copy_rows(slot[4], row_n, static_cast<const char *>(C) + at_n, pitch_n, row_n, p->B, h->max_pitch, h->s_in)) ||
-                !ok(cudaEventRecord(h->ev_in[j], h->s_in)))
-                break;
-            // scan piece k once its inputs are in and slot j's previous y has been copied out
-            if (!ok(cudaStreamWaitEvent(s, h->ev_in[j], 0))) break;
-            if (k >= 2 && !ok(cudaStreamWaitEvent(s, h->ev_out[j], 0))) break;
-            const int frc = sscan_forward_gated(q, slot[0], slot[1], dA, slot[3], slot[4], (k > 0 || h0) ? dh : nullptr,
-                                                delta_bias ? dbias : nullptr, z ? slot[2] : nullptr, slot[5], dh,
-                                                w + h->off_ws[which], s);
-            if (frc != SSCAN_OK) {
-                rc = frc;
-                break;
-            }
-            // y of piece k out of slot j
-            if (!ok(cudaEventRecord(h->ev_comp[j], s)) || !ok(cudaStreamWaitEvent(h->s_out, h->ev_comp[j], 0)) ||
-                !ok(copy_rows(static_cast<char *>(y) + at_d, pitch_d, slot[5], row_d, row_d, p->B, h->max_pitch, h->s_out)) ||
-                !ok(cudaEventRecord(h->ev_out[j], h->s_out)))
-                break;
-        }
-        if (rc == SSCAN_OK && h_final) ok(cudaMemcpyAsync(h_final, dh, n_bdn * 4, cudaMemcpyDefault, h->s_out));
-    } while (false);
-    // `stream` waits for everything queued on the internal streams, on success and on error
-    const bool joined = cudaEventRecord(h->ev_join, h->s_in) == cudaSuccess &&
-                        cudaStreamWaitEvent(s, h->ev_join, 0) == cudaSuccess &&
-                        cudaEventRecord(h->ev_join, h->s_out) == cudaSuccess &&
-                        cudaStreamWaitEvent(s, h->ev_join, 0) == cudaSuccess;
-    if (!joined && rc == SSCAN_OK) rc = SSCAN_ERR_CUDA;
-    return rc;
 }
 
 int sscan_get_status(sscan_plan_t plan, void *stream) {

@@ -211,13 +211,16 @@ def test_split_call_resume_matches_one_call():
 
 
 HOST = [
-    # (B, L, D, N, dtype, h0, zoh, fused): sscan_forward_host, pieces of ceil(L/8) rounded up to 64 tokens
+    # (B, L, D, N, dtype, h0, zoh, fused): sscan_forward_host, pieces of ceil(L/8) rounded up to 64
+    # tokens, or two pieces of batch rows (ceil(B/2) rows, the last one fewer) when L < 512 and B >= 2
     (6, 300, 256, 16, "bf16", True, False, False),   # 5 pieces of 64 + a last piece of 44
     (3, 1000, 96, 32, "f32", True, True, False),     # 8 pieces of 128, the last one 104
     (2, 2048, 64, 16, "f32", False, False, True),    # 8 equal pieces; softplus(delta + bias), silu(z) gate
     (4, 700, 40, 64, "bf16", True, True, True),
-    (5, 1, 300, 16, "f32", True, False, False),      # one token: a single piece
-    (2, 50, 33, 16, "f32", False, True, False),      # shorter than one piece alignment: one piece
+    (5, 1, 300, 16, "f32", True, False, False),      # one token: pieces of 3 and 2 batch rows
+    (2, 50, 33, 16, "f32", False, True, False),      # short: two pieces of one row
+    (11, 100, 64, 16, "bf16", True, True, True),     # short: pieces of 6 and 5 rows; fused
+    (256, 1, 2048, 16, "f32", True, False, False),   # the decode step's shape: two pieces of 128 rows
 ]
 
 
