@@ -118,20 +118,21 @@ __device__ __forceinline__ f2 zoh_coef_pair(f2 dd, f2 e, f2 ia, f2 nia, f2 abar)
     return pack2(fabsf(e0) <= kLim ? s0 : g0, fabsf(e1) <= kLim ? s1 : g1);
 }
 
-// The ZOH coefficient to the precision of bf16 I/O, in one packed operation and a
+// The ZOH coefficient to the precision of bf16 I/O, in two packed operations and a
 // select: d (the z -> 0 limit: relative error |phi(z) - 1| <= |z|/2) when
-// |z| <= 2^-10.5, abar*(1/A) - 1/A beyond (relative error of abar - 1 about
-// 2^-22 / |z|); both below 3.5e-4 relative, against the 2^-9 rounding of a bf16
-// output and the bf16 tolerance of 5e-3 relative L2.  (A = 0 takes the first
-// form: e = 0 there, and ia is not finite.)
-__device__ __forceinline__ f2 zoh_coef_pair_bf16(f2 dd, f2 e, f2 ia, f2 nia, f2 abar) {
-    const f2 big = fma2(abar, ia, nia);
+// |z| <= 2^-10.5, (abar - 1) * (1/A) beyond (abar - 1 is exact for abar in
+// [1/2, 2]; the relative error of abar itself, about 2^-22, becomes 2^-22 / |z|);
+// both below 3.5e-4 relative, against the 2^-9 rounding of a bf16 output and the
+// bf16 tolerance of 5e-3 relative L2.  (A = 0 takes the first form: e = 0 there,
+// and ia is not finite.)
+constexpr float kZohBf16Lim = 9.9606e-4f;  // 2^-10.5 / ln 2: the bound on |e| = |delta A| log2 e
+__device__ __forceinline__ f2 zoh_coef_pair_bf16(f2 dd, f2 e, f2 ia, f2 abar) {
+    const f2 big = mul2(add2(abar, splat2(-1.0f)), ia);
     float e0, e1, d0, d1, g0, g1;
     unpack2(e, e0, e1);
     unpack2(dd, d0, d1);
     unpack2(big, g0, g1);
-    constexpr float kLim = 9.9606e-4f;  // 2^-10.5 / ln 2
-    return pack2(fabsf(e0) <= kLim ? d0 : g0, fabsf(e1) <= kLim ? d1 : g1);
+    return pack2(fabsf(e0) <= kZohBf16Lim ? d0 : g0, fabsf(e1) <= kZohBf16Lim ? d1 : g1);
 }
 
 // softplus(s) = log(1 + e^s) for the fused prologue.  s itself above 20 (the

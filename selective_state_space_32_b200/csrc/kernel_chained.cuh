@@ -160,8 +160,8 @@ __device__ __forceinline__ void discretize(f2 (&ab)[NP], f2 (&bu)[NP], const f2 
                 unpack2(e, e0, e1);
                 ab[p] = pack2(ex2(e0), ex2(e1));
             }
-            if (ZOH && COARSE)  // -1/A from 1/A by its sign bits: no -1/A registers to keep
-                bu[p] = mul2(zoh_coef_pair_bf16(dd, e, iA[p], neg2(iA[p]), ab[p]), mul2(bp, xx));
+            if (ZOH && COARSE)  // (Abar - 1) * (1/A): no -1/A registers to keep
+                bu[p] = mul2(zoh_coef_pair_bf16(dd, e, iA[p], ab[p]), mul2(bp, xx));
             else if (ZOH)
                 bu[p] = mul2(zoh_coef_pair(dd, e, iA[p], nA[p], ab[p]), mul2(bp, xx));
             else

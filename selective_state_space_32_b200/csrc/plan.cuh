@@ -8,7 +8,7 @@
 #include <cstddef>
 #include <cstdint>
 
-enum SscanMode { kGeneric = 0, kChained = 1, kStep = 2 };
+enum SscanMode { kGeneric = 0, kChained = 1, kStep = 2, kTiled = 3 };
 
 struct HostPipe;
 
@@ -21,7 +21,7 @@ struct sscan_plan {
     int *d_status;
     SscanMode mode;
     // chained kernel
-    int cfg;           // index into kChainedCfgs
+    int cfg;           // index into kChainedCfgs (kTiled: into kTiledCfgs)
     bool poly;         // part of the exponents on the FMA pipe
     bool split;        // chains cut into concurrently scanned pieces + look-back fix-up
     bool drop_publish; // failure-detection tests: heads skip publishing (see read_tune)

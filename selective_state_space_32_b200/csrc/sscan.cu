@@ -9,9 +9,12 @@
 //     Abar = exp(delta*A[d,n]);   Bbar u = delta*B[n]*u  (Euler) or
 //     (exp(delta*A)-1)/A*B[n]*u (ZOH);   h = Abar*h + Bbar u;   y = sum_n C[n]*h.
 //
-// Two kernels:
+// Kernels:
 //  * chained (kernel_chained.cuh): persistent, cooperative, one warp per
 //    chain segment, TMA-staged inputs, exactly balanced work per warp;
+//  * tiled (kernel_tiled.cuh): the same recurrence with one block per
+//    block-chain segment, its warps sharing each stage's tiles (shapes whose
+//    per-warp rows are narrower than an L2 fill);
 //  * step (kernel_step.cuh): four states per thread, shaped for the state's
 //    HBM round trip; sequences shorter than the chained kernel's minimum,
 //    the single-token decode step in particular;
@@ -39,6 +42,7 @@
 #include "kernel_decode.cuh"
 #include "kernel_generic.cuh"
 #include "kernel_step.cuh"
+#include "kernel_tiled.cuh"
 #include "plan.cuh"
 #include "sscan.h"
 
@@ -77,6 +81,17 @@ constexpr int kPrefSplitF32[] = {2, 3, 1, 4, 5, 6, 0};
 constexpr int kPrefSplitBF16[] = {0, 2, 3, 1, 4, 5, 6};
 constexpr int kNumCfgs = sizeof(kChainedCfgs) / sizeof(kChainedCfgs[0]);
 
+// Block-tiled shapes (kernel_tiled.cuh): N, NL states per lane, T tokens per
+// stage, STAGES stages per block, WPC consumer warps per block.
+constexpr KCfg kTiledCfgs[] = {
+    {64, 8, 32, 3, 12},  // 0: 48 channels per block, 3 consumer warps per SM sub-partition
+    {64, 8, 16, 4, 16},  // 1: 64 channels per block, 4 per sub-partition
+    {32, 8, 16, 4, 12},  // 2: 96 channels per block
+};
+constexpr int kNumTiledCfgs = sizeof(kTiledCfgs) / sizeof(kTiledCfgs[0]);
+// Shapes the schedule takes without being asked, in order of preference.
+constexpr int kTiledAuto[] = {-1};
+
 std::atomic<uint32_t> g_epoch{1};  // launch tags of the chained kernel (unique per process)
 
 constexpr int kMaxSmem = 227 * 1024;  // dynamic shared memory per block on B200
@@ -97,6 +112,20 @@ int chained_smem_bytes(const KCfg &k, int es) {
     const int warp = (k.STAGES * stage + conv + 127) / 128 * 128;
     const int bars = (2 * k.WPC * k.STAGES * 8 + 127) / 128 * 128;
     return k.WPC * warp + bars;
+}
+
+// Shared memory of a tiled-kernel shape (mirrors TiledCfg::kSmem).
+int tiled_smem_bytes(const KCfg &k, int es) {
+    const int lpc = k.N / k.NL, cpw = 32 / lpc, cpb = k.WPC * cpw;
+    const int kU = k.T * cpb * es, kB = k.T * k.N * es;
+    const int stageF = 2 * kU + 2 * kB + kU;
+    const int rowW = k.N + (lpc >= 4 ? 4 * lpc : 0);
+    const int conv = 2 * k.T * rowW * 4;
+    const int xd = k.T * cpb * 8;
+    const int slot = (stageF + 127) / 128 * 128 + (conv + 127) / 128 * 128 + (xd + 127) / 128 * 128;
+    const int scratch = k.WPC * 2 * k.T * cpw * 4;
+    const int bars = (3 * k.STAGES * 8 + 127) / 128 * 128;
+    return k.STAGES * slot + scratch + bars;
 }
 
 }  // namespace
@@ -136,8 +165,11 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // bounded waits of the warps running the tails must give up and report it),
 // light=<per mille> sets how much shorter the segments of the warps that share
 // an SM sub-partition with the producer warp are (see kLightPermille), decode=0
-// runs a decode step (L = 1) on the step kernel instead of the decode kernel.
-void read_tune(int &cfg, int &poly, int &sms, int &split, int &nopublish, int &light, int &decode) {
+// runs a decode step (L = 1) on the step kernel instead of the decode kernel,
+// tiled=<i> forces the block-tiled shape i (kTiledCfgs), tiled=-1 keeps the
+// schedule off the tiled kernel.
+void read_tune(int &cfg, int &poly, int &sms, int &split, int &nopublish, int &light, int &decode,
+               int &tiled) {
     cfg = -2;
     poly = -1;
     sms = 0;
@@ -145,6 +177,7 @@ void read_tune(int &cfg, int &poly, int &sms, int &split, int &nopublish, int &l
     nopublish = 0;
     light = -1;
     decode = 1;
+    tiled = -2;
     const char *s = getenv("SSCAN_TUNE");
     if (!s) return;
     if (const char *c = strstr(s, "cfg=")) cfg = atoi(c + 4);
@@ -154,6 +187,7 @@ void read_tune(int &cfg, int &poly, int &sms, int &split, int &nopublish, int &l
     if (const char *c = strstr(s, "nopublish=")) nopublish = atoi(c + 10);
     if (const char *c = strstr(s, "light=")) light = atoi(c + 6);
     if (const char *c = strstr(s, "decode=")) decode = atoi(c + 7);
+    if (const char *c = strstr(s, "tiled=")) tiled = atoi(c + 6);
 }
 
 void choose_schedule(sscan_plan *p) {
@@ -161,8 +195,8 @@ void choose_schedule(sscan_plan *p) {
     p->mode = kGeneric;
     p->g_nl = p->N == 16 ? 8 : 16;
     p->g_lpc = static_cast<int>(p->N) / p->g_nl;
-    int want = -2, poly = -1, sms = 0, force_split = 0, nopublish = 0, light = -1, decode = 1;
-    read_tune(want, poly, sms, force_split, nopublish, light, decode);
+    int want = -2, poly = -1, sms = 0, force_split = 0, nopublish = 0, light = -1, decode = 1, tiled = -2;
+    read_tune(want, poly, sms, force_split, nopublish, light, decode, tiled);
     p->drop_publish = nopublish != 0;
     const int blocks = (sms > 0 && sms < p->sm_count) ? sms : p->sm_count;
     // the FMA-pipe exponent measured slower than MUFU alone at every occupancy: off unless asked
@@ -179,6 +213,36 @@ void choose_schedule(sscan_plan *p) {
     if (want == -1) return;
     // the chained kernel needs TMA-compatible rows and int32 TMA row coordinates
     if ((p->D * es) % 16 != 0 || p->B * p->L >= (int64_t(1) << 31) || p->L >= (int64_t(1) << 32)) return;
+    // 0) tiled: block-chains of the block's channels, at least about one per block
+    if (tiled != -1 && want < 0 && !force_split) {
+        const int n_try = tiled >= 0 ? 1 : static_cast<int>(sizeof(kTiledAuto) / sizeof(kTiledAuto[0]));
+        for (int oi = 0; oi < n_try; ++oi) {
+            const int i = tiled >= 0 ? tiled : kTiledAuto[oi];
+            if (i < 0 || i >= kNumTiledCfgs) continue;
+            const KCfg &k = kTiledCfgs[i];
+            if (k.N != p->N || tiled_smem_bytes(k, es) > kMaxSmem) continue;
+            const int64_t cpb = int64_t(32 / (k.N / k.NL)) * k.WPC;
+            const int64_t cpr = ceil_div(p->D, cpb);
+            const int64_t chains = p->B * cpr;
+            if (tiled < 0 && chains * 20 < int64_t(blocks) * 17) continue;
+            p->mode = kTiled;
+            p->split = false;
+            p->cfg = i;
+            p->chains_per_row = cpr;
+            p->chains = chains;
+            p->workers = int64_t(blocks) * k.WPC;
+            p->seg = ceil_div(chains * p->L, blocks);
+            p->seg_shift = 0;
+            p->max_pieces = 0;
+            p->rec_s_off = p->rec_mono_off = 0;
+            // carried state and flag per (block-chain, consumer warp)
+            p->flag_off = align_up(size_t(chains) * k.WPC * 32 * k.NL * sizeof(float), 256);
+            p->flag_bytes = size_t(chains) * k.WPC * sizeof(unsigned long long);
+            p->sink_off = p->flag_off + align_up(p->flag_bytes, 256);
+            p->ws_bytes = p->sink_off + align_up(size_t(p->workers) * 32 * sizeof(float), 256);
+            return;
+        }
+    }
     // 1) chained: enough chains that each is cut at most once (segment >= L)
     // 2) split: fewer chains than warps; cut them into pieces scanned concurrently
     for (int pass = force_split ? 1 : 0; pass < 2; ++pass) {
@@ -476,6 +540,93 @@ int launch_chained(sscan_plan *p, const void *u, const void *dl, const float *A,
     }
 }
 
+// ------------------------------------------------------------- tiled launch
+
+template <class IO, int CFG, bool ZOH, bool FUSED>
+int launch_tiled_t(sscan_plan *p, const void *u, const void *dl, const float *A, const void *Bm,
+                   const void *Cm, const float *h0, void *y, float *hf, void *ws, const Fused &fu,
+                   cudaStream_t s) {
+    constexpr KCfg k = kTiledCfgs[CFG];
+    using Cfg = TiledCfg<IO, k.N, k.NL, k.T, k.STAGES, k.WPC>;
+    auto kern = sscan_tiled_kernel<IO, Cfg, ZOH, FUSED>;
+    if (smem_opt_in<sscan_tiled_kernel<IO, Cfg, ZOH, FUSED>>(Cfg::kSmem) != cudaSuccess) return SSCAN_ERR_CUDA;
+    const int es = sizeof(IO);
+    const void *ptrs[5] = {u, dl, Bm, Cm, fu.z};
+    if (!p->tm_valid || memcmp(ptrs, p->tm_ptr, sizeof ptrs) != 0) {
+        const uint64_t rows = static_cast<uint64_t>(p->B * p->L);
+        if (!encode_map(&p->tm[0], u, es, p->D, rows, Cfg::CPB, Cfg::T) ||
+            !encode_map(&p->tm[1], dl, es, p->D, rows, Cfg::CPB, Cfg::T) ||
+            !encode_map(&p->tm[2], Bm, es, p->N, rows, p->N, Cfg::T) ||
+            !encode_map(&p->tm[3], Cm, es, p->N, rows, p->N, Cfg::T) ||
+            (fu.z != nullptr && !encode_map(&p->tm[4], fu.z, es, p->D, rows, Cfg::CPB, Cfg::T))) {
+            p->tm_valid = false;
+            return SSCAN_ERR_CUDA;
+        }
+        if (fu.z == nullptr) p->tm[4] = p->tm[0];  // never loaded (the kernel sees no gate)
+        memcpy(p->tm_ptr, ptrs, sizeof ptrs);
+        p->tm_valid = true;
+    }
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    unsigned long long *flags = reinterpret_cast<unsigned long long *>(w + p->flag_off);
+    if (ws != p->last_ws) {  // a workspace seen for the first time: clear its flags once
+        if (cudaMemsetAsync(flags, 0, p->flag_bytes, s) != cudaSuccess) return SSCAN_ERR_CUDA;
+        p->last_ws = ws;
+    }
+    uint32_t ep = g_epoch.fetch_add(1);
+    if (ep == 0) ep = g_epoch.fetch_add(1);
+    ChainedParams prm;
+    memset(&prm, 0, sizeof prm);
+    prm.A = A;
+    prm.h0 = h0;
+    prm.y = y;
+    prm.h_final = hf;
+    prm.carry = reinterpret_cast<float *>(w);
+    prm.flags = flags;
+    prm.ysink = w + p->sink_off;
+    prm.drop_publish = p->drop_publish ? 1 : 0;
+    prm.status = p->d_status;
+    prm.epoch_hi = static_cast<unsigned long long>(ep) << 32;
+    prm.L = p->L;
+    prm.D = p->D;
+    prm.chains_per_row = p->chains_per_row;
+    prm.chains = p->chains;
+    prm.seg = p->seg;
+    prm.seg_shift = 0;
+    prm.wpc = 1;  // one segment per block
+    prm.delta_bias = fu.bias;
+    prm.z = fu.z;
+    prm.softplus = fu.softplus ? 1 : 0;
+    void *args[] = {&p->tm[0], &p->tm[1], &p->tm[2], &p->tm[3], &p->tm[4], &prm};
+    const dim3 grid(static_cast<unsigned>(p->workers / k.WPC)), block(Cfg::kThreads);
+    const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kern), grid, block, args,
+                                                      Cfg::kSmem, s);
+    return e == cudaSuccess ? SSCAN_OK : SSCAN_ERR_CUDA;
+}
+
+template <class IO, int CFG>
+int launch_tiled_cfg(sscan_plan *p, const void *u, const void *dl, const float *A, const void *Bm,
+                     const void *Cm, const float *h0, void *y, float *hf, void *ws, const Fused &fu,
+                     cudaStream_t s) {
+    const bool zoh = (p->flags & SSCAN_ZOH) != 0;
+    if (fu.on())
+        return zoh ? launch_tiled_t<IO, CFG, true, true>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s)
+                   : launch_tiled_t<IO, CFG, false, true>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s);
+    return zoh ? launch_tiled_t<IO, CFG, true, false>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s)
+               : launch_tiled_t<IO, CFG, false, false>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s);
+}
+
+template <class IO>
+int launch_tiled(sscan_plan *p, const void *u, const void *dl, const float *A, const void *Bm,
+                 const void *Cm, const float *h0, void *y, float *hf, void *ws, const Fused &fu,
+                 cudaStream_t s) {
+    switch (p->cfg) {
+        case 0: return launch_tiled_cfg<IO, 0>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s);
+        case 1: return launch_tiled_cfg<IO, 1>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s);
+        case 2: return launch_tiled_cfg<IO, 2>(p, u, dl, A, Bm, Cm, h0, y, hf, ws, fu, s);
+        default: return SSCAN_ERR_UNSUPPORTED;
+    }
+}
+
 }  // namespace
 
 void sscan_choose_schedule(sscan_plan *p) { choose_schedule(p); }
@@ -591,7 +742,19 @@ int sscan_plan_describe(sscan_plan_t plan, char *buf, size_t len) {
     if (!plan) return -1;
     char tmp[512];
     int n;
-    if (plan->mode == kChained) {
+    if (plan->mode == kTiled) {
+        const KCfg &k = kTiledCfgs[plan->cfg];
+        n = snprintf(tmp, sizeof tmp,
+                     "kernel=tiled B=%lld L=%lld D=%lld N=%lld dtype=%s zoh=%d states_per_thread=%d "
+                     "threads_per_channel=%d channels_per_warp=%d warps_per_block=%d channels_per_block=%d "
+                     "tokens_per_stage=%d stages=%d split=0 chains=%lld blocks=%lld segment=%lld workspace=%zu "
+                     "sms=%d",
+                     (long long)plan->B, (long long)plan->L, (long long)plan->D, (long long)plan->N,
+                     plan->dtype == SSCAN_F32 ? "f32" : "bf16", (plan->flags & SSCAN_ZOH) ? 1 : 0, k.NL,
+                     k.N / k.NL, 32 / (k.N / k.NL), k.WPC, k.WPC * (32 / (k.N / k.NL)), k.T, k.STAGES,
+                     (long long)plan->chains, (long long)(plan->workers / k.WPC), (long long)plan->seg,
+                     plan->ws_bytes, plan->sm_count);
+    } else if (plan->mode == kChained) {
         const KCfg &k = kChainedCfgs[plan->cfg];
         n = snprintf(tmp, sizeof tmp,
                      "kernel=chained B=%lld L=%lld D=%lld N=%lld dtype=%s zoh=%d states_per_thread=%d "
@@ -670,12 +833,16 @@ int sscan_forward_gated(sscan_plan_t plan, const void *u, const void *delta, con
     if (overlaps(h_final, n_bdn * 4, y, n_bld * es)) return SSCAN_ERR_INVALID;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (p->mode == kChained) {
+    if (p->mode == kChained || p->mode == kTiled) {
         if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SSCAN_ERR_WORKSPACE;
         const size_t sz[10] = {n_bld * es, n_bld * es, n_dn * 4, n_bln * es, n_bln * es,
                                n_bdn * 4, n_bld * es, n_bdn * 4, static_cast<size_t>(p->D) * 4, n_bld * es};
         for (int i = 0; i < 10; ++i)
             if (overlaps(workspace, p->ws_bytes, ptrs[i], sz[i])) return SSCAN_ERR_WORKSPACE;
+        if (p->mode == kTiled)
+            return p->dtype == SSCAN_F32
+                       ? launch_tiled<float>(p, u, delta, A, B, C, h0, y, h_final, workspace, fu, s)
+                       : launch_tiled<uint16_t>(p, u, delta, A, B, C, h0, y, h_final, workspace, fu, s);
         return p->dtype == SSCAN_F32
                    ? launch_chained<float>(p, u, delta, A, B, C, h0, y, h_final, workspace, fu, s)
                    : launch_chained<uint16_t>(p, u, delta, A, B, C, h0, y, h_final, workspace, fu, s);

@@ -5,7 +5,8 @@ The kernels take delta as the raw projection and apply delta <- softplus(delta
 parameters as functions of the input"), and gate the output y <- y * silu(z)
 ("Selective State-Space Models (Mamba) and Hardware-Aware Scans", section 4).
 Every schedule is covered: the chained kernel on forced shapes (chains cut
-between warps, ragged last chain, bf16, ZOH, N = 32 and 64), the split mode,
+between warps, ragged last chain, bf16, ZOH, N = 32 and 64), the block-tiled
+kernel (block-chains cut between blocks), the split mode,
 the generic kernel, decode steps, the default schedule, and sampled rows of the
 full fused workloads.  Tolerances are those of the unfused parity tests.
 """
@@ -89,6 +90,42 @@ def test_fused_chained_forced(case, monkeypatch):
     P.check(hf.cpu().numpy(), hr, dt, "h_final")
     # the same plan without the fused arguments runs the unfused kernel again
     if not sp:
+        y0, hf0 = plan.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"])
+        yr0, hr0 = P.run_oracle(_drop(g, False, False), zoh)
+        P.check(y0.float().cpu().numpy(), yr0, dt, "y unfused")
+        P.check(hf0.cpu().numpy(), hr0, dt, "h_final unfused")
+    plan.close()
+
+
+TILED = [
+    # (B, L, D, N, dtype, h0, zoh, tcfg, blocks, softplus, bias, gate): the block-tiled kernel
+    (2, 300, 200, 64, "bf16", True, True, 0, 3, True, True, True),     # block-chains cut, D % 48 != 0
+    (2, 200, 192, 64, "f32", True, False, 1, 2, True, True, True),     # 16 warps, Euler
+    (2, 200, 200, 32, "f32", True, True, 2, 2, True, False, True),     # N = 32, no bias
+    (2, 300, 96, 64, "bf16", True, True, 0, 3, False, True, False),    # bias only, no softplus
+]
+
+
+@pytest.mark.parametrize("case", TILED, ids=[f"tcfg{c[7]}_B{c[0]}L{c[1]}D{c[2]}N{c[3]}{c[4]}_blk{c[8]}"
+                                            f"{'_zoh' if c[6] else ''}_sp{int(c[9])}b{int(c[10])}g{int(c[11])}"
+                                            for c in TILED])
+def test_fused_tiled_forced(case, monkeypatch):
+    Bt, L, D, N, dt, with_h0, zoh, tcfg, blocks, sp, bias, gate = case
+    g = _drop(W.generate(Bt, L, D, N, dt, 0.1 if with_h0 else 0.0, seed=5500 + L + D, A_jitter=0.3,
+                         fused=True), bias, gate)
+    if not sp:  # without softplus the raw delta must itself be a valid (positive) step
+        g["delta"] = W.generate(Bt, L, D, N, dt, 0.1 if with_h0 else 0.0, seed=5500 + L + D,
+                                A_jitter=0.3)["delta"]
+        if bias:
+            g["delta_bias"] = np.linspace(0.0, 0.05, D).astype(np.float32)
+    monkeypatch.setenv("SSCAN_TUNE", f"tiled={tcfg},sms={blocks}")
+    plan = S.Plan(Bt, L, D, N, _tdt(dt), zoh, delta_softplus=sp)
+    assert "kernel=tiled" in plan.describe(), plan.describe()
+    y, hf, d = _run_plan(plan, g)
+    yr, hr = P.run_oracle(g, zoh, softplus=sp)
+    P.check(y.float().cpu().numpy(), yr, dt, "y")
+    P.check(hf.cpu().numpy(), hr, dt, "h_final")
+    if not sp:  # the same plan without the fused arguments
         y0, hf0 = plan.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"])
         yr0, hr0 = P.run_oracle(_drop(g, False, False), zoh)
         P.check(y0.float().cpu().numpy(), yr0, dt, "y unfused")

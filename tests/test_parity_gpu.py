@@ -101,6 +101,67 @@ def test_chained_kernel_forced(case, monkeypatch):
     plan.close()
 
 
+TILED = [
+    # (B, L, D, N, dtype, h0, zoh, tcfg, blocks): the block-tiled kernel forced onto a small
+    # grid, so that block-chains are cut between blocks (every warp's state handed over).
+    # tcfg indexes the library's tiled shape table (see csrc/sscan.cu).
+    (2, 300, 200, 64, "bf16", True, True, 0, 3),    # 48 channels per block, D % 48 != 0
+    (2, 300, 192, 64, "f32", True, False, 0, 2),    # Euler, fp32 I/O
+    (1, 517, 96, 64, "bf16", False, False, 0, 1),   # one block, ragged last stage
+    (2, 300, 200, 64, "bf16", True, True, 1, 3),    # 64 channels per block (16 warps)
+    (2, 200, 200, 64, "f32", True, True, 1, 2),     # fp32 ZOH (the phi polynomial)
+    (2, 200, 200, 32, "f32", True, True, 2, 2),     # N = 32, 96 channels per block
+    (2, 300, 136, 32, "bf16", True, False, 2, 3),
+    (2, 300, 96, 64, "bf16", True, True, 0, 10),    # segment < L: block-chains cut many times
+    (3, 64, 48, 64, "bf16", False, True, 0, 2),     # L of four stages, one block-chain per row
+]
+
+
+@pytest.mark.parametrize("case", TILED, ids=[f"tcfg{c[7]}_B{c[0]}L{c[1]}D{c[2]}N{c[3]}{c[4]}_blk{c[8]}"
+                                            f"{'_zoh' if c[6] else ''}" for c in TILED])
+def test_tiled_kernel_forced(case, monkeypatch):
+    Bt, L, D, N, dt, with_h0, zoh, tcfg, blocks = case
+    g = W.generate(Bt, L, D, N, dt, 0.1 if with_h0 else 0.0, seed=2500 + L + D, A_jitter=0.3)
+    monkeypatch.setenv("SSCAN_TUNE", f"tiled={tcfg},sms={blocks}")
+    plan = S.Plan(Bt, L, D, N, torch.float32 if dt == "f32" else torch.bfloat16, zoh)
+    assert "kernel=tiled" in plan.describe(), plan.describe()
+    d = P.to_device(g)
+    y, hf = plan.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"])
+    assert plan.status() == S.OK
+    yr, hr = P.run_oracle(g, zoh)
+    P.check(y.float().cpu().numpy(), yr, dt, "y")
+    P.check(hf.cpu().numpy(), hr, dt, "h_final")
+    # a second call through the same plan and workspace (new launch epoch) is identical
+    y2, hf2 = plan.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"])
+    assert plan.status() == S.OK
+    assert torch.equal(y, y2) and torch.equal(hf, hf2)
+    plan.close()
+
+
+def test_tiled_lost_carry_times_out_and_is_reported(monkeypatch):
+    """The tiled kernel's failure detection: block-chain heads skip publishing their
+    warps' states, the tails' bounded waits give up, the status word reports it, and the
+    next call through a fresh plan is correct."""
+    import time
+    g = W.generate(2, 300, 96, 64, "bf16", 0.1, seed=78)
+    d = P.to_device(g)
+    monkeypatch.setenv("SSCAN_TUNE", "tiled=0,sms=3,nopublish=1")
+    plan = S.Plan(2, 300, 96, 64, torch.bfloat16, True)
+    assert "kernel=tiled" in plan.describe()
+    t0 = time.time()
+    plan.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"])
+    assert plan.status() == S.ERR_TIMEOUT
+    assert time.time() - t0 < 60
+    plan.close()
+    monkeypatch.setenv("SSCAN_TUNE", "tiled=0,sms=3")
+    plan = S.Plan(2, 300, 96, 64, torch.bfloat16, True)
+    y, hf = plan.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"])
+    assert plan.status() == S.OK
+    yr, hr = P.run_oracle(g, True)
+    P.check(y.float().cpu().numpy(), yr, "bf16", "y after a failed call")
+    plan.close()
+
+
 SPLIT = [
     # (B, L, D, N, dtype, h0, zoh, reset_frac, blocks, negate): split mode forced on a small
     # grid: pieces scanned from zero, exact carry-in by look-back, bounded fix-up of y
