@@ -120,14 +120,18 @@ __device__ __forceinline__ f2 zoh_coef_pair(f2 dd, f2 e, f2 ia, f2 nia, f2 abar)
 
 // The ZOH coefficient to the precision of bf16 I/O, in two packed operations and a
 // select: d (the z -> 0 limit: relative error |phi(z) - 1| <= |z|/2) when
-// |z| <= 2^-10.5, (abar - 1) * (1/A) beyond (abar - 1 is exact for abar in
-// [1/2, 2]; the relative error of abar itself, about 2^-22, becomes 2^-22 / |z|);
-// both below 3.5e-4 relative, against the 2^-9 rounding of a bf16 output and the
-// bf16 tolerance of 5e-3 relative L2.  (A = 0 takes the first form: e = 0 there,
-// and ia is not finite.)
+// |z| <= 2^-10.5, (abar - 1)/A beyond, as (abar - 1) * (1/A) (abar - 1 is exact
+// for abar in [1/2, 2]) or, with FMA, as abar * (1/A) - 1/A in one fused
+// operation (-1/A from the sign bits of 1/A); the relative error of abar itself,
+// about 2^-22, becomes 2^-22 / |z|.  Both forms stay below 3.5e-4 relative,
+// against the 2^-9 rounding of a bf16 output and the bf16 tolerance of 5e-3
+// relative L2.  (A = 0 takes the first form: e = 0 there, and ia is not finite.)
+// The chained kernel measured faster with the first form on B200, the tiled one
+// with the second.
 constexpr float kZohBf16Lim = 9.9606e-4f;  // 2^-10.5 / ln 2: the bound on |e| = |delta A| log2 e
+template <bool FMA = false>
 __device__ __forceinline__ f2 zoh_coef_pair_bf16(f2 dd, f2 e, f2 ia, f2 abar) {
-    const f2 big = mul2(add2(abar, splat2(-1.0f)), ia);
+    const f2 big = FMA ? fma2(abar, ia, neg2(ia)) : mul2(add2(abar, splat2(-1.0f)), ia);
     float e0, e1, d0, d1, g0, g1;
     unpack2(e, e0, e1);
     unpack2(dd, d0, d1);

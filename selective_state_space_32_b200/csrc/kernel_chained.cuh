@@ -132,8 +132,8 @@ struct ChainedCfg {
 // (sequential) state updates and the MUFU latency overlaps them.  PAR is the
 // token's parity; it selects which pairs take 2^x on the FMA pipe (a quarter
 // of all pairs across two tokens).  COARSE (bf16 I/O) takes the ZOH coefficient
-// to bf16 precision (zoh_coef_pair_bf16).
-template <int NP, bool ZOH, bool POLY, int PAR, bool COARSE = false>
+// to bf16 precision (zoh_coef_pair_bf16; CFMA: its fused multiply-add form).
+template <int NP, bool ZOH, bool POLY, int PAR, bool COARSE = false, bool CFMA = false>
 __device__ __forceinline__ void discretize(f2 (&ab)[NP], f2 (&bu)[NP], const f2 (&A2)[NP], const f2 (&nA)[NP],
                                            const f2 (&iA)[NP], float cap, float x, float dl,
                                            const float *Bs) {
@@ -160,8 +160,8 @@ __device__ __forceinline__ void discretize(f2 (&ab)[NP], f2 (&bu)[NP], const f2 
                 unpack2(e, e0, e1);
                 ab[p] = pack2(ex2(e0), ex2(e1));
             }
-            if (ZOH && COARSE)  // (Abar - 1) * (1/A): no -1/A registers to keep
-                bu[p] = mul2(zoh_coef_pair_bf16(dd, e, iA[p], ab[p]), mul2(bp, xx));
+            if (ZOH && COARSE)  // no -1/A registers to keep
+                bu[p] = mul2(zoh_coef_pair_bf16<CFMA>(dd, e, iA[p], ab[p]), mul2(bp, xx));
             else if (ZOH)
                 bu[p] = mul2(zoh_coef_pair(dd, e, iA[p], nA[p], ab[p]), mul2(bp, xx));
             else

@@ -17,9 +17,8 @@
 //
 // Roles.  Warp WPC (the producer) issues the 2-D TMA loads of every stage
 // (u, delta [T][CPB]; B, C [T][N]) on a "full" mbarrier, waits for each stage to
-// land, copies its B and C tiles into padded fp32 rows (bf16 widened) and its
-// u and delta tiles into one tile of (x, delta) fp32 pairs, and arrives on the
-// stage's "ready" mbarrier.  Consumer warp w runs channels
+// land, copies its B and C tiles into padded fp32 rows (bf16 widened) and
+// arrives on the stage's "ready" mbarrier.  Consumer warp w runs channels
 // w*CPW .. w*CPW + CPW - 1 of the block-chain with the lane layout of the
 // chained kernel (LPC lanes per channel, NL states per lane in registers), and
 // arrives on the stage's "empty" mbarrier (WPC arrivals release the slot).
@@ -59,9 +58,7 @@ struct TiledCfg {
     static constexpr int kRowW = N + LPC * kPadG;
     static constexpr int kConv = 2 * T * kRowW * 4;
     static constexpr int kStageA = (kStageF + 127) / 128 * 128;
-    static constexpr int kXdOff = kStageA + (kConv + 127) / 128 * 128;  // (u, delta) as fp32 pairs [T][CPB]
-    static constexpr int kXd = T * CPB * 8;
-    static constexpr int kSlot = kXdOff + (kXd + 127) / 128 * 128;
+    static constexpr int kSlot = kStageA + (kConv + 127) / 128 * 128;
     // fused calls: each consumer warp's delta' = softplus(delta + bias) and silu(z), fp32 [T][CPW]
     static constexpr int kDsf = T * CPW * 4;
     static constexpr int kScratch = WPC * 2 * kDsf;
@@ -78,8 +75,8 @@ struct TiledCfg {
 };
 
 // The producer warp: TMA issue in the block's processing order, at most STAGES
-// stages ahead of the consumers, and the fp32 copies of every landed stage's
-// tiles.  All lanes walk the same stages; lane 0 issues the copies.  On a wait
+// stages ahead of the consumers, and the fp32 copy of every landed stage's B and
+// C tiles.  All lanes walk the same stages; lane 0 issues the copies.  On a wait
 // that gives up it records the failure and waits (bounded) for its copies in
 // flight before returning.
 template <class IO, class Cfg, bool FUSED>
@@ -189,30 +186,6 @@ __device__ __forceinline__ void tiled_produce(const CUtensorMap *tm_u, const CUt
                                     __uint_as_float(vc.w << 16), __uint_as_float(vc.w & 0xffff0000u));
             }
         }
-        // u and delta as (x, delta) fp32 pairs: one 8-byte load per token for a consumer lane
-        {
-            const uint4 *ru = reinterpret_cast<const uint4 *>(slot);
-            const uint4 *rd = reinterpret_cast<const uint4 *>(slot + Cfg::kU);
-            float4 *oxd = reinterpret_cast<float4 *>(slot + Cfg::kXdOff);
-            constexpr int kXChunks = T * CPB / kPer;  // 16-byte chunks of the u (and delta) tile
-#pragma unroll 2
-            for (int q = lane; q < kXChunks; q += 32) {
-                const uint4 vu = ru[q], vd = rd[q];
-                float4 *o = oxd + q * (kPer / 2);  // kPer pairs = kPer / 2 float4
-                if constexpr (Cfg::ES == 4) {
-                    o[0] = make_float4(__uint_as_float(vu.x), __uint_as_float(vd.x), __uint_as_float(vu.y),
-                                       __uint_as_float(vd.y));
-                    o[1] = make_float4(__uint_as_float(vu.z), __uint_as_float(vd.z), __uint_as_float(vu.w),
-                                       __uint_as_float(vd.w));
-                } else {
-                    const uint32_t wu[4] = {vu.x, vu.y, vu.z, vu.w}, wd[4] = {vd.x, vd.y, vd.z, vd.w};
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        o[k] = make_float4(__uint_as_float(wu[k] << 16), __uint_as_float(wd[k] << 16),
-                                           __uint_as_float(wu[k] & 0xffff0000u), __uint_as_float(wd[k] & 0xffff0000u));
-                }
-            }
-        }
         __syncwarp();  // every lane's rows before the arrive (release)
         if (lane == 0) mbar_arrive(&ready[s]);
         ++r_w;
@@ -229,17 +202,17 @@ __device__ __forceinline__ void tiled_produce(const CUtensorMap *tm_u, const CUt
 
 // Fused calls: a consumer warp's delta' = softplus(delta + bias) (or delta + bias)
 // and silu(z) (or 1) for its CPW channels of one stage, from the block's
-// (x, delta) and z tiles into its own fp32 [T][CPW] tiles.  Entry i = lane + 32k is
+// [T][CPB] tiles into its own fp32 [T][CPW] tiles.  Entry i = lane + 32k is
 // token i / CPW, channel i % CPW = lane % CPW (32 is a multiple of CPW).
 template <class IO, class Cfg>
-__device__ __forceinline__ void tiled_fused_tile(const float2 *xd, const IO *zs, float *dsf, float *gsf, int ch0,
+__device__ __forceinline__ void tiled_fused_tile(const IO *dsm, const IO *zs, float *dsf, float *gsf, int ch0,
                                                  float biasv, bool softplus, bool gate, int lane) {
     constexpr int CPW = Cfg::CPW, CPB = Cfg::CPB, kPer = Cfg::T * CPW / 32;
 #pragma unroll
     for (int k = 0; k < kPer; ++k) {
         const int i = lane + 32 * k;
         const int src = (i / CPW) * CPB + ch0 + i % CPW;
-        const float v = xd[src].y + biasv;
+        const float v = Io<IO>::widen(dsm[src]) + biasv;
         dsf[i] = softplus ? softplus_f(v) : v;
         gsf[i] = gate ? silu_f(Io<IO>::widen(zs[src])) : 1.0f;
     }
@@ -371,17 +344,18 @@ sscan_tiled_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_consta
                 break;
             }
             const unsigned char *slot = smem + s * Cfg::kSlot;
-            const float2 *xds = reinterpret_cast<const float2 *>(slot + Cfg::kXdOff) + ch;  // (x, delta)
+            const IO *us = reinterpret_cast<const IO *>(slot) + ch;
+            const IO *dsm = reinterpret_cast<const IO *>(slot + Cfg::kU) + ch;
             const float *Bs = reinterpret_cast<const float *>(slot + Cfg::kStageA) + gofs;
             const float *Cs = Bs + T * RS;
             if (FUSED) {
-                tiled_fused_tile<IO, Cfg>(reinterpret_cast<const float2 *>(slot + Cfg::kXdOff),
+                tiled_fused_tile<IO, Cfg>(reinterpret_cast<const IO *>(slot + Cfg::kU),
                                           reinterpret_cast<const IO *>(slot + Cfg::kStage), dsf, gsf, warp * CPW,
                                           biasv, P.softplus != 0, gate, lane);
                 __syncwarp();
             }
-            auto delta_at = [&](int j1) { return FUSED ? dsf[j1 * CPW + cl] : xds[j1 * CPB].y; };
-            auto x_at = [&](int j1) { return xds[j1 * CPB].x; };
+            auto delta_at = [&](int j1) { return FUSED ? dsf[j1 * CPW + cl] : Io<IO>::widen(dsm[j1 * CPB]); };
+            auto x_at = [&](int j1) { return Io<IO>::widen(us[j1 * CPB]); };
             const int nsteps = static_cast<int>(te - t0 < T ? te - t0 : T);
             IO *yp = ybase + t0 * ystr;
             int j = 0;
@@ -417,7 +391,7 @@ sscan_tiled_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_consta
                 f2 ab[GZ][NP], bu[GZ][NP];
 #pragma unroll
                 for (int q = 0; q < GZ; ++q)
-                    discretize<NP, true, false, 0, Cfg::ES == 2>(ab[q], bu[q], A2, A1, iA, 0.0f,
+                    discretize<NP, true, false, 0, Cfg::ES == 2, true>(ab[q], bu[q], A2, A1, iA, 0.0f,
                                                                  x_at(j0 + q), delta_at(j0 + q),
                                                                  Bs + (j0 + q) * RS);
                 float yv[GZ];
@@ -454,7 +428,7 @@ sscan_tiled_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_consta
                 f2 ab[NP], bu[NP];
                 const float x = x_at(j);
                 const float dl = delta_at(j);
-                discretize<NP, ZOH, false, 0, Cfg::ES == 2>(ab, bu, A2, A1, iA, 0.0f, x, dl, Bs + j * RS);
+                discretize<NP, ZOH, false, 0, Cfg::ES == 2, true>(ab, bu, A2, A1, iA, 0.0f, x, dl, Bs + j * RS);
                 float yv = advance<NP>(h, ab, bu, Cs + j * RS);
 #pragma unroll
                 for (int o = 1; o < LPC; o <<= 1) yv += __shfl_xor_sync(0xffffffffu, yv, o);

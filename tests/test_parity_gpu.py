@@ -228,13 +228,15 @@ def test_lost_carry_times_out_and_is_reported(monkeypatch):
 
 
 def test_default_schedules():
-    """The full-size workloads get the chained kernel; the 2048-channel long sequence is split."""
-    for name, want in [("mamba130m_f32", "split=0"), ("mamba1p4b_bf16", "split=0"),
-                       ("zoh_n64_bf16", "split=0"), ("longseq_bf16", "split=1")]:
+    """The full-size N = 16 workloads get the chained kernel (the 2048-channel long sequence
+    split), the N = 64 bf16 one the block-tiled kernel."""
+    for name, want in [("mamba130m_f32", "kernel=chained"), ("mamba1p4b_bf16", "kernel=chained"),
+                       ("zoh_n64_bf16", "kernel=tiled"), ("longseq_bf16", "kernel=chained")]:
         w = W.WORKLOADS[name]
         plan = S.Plan(w.B, w.L, w.D, w.N, torch.float32 if w.dtype == "f32" else torch.bfloat16,
                       w.zoh)
-        assert "kernel=chained" in plan.describe() and want in plan.describe(), (name, plan.describe())
+        split = "split=1" if name == "longseq_bf16" else "split=0"
+        assert want in plan.describe() and split in plan.describe(), (name, plan.describe())
         plan.close()
 
 

@@ -160,13 +160,14 @@ def test_noalloc_reports_a_wait_that_gave_up(monkeypatch):
 
 
 def test_noalloc_rejects_workspace_beyond_the_fixed_array():
-    """64 batch rows x 2048 channels (N = 64, bf16): the default chained schedule keeps
-    a carry slot per 8-channel chain, over 32 MiB in all, so the call is rejected before
-    any launch.  The buffers are real device buffers of the stated shape, so even a
-    failed check could not make a kernel touch memory it does not own."""
+    """64 batch rows x 2048 channels (N = 64, bf16): the default block-tiled schedule
+    keeps a carry slot per warp of every 48-channel block-chain, over 32 MiB in all, so
+    the call is rejected before any launch.  The buffers are real device buffers of the
+    stated shape, so even a failed check could not make a kernel touch memory it does
+    not own."""
     Bt, L, D, N = 64, 64, 2048, 64
     plan = S.Plan(Bt, L, D, N, torch.bfloat16)
-    assert "kernel=chained" in plan.describe(), plan.describe()
+    assert "kernel=tiled" in plan.describe(), plan.describe()
     assert plan.workspace_bytes > WORKSPACE_ROOM, plan.workspace_bytes
     plan.close()
     g = W.generate(Bt, L, D, N, "bf16", seed=99)
