@@ -38,8 +38,9 @@
  * device can see (a bounded wait that gave up) are latched in the plan's
  * status word and read back with sscan_get_status.
  *
- * CUDA graphs.  A launch of the chained schedule (sscan_plan_describe says
- * "kernel=chained") tags its carry flags with a tag the host picks per call,
+ * CUDA graphs.  A launch of the chained or tiled schedules (sscan_plan_describe
+ * says "kernel=chained" or "kernel=tiled") tags its carry flags with a tag the
+ * host picks per call,
  * so a graph that captured it would replay the same tag and could read a
  * carried state left by an earlier replay: do not replay such calls from a
  * graph.  The decode, step and generic schedules keep no state between
