@@ -226,13 +226,50 @@ sscan_backward_kernel(const BwdParams P) {
 
     // ---- pass 1: forward, keeping the state entering every chunk ----
     // (chunk by chunk: a chunk's loads sit in one straight-line block, ahead of its
-    // dependent updates)
-    float h[S];
+    // dependent updates).  States are held as packed pairs: the Euler updates run on
+    // f32x2 instructions; ZOH works on the unpacked values.
+    constexpr int SP = S / 2;  // state pairs per lane
+    static_assert(S % 2 == 0, "states per lane come in pairs");
+    f2 a2p[SP], a1p[SP];
+#pragma unroll
+    for (int p = 0; p < SP; ++p) {
+        a2p[p] = pack2(a2[2 * p], a2[2 * p + 1]);
+        a1p[p] = pack2(a1[2 * p], a1[2 * p + 1]);
+    }
+    auto abar_pair = [&](float dl, int p) {
+        float e0, e1;
+        unpack2(mul2(splat2(dl), a2p[p]), e0, e1);
+        return pack2(ex2(e0), ex2(e1));
+    };
+    auto ld_pairs = [&](const float *src, f2 (&v)[SP], bool ro) {
+        float t[S];
+        ldv<S>(src, t, ro);
+#pragma unroll
+        for (int p = 0; p < SP; ++p) v[p] = pack2(t[2 * p], t[2 * p + 1]);
+    };
+    auto st_pairs = [&](float *dst, const f2 (&v)[SP]) {
+        float t[S];
+#pragma unroll
+        for (int p = 0; p < SP; ++p) unpack2(v[p], t[2 * p], t[2 * p + 1]);
+        stv<S>(dst, t);
+    };
+    // ZOH state update of one pair (scalar: the coefficient's series need the single values)
+    auto zoh_step = [&](f2 hp, int p, float dl, float x, float b0, float b1, f2 &abp) {
+        float h0v, h1v;
+        unpack2(hp, h0v, h1v);
+        const float ab0 = ex2(dl * a2[2 * p]), ab1 = ex2(dl * a2[2 * p + 1]);
+        float beta0, beta1, q0, q1, q2;
+        coefs(2 * p, dl, ab0, b0, beta0, q0, q1, q2);
+        coefs(2 * p + 1, dl, ab1, b1, beta1, q0, q1, q2);
+        abp = pack2(ab0, ab1);
+        return pack2(fmaf(ab0, h0v, beta0 * x), fmaf(ab1, h1v, beta1 * x));
+    };
+    f2 h[SP];
     if (P.h0) {
-        ldv<S>(P.h0 + (b * D + dc) * N + n0, h, false);
+        ld_pairs(P.h0 + (b * D + dc) * N + n0, h, false);
     } else {
 #pragma unroll
-        for (int i = 0; i < S; ++i) h[i] = 0.0f;
+        for (int p = 0; p < SP; ++p) h[p] = splat2(0.0f);
     }
     prefetch_chunk(0, true, false);
     prefetch_chunk(1, false, false);
@@ -241,7 +278,7 @@ sscan_backward_kernel(const BwdParams P) {
         const int nt = static_cast<int>(L - t0 < KC ? L - t0 : KC);
         prefetch_chunk(c + 1, true, false);
         prefetch_chunk(c + 2, false, false);
-        stv<S>(ck + c * N, h);
+        st_pairs(ck + c * N, h);
         float xs[KC], ds[KC], Bs[KC][S];
 #pragma unroll
         for (int k = 0; k < KC; ++k) {
@@ -254,16 +291,14 @@ sscan_backward_kernel(const BwdParams P) {
 #pragma unroll
         for (int k = 0; k < KC; ++k) {
             if (k < nt) {
-                const float dx = ds[k] * xs[k];  // Euler: Bbar u = B (delta u)
+                const f2 dx2 = splat2(ds[k] * xs[k]);  // Euler: Bbar u = B (delta u)
 #pragma unroll
-                for (int i = 0; i < S; ++i) {
-                    const float abar = ex2(ds[k] * a2[i]);
+                for (int p = 0; p < SP; ++p) {
                     if constexpr (ZOH) {
-                        float beta, q0, q1, q2;
-                        coefs(i, ds[k], abar, Bs[k][i], beta, q0, q1, q2);
-                        h[i] = fmaf(abar, h[i], beta * xs[k]);
+                        f2 abp;
+                        h[p] = zoh_step(h[p], p, ds[k], xs[k], Bs[k][2 * p], Bs[k][2 * p + 1], abp);
                     } else {
-                        h[i] = fmaf(abar, h[i], Bs[k][i] * dx);
+                        h[p] = fma2(abar_pair(ds[k], p), h[p], mul2(pack2(Bs[k][2 * p], Bs[k][2 * p + 1]), dx2));
                     }
                 }
             }
@@ -271,15 +306,15 @@ sscan_backward_kernel(const BwdParams P) {
     }
 
     // ---- pass 2: reverse sweep over the chunks ----
-    float gs[S], dacc[S];
+    f2 gs[SP], dacc[SP];
     if (P.dhf && valid) {
-        ldv<S>(P.dhf + (b * D + dc) * N + n0, gs, false);
+        ld_pairs(P.dhf + (b * D + dc) * N + n0, gs, false);
     } else {
 #pragma unroll
-        for (int i = 0; i < S; ++i) gs[i] = 0.0f;
+        for (int p = 0; p < SP; ++p) gs[p] = splat2(0.0f);
     }
 #pragma unroll
-    for (int i = 0; i < S; ++i) dacc[i] = 0.0f;
+    for (int p = 0; p < SP; ++p) dacc[p] = splat2(0.0f);
     float dbias_acc = 0.0f;
     prefetch_chunk(P.nchunks - 1, true, true);
     for (int64_t c = P.nchunks - 1; c >= 0; --c) {
@@ -289,12 +324,12 @@ sscan_backward_kernel(const BwdParams P) {
         prefetch_chunk(c - 2, false, true);
         if (c >= 1) prefetch_l1(ck + (c - 1) * N);
         // recompute the chunk's states h_{t0 .. t0+nt-1} (and each token's Abar) from its checkpoint
-        float h_in[S], hk[KC][S], ab[KA][S];
-        ldv<S>(ck + c * N, h_in, false);
+        f2 h_in[SP], hk[KC][SP], ab[KA][SP];
+        ld_pairs(ck + c * N, h_in, false);
         {
-            float hc[S];
+            f2 hc[SP];
 #pragma unroll
-            for (int i = 0; i < S; ++i) hc[i] = h_in[i];
+            for (int p = 0; p < SP; ++p) hc[p] = h_in[p];
 #pragma unroll
             for (int k = 0; k < KC; ++k) {
                 const int64_t t = t0 + (k < nt ? k : nt - 1);  // loads need not wait behind work
@@ -303,21 +338,19 @@ sscan_backward_kernel(const BwdParams P) {
                 const float x = Io<IO>::widen(Io<IO>::ld(u + t * D));
                 float Bv[S];
                 ldv_io<IO, S>(Bp + t * N, Bv);
-                const float dx = dl * x;
+                const f2 dx2 = splat2(dl * x);
 #pragma unroll
-                for (int i = 0; i < S; ++i) {
-                    const float abar = ex2(dl * a2[i]);
-                    float bu;
+                for (int p = 0; p < SP; ++p) {
+                    f2 abp, hn;
                     if constexpr (ZOH) {
-                        float beta, q0, q1, q2;
-                        coefs(i, dl, abar, Bv[i], beta, q0, q1, q2);
-                        bu = beta * x;
+                        hn = zoh_step(hc[p], p, dl, x, Bv[2 * p], Bv[2 * p + 1], abp);
                     } else {
-                        bu = Bv[i] * dx;
+                        abp = abar_pair(dl, p);
+                        hn = fma2(abp, hc[p], mul2(pack2(Bv[2 * p], Bv[2 * p + 1]), dx2));
                     }
-                    if (k < nt) hc[i] = fmaf(abar, hc[i], bu);
-                    hk[k][i] = hc[i];
-                    if constexpr (kKeepAbar) ab[k][i] = abar;
+                    if (k < nt) hc[p] = hn;
+                    hk[k][p] = hc[p];
+                    if constexpr (kKeepAbar) ab[k][p] = abp;
                 }
             }
         }
@@ -340,57 +373,79 @@ sscan_backward_kernel(const BwdParams P) {
                 if (FUSED && zp != nullptr) {
                     // the gate: this lane's share of the scan's own output ys = C . h_t
 #pragma unroll
-                    for (int i = 0; i < S; ++i) ysp = fmaf(Cv[i], hk[k][i], ysp);
+                    for (int p = 0; p < SP; ++p) {
+                        float h0v, h1v;
+                        unpack2(hk[k][p], h0v, h1v);
+                        ysp = fmaf(Cv[2 * p], h0v, ysp);
+                        ysp = fmaf(Cv[2 * p + 1], h1v, ysp);
+                    }
                     const float sz = 1.0f / (1.0f + ex2(-zraw * 1.4426950408889634f));
                     dyt *= zraw * sz;  // dy of the scan = dy silu(z)
                 }
                 float dut = 0.0f, ddt = 0.0f;
-                float vb[S], vc[S];
+                f2 vb[SP], vc[SP];
+                const f2 dy2 = splat2(dyt);
                 if constexpr (ZOH) {
 #pragma unroll
-                    for (int i = 0; i < S; ++i) {
-                        const float hprev = k > 0 ? hk[k > 0 ? k - 1 : 0][i] : h_in[i];
-                        float abar;
-                        if constexpr (kKeepAbar) abar = ab[k][i];
-                        else abar = ex2(dl * a2[i]);
-                        float beta, dbdl, dbda, dbdb;
-                        coefs(i, dl, abar, Bv[i], beta, dbdl, dbda, dbdb);
-                        gs[i] = fmaf(Cv[i], dyt, gs[i]);
-                        dut = fmaf(gs[i], beta, dut);
-                        ddt = fmaf(gs[i], fmaf(hprev * a1[i], abar, x * dbdl), ddt);
-                        dacc[i] = fmaf(gs[i], fmaf(hprev * dl, abar, x * dbda), dacc[i]);
-                        vb[i] = gs[i] * x * dbdb;
-                        vc[i] = dyt * hk[k][i];
-                        gs[i] *= abar;
+                    for (int p = 0; p < SP; ++p) {
+                        float hp0, hp1, hk0, hk1, g0, g1, da0, da1;
+                        unpack2(k > 0 ? hk[k > 0 ? k - 1 : 0][p] : h_in[p], hp0, hp1);
+                        unpack2(hk[k][p], hk0, hk1);
+                        unpack2(gs[p], g0, g1);
+                        unpack2(dacc[p], da0, da1);
+                        float abv[2];
+                        if constexpr (kKeepAbar) unpack2(ab[k][p], abv[0], abv[1]);
+                        else { abv[0] = ex2(dl * a2[2 * p]); abv[1] = ex2(dl * a2[2 * p + 1]); }
+                        float gv[2] = {g0, g1}, dav[2] = {da0, da1}, vbv[2], vcv[2];
+                        const float hpv[2] = {hp0, hp1}, hkv[2] = {hk0, hk1};
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) {
+                            const int i = 2 * p + q;
+                            float beta, dbdl, dbda, dbdb;
+                            coefs(i, dl, abv[q], Bv[i], beta, dbdl, dbda, dbdb);
+                            gv[q] = fmaf(Cv[i], dyt, gv[q]);
+                            dut = fmaf(gv[q], beta, dut);
+                            ddt = fmaf(gv[q], fmaf(hpv[q] * a1[i], abv[q], x * dbdl), ddt);
+                            dav[q] = fmaf(gv[q], fmaf(hpv[q] * dl, abv[q], x * dbda), dav[q]);
+                            vbv[q] = gv[q] * x * dbdb;
+                            vcv[q] = dyt * hkv[q];
+                            gv[q] *= abv[q];
+                        }
+                        gs[p] = pack2(gv[0], gv[1]);
+                        dacc[p] = pack2(dav[0], dav[1]);
+                        vb[p] = pack2(vbv[0], vbv[1]);
+                        vc[p] = pack2(vcv[0], vcv[1]);
                     }
                 } else {
                     // Euler (beta = delta B): du = delta sum g B, ddelta = sum g hprev A Abar + u sum g B,
                     // dA += g hprev delta Abar, dB += g u delta; the shared factors once per state
-                    const float xdl = x * dl;
-                    float sgb = 0.0f, sqa = 0.0f;
+                    const f2 xdl2 = splat2(x * dl), dl2 = splat2(dl);
+                    f2 sgb = splat2(0.0f), sqa = splat2(0.0f);
 #pragma unroll
-                    for (int i = 0; i < S; ++i) {
-                        const float hprev = k > 0 ? hk[k > 0 ? k - 1 : 0][i] : h_in[i];
-                        float abar;
-                        if constexpr (kKeepAbar) abar = ab[k][i];
-                        else abar = ex2(dl * a2[i]);
-                        gs[i] = fmaf(Cv[i], dyt, gs[i]);
-                        sgb = fmaf(gs[i], Bv[i], sgb);
-                        const float q = gs[i] * hprev * abar;
-                        sqa = fmaf(q, a1[i], sqa);
-                        dacc[i] = fmaf(q, dl, dacc[i]);
-                        vb[i] = gs[i] * xdl;
-                        vc[i] = dyt * hk[k][i];
-                        gs[i] *= abar;
+                    for (int p = 0; p < SP; ++p) {
+                        const f2 hprev = k > 0 ? hk[k > 0 ? k - 1 : 0][p] : h_in[p];
+                        const f2 abp = kKeepAbar ? ab[k > KA - 1 ? KA - 1 : k][p] : abar_pair(dl, p);
+                        gs[p] = fma2(pack2(Cv[2 * p], Cv[2 * p + 1]), dy2, gs[p]);
+                        sgb = fma2(gs[p], pack2(Bv[2 * p], Bv[2 * p + 1]), sgb);
+                        const f2 q = mul2(mul2(gs[p], hprev), abp);
+                        sqa = fma2(q, a1p[p], sqa);
+                        dacc[p] = fma2(q, dl2, dacc[p]);
+                        vb[p] = mul2(gs[p], xdl2);
+                        vc[p] = mul2(dy2, hk[k][p]);
+                        gs[p] = mul2(gs[p], abp);
                     }
-                    dut = dl * sgb;
-                    ddt = fmaf(x, sgb, sqa);
+                    float sb0, sb1, sq0, sq1;
+                    unpack2(sgb, sb0, sb1);
+                    unpack2(sqa, sq0, sq1);
+                    const float sgbv = sb0 + sb1;
+                    dut = dl * sgbv;
+                    ddt = fmaf(x, sgbv, sq0 + sq1);
                 }
                 s_tok[0][k][threadIdx.x] = dut;
                 s_tok[1][k][threadIdx.x] = ddt * sg;  // the gradient of the raw step (softplus' = sigmoid)
                 if (FUSED && zp != nullptr) s_tok[2][k][threadIdx.x] = ysp;
-                stv<S>(&s_vb[k][threadIdx.x * S], vb);
-                stv<S>(&s_vc[k][threadIdx.x * S], vc);
+                st_pairs(&s_vb[k][threadIdx.x * S], vb);
+                st_pairs(&s_vc[k][threadIdx.x * S], vc);
             }
         }
         __syncthreads();
@@ -433,8 +488,11 @@ sscan_backward_kernel(const BwdParams P) {
         __syncthreads();
     }
     if (valid) {
-        if (P.dh0 != nullptr) stv<S>(P.dh0 + (b * D + d) * N + n0, gs);
-        atomic_addv<S>(P.dA + d * N + n0, dacc);
+        if (P.dh0 != nullptr) st_pairs(P.dh0 + (b * D + d) * N + n0, gs);
+        float da[S];
+#pragma unroll
+        for (int p = 0; p < SP; ++p) unpack2(dacc[p], da[2 * p], da[2 * p + 1]);
+        atomic_addv<S>(P.dA + d * N + n0, da);
     }
     if (FUSED && P.dbias != nullptr && threadIdx.x < KC * CPB) {
         const int64_t dj = static_cast<int64_t>(blockIdx.x) * CPB + threadIdx.x % CPB;
