@@ -16,12 +16,13 @@
 //    block-chain segment, its warps sharing each stage's tiles (shapes whose
 //    per-warp rows are narrower than an L2 fill);
 //  * step (kernel_step.cuh): four states per thread, shaped for the state's
-//    HBM round trip; sequences shorter than the chained kernel's minimum,
-//    the single-token decode step in particular;
+//    HBM round trip; sequences shorter than the chained kernel's minimum
+//    (the decode kernel, kernel_decode.cuh, takes the single-token step with
+//    a state);
 //  * generic (kernel_generic.cuh): one thread per (channel, state group),
 //    plain loads; for the longer shapes the chained kernel cannot take.
-// Both keep every (b,d) state row in registers; the [B,L,D,N] tensors never
-// reach memory.  The path is ALU bound on B200 (one 2^x and four FMA-pipe
+// Every one keeps each (b,d) state row in registers; the [B,L,D,N] tensors
+// never reach memory.  The path is ALU bound on B200 (one 2^x and four FMA-pipe
 // operations per state update against 1-3 bytes of HBM traffic), so there are
 // no tensor-core stages.
 #include <cuda.h>
