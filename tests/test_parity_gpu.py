@@ -284,6 +284,7 @@ HOST = [
     (2, 50, 33, 16, "f32", False, True, False),      # short: two pieces of one row
     (11, 100, 64, 16, "bf16", True, True, True),     # short: pieces of 6 and 5 rows; fused
     (256, 1, 2048, 16, "f32", True, False, False),   # the decode step's shape: two pieces of 128 rows
+    (4, 512, 2048, 64, "bf16", True, True, False),   # 8 pieces of 64 tokens, each on the block-tiled kernel
 ]
 
 

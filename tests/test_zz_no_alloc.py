@@ -74,6 +74,7 @@ CASES = [
     (4, 512, 2048, 16, "f32", True, False, 0.0, None),           # chained, cuts between warps
     (1, 4096, 64, 16, "bf16", True, False, 0.32, "split=1,sms=8"),  # split mode with fix-up
     (2, 300, 96, 64, "bf16", False, True, 0.0, None),            # ZOH, N = 64
+    (4, 64, 2048, 64, "bf16", True, True, 0.0, None),            # block-tiled kernel (N = 64)
     (1, 100, 70, 16, "f32", True, False, 0.0, None),             # generic kernel (D*4 % 16 != 0)
 ]
 
