@@ -38,7 +38,11 @@
 // into dB and dC: the blocks of a batch row walk the same tokens at the same
 // time, so atomics on dB and dC would all meet on the same few lines.  dA
 // needs no cross-lane sum (one atomic per lane at the end).  The recompute
-// keeps each token's Abar in registers for the reverse sweep.
+// keeps each token's Abar in registers for the reverse sweep.  When every row
+// of the block's channels is 4-byte aligned (fp32, or bf16 with an even D) the
+// chunk's inputs are staged in shared memory by cp.async one chunk ahead
+// (STAGED: the L1 kept only about a third of the prefetched rows, and the
+// reverse sweep waited on L2 for the rest).
 #pragma once
 
 #include "device_utils.cuh"
@@ -113,6 +117,43 @@ __device__ __forceinline__ void prefetch_l1(const void *p) {
     asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
 }
 
+// 4-byte asynchronous global -> shared copies (cp.async, no register staging)
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// S consecutive values of a staged B or C row (shared memory, I/O type), widened to fp32
+template <class IO, int S> __device__ __forceinline__ void ldv_sm(const IO *p, float (&v)[S]) {
+    static_assert(S == 4, "four states per lane");
+    if constexpr (sizeof(IO) == 4) {
+        const float4 t = *reinterpret_cast<const float4 *>(p);
+        v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+    } else {
+        const uint2 t = *reinterpret_cast<const uint2 *>(p);
+        v[0] = __uint_as_float(t.x << 16); v[1] = __uint_as_float(t.x & 0xffff0000u);
+        v[2] = __uint_as_float(t.y << 16); v[3] = __uint_as_float(t.y & 0xffff0000u);
+    }
+}
+
+// One buffer of a chunk's staged inputs, in the I/O type: delta, u, dy, z as
+// [KC][CPB] (the block's channels fastest), B and C as [KC][N].
+template <class IO, int N, int S>
+struct BwdStage {
+    static constexpr int CPB = bwd_block_channels_s(N, S), KC = kChunk;
+    static constexpr int kDl = 0, kU = KC * CPB, kDy = 2 * KC * CPB, kZ = 3 * KC * CPB;
+    static constexpr int kB = 4 * KC * CPB, kC = kB + KC * N;
+    static constexpr int kElems = ((kC + KC * N) * int(sizeof(IO)) + 15) / 16 * 16 / int(sizeof(IO));
+};
+// dynamic shared memory of the backward kernel: the per-chunk partials, and two
+// staging buffers when STAGED
+template <class IO, int N, int S, bool STAGED>
+constexpr int bwd_smem_bytes() {
+    return (3 * kChunk * kBwdThreads + 2 * kChunk * kBwdThreads * S) * 4 +
+           (STAGED ? 2 * BwdStage<IO, N, S>::kElems * int(sizeof(IO)) : 0);
+}
+
 // Sum of LPC consecutive floats in shared memory (16-byte aligned when LPC >= 4).
 template <int LPC> __device__ __forceinline__ float sum_lanes(const float *p) {
     float acc = 0.0f;
@@ -129,7 +170,7 @@ template <int LPC> __device__ __forceinline__ float sum_lanes(const float *p) {
     return acc;
 }
 
-template <class IO, int N, int S, bool ZOH, bool FUSED>
+template <class IO, int N, int S, bool ZOH, bool FUSED, bool STAGED>
 __global__ void __launch_bounds__(kBwdThreads, bwd_min_blocks<S>())
 sscan_backward_kernel(const BwdParams P) {
     constexpr int LPC = N / S, CPW = 32 / LPC, CPB = kBwdWarps * CPW, KC = kChunk;
@@ -139,8 +180,14 @@ sscan_backward_kernel(const BwdParams P) {
     constexpr int KA = kKeepAbar ? KC : 1;
     // per chunk: each lane's partials of du, ddelta (of the raw step) and the gate's ys per
     // token, and its S contributions to dB and dC per token ([k][channel][N] order)
-    __shared__ __align__(16) float s_tok[3][KC][kBwdThreads];
-    __shared__ __align__(16) float s_vb[KC][kBwdThreads * S], s_vc[KC][kBwdThreads * S];
+    extern __shared__ __align__(16) unsigned char bsm[];
+    float(*s_tok)[KC][kBwdThreads] = reinterpret_cast<float(*)[KC][kBwdThreads]>(bsm);
+    float(*s_vb)[kBwdThreads * S] =
+        reinterpret_cast<float(*)[kBwdThreads * S]>(bsm + 3 * KC * kBwdThreads * 4);
+    float(*s_vc)[kBwdThreads * S] = s_vb + KC;
+    // STAGED: two buffers of a chunk's inputs (BwdStage), filled by cp.async a chunk ahead
+    using St = BwdStage<IO, N, S>;
+    IO *stage_base = reinterpret_cast<IO *>(bsm + (3 * KC * kBwdThreads + 2 * KC * kBwdThreads * S) * 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cl = lane / LPC, g = lane % LPC, n0 = S * g;
     const int64_t L = P.L, D = P.D;
@@ -164,9 +211,9 @@ sscan_backward_kernel(const BwdParams P) {
         ia[i] = a1[i] != 0.0f ? 1.0f / a1[i] : 0.0f;
     }
     const float biasv = FUSED && P.bias ? __ldg(P.bias + dc) : 0.0f;
-    // the step the scan uses, and (fused) softplus' = sigmoid of its argument
-    auto step = [&](int64_t t, float &sig) {
-        const float raw = Io<IO>::widen(Io<IO>::ld(dl_in + t * D));
+    // the step the scan uses, and (fused) softplus' = sigmoid of its argument, from the raw
+    // delta of this lane's channel
+    auto step_raw = [&](float raw, float &sig) {
         if (!FUSED) {
             sig = 1.0f;
             return raw;
@@ -224,6 +271,72 @@ sscan_backward_kernel(const BwdParams P) {
         }
     };
 
+    // STAGED: chunk c's inputs into buffer `buf` with 4-byte cp.async copies, issued by
+    // all threads (consecutive threads take consecutive words of a token row: coalesced),
+    // one commit group per chunk; the caller waits and synchronises before reading.
+    // Tokens past the sequence's end repeat its last token (unused); words past D read the
+    // row's last word (D is a multiple of the elements per word), lanes there add nothing.
+    constexpr int EPW = 4 / int(sizeof(IO));  // elements per 4-byte word
+    const int64_t d0 = static_cast<int64_t>(blockIdx.x) * CPB;
+    const IO *dl_row = static_cast<const IO *>(P.delta) + b * L * D;
+    const IO *u_row = static_cast<const IO *>(P.u) + b * L * D;
+    const IO *dy_row = static_cast<const IO *>(P.dy) + b * L * D;
+    const IO *z_row = FUSED && P.z ? static_cast<const IO *>(P.z) + b * L * D : nullptr;
+    const IO *B_row = static_cast<const IO *>(P.Bm) + b * L * N;
+    const IO *C_row = static_cast<const IO *>(P.Cm) + b * L * N;
+    auto issue = [&](int64_t c, int buf, bool rev) {
+        IO *sb = stage_base + buf * St::kElems;
+        const int64_t t0 = c * KC;
+        const int nt = static_cast<int>(L - t0 < KC ? L - t0 : KC);
+        constexpr int WPR = CPB / EPW;  // words per token row of the block's channels
+        for (int e = threadIdx.x; e < KC * WPR; e += kBwdThreads) {
+            const int k = e / WPR, w = e % WPR;
+            const int64_t t = t0 + (k < nt ? k : nt - 1);
+            const int64_t col = d0 + w * EPW < D ? d0 + w * EPW : D - EPW;
+            const int64_t gi = t * D + col;
+            const int si = k * CPB + w * EPW;
+            cp_async4(sb + St::kDl + si, dl_row + gi);
+            cp_async4(sb + St::kU + si, u_row + gi);
+            if (rev) {
+                cp_async4(sb + St::kDy + si, dy_row + gi);
+                if (FUSED && z_row != nullptr) cp_async4(sb + St::kZ + si, z_row + gi);
+            }
+        }
+        constexpr int WPN = N / EPW;
+        for (int e = threadIdx.x; e < (rev ? 2 : 1) * KC * WPN; e += kBwdThreads) {
+            const int which = e / (KC * WPN), r = e % (KC * WPN), k = r / WPN, w = r % WPN;
+            const int64_t t = t0 + (k < nt ? k : nt - 1);
+            cp_async4(sb + (which ? St::kC : St::kB) + k * N + w * EPW, (which ? C_row : B_row) + t * N + w * EPW);
+        }
+        cp_async_commit();
+    };
+    const int ch = warp * CPW + cl;  // this lane's channel within the block
+    // token k of chunk c (token t): staged or straight from global memory
+    auto in_dl = [&](const IO *sb, int k, int64_t t) {
+        if constexpr (STAGED) return Io<IO>::widen(sb[St::kDl + k * CPB + ch]);
+        else return Io<IO>::widen(Io<IO>::ld(dl_in + t * D));
+    };
+    auto in_x = [&](const IO *sb, int k, int64_t t) {
+        if constexpr (STAGED) return Io<IO>::widen(sb[St::kU + k * CPB + ch]);
+        else return Io<IO>::widen(Io<IO>::ld(u + t * D));
+    };
+    auto in_dy = [&](const IO *sb, int k, int64_t t) {
+        if constexpr (STAGED) return Io<IO>::widen(sb[St::kDy + k * CPB + ch]);
+        else return Io<IO>::widen(Io<IO>::ld(dyp + t * D));
+    };
+    auto in_z = [&](const IO *sb, int k, int64_t t) {
+        if constexpr (STAGED) return Io<IO>::widen(sb[St::kZ + k * CPB + ch]);
+        else return Io<IO>::widen(Io<IO>::ld(zp + t * D));
+    };
+    auto in_B = [&](const IO *sb, int k, int64_t t, float (&v)[S]) {
+        if constexpr (STAGED) ldv_sm<IO, S>(sb + St::kB + k * N + n0, v);
+        else ldv_io<IO, S>(Bp + t * N, v);
+    };
+    auto in_C = [&](const IO *sb, int k, int64_t t, float (&v)[S]) {
+        if constexpr (STAGED) ldv_sm<IO, S>(sb + St::kC + k * N + n0, v);
+        else ldv_io<IO, S>(Cp + t * N, v);
+    };
+
     // ---- pass 1: forward, keeping the state entering every chunk ----
     // (chunk by chunk: a chunk's loads sit in one straight-line block, ahead of its
     // dependent updates).  States are held as packed pairs: the Euler updates run on
@@ -271,22 +384,37 @@ sscan_backward_kernel(const BwdParams P) {
 #pragma unroll
         for (int p = 0; p < SP; ++p) h[p] = splat2(0.0f);
     }
-    prefetch_chunk(0, true, false);
-    prefetch_chunk(1, false, false);
+    if constexpr (STAGED) {
+        prefetch_chunk(1, false, false);
+        issue(0, 0, false);
+    } else {
+        prefetch_chunk(0, true, false);
+        prefetch_chunk(1, false, false);
+    }
     for (int64_t c = 0; c < P.nchunks; ++c) {
         const int64_t t0 = c * KC;
         const int nt = static_cast<int>(L - t0 < KC ? L - t0 : KC);
-        prefetch_chunk(c + 1, true, false);
-        prefetch_chunk(c + 2, false, false);
+        const IO *sb = stage_base + (c & 1) * St::kElems;
+        if constexpr (STAGED) {
+            // chunk c has landed (this thread's copies), then every thread's; every thread is
+            // also done with chunk c - 1, whose buffer takes chunk c + 1
+            cp_async_wait_all();
+            __syncthreads();
+            if (c + 1 < P.nchunks) issue(c + 1, (c + 1) & 1, false);
+            prefetch_chunk(c + 2, false, false);
+        } else {
+            prefetch_chunk(c + 1, true, false);
+            prefetch_chunk(c + 2, false, false);
+        }
         st_pairs(ck + c * N, h);
         float xs[KC], ds[KC], Bs[KC][S];
 #pragma unroll
         for (int k = 0; k < KC; ++k) {
             const int64_t t = t0 + (k < nt ? k : nt - 1);
             float sg;
-            ds[k] = step(t, sg);
-            xs[k] = Io<IO>::widen(Io<IO>::ld(u + t * D));
-            ldv_io<IO, S>(Bp + t * N, Bs[k]);
+            ds[k] = step_raw(in_dl(sb, k, t), sg);
+            xs[k] = in_x(sb, k, t);
+            in_B(sb, k, t, Bs[k]);
         }
 #pragma unroll
         for (int k = 0; k < KC; ++k) {
@@ -316,12 +444,28 @@ sscan_backward_kernel(const BwdParams P) {
 #pragma unroll
     for (int p = 0; p < SP; ++p) dacc[p] = splat2(0.0f);
     float dbias_acc = 0.0f;
-    prefetch_chunk(P.nchunks - 1, true, true);
+    if constexpr (STAGED) {
+        __syncthreads();  // every thread is done with the forward pass's buffers
+        prefetch_chunk(P.nchunks - 2, false, true);
+        issue(P.nchunks - 1, (P.nchunks - 1) & 1, true);
+    } else {
+        prefetch_chunk(P.nchunks - 1, true, true);
+    }
     for (int64_t c = P.nchunks - 1; c >= 0; --c) {
         const int64_t t0 = c * KC;
         const int nt = static_cast<int>(L - t0 < KC ? L - t0 : KC);
-        prefetch_chunk(c - 1, true, true);
-        prefetch_chunk(c - 2, false, true);
+        const IO *sb = stage_base + (c & 1) * St::kElems;
+        if constexpr (STAGED) {
+            // chunk c has landed; every thread is done with chunk c + 1 (its buffer takes
+            // chunk c - 1) and with the previous chunk's sums in shared memory
+            cp_async_wait_all();
+            __syncthreads();
+            if (c >= 1) issue(c - 1, (c - 1) & 1, true);
+            prefetch_chunk(c - 2, false, true);
+        } else {
+            prefetch_chunk(c - 1, true, true);
+            prefetch_chunk(c - 2, false, true);
+        }
         if (c >= 1) prefetch_l1(ck + (c - 1) * N);
         // recompute the chunk's states h_{t0 .. t0+nt-1} (and each token's Abar) from its checkpoint
         f2 h_in[SP], hk[KC][SP], ab[KA][SP];
@@ -334,10 +478,10 @@ sscan_backward_kernel(const BwdParams P) {
             for (int k = 0; k < KC; ++k) {
                 const int64_t t = t0 + (k < nt ? k : nt - 1);  // loads need not wait behind work
                 float sg;
-                const float dl = step(t, sg);
-                const float x = Io<IO>::widen(Io<IO>::ld(u + t * D));
+                const float dl = step_raw(in_dl(sb, k, t), sg);
+                const float x = in_x(sb, k, t);
                 float Bv[S];
-                ldv_io<IO, S>(Bp + t * N, Bv);
+                in_B(sb, k, t, Bv);
                 const f2 dx2 = splat2(dl * x);
 #pragma unroll
                 for (int p = 0; p < SP; ++p) {
@@ -361,13 +505,13 @@ sscan_backward_kernel(const BwdParams P) {
             // token, unused), so the loads need not wait behind the previous token's work
             const int64_t t = t0 + (k < nt ? k : nt - 1);
             float sg;
-            const float dl = step(t, sg);
-            const float x = Io<IO>::widen(Io<IO>::ld(u + t * D));
-            float dyt = valid ? Io<IO>::widen(Io<IO>::ld(dyp + t * D)) : 0.0f;  // idle lanes add nothing
+            const float dl = step_raw(in_dl(sb, k, t), sg);
+            const float x = in_x(sb, k, t);
+            float dyt = valid ? in_dy(sb, k, t) : 0.0f;  // idle lanes add nothing
             float Bv[S], Cv[S];
-            ldv_io<IO, S>(Bp + t * N, Bv);
-            ldv_io<IO, S>(Cp + t * N, Cv);
-            const float zraw = (FUSED && zp != nullptr) ? Io<IO>::widen(Io<IO>::ld(zp + t * D)) : 0.0f;
+            in_B(sb, k, t, Bv);
+            in_C(sb, k, t, Cv);
+            const float zraw = (FUSED && zp != nullptr) ? in_z(sb, k, t) : 0.0f;
             if (k < nt) {
                 float ysp = 0.0f;
                 if (FUSED && zp != nullptr) {
@@ -485,7 +629,9 @@ sscan_backward_kernel(const BwdParams P) {
             }
             *reinterpret_cast<float4 *>(plane + ((b * L + t0 + k) * 2 + which) * N + 4 * q) = acc;
         }
-        __syncthreads();
+        // every thread done with this chunk's sums before the next chunk writes them (STAGED:
+        // the barrier at the top of the next chunk)
+        if constexpr (!STAGED) __syncthreads();
     }
     if (valid) {
         if (P.dh0 != nullptr) st_pairs(P.dh0 + (b * D + d) * N + n0, gs);

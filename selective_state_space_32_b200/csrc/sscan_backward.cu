@@ -39,11 +39,20 @@ size_t bwd_ckpt_bytes(int64_t B, int64_t L, int64_t D, int64_t N) {
     return (bytes + 255) / 256 * 256;
 }
 
+template <class IO, int N, int S, bool ZOH, bool FUSED, bool STAGED>
+int launch_backward_k(int64_t B, const BwdParams &prm, cudaStream_t s) {
+    const dim3 grid(static_cast<unsigned>(prm.Dpad / bwd_block_channels_s(N, S)), static_cast<unsigned>(B));
+    constexpr int smem = bwd_smem_bytes<IO, N, S, STAGED>();
+    if (smem_opt_in<sscan_backward_kernel<IO, N, S, ZOH, FUSED, STAGED>>(smem) != cudaSuccess) return SSCAN_ERR_CUDA;
+    sscan_backward_kernel<IO, N, S, ZOH, FUSED, STAGED><<<grid, kBwdThreads, smem, s>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? SSCAN_OK : SSCAN_ERR_CUDA;
+}
+
+// The staged kernel copies 4-byte words of every row: fp32, or bf16 with an even D.
 template <class IO, int N, int S, bool ZOH, bool FUSED>
 int launch_backward_t(int64_t B, const BwdParams &prm, cudaStream_t s) {
-    const dim3 grid(static_cast<unsigned>(prm.Dpad / bwd_block_channels_s(N, S)), static_cast<unsigned>(B));
-    sscan_backward_kernel<IO, N, S, ZOH, FUSED><<<grid, kBwdThreads, 0, s>>>(prm);
-    return cudaGetLastError() == cudaSuccess ? SSCAN_OK : SSCAN_ERR_CUDA;
+    if (sizeof(IO) == 4 || prm.D % 2 == 0) return launch_backward_k<IO, N, S, ZOH, FUSED, true>(B, prm, s);
+    return launch_backward_k<IO, N, S, ZOH, FUSED, false>(B, prm, s);
 }
 
 template <class IO, int N, int S>

@@ -86,6 +86,7 @@ CASES = [
     (2, 130, 36, 32, "bf16", True, True, False, False),
     (2, 50, 21, 64, "f32", True, True, True, True),        # N = 64, ZOH with A = 0, ragged D
     (1, 200, 40, 64, "bf16", False, True, True, False),
+    (2, 77, 45, 16, "bf16", True, True, False, False),     # odd D with bf16: rows not 4-byte aligned, unstaged
 ]
 
 
@@ -120,6 +121,7 @@ FUSED = [
     (2, 90, 96, 16, "bf16", False, True, True, True),
     (2, 40, 48, 16, "f32", False, False, True, False),      # bias only, no softplus, no gate
     (1, 33, 16, 16, "f32", False, True, True, False),       # softplus + bias, no gate
+    (2, 50, 33, 16, "bf16", False, True, True, True),       # odd D with bf16 (unstaged)
 ]
 
 
