@@ -148,9 +148,14 @@ struct BwdStage {
 };
 // dynamic shared memory of the backward kernel: the per-chunk partials, and two
 // staging buffers when STAGED
+// A row of the per-token dB / dC contributions ([channel][N] of one token): 16 floats of
+// padding put consecutive tokens' rows on opposite halves of the banks, so the
+// threads of the channel sums (one per token and four states) read 16-byte words
+// spread over all 32 banks.
+template <int S> constexpr int bwd_vrow() { return kBwdThreads * S + 16; }
 template <class IO, int N, int S, bool STAGED>
 constexpr int bwd_smem_bytes() {
-    return (3 * kChunk * kBwdThreads + 2 * kChunk * kBwdThreads * S) * 4 +
+    return (3 * kChunk * kBwdThreads + 2 * kChunk * bwd_vrow<S>()) * 4 +
            (STAGED ? 2 * BwdStage<IO, N, S>::kElems * int(sizeof(IO)) : 0);
 }
 
@@ -182,12 +187,12 @@ sscan_backward_kernel(const BwdParams P) {
     // token, and its S contributions to dB and dC per token ([k][channel][N] order)
     extern __shared__ __align__(16) unsigned char bsm[];
     float(*s_tok)[KC][kBwdThreads] = reinterpret_cast<float(*)[KC][kBwdThreads]>(bsm);
-    float(*s_vb)[kBwdThreads * S] =
-        reinterpret_cast<float(*)[kBwdThreads * S]>(bsm + 3 * KC * kBwdThreads * 4);
-    float(*s_vc)[kBwdThreads * S] = s_vb + KC;
+    constexpr int VR = bwd_vrow<S>();
+    float(*s_vb)[VR] = reinterpret_cast<float(*)[VR]>(bsm + 3 * KC * kBwdThreads * 4);
+    float(*s_vc)[VR] = s_vb + KC;
     // STAGED: two buffers of a chunk's inputs (BwdStage), filled by cp.async a chunk ahead
     using St = BwdStage<IO, N, S>;
-    IO *stage_base = reinterpret_cast<IO *>(bsm + (3 * KC * kBwdThreads + 2 * KC * kBwdThreads * S) * 4);
+    IO *stage_base = reinterpret_cast<IO *>(bsm + (3 * KC * kBwdThreads + 2 * KC * VR) * 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cl = lane / LPC, g = lane % LPC, n0 = S * g;
     const int64_t L = P.L, D = P.D;
