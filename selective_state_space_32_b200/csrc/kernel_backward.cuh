@@ -619,20 +619,29 @@ sscan_backward_kernel(const BwdParams P) {
             }
         }
         // dB, dC of each (token, four states): summed over the block's channels (the
-        // contributions sit in [k][channel][N] order) into this block's plane
+        // contributions sit in [k][channel][N] order) into this block's plane.  Two adjacent
+        // lanes share an item, one over the even channels and one over the odd, and meet by a
+        // shuffle (2 KC N/4 items: a multiple of the block's threads, so every lane takes part
+        // in every shuffle; rows past the chunk's end are summed and not stored).
         constexpr int kQ = N / 4;
+        static_assert((4 * KC * kQ) % kBwdThreads == 0 && CPB % 2 == 0, "two lanes per item, every lane busy");
         float *plane = P.part + static_cast<int64_t>(blockIdx.x) * gridDim.y * L * 2 * N;
-        for (int e = threadIdx.x; e < 2 * KC * kQ; e += kBwdThreads) {
-            const int which = e / (KC * kQ), r = e % (KC * kQ), k = r / kQ, q = r % kQ;
-            if (k >= nt) continue;
-            const float *src = (which ? &s_vc[k][0] : &s_vb[k][0]) + 4 * q;
+        for (int e = threadIdx.x; e < 4 * KC * kQ; e += kBwdThreads) {
+            const int item = e >> 1, half = e & 1;
+            const int which = item / (KC * kQ), r = item % (KC * kQ), k = r / kQ, q = r % kQ;
+            const float *src = (which ? &s_vc[k][0] : &s_vb[k][0]) + 4 * q + half * N;
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
-            for (int j = 0; j < CPB; ++j) {
-                const float4 v = *reinterpret_cast<const float4 *>(src + j * N);
+            for (int j = 0; j < CPB / 2; ++j) {
+                const float4 v = *reinterpret_cast<const float4 *>(src + 2 * j * N);
                 acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
             }
-            *reinterpret_cast<float4 *>(plane + ((b * L + t0 + k) * 2 + which) * N + 4 * q) = acc;
+            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 1);
+            acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 1);
+            acc.z += __shfl_xor_sync(0xffffffffu, acc.z, 1);
+            acc.w += __shfl_xor_sync(0xffffffffu, acc.w, 1);
+            if (half == 0 && k < nt)
+                *reinterpret_cast<float4 *>(plane + ((b * L + t0 + k) * 2 + which) * N + 4 * q) = acc;
         }
         // every thread done with this chunk's sums before the next chunk writes them (STAGED:
         // the barrier at the top of the next chunk)
