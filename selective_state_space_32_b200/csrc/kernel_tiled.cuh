@@ -33,6 +33,8 @@
 // the chained kernel's (discretize / advance, kernel_chained.cuh).
 #pragma once
 
+#include <type_traits>
+
 #include "kernel_chained.cuh"
 
 namespace sscan {
@@ -73,6 +75,37 @@ struct TiledCfg {
     static_assert(T % 8 == 0, "token groups divide a stage");
     static_assert(T * CPW % 32 == 0 && kScratch % 128 == 0, "fused tile entries per lane");
 };
+
+// Exact ZOH at bf16 precision without a select, for a warp whose every A is <= 0:
+// the coefficient (Abar - 1)/A as min(Abar (1/A) - (1 + 2^-21)/A, delta).  The bias
+// 2^-21/|A| exceeds the error of Abar (ex2.approx, about 2^-22) and makes the first
+// form an upper bound of the exact c = delta phi(delta A) in the signed sense, and
+// c <= delta for A <= 0, so where the first form has lost its relative accuracy
+// (|delta A| below about 2^-10) the min takes delta (relative error |delta A|/2),
+// and elsewhere the first form (relative error 2^-21 / |delta A|): at most about
+// 2^-11, against the 2^-9 rounding of a bf16 output.  A = 0: 1/A is infinite, the
+// first form NaN, and fminf returns delta, the exact limit.
+template <int NP>
+__device__ __forceinline__ void discretize_zoh_min(f2 (&ab)[NP], f2 (&bu)[NP], const f2 (&A2)[NP],
+                                                   const f2 (&iA)[NP], float x, float dl, const float *Bs) {
+    const f2 dd = splat2(dl), xx = splat2(x);
+    const f2 kBias = splat2(-(1.0f + 0x1p-21f));
+#pragma unroll
+    for (int i = 0; i < NP / 2; ++i) {
+        const float4 bv = reinterpret_cast<const float4 *>(Bs)[i];
+        const f2 b01 = pack2(bv.x, bv.y), b23 = pack2(bv.z, bv.w);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int p = 2 * i + q;
+            float e0, e1;
+            unpack2(mul2(dd, A2[p]), e0, e1);
+            ab[p] = pack2(ex2(e0), ex2(e1));
+            float c0, c1;
+            unpack2(fma2(ab[p], iA[p], mul2(iA[p], kBias)), c0, c1);
+            bu[p] = mul2(pack2(fminf(c0, dl), fminf(c1, dl)), mul2(q ? b23 : b01, xx));
+        }
+    }
+}
 
 // The producer warp: TMA issue in the block's processing order, at most STAGES
 // stages ahead of the consumers, and the fp32 copy of every landed stage's B and
@@ -333,6 +366,18 @@ sscan_tiled_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_consta
             const int64_t dp = cg * CPB + warp * CPW + lane % CPW;
             biasv = dp < D ? __ldg(P.delta_bias + dp) : 0.0f;
         }
+        // bf16 ZOH: the select-free coefficient when every A of the warp is <= 0 (decided
+        // once per part, the same for every stage: two copies of the stage loop)
+        bool a_nonpos = true;
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+            float x0, x1;
+            unpack2(A2[p], x0, x1);
+            a_nonpos = a_nonpos && x0 <= 0.0f && x1 <= 0.0f;
+        }
+        a_nonpos = __all_sync(0xffffffffu, a_nonpos);
+        auto stages = [&](auto min_tag) {
+        constexpr bool MINF = decltype(min_tag)::value;
         for (int64_t t0 = ts; t0 < te; t0 += T) {
             const int s = static_cast<int>(consumed % STAGES);
             const uint32_t par = static_cast<uint32_t>((consumed / STAGES) & 1);
@@ -390,10 +435,15 @@ sscan_tiled_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_consta
                 const bool g_store = LPC <= GZ || (g & (LPC / GZ - 1)) == 0;
                 f2 ab[GZ][NP], bu[GZ][NP];
 #pragma unroll
-                for (int q = 0; q < GZ; ++q)
-                    discretize<NP, true, false, 0, Cfg::ES == 2, true>(ab[q], bu[q], A2, A1, iA, 0.0f,
-                                                                 x_at(j0 + q), delta_at(j0 + q),
-                                                                 Bs + (j0 + q) * RS);
+                for (int q = 0; q < GZ; ++q) {
+                    if constexpr (MINF)
+                        discretize_zoh_min<NP>(ab[q], bu[q], A2, iA, x_at(j0 + q), delta_at(j0 + q),
+                                               Bs + (j0 + q) * RS);
+                    else
+                        discretize<NP, true, false, 0, Cfg::ES == 2, true>(ab[q], bu[q], A2, A1, iA, 0.0f,
+                                                                     x_at(j0 + q), delta_at(j0 + q),
+                                                                     Bs + (j0 + q) * RS);
+                }
                 float yv[GZ];
 #pragma unroll
                 for (int q = 0; q < GZ; ++q) yv[q] = advance<NP>(h, ab[q], bu[q], Cs + (j0 + q) * RS);
@@ -440,6 +490,11 @@ sscan_tiled_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_consta
             if (lane == 0) mbar_arrive(&empty[s]);
             ++consumed;
         }
+        };
+        if (ZOH && Cfg::ES == 2 && a_nonpos)
+            stages(std::true_type());
+        else
+            stages(std::false_type());
         if (failed) break;
 
         if (te < L && !P.drop_publish) {

@@ -138,6 +138,32 @@ def test_tiled_kernel_forced(case, monkeypatch):
     plan.close()
 
 
+@pytest.mark.parametrize("a_case", ["zero", "positive"])
+def test_tiled_zoh_bf16_sign_of_A(a_case, monkeypatch):
+    """The tiled kernel's bf16 ZOH coefficient: warps whose every A is <= 0 take the
+    select-free form min(Abar/A - (1 + 2^-21)/A, delta), which must give delta where A = 0
+    (the first form is NaN there); a warp with a positive A takes the select."""
+    Bt, L, D, N = 2, 300, 96, 64
+    g = W.generate(Bt, L, D, N, "bf16", 0.1, seed=2600, A_jitter=0.3)
+    A = g["A"].copy()
+    if a_case == "zero":
+        A[:, 0] = 0.0          # every channel's first state, in every warp
+        A[7, 5:9] = 0.0
+    else:
+        A[5, 3] = 0.05         # one growing state in the first warp of a block-chain
+    g["A"] = A
+    monkeypatch.setenv("SSCAN_TUNE", "tiled=0,sms=3")
+    plan = S.Plan(Bt, L, D, N, torch.bfloat16, True)
+    assert "kernel=tiled" in plan.describe(), plan.describe()
+    d = P.to_device(g)
+    y, hf = plan.forward(d["u"], d["delta"], d["A"], d["B"], d["C"], d["h0"])
+    assert plan.status() == S.OK
+    yr, hr = P.run_oracle(g, True)
+    P.check(y.float().cpu().numpy(), yr, "bf16", "y")
+    P.check(hf.cpu().numpy(), hr, "bf16", "h_final")
+    plan.close()
+
+
 def test_tiled_lost_carry_times_out_and_is_reported(monkeypatch):
     """The tiled kernel's failure detection: block-chain heads skip publishing their
     warps' states, the tails' bounded waits give up, the status word reports it, and the
