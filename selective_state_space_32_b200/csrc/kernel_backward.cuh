@@ -121,6 +121,9 @@ __device__ __forceinline__ void prefetch_l1(const void *p) {
 __device__ __forceinline__ void cp_async4(void *dst, const void *src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
@@ -156,7 +159,7 @@ template <int S> constexpr int bwd_vrow() { return kBwdThreads * S + 16; }
 template <class IO, int N, int S, bool STAGED>
 constexpr int bwd_smem_bytes() {
     return (3 * kChunk * kBwdThreads + 2 * kChunk * bwd_vrow<S>()) * 4 +
-           (STAGED ? 2 * BwdStage<IO, N, S>::kElems * int(sizeof(IO)) : 0);
+           (STAGED ? 2 * BwdStage<IO, N, S>::kElems * int(sizeof(IO)) + 2 * kBwdThreads * S * 4 : 0);
 }
 
 // Sum of LPC consecutive floats in shared memory (16-byte aligned when LPC >= 4).
@@ -193,6 +196,8 @@ sscan_backward_kernel(const BwdParams P) {
     // STAGED: two buffers of a chunk's inputs (BwdStage), filled by cp.async a chunk ahead
     using St = BwdStage<IO, N, S>;
     IO *stage_base = reinterpret_cast<IO *>(bsm + (3 * KC * kBwdThreads + 2 * KC * VR) * 4);
+    // STAGED: two buffers of each lane's checkpoint for the reverse sweep, [buffer][thread][S]
+    float *ck_stage = reinterpret_cast<float *>(stage_base + 2 * St::kElems);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cl = lane / LPC, g = lane % LPC, n0 = S * g;
     const int64_t L = P.L, D = P.D;
@@ -314,6 +319,7 @@ sscan_backward_kernel(const BwdParams P) {
             const int64_t t = t0 + (k < nt ? k : nt - 1);
             cp_async4(sb + (which ? St::kC : St::kB) + k * N + w * EPW, (which ? C_row : B_row) + t * N + w * EPW);
         }
+        if (rev) cp_async16(ck_stage + (buf * kBwdThreads + threadIdx.x) * S, ck + c * N);  // this lane's own
         cp_async_commit();
     };
     const int ch = warp * CPW + cl;  // this lane's channel within the block
@@ -468,10 +474,16 @@ sscan_backward_kernel(const BwdParams P) {
             prefetch_chunk(c - 1, true, true);
             prefetch_chunk(c - 2, false, true);
         }
-        if (c >= 1) prefetch_l1(ck + (c - 1) * N);
+        if (!STAGED && c >= 1) prefetch_l1(ck + (c - 1) * N);
         // recompute the chunk's states h_{t0 .. t0+nt-1} (and each token's Abar) from its checkpoint
         f2 h_in[SP], hk[KC][SP], ab[KA][SP];
-        ld_pairs(ck + c * N, h_in, false);
+        if constexpr (STAGED) {
+            const float4 v = *reinterpret_cast<const float4 *>(ck_stage + ((c & 1) * kBwdThreads + threadIdx.x) * S);
+            h_in[0] = pack2(v.x, v.y);
+            h_in[1] = pack2(v.z, v.w);
+        } else {
+            ld_pairs(ck + c * N, h_in, false);
+        }
         {
             f2 hc[SP];
 #pragma unroll
