@@ -30,7 +30,9 @@
 // warp's state at the cut; the later block runs the tail last, each warp
 // reading its own part (epoch-tagged flags, bounded waits; the grid is launched
 // cooperatively, so every block is resident).  Arithmetic per state update is
-// the chained kernel's (discretize / advance, kernel_chained.cuh).
+// the chained kernel's (discretize / advance, kernel_chained.cuh), except the
+// bf16-precision ZOH coefficient of warps whose every A is <= 0, which takes a
+// select-free form (discretize_zoh_min).
 #pragma once
 
 #include <type_traits>
